@@ -1,0 +1,437 @@
+#!/usr/bin/env python
+"""Benchmark: DF11 decompression of BF16 weights on B200.
+
+A step is one pass of the whole decode path over one stream: one kernel launch
+that rebuilds every matrix of a Llama-3.1-8B-shaped transformer block
+(218,112,000 BF16 weights, one shared code table) from its DF11 stream, with
+the compressed arrays already resident in HBM.  The workload's inputs and
+output (~726 MB per step) exceed the 126 MB L2, so no flush is needed between
+steps.  Every timed output is compared bit for bit with the original weights.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config c3]
+  python bench.py --impl reference ...   # the CPU oracle on the host cores
+
+Under torchrun (N > 1) every rank decompresses its own block (other seeds):
+independent streams, no data-path collective ("weak" scaling); the timed
+region is bracketed by barriers and the slowest rank's time is reported.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import platform
+import re
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decompressed BF16 GB/s on 1 B200 (bit-exact), % of HBM roofline"
+UNIT = "GB/s"
+FALLBACK_HBM_GBS = 6650.0
+KERNEL_SOURCE = os.path.join(ROOT, "lossless_entropy_coded_dfloat11_b200", "csrc", "df11_decode.cu")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_kernel_llama8b_block.txt")
+
+CONFIGS = {
+    "c1": "matrix_1k: one 1024x1024 BF16 matrix, N(0, 0.02)",
+    "c2": "matrix_outliers: one 14336x4096 BF16 matrix, N(0, 0.02), 0.1% Laplace(0, 0.5) outliers, 0.01% zeros",
+    "c3": "llama3.1-8b-block: q/o 4096x4096, k/v 1024x4096, gate/up 14336x4096, down 4096x14336, "
+          "2 RMSNorm 4096; 218,112,000 BF16 weights, one table, one launch",
+    "c4": "8 llama3.1-70b-blocks: hidden 8192, intermediate 28672, kv 1024x8192; 855,654,400 weights "
+          "per block, each block one launch into one reused buffer",
+}
+
+
+# --------------------------------------------------------------------------- #
+# helpers shared with the CPU tests                                           #
+# --------------------------------------------------------------------------- #
+def aggregate(per_rank_elapsed_ms: list[float], bytes_per_rank_step: int, steps: int) -> dict:
+    """Whole-job throughput: all ranks' bytes over the slowest rank's time."""
+    t = max(per_rank_elapsed_ms)
+    total = bytes_per_rank_step * steps * len(per_rank_elapsed_ms)
+    return {"ms": t, "gbs": total / (t * 1e-3) / 1e9, "ms_per_step": t / steps}
+
+
+def rank_seed_offset(rank: int) -> int:
+    """Each rank draws its own block (seeds shifted by 1000 per rank)."""
+    return 1000 * rank
+
+
+def measured_peak_gbs() -> tuple[float, str]:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            v = float(json.load(f)["hbm_gbs"])
+        return v, "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def recorded_traffic() -> float | None:
+    """DRAM bytes per launch from the committed ncu summary, only while the
+    kernel source still matches the one that was profiled."""
+    try:
+        text = open(TRAFFIC_FILE).read()
+    except OSError:
+        return None
+    m_sha = re.search(r"kernel_source_sha256:\s*([0-9a-f]{64})", text)
+    m_tr = re.search(r"traffic_bytes_per_launch_full_size:\s*([0-9.eE+]+)", text)
+    if not m_sha or not m_tr:
+        return None
+    sha = hashlib.sha256(open(KERNEL_SOURCE, "rb").read()).hexdigest()
+    return float(m_tr.group(1)) if sha == m_sha.group(1) else None
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int, interval_s: float = 0.005):
+        self.interval = interval_s
+        self.samples, self.reasons = [], 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        self.handle = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.handle = self._handle(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM)
+        except Exception:  # NVML missing: no clock record
+            self.handle = None
+
+    def _handle(self, idx):
+        import torch
+        p = self.nvml
+        props = torch.cuda.get_device_properties(idx)
+        bus = getattr(props, "pci_bus_id", None)
+        if bus is not None:
+            try:
+                busid = "%08X:%02X:%02X.0" % (getattr(props, "pci_domain_id", 0), bus,
+                                               getattr(props, "pci_device_id", 0))
+                return p.nvmlDeviceGetHandleByPciBusId(busid)
+            except Exception:
+                pass
+        return p.nvmlDeviceGetHandleByIndex(idx)
+
+    def _run(self):
+        p = self.nvml
+        while not self._stop.is_set():
+            try:
+                self.samples.append(p.nvmlDeviceGetClockInfo(self.handle, p.NVML_CLOCK_SM))
+                self.reasons |= int(p.nvmlDeviceGetCurrentClocksEventReasons(self.handle))
+            except Exception:
+                pass
+            time.sleep(self.interval)
+
+    def __enter__(self):
+        if self.handle is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thread:
+            self._thread.join()
+
+    def record(self) -> dict | None:
+        if self.handle is None or not self.samples:
+            return None
+        s = sorted(self.samples)
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": s[len(s) // 2], "sm_max_mhz": self.max_mhz, "reasons": names,
+                "samples": len(s)}
+
+
+def cpu_model() -> str:
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return platform.processor() or "unknown"
+
+
+# --------------------------------------------------------------------------- #
+# workloads                                                                   #
+# --------------------------------------------------------------------------- #
+def make_workloads(config: str, rank: int, device: str):
+    from lossless_entropy_coded_dfloat11_b200 import inputs as I
+    off = rank_seed_offset(rank)
+    if config == "c1":
+        return [I.Workload("matrix_1k", ["w"], [I.gaussian((1024, 1024), 0.02, 1 + off, device=device)])]
+    if config == "c2":
+        return [I.matrix_outliers(seed=2 + off, device=device)]
+    if config == "c3":
+        return [I.llama_block(I.LLAMA_8B, seed_base=3 + off, device=device)]
+    if config == "c4":
+        return [I.llama_block(I.LLAMA_70B, seed_base=100 + 16 * b + off, device=device) for b in range(8)]
+    raise ValueError(config)
+
+
+def reference_sample(config: str, n_target: int):
+    """Host-side sample for the CPU oracle: the first n_target elements of the
+    workload's concatenated matrices, drawn with the CPU generator."""
+    import numpy as np
+    from lossless_entropy_coded_dfloat11_b200 import inputs as I
+    if config == "c4":
+        cfg, base = I.LLAMA_70B, 100
+    elif config == "c3":
+        cfg, base = I.LLAMA_8B, 3
+    else:
+        w = I.matrix_1k() if config == "c1" else I.matrix_outliers()
+        return w.flat_u16()[:n_target]
+    parts, have = [], 0
+    for k, (name, shape) in enumerate(I.block_shapes(**cfg)):
+        if have >= n_target:
+            break
+        if len(shape) == 1:
+            t = I.gaussian(shape, 0.05, base + k, mean=1.0)
+        else:
+            t = I.gaussian(shape, 1.0 / (shape[1] ** 0.5), base + k)
+        parts.append(t.reshape(-1).view(__import__("torch").int16).numpy().view(np.uint16)[: n_target - have])
+        have += parts[-1].size
+    return np.concatenate(parts)
+
+
+def time_oracle_decode(x, steps: int, warmup: int):
+    """Oracle (single-threaded C, as it stands) decode of a fixed sample."""
+    import numpy as np
+    import oracle
+    s = oracle.encode(x)
+    for _ in range(warmup):
+        oracle.decode(s)
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        y = oracle.decode(s)
+    dt = time.perf_counter() - t0
+    assert np.array_equal(y, x), "oracle round trip failed"
+    return dt, s
+
+
+# --------------------------------------------------------------------------- #
+# arms                                                                        #
+# --------------------------------------------------------------------------- #
+def run_reference(args, rank: int, world: int) -> None:
+    if rank != 0:
+        return
+    n_sample = args.ref_sample
+    x = reference_sample(args.config, n_sample)
+    dt, s = time_oracle_decode(x, args.steps, args.warmup)
+    value = 2 * x.size * args.steps / dt / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u8",
+        "data": "synthetic",
+        "config": {"workload": CONFIGS[args.config], "reference_sample_elements": int(x.size)},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": f"oracle bit-serial decode of the first {x.size} elements of the "
+                                   f"workload per step, single thread on {cpu_model()} "
+                                   f"({os.cpu_count()} host cores present)"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_native(args, rank: int, world: int, local_rank: int) -> None:
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    import lossless_entropy_coded_dfloat11_b200 as df11
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    df11.load_library()
+
+    # ---- build the compressed workload on this GPU ------------------------
+    workloads = make_workloads(args.config, rank, "cuda")
+    streams, originals = [], []
+    for w in workloads:
+        cs = df11.compress(w.tensors, names=w.names)
+        streams.append(cs)
+        originals.append(torch.cat([t.reshape(-1) for t in w.tensors]).view(torch.int16)
+                         if len(workloads) == 1 else None)
+        if len(workloads) > 1:
+            # keep a fingerprint per block instead of all 6.9B weights
+            originals[-1] = [t.reshape(-1).view(torch.int16)[:: 4093].clone() for t in w.tensors]
+        del w
+    torch.cuda.synchronize()
+    n_max = max(cs.n_elems for cs in streams)
+    out = torch.empty(n_max, dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream()
+    out_bytes = sum(2 * cs.n_elems for cs in streams)
+    alg_bytes = sum(cs.read_bytes() + 2 * cs.n_elems for cs in streams)
+    launches_per_step = len(streams)
+
+    def step():
+        for cs in streams:
+            df11.decompress(cs, out=out[: cs.n_elems], stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    # ---- timed region -------------------------------------------------------
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local_rank)
+    with sampler:
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    elapsed = ev0.elapsed_time(ev1)
+
+    # ---- bit-exact check of the last step's output --------------------------
+    exact = True
+    if len(streams) == 1:
+        exact = bool(torch.equal(out[: streams[0].n_elems].view(torch.int16), originals[0]))
+    else:
+        for cs, fp in zip(streams, originals):
+            step_out = df11.decompress(cs, out=out[: cs.n_elems], stream=stream)
+            for v, f in zip(cs.views(step_out), fp):
+                exact &= bool(torch.equal(v.reshape(-1).view(torch.int16)[:: 4093], f))
+    torch.cuda.synchronize()
+
+    per_rank = [elapsed]
+    if world > 1:
+        t = torch.tensor([elapsed], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        per_rank = [float(t.item())] * world
+        e = torch.tensor([1 if exact else 0], device=dev, dtype=torch.int32)
+        dist.all_reduce(e, op=dist.ReduceOp.MIN)
+        exact = bool(e.item())
+    agg = aggregate(per_rank, out_bytes, args.steps)
+
+    # ---- end to end: host buffers through the public API --------------------
+    e2e = None
+    if not args.no_e2e and len(streams) == 1:
+        hs = df11.HostStream(streams[0])
+        for _ in range(2):
+            hs.run(stream)
+        torch.cuda.synchronize()
+        k = args.e2e_steps
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(k):
+            res = hs.run(stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ems = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([ems], device=dev, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ems = float(t.item())
+        e2e_exact = bool(torch.equal(res.view(torch.int16), originals[0].cpu()))
+        e2e = {"value": 2 * streams[0].n_elems * k * world / (ems * 1e-3) / 1e9, "unit": UNIT,
+               "h2d_bytes_per_step": hs.h2d_bytes(), "d2h_bytes_per_step": hs.d2h_bytes(),
+               "steps": k, "bit_exact": e2e_exact}
+        del hs
+
+    # ---- CPU baseline (oracle, rank 0, one GPU) ----------------------------
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        n_sample = min(args.cpu_sample, streams[0].n_elems)
+        if len(streams) == 1:
+            x = originals[0][:n_sample].cpu().numpy().view(np.uint16)
+        else:
+            x = reference_sample(args.config, n_sample)
+        dt, _ = time_oracle_decode(x, 1, 0)
+        cpu = {"value": 2 * x.size / dt / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
+               "sample": f"first {x.size} elements of the workload, oracle bit-serial decode, one "
+                         f"thread on {cpu_model()} ({os.cpu_count()} host cores present)",
+               "seconds": dt}
+
+    if rank != 0:
+        return
+    peak, peak_kind = measured_peak_gbs()
+    launch_ms = elapsed / (args.steps * launches_per_step)
+    achieved = (alg_bytes / launches_per_step) / (launch_ms * 1e-3) / 1e9
+    traffic = recorded_traffic() if args.config == "c3" else None
+    cs0 = streams[0]
+    line = {
+        "metric": METRIC, "value": agg["gbs"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": agg["ms_per_step"], "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "u8", "data": "synthetic",
+        "config": {"workload": CONFIGS[args.config], "elements_per_step": sum(c.n_elems for c in streams),
+                   "threads_per_block": cs0.threads_per_block, "launches_per_step": launches_per_step,
+                   "l2": "no flush: compressed input + BF16 output per step exceed the 126 MB L2",
+                   "parallelism": f"replicas x{world} (independent streams per rank)"},
+        "bit_exact": exact,
+        "elements_per_s": agg["gbs"] * 1e9 / 2,
+        "compression_ratio": sum(c.compressed_bytes() for c in streams) / out_bytes,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": traffic,
+                     "peak_kind": f"{peak_kind} (copy bandwidth)",
+                     "algorithmic_bytes_per_launch": alg_bytes / launches_per_step,
+                     "frac_of_8000_nominal": achieved / 8000.0},
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": args.steps * launches_per_step,
+        "clocks": sampler.record(),
+        "when": datetime.datetime.now(datetime.timezone.utc).isoformat(timespec="seconds"),
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--config", choices=sorted(CONFIGS), default="c3")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--cpu-sample", type=int, default=218_112_000,
+                    help="elements the CPU baseline decodes (bounded sample)")
+    ap.add_argument("--ref-sample", type=int, default=1_000_000,
+                    help="elements per step in the reference arm")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("at least 3 warm-up steps")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        run_native(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

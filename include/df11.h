@@ -1,0 +1,178 @@
+/*
+ * df11.h -- C ABI of the DF11 (DFloat11) codec for BF16 weights on B200.
+ *
+ * What the format is ("DFloat11: compressao sem perda para inferencia em GPU
+ * que reduz LLMs para 70% do tamanho", section "O formato DFloat11"; abstract
+ * of "70% Size, 100% Accuracy: Lossless LLM Compression for Efficient GPU
+ * Inference via Dynamic-Length Float"): every BF16 value is split into its
+ * 8-bit exponent and a byte holding sign and mantissa.  The exponents are
+ * Huffman-coded into the bit-packed EncodedExponent array; the sign+mantissa
+ * bytes are kept raw in PackedSignMantissa.  Decoding rebuilds the original
+ * BF16 bits exactly.
+ *
+ * Decoder metadata (section "Kernel de GPU em 2 etapas e metadados
+ * auxiliares"): each GPU thread owns an 8-byte window of EncodedExponent and
+ * decodes the codes that start in it; a 5-bit Gaps entry per thread gives the
+ * offset of its first code, and one 32-bit output position per thread block
+ * gives where the block's decoded elements go.
+ *
+ * Byte layout (readings of points the pages leave open):
+ *   - PackedSignMantissa byte = sign << 7 | mantissa (7 bits).
+ *   - EncodedExponent is MSB-first: stream bit p is bit 7 - p%8 of byte p/8.
+ *   - Codes are canonical: present exponents sorted by (length, value), the
+ *     first code is all zeros, each next code is (previous + 1) shifted left
+ *     by the length increase.  Lengths are the optimal prefix code with at
+ *     most max_code_len (<= 32) bits, computed by package-merge; on equal
+ *     counts the lower exponent value counts as the lighter symbol, and a
+ *     leaf sorts before a package of equal weight.  One present exponent
+ *     gets the 1-bit code "0".
+ *   - n_threads = ceil(total_bits / 64), n_blocks = ceil(n_threads / T).
+ *   - Gaps: n_threads 5-bit fields, field t at array bits 5t..5t+4, array bit
+ *     q being bit q%8 of byte q/8.  gap[t] = (first code start >= 64t, or
+ *     total_bits if none) - 64t, always in [0, 31].
+ *   - Block offsets: uint32 off[n_blocks + 1]; off[b] = number of codes that
+ *     start before stream bit 64*T*b; off[n_blocks] = n_elems.
+ *   - Buffer sizes (all zero-padded): bytes_exp = 8*T*n_blocks + 16,
+ *     bytes_sm = n_elems rounded up to 16, bytes_gaps = ceil(5*T*n_blocks/8)
+ *     + 8 rounded up to 16, bytes_off = 4*(n_blocks + 1).
+ *
+ * Ownership: every buffer belongs to the caller.  Device pointers must be
+ * 16-byte aligned.  No entry point allocates device memory; the compress
+ * entry points use a caller-provided device workspace.
+ *
+ * Errors: every call returns a df11_status; nothing aborts or throws across
+ * the ABI.  df11_last_error() returns a message for the last failing call on
+ * the calling host thread.  A stream that is inconsistent with its metadata is
+ * reported by the kernel through the optional device status word (a bitwise
+ * OR of df11_status values, 0 when clean) and never traps.
+ */
+#ifndef DF11_H
+#define DF11_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define DF11_VERSION 1
+#define DF11_WINDOW_BYTES 8
+#define DF11_MAX_CODE_LEN 32
+#define DF11_MAX_SEGMENTS 64
+
+typedef enum {
+    DF11_OK = 0,
+    DF11_ERR_INVALID = 1,   /* bad argument, misaligned pointer, bad table   */
+    DF11_ERR_CUDA = 2,      /* a CUDA runtime call failed                    */
+    DF11_ERR_CORRUPT = 3,   /* stream disagrees with its Gaps / block offsets */
+    DF11_ERR_TOO_LARGE = 4, /* n_elems >= 2^32 (block offsets are 32-bit)    */
+    DF11_ERR_CAPACITY = 5   /* a buffer is smaller than the header needs     */
+} df11_status;
+
+/* Host-side description of one DF11 stream: one matrix, or every matrix of a
+ * transformer block concatenated in order (one shared code table). */
+typedef struct {
+    uint32_t version;            /* DF11_VERSION                               */
+    uint32_t window_bytes;       /* 8                                          */
+    uint32_t threads_per_block;  /* T: 64, 128, 256, 512 or 1024               */
+    uint32_t max_code_len;       /* L used to build the code, 1..32            */
+    uint64_t n_elems;            /* BF16 elements, < 2^32                      */
+    uint64_t total_bits;         /* bits in EncodedExponent                    */
+    uint64_t n_threads;          /* ceil(total_bits / 64)                      */
+    uint64_t n_blocks;           /* ceil(n_threads / T)                        */
+    uint8_t code_len[256];       /* code length per exponent value, 0 = absent */
+    uint32_t n_segments;         /* matrices in the stream, 1..64              */
+    uint32_t reserved;
+    uint64_t seg_elem_off[DF11_MAX_SEGMENTS + 1]; /* segment k = elements
+                                    [seg_elem_off[k], seg_elem_off[k+1])       */
+    uint64_t bytes_exp;          /* EncodedExponent buffer size                */
+    uint64_t bytes_sm;           /* PackedSignMantissa buffer size             */
+    uint64_t bytes_gaps;         /* Gaps buffer size                           */
+    uint64_t bytes_off;          /* block offsets buffer size                  */
+    uint64_t bytes_lut;          /* decode tables size (df11_build_lut)        */
+} df11_header;
+
+/* Library version (DF11_VERSION). */
+int df11_version(void);
+
+/* Message for the last failing call on this host thread ("" if none). */
+const char* df11_last_error(void);
+
+/* Optimal length-limited code lengths for an exponent histogram
+ * ("O formato DFloat11": a Huffman code over the exponent distribution, here
+ * with at most max_code_len bits).  Host only, no GPU needed.
+ *   hist[256]      in: count per exponent value
+ *   max_code_len   in: 1..32, 2^max_code_len >= number of present values
+ *   code_len[256]  out: length per value, 0 where hist is 0
+ * Returns DF11_ERR_INVALID on a bad limit. */
+df11_status df11_code_lengths(const uint64_t* hist, uint32_t max_code_len, uint8_t* code_len);
+
+/* Fill a header for a given code table and sizes (used for streams made
+ * elsewhere, e.g. read from disk).  Host only.
+ *   code_len[256]       in: lengths; must form a prefix code (Kraft <= 1,
+ *                           equality required for >= 2 present values)
+ *   n_elems, total_bits in: element count (< 2^32) and stream length in bits
+ *   threads_per_block   in: T (64..1024, power of two)
+ *   seg_counts[n_segs]  in: elements per segment, summing to n_elems; NULL
+ *                           with n_segs = 1 means one segment
+ * Validates and fills every size field, including bytes_lut. */
+df11_status df11_header_init(df11_header* hdr, const uint8_t* code_len, uint64_t n_elems,
+                             uint64_t total_bits, uint32_t threads_per_block,
+                             uint32_t max_code_len, const uint64_t* seg_counts,
+                             uint32_t n_segs);
+
+/* Build the decoder's tables for hdr->code_len into host memory h_lut
+ * (capacity cap >= hdr->bytes_lut).  The caller copies them to the device
+ * once per stream; df11_decompress reads them from there.  Host only.
+ * (Section "Decodificacao com LUT hierarquica": compact lookup tables that
+ * fit in on-chip memory, used instead of a bit-level tree walk.) */
+df11_status df11_build_lut(const df11_header* hdr, void* h_lut, uint64_t cap);
+
+/* Device workspace the compress entry points need for n_elems elements. */
+df11_status df11_compress_workspace_size(uint64_t n_elems, uint64_t* bytes);
+
+/* Compress, step 1 of 2 ("O formato DFloat11"): exponent histogram on the
+ * GPU, then the code built on the host; fills *hdr (code_len, total_bits and
+ * every buffer size).  Synchronises `stream` once (histogram readback).
+ *   d_segs[n_segs]      in: device pointers to BF16 data, 16-byte aligned
+ *   seg_counts[n_segs]  in: elements per segment (sum < 2^32); n_segs 1..64
+ *   threads_per_block   in: T; max_code_len in: L (1..32; 32 = the pages')
+ *   d_workspace         in: device scratch of >= workspace_bytes bytes
+ *   stream              in: cudaStream_t (NULL = default stream) */
+df11_status df11_compress_plan(const void* const* d_segs, const uint64_t* seg_counts,
+                               uint32_t n_segs, uint32_t threads_per_block,
+                               uint32_t max_code_len, void* d_workspace,
+                               uint64_t workspace_bytes, df11_header* hdr, void* stream);
+
+/* Compress, step 2 of 2: bit-pack kernel.  Writes EncodedExponent,
+ * PackedSignMantissa, Gaps and block offsets into caller buffers of at least
+ * the header's sizes, and the decode tables into d_lut (hdr->bytes_lut).
+ * Asynchronous on `stream`; d_segs must hold the data the plan saw. */
+df11_status df11_compress_encode(const void* const* d_segs, const df11_header* hdr,
+                                 void* d_workspace, uint64_t workspace_bytes, uint8_t* d_exp,
+                                 uint8_t* d_sm, uint8_t* d_gaps, uint32_t* d_block_off,
+                                 void* d_lut, void* stream);
+
+/* Decompress one stream -- every matrix of a transformer block -- in one
+ * kernel launch ("Descompressao por bloco de transformer"; two-phase kernel of
+ * "Kernel de GPU em 2 etapas e metadados auxiliares").
+ *   d_exp, d_sm, d_gaps, d_block_off  in: the stream's device arrays
+ *   d_lut       in: device copy of df11_build_lut's output for this header
+ *   d_out       out: n_elems BF16 values (uint16 bit patterns), contiguous;
+ *               segment k starts at element seg_elem_off[k]
+ *   d_status    in/out, may be NULL: device word OR-ed with DF11_ERR_CORRUPT
+ *               if the stream disagrees with its metadata (the caller zeroes it)
+ *   stream      cudaStream_t (NULL = default stream)
+ * Asynchronous: no allocation, no host synchronisation.  n_elems = 0 is a
+ * no-op. */
+df11_status df11_decompress(const df11_header* hdr, const uint8_t* d_exp, const uint8_t* d_sm,
+                            const uint8_t* d_gaps, const uint32_t* d_block_off,
+                            const void* d_lut, uint16_t* d_out, uint32_t* d_status,
+                            void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DF11_H */

@@ -1,0 +1,14 @@
+"""DF11 (DFloat11) lossless BF16 weight codec for NVIDIA B200 (sm_100a).
+
+The codec runs in libdf11.so (hand-written CUDA kernels plus a C++ code
+builder behind the C ABI of include/df11.h); this package allocates
+caller-owned buffers with PyTorch and passes pointers.  Importing it does not
+load the library; the first call does, and raises if it is missing.
+"""
+from .codec import (CompressedStream, HostStream, build_lut, code_lengths, compress, decompress,
+                    from_arrays, make_header, to_host, workspace_bytes)
+from ._binding import DF11Error, EXPORTED, load as load_library, library_path
+
+__all__ = ["CompressedStream", "HostStream", "build_lut", "code_lengths", "compress", "decompress",
+           "from_arrays", "make_header", "to_host", "workspace_bytes", "DF11Error", "EXPORTED",
+           "load_library", "library_path"]

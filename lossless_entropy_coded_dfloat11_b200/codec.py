@@ -1,0 +1,239 @@
+"""PyTorch-facing API of the DF11 codec.
+
+PyTorch provides device memory and streams; every step of compression and
+decompression runs in libdf11.so (CUDA kernels for sm_100a plus the host-side
+code builder).  The functions here only allocate caller-owned buffers with
+torch and pass raw pointers through the C ABI of include/df11.h.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+from dataclasses import dataclass, field
+
+import numpy as np
+import torch
+
+from . import _binding as B
+
+
+def _stream_handle(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(int(stream.cuda_stream))
+
+
+def _ptr(t: torch.Tensor) -> ctypes.c_void_p:
+    return ctypes.c_void_p(int(t.data_ptr()))
+
+
+def _np_ptr(a: np.ndarray) -> ctypes.c_void_p:
+    return ctypes.c_void_p(int(a.ctypes.data))
+
+
+@dataclass
+class CompressedStream:
+    """One DF11 stream on the device: a matrix, or every matrix of a
+    transformer block sharing one code table."""
+    header: B.Header
+    exp: torch.Tensor        # uint8  EncodedExponent
+    sm: torch.Tensor         # uint8  PackedSignMantissa
+    gaps: torch.Tensor       # uint8  5-bit Gaps
+    block_off: torch.Tensor  # int32 storage of uint32 block offsets
+    lut: torch.Tensor        # uint8  decode tables (df11_build_lut)
+    names: list = field(default_factory=list)
+    shapes: list = field(default_factory=list)
+
+    @property
+    def n_elems(self) -> int:
+        return int(self.header.n_elems)
+
+    @property
+    def total_bits(self) -> int:
+        return int(self.header.total_bits)
+
+    @property
+    def threads_per_block(self) -> int:
+        return int(self.header.threads_per_block)
+
+    @property
+    def code_len(self) -> np.ndarray:
+        return np.frombuffer(bytes(self.header.code_len), dtype=np.uint8).copy()
+
+    def compressed_bytes(self) -> int:
+        """Bytes of the format's arrays without padding: code bits, one byte
+        per element, 5 bits per thread, 4 bytes per thread-block position and
+        the 256-byte code-length table."""
+        h = self.header
+        return ((h.total_bits + 7) // 8 + h.n_elems + (5 * h.n_threads + 7) // 8
+                + 4 * (h.n_blocks + 1) + 256)
+
+    def read_bytes(self) -> int:
+        """Bytes one decompress reads from HBM (the format's arrays as the
+        kernel fetches them, plus the decode tables once per CTA from L2)."""
+        h = self.header
+        return (h.total_bits + 7) // 8 + h.n_elems + (5 * h.n_threads + 7) // 8 + 4 * (h.n_blocks + 1)
+
+    def views(self, flat: torch.Tensor) -> list[torch.Tensor]:
+        """Per-matrix views of a decompressed flat buffer."""
+        out = []
+        for k, shape in enumerate(self.shapes):
+            a, b = int(self.header.seg_elem_off[k]), int(self.header.seg_elem_off[k + 1])
+            out.append(flat[a:b].view(shape))
+        return out
+
+
+def code_lengths(hist: np.ndarray, max_code_len: int = 32) -> np.ndarray:
+    """The library's host code builder (package-merge), for tests."""
+    h = np.ascontiguousarray(hist, dtype=np.uint64)
+    out = np.zeros(256, dtype=np.uint8)
+    B.call("df11_code_lengths", _np_ptr(h), max_code_len, _np_ptr(out))
+    return out
+
+
+def make_header(code_len: np.ndarray, n_elems: int, total_bits: int, threads_per_block: int = 256,
+                max_code_len: int = 32, seg_counts=None) -> B.Header:
+    hdr = B.Header()
+    ln = np.ascontiguousarray(code_len, dtype=np.uint8)
+    if seg_counts is None:
+        seg_counts = [n_elems]
+    counts = np.ascontiguousarray(seg_counts, dtype=np.uint64)
+    B.call("df11_header_init", ctypes.byref(hdr), _np_ptr(ln), n_elems, total_bits, threads_per_block,
+           max_code_len, _np_ptr(counts), len(counts))
+    return hdr
+
+
+def build_lut(header: B.Header) -> np.ndarray:
+    out = np.zeros(int(header.bytes_lut), dtype=np.uint8)
+    B.call("df11_build_lut", ctypes.byref(header), _np_ptr(out), out.size)
+    return out
+
+
+def workspace_bytes(n_elems: int) -> int:
+    v = ctypes.c_uint64()
+    B.call("df11_compress_workspace_size", n_elems, ctypes.byref(v))
+    return int(v.value)
+
+
+def _as_segments(tensors):
+    if isinstance(tensors, torch.Tensor):
+        tensors = [tensors]
+    segs = []
+    for t in tensors:
+        if t.dtype != torch.bfloat16:
+            raise TypeError(f"DF11 compresses bfloat16 tensors, got {t.dtype}")
+        if not t.is_cuda:
+            raise ValueError("compress expects CUDA tensors")
+        segs.append(t.contiguous())
+    return segs
+
+
+def compress(tensors, names=None, threads_per_block: int = 256, max_code_len: int = 32,
+             stream=None) -> CompressedStream:
+    """Compress one BF16 tensor, or a list (a transformer block) into one
+    stream with a shared code table: histogram kernel, host code builder,
+    bit-pack kernel.  Synchronises the stream once (histogram readback)."""
+    segs = _as_segments(tensors)
+    device = segs[0].device
+    n = sum(t.numel() for t in segs)
+    ws = torch.empty(max(workspace_bytes(n), 16), dtype=torch.uint8, device=device)
+    ptrs = (ctypes.c_void_p * len(segs))(*[int(t.data_ptr()) for t in segs])
+    counts = (ctypes.c_uint64 * len(segs))(*[t.numel() for t in segs])
+    hdr = B.Header()
+    sh = _stream_handle(stream)
+    B.call("df11_compress_plan", ptrs, counts, len(segs), threads_per_block, max_code_len, _ptr(ws),
+           ws.numel(), ctypes.byref(hdr), sh)
+    exp = torch.empty(int(hdr.bytes_exp), dtype=torch.uint8, device=device)
+    sm = torch.empty(int(hdr.bytes_sm) or 16, dtype=torch.uint8, device=device)
+    gaps = torch.empty(int(hdr.bytes_gaps), dtype=torch.uint8, device=device)
+    off = torch.empty(int(hdr.n_blocks) + 1, dtype=torch.int32, device=device)
+    lut = torch.empty(int(hdr.bytes_lut), dtype=torch.uint8, device=device)
+    B.call("df11_compress_encode", ptrs, ctypes.byref(hdr), _ptr(ws), ws.numel(), _ptr(exp), _ptr(sm),
+           _ptr(gaps), _ptr(off), _ptr(lut), sh)
+    # keep the workspace alive until the queued kernels have consumed it
+    (stream or torch.cuda.current_stream()).synchronize()
+    return CompressedStream(hdr, exp, sm, gaps, off, lut,
+                            names=list(names) if names else [f"t{k}" for k in range(len(segs))],
+                            shapes=[tuple(t.shape) for t in segs])
+
+
+def from_arrays(code_len: np.ndarray, n_elems: int, total_bits: int, threads_per_block: int,
+                exp: np.ndarray, sm: np.ndarray, gaps: np.ndarray, block_off: np.ndarray,
+                max_code_len: int = 32, seg_counts=None, shapes=None, device="cuda") -> CompressedStream:
+    """Upload a stream made elsewhere (another encoder, a file)."""
+    hdr = make_header(code_len, n_elems, total_bits, threads_per_block, max_code_len, seg_counts)
+    for name, arr, need in (("exp", exp, hdr.bytes_exp), ("sm", sm, hdr.bytes_sm),
+                            ("gaps", gaps, hdr.bytes_gaps), ("block_off", block_off, hdr.n_blocks + 1)):
+        if arr.size < need:
+            raise ValueError(f"{name}: {arr.size} entries, header needs {need}")
+    lut = build_lut(hdr)
+
+    def up(a, dtype=torch.uint8):
+        a = np.ascontiguousarray(a)
+        if a.size == 0:
+            return torch.zeros(16, dtype=dtype, device=device)
+        return torch.from_numpy(a.view(np.int32) if dtype == torch.int32 else a).to(device)
+
+    shapes = shapes or [(int(c),) for c in (seg_counts or [n_elems])]
+    return CompressedStream(hdr, up(exp), up(sm), up(gaps),
+                            up(np.ascontiguousarray(block_off, dtype=np.uint32), torch.int32), up(lut),
+                            names=[f"t{k}" for k in range(len(shapes))], shapes=shapes)
+
+
+def to_host(cs: CompressedStream) -> dict:
+    """The stream's arrays as numpy (for another decoder)."""
+    h = cs.header
+    return dict(code_len=cs.code_len, n_elems=int(h.n_elems), total_bits=int(h.total_bits),
+                threads_per_block=int(h.threads_per_block), n_threads=int(h.n_threads),
+                n_blocks=int(h.n_blocks),
+                exp=cs.exp.cpu().numpy()[: int(h.bytes_exp)],
+                sm=cs.sm.cpu().numpy()[: int(h.bytes_sm)],
+                gaps=cs.gaps.cpu().numpy()[: int(h.bytes_gaps)],
+                block_off=cs.block_off.cpu().numpy().view(np.uint32)[: int(h.n_blocks) + 1])
+
+
+def decompress(cs: CompressedStream, out: torch.Tensor | None = None, status: torch.Tensor | None = None,
+               stream=None) -> torch.Tensor:
+    """One kernel launch rebuilding all n_elems BF16 values of the stream.
+    Asynchronous; `out` (bfloat16, n_elems, contiguous) may be reused across
+    calls.  `status` (int32 device word, zeroed by the caller) receives
+    DF11_ERR_CORRUPT if the stream disagrees with its metadata."""
+    n = cs.n_elems
+    if out is None:
+        out = torch.empty(max(n, 1), dtype=torch.bfloat16, device=cs.exp.device)[:n]
+    if out.dtype != torch.bfloat16 or not out.is_contiguous() or out.numel() < n:
+        raise ValueError("out must be a contiguous bfloat16 tensor with n_elems elements")
+    B.call("df11_decompress", ctypes.byref(cs.header), _ptr(cs.exp), _ptr(cs.sm), _ptr(cs.gaps),
+           _ptr(cs.block_off), _ptr(cs.lut), _ptr(out),
+           _ptr(status) if status is not None else ctypes.c_void_p(0), _stream_handle(stream))
+    return out
+
+
+class HostStream:
+    """A stream kept in pinned host memory, decompressed end to end: copy the
+    compressed arrays to the device, decode, copy the BF16 result back."""
+
+    def __init__(self, cs: CompressedStream):
+        self.header = cs.header
+        self.host = {k: getattr(cs, k).cpu().pin_memory() for k in ("exp", "sm", "gaps", "block_off", "lut")}
+        dev = cs.exp.device
+        self.dev = {k: torch.empty_like(v, device=dev) for k, v in self.host.items()}
+        self.dev_stream = CompressedStream(cs.header, self.dev["exp"], self.dev["sm"], self.dev["gaps"],
+                                           self.dev["block_off"], self.dev["lut"], cs.names, cs.shapes)
+        self.out_dev = torch.empty(max(cs.n_elems, 1), dtype=torch.bfloat16, device=dev)[: cs.n_elems]
+        self.out_host = torch.empty(max(cs.n_elems, 1), dtype=torch.bfloat16).pin_memory()[: cs.n_elems]
+
+    def h2d_bytes(self) -> int:
+        return sum(v.numel() * v.element_size() for v in self.host.values())
+
+    def d2h_bytes(self) -> int:
+        return 2 * int(self.header.n_elems)
+
+    def run(self, stream=None) -> torch.Tensor:
+        s = stream or torch.cuda.current_stream()
+        with torch.cuda.stream(s):
+            for k, v in self.host.items():
+                self.dev[k].copy_(v, non_blocking=True)
+            decompress(self.dev_stream, self.out_dev, stream=s)
+            self.out_host.copy_(self.out_dev, non_blocking=True)
+        return self.out_host

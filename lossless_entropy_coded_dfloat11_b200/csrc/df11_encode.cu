@@ -1,0 +1,435 @@
+// DF11 compression on the GPU: exponent histogram, then (after the host has
+// built the code) per-chunk code-bit totals, their prefix sum, and the
+// bit-pack kernel that writes EncodedExponent, PackedSignMantissa, Gaps and
+// the per-thread-block output positions.
+//
+// Format: "DFloat11: compressao sem perda para inferencia em GPU que reduz
+// LLMs para 70% do tamanho", sections "O formato DFloat11" (Huffman-coded
+// exponents, raw sign+mantissa bytes) and "Kernel de GPU em 2 etapas e
+// metadados auxiliares" (8-byte thread windows, 5-bit gaps, one output
+// position per thread block).
+#include <cuda_runtime.h>
+
+#include <cstring>
+#include <vector>
+
+#include "df11_internal.h"
+
+namespace df11 {
+
+df11_status check_header(const df11_header* h);
+
+namespace {
+
+struct SegTable {
+    const uint16_t* ptr[DF11_MAX_SEGMENTS];
+    uint64_t start[DF11_MAX_SEGMENTS + 1];
+    uint32_t n;
+};
+
+struct CodeTable {
+    uint32_t code[256];
+    uint8_t len[256];
+};
+
+// ---------------------------------------------------------------------------
+// Histogram of the exponent field of one segment; per-warp shared-memory
+// histograms, flushed into 64-bit global counters.
+// ---------------------------------------------------------------------------
+constexpr int kHistThreads = 256;
+
+__global__ void __launch_bounds__(kHistThreads) histogram_kernel(const uint16_t* __restrict__ x, uint64_t n,
+                                                                 unsigned long long* __restrict__ hist) {
+    __shared__ uint32_t sh[kHistThreads / 32][256];
+    uint32_t* mine = sh[threadIdx.x >> 5];
+    for (int i = threadIdx.x; i < (kHistThreads / 32) * 256; i += kHistThreads) (&sh[0][0])[i] = 0;
+    __syncthreads();
+    const uint64_t nvec = n / 8;
+    const uint4* xv = reinterpret_cast<const uint4*>(x);
+    const uint64_t stride = uint64_t(gridDim.x) * kHistThreads;
+    for (uint64_t v = uint64_t(blockIdx.x) * kHistThreads + threadIdx.x; v < nvec; v += stride) {
+        const uint4 q = __ldcs(xv + v);
+        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+        for (int k = 0; k < 4; k++) {
+            atomicAdd(&mine[(w[k] >> 7) & 0xFFu], 1u);
+            atomicAdd(&mine[(w[k] >> 23) & 0xFFu], 1u);
+        }
+    }
+    for (uint64_t i = nvec * 8 + uint64_t(blockIdx.x) * kHistThreads + threadIdx.x; i < n; i += stride)
+        atomicAdd(&mine[(x[i] >> 7) & 0xFFu], 1u);
+    __syncthreads();
+    for (int s = threadIdx.x; s < 256; s += kHistThreads) {
+        uint64_t t = 0;
+        for (int w = 0; w < kHistThreads / 32; w++) t += sh[w][s];
+        if (t) atomicAdd(hist + s, (unsigned long long)t);
+    }
+}
+
+// Element i of the concatenated segments.
+__device__ __forceinline__ uint16_t load_elem(const SegTable& sg, uint64_t i, uint32_t& seg) {
+    while (seg + 1 < sg.n && i >= sg.start[seg + 1]) seg++;
+    return sg.ptr[seg][i - sg.start[seg]];
+}
+
+__device__ __forceinline__ uint32_t find_seg(const SegTable& sg, uint64_t i) {
+    uint32_t lo = 0, hi = sg.n - 1;
+    while (lo < hi) {
+        const uint32_t mid = (lo + hi + 1) >> 1;
+        if (sg.start[mid] <= i) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+
+// Loads the kEncPerThread elements of this thread (those past n read as 0).
+__device__ __forceinline__ void load_chunk(const SegTable& sg, uint64_t i0, uint64_t n,
+                                           uint16_t (&x)[kEncPerThread]) {
+    uint32_t seg = find_seg(sg, i0 < n ? i0 : n - 1);
+    const uint64_t rel = i0 - sg.start[seg];
+    const uint16_t* p = sg.ptr[seg] + rel;
+    if (i0 + kEncPerThread <= sg.start[seg + 1] && (reinterpret_cast<uintptr_t>(p) & 15u) == 0) {
+        const uint4 a = __ldcs(reinterpret_cast<const uint4*>(p));
+        const uint4 b = __ldcs(reinterpret_cast<const uint4*>(p) + 1);
+        const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+        for (int k = 0; k < 8; k++) {
+            x[2 * k] = uint16_t(w[k]);
+            x[2 * k + 1] = uint16_t(w[k] >> 16);
+        }
+    } else {
+#pragma unroll
+        for (int k = 0; k < int(kEncPerThread); k++) {
+            const uint64_t i = i0 + k;
+            x[k] = i < n ? load_elem(sg, i, seg) : uint16_t(0);
+        }
+    }
+}
+
+// Block-wide exclusive scan of one value per thread; also returns the total.
+template <int NT>
+__device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* s_warp, uint32_t& total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    uint32_t incl = v;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+        if (lane >= d) incl += y;
+    }
+    if (lane == 31) s_warp[warp] = incl;
+    __syncthreads();
+    uint32_t before = 0, tot = 0;
+#pragma unroll
+    for (int w = 0; w < NT / 32; w++) {
+        const uint32_t t = s_warp[w];
+        tot += t;
+        before += (w < warp) ? t : 0u;
+    }
+    total = tot;
+    return before + incl - v;
+}
+
+// ---------------------------------------------------------------------------
+// Bits of code per chunk of kEncChunk elements.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kEncThreads) chunk_bits_kernel(const __grid_constant__ SegTable sg,
+                                                                 const __grid_constant__ CodeTable ct,
+                                                                 uint64_t n, uint32_t* __restrict__ chunk_bits) {
+    __shared__ uint32_t s_warp[kEncThreads / 32];
+    const uint64_t i0 = uint64_t(blockIdx.x) * kEncChunk + uint64_t(threadIdx.x) * kEncPerThread;
+    uint32_t bits = 0;
+    if (i0 < n) {
+        uint16_t x[kEncPerThread];
+        load_chunk(sg, i0, n, x);
+#pragma unroll
+        for (int k = 0; k < int(kEncPerThread); k++)
+            if (i0 + k < n) bits += ct.len[(x[k] >> 7) & 0xFFu];
+    }
+    uint32_t total;
+    block_exclusive_scan<kEncThreads>(bits, s_warp, total);
+    if (threadIdx.x == 0) chunk_bits[blockIdx.x] = total;
+}
+
+// Exclusive prefix sum of the chunk totals (one CTA; a few thousand chunks
+// per stream at most a million).
+constexpr int kScanThreads = 1024;
+__global__ void __launch_bounds__(kScanThreads) chunk_scan_kernel(const uint32_t* __restrict__ chunk_bits,
+                                                                  uint64_t n_chunks,
+                                                                  unsigned long long* __restrict__ chunk_start) {
+    __shared__ unsigned long long s_part[kScanThreads];
+    const uint64_t per = (n_chunks + kScanThreads - 1) / kScanThreads;
+    const uint64_t lo = per * threadIdx.x;
+    const uint64_t hi = lo + per < n_chunks ? lo + per : n_chunks;
+    unsigned long long sum = 0;
+    for (uint64_t c = lo; c < hi; c++) sum += chunk_bits[c];
+    s_part[threadIdx.x] = sum;
+    __syncthreads();
+    // Hillis-Steele over 1024 partial sums
+    for (int d = 1; d < kScanThreads; d <<= 1) {
+        const unsigned long long y = threadIdx.x >= d ? s_part[threadIdx.x - d] : 0ull;
+        __syncthreads();
+        s_part[threadIdx.x] += y;
+        __syncthreads();
+    }
+    unsigned long long run = s_part[threadIdx.x] - sum;
+    for (uint64_t c = lo; c < hi; c++) {
+        chunk_start[c] = run;
+        run += chunk_bits[c];
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Bit-pack: codes are OR-ed into a shared-memory image of the chunk's words,
+// interior words are stored, the two boundary words (shared with the
+// neighbouring chunks) are OR-ed into global memory.  The same pass writes
+// the sign+mantissa bytes, each window's gap and each thread block's output
+// position, using only the element's own start bit s and length l:
+//   * a code that starts inside window w-1 and runs into window w sets
+//     gap[w] = s + l - 64w (gaps of windows that begin exactly at a code start
+//     stay 0);
+//   * a code that starts exactly at bit 64*T*b sets off[b] = i, one that runs
+//     over that bit sets off[b] = i + 1.
+// ---------------------------------------------------------------------------
+constexpr int kPackWords = kEncChunk + 4;  // 32 bits per element at most, plus the misalignment
+
+__global__ void __launch_bounds__(kEncThreads) pack_kernel(const __grid_constant__ SegTable sg,
+                                                           const __grid_constant__ CodeTable ct, uint64_t n,
+                                                           uint32_t log2_block_bits,
+                                                           const unsigned long long* __restrict__ chunk_start,
+                                                           uint32_t* __restrict__ exp32, uint8_t* __restrict__ sm,
+                                                           uint32_t* __restrict__ gaps32,
+                                                           uint32_t* __restrict__ block_off, uint64_t n_blocks) {
+    __shared__ uint32_t s_words[kPackWords];
+    __shared__ uint32_t s_warp[kEncThreads / 32];
+    const uint64_t i0 = uint64_t(blockIdx.x) * kEncChunk + uint64_t(threadIdx.x) * kEncPerThread;
+    uint16_t x[kEncPerThread];
+    uint32_t bits = 0;
+    if (i0 < n) {
+        load_chunk(sg, i0, n, x);
+#pragma unroll
+        for (int k = 0; k < int(kEncPerThread); k++)
+            if (i0 + k < n) bits += ct.len[(x[k] >> 7) & 0xFFu];
+    }
+    for (int j = threadIdx.x; j < kPackWords; j += kEncThreads) s_words[j] = 0;
+    uint32_t chunk_total;
+    const uint32_t my_off = block_exclusive_scan<kEncThreads>(bits, s_warp, chunk_total);
+    const uint64_t S = chunk_start[blockIdx.x];
+    const uint32_t lead = uint32_t(S & 31u);
+
+    if (i0 < n) {
+        uint32_t q = lead + my_off;  // bit position relative to word S/32
+        uint8_t smb[kEncPerThread];
+#pragma unroll
+        for (int k = 0; k < int(kEncPerThread); k++) {
+            const uint64_t i = i0 + k;
+            const uint32_t xv = x[k];
+            smb[k] = uint8_t(((xv >> 8) & 0x80u) | (xv & 0x7Fu));
+            if (i >= n) continue;
+            const uint32_t e = (xv >> 7) & 0xFFu;
+            const uint32_t l = ct.len[e];
+            const uint32_t code = ct.code[e];
+            const uint32_t o = q & 31u;
+            if (o + l <= 32) {
+                atomicOr(&s_words[q >> 5], code << (32 - o - l));
+            } else {
+                atomicOr(&s_words[q >> 5], code >> (o + l - 32));
+                atomicOr(&s_words[(q >> 5) + 1], code << (64 - o - l));
+            }
+            // gaps and block offsets from the absolute start bit
+            const uint64_t s = (S & ~uint64_t(31)) + q;
+            const uint64_t last = s + l - 1;
+            if ((s & 63) != 0 && (s >> 6) != (last >> 6)) {
+                const uint64_t w = (s >> 6) + 1;
+                const uint32_t g = uint32_t(s + l - 64 * w);
+                const uint64_t gb = 5 * w;
+                const uint32_t sh = uint32_t(gb & 31);
+                atomicOr(gaps32 + (gb >> 5), g << sh);
+                if (sh > 27) atomicOr(gaps32 + (gb >> 5) + 1, g >> (32 - sh));
+            }
+            const uint64_t bb = s >> log2_block_bits;
+            if ((s & ((uint64_t(1) << log2_block_bits) - 1)) == 0) {
+                block_off[bb] = uint32_t(i);
+            } else if ((last >> log2_block_bits) != bb) {
+                block_off[bb + 1] = uint32_t(i + 1);
+            }
+            if (i == n - 1) block_off[n_blocks] = uint32_t(n);
+            q += l;
+        }
+        // sign+mantissa bytes
+        if (i0 + kEncPerThread <= n) {
+            uint4 v;
+            v.x = smb[0] | (smb[1] << 8) | (smb[2] << 16) | (uint32_t(smb[3]) << 24);
+            v.y = smb[4] | (smb[5] << 8) | (smb[6] << 16) | (uint32_t(smb[7]) << 24);
+            v.z = smb[8] | (smb[9] << 8) | (smb[10] << 16) | (uint32_t(smb[11]) << 24);
+            v.w = smb[12] | (smb[13] << 8) | (smb[14] << 16) | (uint32_t(smb[15]) << 24);
+            *reinterpret_cast<uint4*>(sm + i0) = v;
+        } else {
+            for (int k = 0; k < int(kEncPerThread); k++)
+                if (i0 + k < n) sm[i0 + k] = smb[k];
+        }
+    }
+    __syncthreads();
+    const uint32_t nwords = (lead + chunk_total + 31) >> 5;
+    const uint64_t W0 = S >> 5;
+    for (uint32_t j = threadIdx.x; j < nwords; j += kEncThreads) {
+        const uint32_t v = __byte_perm(s_words[j], 0, 0x0123);  // MSB-first bytes
+        if (j == 0 || j == nwords - 1) {
+            if (v) atomicOr(exp32 + W0 + j, v);
+        } else {
+            exp32[W0 + j] = v;
+        }
+    }
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct Workspace {
+    unsigned long long* hist;
+    uint32_t* chunk_bits;
+    unsigned long long* chunk_start;
+};
+
+df11_status carve(void* ws, uint64_t ws_bytes, uint64_t n_elems, Workspace* w) {
+    uint64_t need = 0;
+    df11_compress_workspace_size(n_elems, &need);
+    if (!ws) return fail(DF11_ERR_INVALID, "null workspace");
+    if (!aligned16(ws)) return fail(DF11_ERR_INVALID, "workspace must be 16-byte aligned");
+    if (ws_bytes < need)
+        return fail(DF11_ERR_CAPACITY, "workspace of %llu bytes, need %llu", (unsigned long long)ws_bytes,
+                    (unsigned long long)need);
+    const uint64_t chunks = (n_elems + kEncChunk - 1) / kEncChunk;
+    uint8_t* p = static_cast<uint8_t*>(ws);
+    w->hist = reinterpret_cast<unsigned long long*>(p);
+    w->chunk_bits = reinterpret_cast<uint32_t*>(p + 2048);
+    w->chunk_start = reinterpret_cast<unsigned long long*>(p + 2048 + align16(4 * chunks));
+    return DF11_OK;
+}
+
+df11_status cuda_fail(const char* what, cudaError_t e) {
+    return fail(DF11_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+df11_status build_segtable(const void* const* d_segs, const uint64_t* counts, uint32_t n_segs, SegTable* sg,
+                           uint64_t* n_total) {
+    if (!d_segs || !counts) return fail(DF11_ERR_INVALID, "null segment arrays");
+    if (n_segs < 1 || n_segs > DF11_MAX_SEGMENTS)
+        return fail(DF11_ERR_INVALID, "n_segs %u outside 1..%d", n_segs, DF11_MAX_SEGMENTS);
+    std::memset(sg, 0, sizeof(*sg));
+    uint64_t acc = 0;
+    for (uint32_t k = 0; k < n_segs; k++) {
+        if (counts[k] && !d_segs[k]) return fail(DF11_ERR_INVALID, "null segment %u", k);
+        if (counts[k] && !aligned16(d_segs[k]))
+            return fail(DF11_ERR_INVALID, "segment %u is not 16-byte aligned", k);
+        sg->ptr[k] = static_cast<const uint16_t*>(d_segs[k]);
+        sg->start[k] = acc;
+        acc += counts[k];
+    }
+    sg->start[n_segs] = acc;
+    sg->n = n_segs;
+    if (acc >= (uint64_t(1) << 32)) return fail(DF11_ERR_TOO_LARGE, "more than 2^32 - 1 elements");
+    *n_total = acc;
+    return DF11_OK;
+}
+
+}  // namespace
+}  // namespace df11
+
+using namespace df11;
+
+extern "C" df11_status df11_compress_plan(const void* const* d_segs, const uint64_t* seg_counts, uint32_t n_segs,
+                                          uint32_t threads_per_block, uint32_t max_code_len, void* d_workspace,
+                                          uint64_t workspace_bytes, df11_header* hdr, void* stream) {
+    if (!hdr) return fail(DF11_ERR_INVALID, "null header");
+    SegTable sg;
+    uint64_t n = 0;
+    df11_status st = build_segtable(d_segs, seg_counts, n_segs, &sg, &n);
+    if (st != DF11_OK) return st;
+    Workspace w;
+    st = carve(d_workspace, workspace_bytes, n, &w);
+    if (st != DF11_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemsetAsync(w.hist, 0, 2048, s);
+    if (e != cudaSuccess) return cuda_fail("histogram clear", e);
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    for (uint32_t k = 0; k < n_segs; k++) {
+        const uint64_t cnt = seg_counts[k];
+        if (!cnt) continue;
+        const uint64_t vec_blocks = (cnt / 8 + kHistThreads - 1) / kHistThreads;
+        uint64_t grid = vec_blocks < uint64_t(4 * sms) ? vec_blocks : uint64_t(4 * sms);
+        if (grid == 0) grid = 1;
+        histogram_kernel<<<unsigned(grid), kHistThreads, 0, s>>>(sg.ptr[k], cnt, w.hist);
+    }
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail("histogram launch", e);
+    uint64_t hist[256];
+    e = cudaMemcpyAsync(hist, w.hist, sizeof(hist), cudaMemcpyDeviceToHost, s);
+    if (e != cudaSuccess) return cuda_fail("histogram readback", e);
+    e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail("histogram sync", e);
+    uint8_t len[256];
+    st = df11_code_lengths(hist, max_code_len, len);
+    if (st != DF11_OK) return st;
+    uint64_t bits = 0;
+    for (int v = 0; v < 256; v++) bits += hist[v] * len[v];
+    return df11_header_init(hdr, len, n, bits, threads_per_block, max_code_len, seg_counts, n_segs);
+}
+
+extern "C" df11_status df11_compress_encode(const void* const* d_segs, const df11_header* hdr, void* d_workspace,
+                                            uint64_t workspace_bytes, uint8_t* d_exp, uint8_t* d_sm,
+                                            uint8_t* d_gaps, uint32_t* d_block_off, void* d_lut,
+                                            void* stream) {
+    df11_status st = check_header(hdr);
+    if (st != DF11_OK) return st;
+    uint64_t counts[DF11_MAX_SEGMENTS];
+    if (hdr->n_segments < 1 || hdr->n_segments > DF11_MAX_SEGMENTS)
+        return fail(DF11_ERR_INVALID, "header n_segments %u", hdr->n_segments);
+    for (uint32_t k = 0; k < hdr->n_segments; k++) counts[k] = hdr->seg_elem_off[k + 1] - hdr->seg_elem_off[k];
+    SegTable sg;
+    uint64_t n = 0;
+    st = build_segtable(d_segs, counts, hdr->n_segments, &sg, &n);
+    if (st != DF11_OK) return st;
+    if (n != hdr->n_elems) return fail(DF11_ERR_INVALID, "segments disagree with header n_elems");
+    if (!d_exp || !d_sm || !d_gaps || !d_block_off || !d_lut)
+        return fail(DF11_ERR_INVALID, "df11_compress_encode: null output pointer");
+    if (!aligned16(d_exp) || !aligned16(d_sm) || !aligned16(d_gaps) || !aligned16(d_block_off) ||
+        !aligned16(d_lut))
+        return fail(DF11_ERR_INVALID, "df11_compress_encode: outputs must be 16-byte aligned");
+    Workspace w;
+    st = carve(d_workspace, workspace_bytes, n, &w);
+    if (st != DF11_OK) return st;
+
+    CodeTable ct;
+    std::memcpy(ct.len, hdr->code_len, 256);
+    if (!canonical_codes(hdr->code_len, ct.code)) return fail(DF11_ERR_INVALID, "code lengths overflow");
+    std::vector<uint8_t> lut(kLutBytes);
+    st = df11_build_lut(hdr, lut.data(), lut.size());
+    if (st != DF11_OK) return st;
+
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    if ((e = cudaMemcpyAsync(d_lut, lut.data(), kLutBytes, cudaMemcpyHostToDevice, s)) != cudaSuccess)
+        return cuda_fail("table upload", e);
+    if ((e = cudaMemsetAsync(d_exp, 0, hdr->bytes_exp, s)) != cudaSuccess) return cuda_fail("clear exp", e);
+    if ((e = cudaMemsetAsync(d_gaps, 0, hdr->bytes_gaps, s)) != cudaSuccess) return cuda_fail("clear gaps", e);
+    if ((e = cudaMemsetAsync(d_block_off, 0, hdr->bytes_off, s)) != cudaSuccess) return cuda_fail("clear off", e);
+    const uint64_t sm_tail = n & ~uint64_t(15);
+    if (hdr->bytes_sm > sm_tail &&
+        (e = cudaMemsetAsync(d_sm + sm_tail, 0, hdr->bytes_sm - sm_tail, s)) != cudaSuccess)
+        return cuda_fail("clear sm tail", e);
+    if (n == 0) return DF11_OK;
+
+    const uint64_t chunks = (n + kEncChunk - 1) / kEncChunk;
+    if (chunks >= (uint64_t(1) << 31)) return fail(DF11_ERR_TOO_LARGE, "too many chunks");
+    chunk_bits_kernel<<<unsigned(chunks), kEncThreads, 0, s>>>(sg, ct, n, w.chunk_bits);
+    chunk_scan_kernel<<<1, kScanThreads, 0, s>>>(w.chunk_bits, chunks, w.chunk_start);
+    uint32_t log2_bb = 6;
+    while ((1u << (log2_bb - 6)) < hdr->threads_per_block) log2_bb++;
+    pack_kernel<<<unsigned(chunks), kEncThreads, 0, s>>>(sg, ct, n, log2_bb, w.chunk_start,
+                                                         reinterpret_cast<uint32_t*>(d_exp), d_sm,
+                                                         reinterpret_cast<uint32_t*>(d_gaps), d_block_off,
+                                                         hdr->n_blocks);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail("encode launch", e);
+    return DF11_OK;
+}

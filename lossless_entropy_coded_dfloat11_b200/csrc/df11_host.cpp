@@ -1,0 +1,299 @@
+// Host side of the DF11 library: error reporting, the length-limited code
+// builder, canonical codes, header validation and the decode-table builder.
+// Sources: "DFloat11: compressao sem perda para inferencia em GPU que reduz
+// LLMs para 70% do tamanho" -- "O formato DFloat11" (Huffman code over the
+// exponents), "Decodificacao com LUT hierarquica" (compact decode tables),
+// "Kernel de GPU em 2 etapas e metadados auxiliares" (8-byte windows, 5-bit
+// gaps, 32-bit codes at most, per-thread-block output positions).
+#include <algorithm>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <vector>
+
+#include "df11_internal.h"
+
+namespace df11 {
+
+static thread_local char g_err[512] = "";
+
+df11_status fail(df11_status st, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    std::vsnprintf(g_err, sizeof(g_err), fmt, ap);
+    va_end(ap);
+    return st;
+}
+
+bool canonical_codes(const uint8_t* len, uint32_t* code) {
+    // count per length, then the first code of each length, then hand out
+    // codes in increasing value order inside each length
+    uint64_t bl_count[34] = {0};
+    for (int s = 0; s < 256; s++) {
+        code[s] = 0;
+        if (len[s] > 32) return false;
+        if (len[s]) bl_count[len[s]]++;
+    }
+    uint64_t next[34] = {0};
+    uint64_t c = 0;
+    for (int l = 1; l <= 32; l++) {
+        c = (c + bl_count[l - 1]) << 1;
+        next[l] = c;
+    }
+    for (int s = 0; s < 256; s++) {
+        int l = len[s];
+        if (!l) continue;
+        uint64_t v = next[l]++;
+        if (v >> l) return false;  // more codes than the length allows
+        code[s] = uint32_t(v);
+    }
+    return true;
+}
+
+void fill_sizes(df11_header* h) {
+    const uint64_t T = h->threads_per_block;
+    h->n_threads = (h->total_bits + 63) / 64;
+    h->n_blocks = (h->n_threads + T - 1) / T;
+    h->bytes_exp = 8 * T * h->n_blocks + 16;
+    h->bytes_sm = (h->n_elems + 15) & ~uint64_t(15);
+    h->bytes_gaps = align16((5 * T * h->n_blocks + 7) / 8 + 8);
+    h->bytes_off = 4 * (h->n_blocks + 1);
+    h->bytes_lut = kLutBytes;
+}
+
+// Kraft sum in units of 2^-32; returns false on lengths > 32.
+static bool kraft_units(const uint8_t* len, uint64_t* units, int* n_present) {
+    uint64_t u = 0;
+    int m = 0;
+    for (int s = 0; s < 256; s++) {
+        if (!len[s]) continue;
+        if (len[s] > 32) return false;
+        u += uint64_t(1) << (32 - len[s]);
+        m++;
+    }
+    *units = u;
+    *n_present = m;
+    return true;
+}
+
+}  // namespace df11
+
+using namespace df11;
+
+extern "C" {
+
+int df11_version(void) { return DF11_VERSION; }
+
+const char* df11_last_error(void) { return g_err; }
+
+// Package-merge for optimal length-limited prefix codes.  Each present symbol
+// has one coin per depth 1..L (value = its count); the cheapest coins whose
+// depths' weights 2^-d sum to m-1 give the lengths.  The list of depth d is
+// the depth-d coins merged with pairs of consecutive depth-(d+1) items.
+// Instead of expanding the chosen packages, count down: if the first k items
+// of depth d hold j leaves, those are the j lightest symbols (the merge keeps
+// leaf order), each gains one bit, and the k - j packages stand for the first
+// 2(k - j) items of depth d+1.
+df11_status df11_code_lengths(const uint64_t* hist, uint32_t max_code_len, uint8_t* code_len) {
+    if (!hist || !code_len) return fail(DF11_ERR_INVALID, "df11_code_lengths: null pointer");
+    std::memset(code_len, 0, 256);
+    std::vector<int> sym;
+    for (int s = 0; s < 256; s++)
+        if (hist[s]) sym.push_back(s);
+    const int m = int(sym.size());
+    if (m == 0) return DF11_OK;
+    if (max_code_len < 1 || max_code_len > 32)
+        return fail(DF11_ERR_INVALID, "df11_code_lengths: max_code_len %u outside 1..32", max_code_len);
+    if (m == 1) {
+        code_len[sym[0]] = 1;
+        return DF11_OK;
+    }
+    const int L = int(max_code_len);
+    if (L < 9 && (1 << L) < m)
+        return fail(DF11_ERR_INVALID, "df11_code_lengths: %d values do not fit in %d-bit codes", m, L);
+    // lighter first; equal counts: lower value first
+    std::stable_sort(sym.begin(), sym.end(), [&](int a, int b) { return hist[a] < hist[b]; });
+
+    // is_leaf[d][i]: item i of the depth-d list is a leaf coin
+    std::vector<std::vector<uint8_t>> is_leaf(L + 1);
+    std::vector<uint64_t> prev(m), cur;
+    for (int i = 0; i < m; i++) prev[i] = hist[sym[i]];
+    is_leaf[L].assign(m, 1);
+    for (int d = L - 1; d >= 1; d--) {
+        const size_t npk = prev.size() / 2;
+        cur.clear();
+        is_leaf[d].clear();
+        size_t li = 0, pi = 0;
+        while (li < size_t(m) || pi < npk) {
+            const bool have_pk = pi < npk;
+            const uint64_t pw = have_pk ? prev[2 * pi] + prev[2 * pi + 1] : 0;
+            if (li < size_t(m) && (!have_pk || hist[sym[li]] <= pw)) {
+                cur.push_back(hist[sym[li++]]);
+                is_leaf[d].push_back(1);
+            } else {
+                cur.push_back(pw);
+                is_leaf[d].push_back(0);
+                pi++;
+            }
+        }
+        prev.swap(cur);
+    }
+    size_t k = size_t(2 * (m - 1));
+    if (is_leaf[1].size() < k) return fail(DF11_ERR_INVALID, "df11_code_lengths: too few items");
+    for (int d = 1; d <= L && k; d++) {
+        size_t j = 0;
+        for (size_t i = 0; i < k; i++) j += is_leaf[d][i];
+        for (size_t i = 0; i < j; i++) code_len[sym[i]]++;
+        k = 2 * (k - j);
+    }
+    return DF11_OK;
+}
+
+df11_status df11_header_init(df11_header* hdr, const uint8_t* code_len, uint64_t n_elems,
+                             uint64_t total_bits, uint32_t threads_per_block,
+                             uint32_t max_code_len, const uint64_t* seg_counts,
+                             uint32_t n_segs) {
+    if (!hdr || !code_len) return fail(DF11_ERR_INVALID, "df11_header_init: null pointer");
+    const uint32_t T = threads_per_block;
+    if (T < 64 || T > 1024 || (T & (T - 1)))
+        return fail(DF11_ERR_INVALID, "threads_per_block %u is not a power of two in 64..1024", T);
+    if (max_code_len < 1 || max_code_len > 32)
+        return fail(DF11_ERR_INVALID, "max_code_len %u outside 1..32", max_code_len);
+    if (n_elems >= (uint64_t(1) << 32))
+        return fail(DF11_ERR_TOO_LARGE, "n_elems %llu does not fit the 32-bit block offsets",
+                    (unsigned long long)n_elems);
+    if (n_segs < 1 || n_segs > DF11_MAX_SEGMENTS)
+        return fail(DF11_ERR_INVALID, "n_segments %u outside 1..%d", n_segs, DF11_MAX_SEGMENTS);
+    uint64_t units;
+    int m;
+    if (!kraft_units(code_len, &units, &m))
+        return fail(DF11_ERR_INVALID, "code length above 32");
+    for (int s = 0; s < 256; s++)
+        if (code_len[s] > max_code_len)
+            return fail(DF11_ERR_INVALID, "code length %u above max_code_len %u", code_len[s], max_code_len);
+    if (n_elems > 0 && m == 0) return fail(DF11_ERR_INVALID, "empty code table for a non-empty stream");
+    if (m == 1 && units != (uint64_t(1) << 31))
+        return fail(DF11_ERR_INVALID, "a single present value must have the 1-bit code");
+    if (m >= 2 && units != (uint64_t(1) << 32))
+        return fail(DF11_ERR_INVALID, "code lengths are not a complete prefix code (Kraft sum != 1)");
+    if (n_elems && (total_bits < n_elems || total_bits > 32 * n_elems))
+        return fail(DF11_ERR_INVALID, "total_bits %llu inconsistent with %llu elements",
+                    (unsigned long long)total_bits, (unsigned long long)n_elems);
+    if (!n_elems && total_bits) return fail(DF11_ERR_INVALID, "bits without elements");
+
+    std::memset(hdr, 0, sizeof(*hdr));
+    hdr->version = DF11_VERSION;
+    hdr->window_bytes = DF11_WINDOW_BYTES;
+    hdr->threads_per_block = T;
+    hdr->max_code_len = max_code_len;
+    hdr->n_elems = n_elems;
+    hdr->total_bits = total_bits;
+    std::memcpy(hdr->code_len, code_len, 256);
+    hdr->n_segments = n_segs;
+    uint64_t acc = 0;
+    for (uint32_t k = 0; k < n_segs; k++) {
+        hdr->seg_elem_off[k] = acc;
+        acc += seg_counts ? seg_counts[k] : n_elems;
+    }
+    hdr->seg_elem_off[n_segs] = acc;
+    if (acc != n_elems) return fail(DF11_ERR_INVALID, "segment counts do not add up to n_elems");
+    fill_sizes(hdr);
+    return DF11_OK;
+}
+
+// Decode tables for hdr->code_len, in the layout of df11_internal.h.
+df11_status df11_build_lut(const df11_header* hdr, void* h_lut, uint64_t cap) {
+    if (!hdr || !h_lut) return fail(DF11_ERR_INVALID, "df11_build_lut: null pointer");
+    if (cap < kLutBytes) return fail(DF11_ERR_CAPACITY, "df11_build_lut: need %llu bytes",
+                                     (unsigned long long)kLutBytes);
+    const uint8_t* len = hdr->code_len;
+    uint32_t code[256];
+    if (!canonical_codes(len, code)) return fail(DF11_ERR_INVALID, "code lengths overflow");
+
+    uint8_t* blob = static_cast<uint8_t*>(h_lut);
+    std::memset(blob, 0, kLutBytes);
+    LutHeader lh{};
+    lh.magic = kLutMagic;
+    lh.count_bits = kCountBits;
+    lh.decode_bits = kDecodeBits;
+
+    // per-length counts and first codes
+    uint64_t count[34] = {0}, first[34] = {0};
+    for (int s = 0; s < 256; s++)
+        if (len[s]) count[len[s]]++;
+    uint64_t c = 0;
+    for (int l = 1; l <= 32; l++) {
+        c = (c + count[l - 1]) << 1;
+        first[l] = c;
+    }
+    // symbols sorted by (length, value); base = codes shorter than l
+    uint8_t* syms = blob + kLutOffSyms;
+    uint32_t base[34] = {0};
+    int n = 0;
+    lh.min_len = 0;
+    lh.max_len = 0;
+    for (int l = 1; l <= 32; l++) {
+        base[l] = uint32_t(n);
+        for (int s = 0; s < 256; s++)
+            if (len[s] == l) syms[n++] = uint8_t(s);
+        if (count[l] && !lh.min_len) lh.min_len = l;
+        if (count[l]) lh.max_len = l;
+    }
+    lh.n_syms = uint32_t(n);
+    uint64_t* lj_end = reinterpret_cast<uint64_t*>(blob + kLutOffLjEnd);
+    uint32_t* delta = reinterpret_cast<uint32_t*>(blob + kLutOffDelta);
+    lj_end[0] = 0;
+    for (int l = 1; l <= 32; l++) {
+        lj_end[l] = (first[l] + count[l]) << (32 - l);
+        delta[l] = base[l] - uint32_t(first[l]);  // wraps; used modulo 2^32
+    }
+
+    // length of the code at the top of a 32-bit left-justified peek, 0 if none
+    auto code_length = [&](uint64_t peek32) -> int {
+        for (int l = 1; l <= 32; l++)
+            if (peek32 < lj_end[l]) return l;
+        return 0;
+    };
+
+    uint16_t* ctab = reinterpret_cast<uint16_t*>(blob + kLutOffCount);
+    for (uint32_t v = 0; v < (1u << kCountBits); v++) {
+        uint32_t mask = 0;
+        int pos = 0;
+        while (pos < kCountBits) {
+            uint64_t peek = (uint64_t(v) << (32 - kCountBits + pos)) & 0xFFFFFFFFull;
+            int l = code_length(peek);
+            if (l == 0 || pos + l > kCountBits) break;
+            mask |= 1u << pos;
+            pos += l;
+        }
+        ctab[v] = uint16_t(mask | (uint32_t(pos) << 12));
+    }
+    uint32_t* dtab = reinterpret_cast<uint32_t*>(blob + kLutOffDecode);
+    for (uint32_t v = 0; v < (1u << kDecodeBits); v++) {
+        uint32_t entry = 0, nsym = 0;
+        int pos = 0;
+        while (nsym < 3 && pos < kDecodeBits) {
+            uint64_t peek = (uint64_t(v) << (32 - kDecodeBits + pos)) & 0xFFFFFFFFull;
+            int l = code_length(peek);
+            if (l == 0 || pos + l > kDecodeBits) break;
+            uint32_t value = uint32_t(peek >> (32 - l));
+            uint32_t s = syms[(value + delta[l]) & 0xFFu];
+            entry |= s << (8 * nsym);
+            nsym++;
+            pos += l;
+        }
+        dtab[v] = nsym ? (entry | (nsym << 24) | (uint32_t(pos) << 26)) : 0u;
+    }
+    std::memcpy(blob, &lh, sizeof(lh));
+    return DF11_OK;
+}
+
+df11_status df11_compress_workspace_size(uint64_t n_elems, uint64_t* bytes) {
+    if (!bytes) return fail(DF11_ERR_INVALID, "df11_compress_workspace_size: null pointer");
+    const uint64_t chunks = (n_elems + kEncChunk - 1) / kEncChunk;
+    // histogram (256 x u64) + per-chunk bit counts (u32) + chunk starts (u64)
+    *bytes = 2048 + align16(4 * chunks) + align16(8 * chunks) + 64;
+    return DF11_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,191 @@
+"""CPU-only checks of the C-ABI library: it loads, exports every entry point
+that include/df11.h declares, and its host logic (code builder, header
+validation, decode tables) agrees with the oracle.  No kernel runs here."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+import lossless_entropy_coded_dfloat11_b200 as df11
+from lossless_entropy_coded_dfloat11_b200 import _binding as B
+from lossless_entropy_coded_dfloat11_b200 import inputs
+from tests.conftest import ROOT
+
+HEADER = os.path.join(ROOT, "include", "df11.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(df11_[a-z_]+)\s*\(", text)))
+
+
+def test_library_loads_and_exports_every_declared_symbol():
+    lib = df11.load_library()
+    names = declared_functions()
+    assert len(names) >= 9
+    for name in names:
+        assert hasattr(lib, name), name
+    assert set(names) == set(B.EXPORTED)
+    assert lib.df11_version() == 1
+
+
+def test_header_struct_layout_matches_c():
+    assert ctypes.sizeof(B.Header) == 872
+    assert B.Header.code_len.offset == 48
+    assert B.Header.seg_elem_off.offset == 312
+    assert B.Header.bytes_lut.offset == 864
+
+
+def hist_of(weights, symbols):
+    h = np.zeros(256, dtype=np.uint64)
+    h[list(symbols)] = weights
+    return h
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_code_lengths_identical_to_oracle(seed):
+    """The library and the oracle implement package-merge separately with the
+    same tie rule, so their lengths must be identical, not just equally good."""
+    rng = np.random.default_rng(seed)
+    m = int(rng.integers(1, 257))
+    syms = rng.choice(256, size=m, replace=False)
+    kind = seed % 4
+    if kind == 0:
+        w = rng.integers(1, 10, size=m)          # many ties
+    elif kind == 1:
+        w = rng.zipf(1.1, size=m).clip(max=10 ** 12)
+    elif kind == 2:
+        w = rng.integers(1, 2 ** 40, size=m)
+    else:
+        w = np.full(m, 7)
+    h = hist_of(w, syms)
+    minL = max(1, int(np.ceil(np.log2(max(m, 2)))))
+    for L in sorted({minL, minL + 1, 12, 16, 24, 32}):
+        if L > 32:
+            continue
+        np.testing.assert_array_equal(df11.code_lengths(h, L), oracle.code_lengths(h, L))
+
+
+def test_code_lengths_fibonacci_and_workloads():
+    fib = [1, 1]
+    while len(fib) < 40:
+        fib.append(fib[-1] + fib[-2])
+    h = hist_of(fib, range(200, 240))
+    for L in (6, 12, 20, 32):
+        np.testing.assert_array_equal(df11.code_lengths(h, L), oracle.code_lengths(h, L))
+    for w in (inputs.matrix_1k(), inputs.edge_case(65537, "zipf", 515), inputs.all_patterns()):
+        h = oracle.histogram(w.flat_u16())
+        np.testing.assert_array_equal(df11.code_lengths(h, 32), oracle.code_lengths(h, 32))
+
+
+def test_code_lengths_rejects_bad_limits():
+    h = hist_of([1] * 5, range(5))
+    with pytest.raises(df11.DF11Error):
+        df11.code_lengths(h, 2)        # 5 values do not fit 2-bit codes
+    with pytest.raises(df11.DF11Error):
+        df11.code_lengths(h, 33)
+
+
+@pytest.mark.parametrize("T", [64, 256, 1024])
+def test_header_sizes_match_oracle(T):
+    x = inputs.edge_case(4097, "zipf", 514).flat_u16()
+    s = oracle.encode(x, threads_per_block=T)
+    hdr = df11.make_header(s.code_len, s.n_elems, s.total_bits, T)
+    sz = oracle.sizes(oracle.histogram(x), s.code_len, T)
+    assert (hdr.n_threads, hdr.n_blocks) == (sz["n_threads"], sz["n_blocks"])
+    assert (hdr.bytes_exp, hdr.bytes_sm, hdr.bytes_gaps, hdr.bytes_off) == (
+        sz["bytes_exp"], sz["bytes_sm"], sz["bytes_gaps"], sz["bytes_off"])
+
+
+def test_header_validation():
+    ln = np.zeros(256, dtype=np.uint8)
+    ln[[1, 2, 3]] = [1, 2, 2]
+    df11.make_header(ln, 10, 15, 256)
+    bad = ln.copy()
+    bad[4] = 3                                   # Kraft sum above 1
+    with pytest.raises(df11.DF11Error):
+        df11.make_header(bad, 10, 15, 256)
+    bad = ln.copy()
+    bad[3] = 3                                   # incomplete code
+    with pytest.raises(df11.DF11Error):
+        df11.make_header(bad, 10, 15, 256)
+    with pytest.raises(df11.DF11Error):
+        df11.make_header(ln, 10, 15, 96)         # T not a power of two
+    with pytest.raises(df11.DF11Error) as e:
+        df11.make_header(ln, 2 ** 32, 2 ** 33, 256)
+    assert e.value.code == B.DF11_ERR_TOO_LARGE
+    with pytest.raises(df11.DF11Error):
+        df11.make_header(ln, 10, 5, 256)         # fewer bits than elements
+    one = np.zeros(256, dtype=np.uint8)
+    one[9] = 1
+    df11.make_header(one, 3, 3, 64)              # single value: code "0"
+    one[9] = 2
+    with pytest.raises(df11.DF11Error):
+        df11.make_header(one, 3, 6, 64)
+
+
+LUT_COUNT_BITS = 12
+LUT_DECODE_BITS = 12
+OFF_COUNT = 736          # after the 64-byte header, lj_end[33], delta[33], syms[256]
+OFF_DECODE = OFF_COUNT + 2 * 4096
+
+
+def _oracle_prefix_decoder(code_len):
+    codes = oracle.canonical_codes(code_len)
+    table = {format(int(codes[s]), "0%db" % int(code_len[s])): int(s)
+             for s in range(256) if code_len[s]}
+    return table
+
+
+def _decode_bits(table, bits, limit):
+    """Complete codes at the front of the bit string (oracle codes)."""
+    out, pos = [], 0
+    while True:
+        for l in range(1, len(bits) - pos + 1):
+            sym = table.get(bits[pos:pos + l])
+            if sym is not None:
+                break
+        else:
+            return out, pos
+        if len(out) == limit:
+            return out, pos
+        out.append((sym, pos))
+        pos += l
+
+
+@pytest.mark.parametrize("source", ["matrix_1k", "zipf", "one_value", "fibonacci"])
+def test_decode_tables_agree_with_oracle_codes(source):
+    """Every level-1 entry must describe exactly the complete oracle codes at
+    the front of its 12-bit index."""
+    if source == "matrix_1k":
+        x = inputs.matrix_1k().flat_u16()
+    elif source == "fibonacci":
+        x = inputs.fibonacci().flat_u16()
+    else:
+        x = inputs.edge_case(65537, source, 515).flat_u16()
+    s = oracle.encode(x)
+    hdr = df11.make_header(s.code_len, s.n_elems, s.total_bits, 256)
+    lut = df11.build_lut(hdr)
+    assert lut[:4].tobytes() == b"DF11"
+    ctab = lut[OFF_COUNT:OFF_COUNT + 2 * 4096].view(np.uint16)
+    dtab = lut[OFF_DECODE:OFF_DECODE + 4 * 4096].view(np.uint32)
+    table = _oracle_prefix_decoder(s.code_len)
+    rng = np.random.default_rng(3)
+    for v in list(range(64)) + list(rng.integers(0, 4096, size=400)) + list(range(4032, 4096)):
+        bits = format(int(v), "012b")
+        codes, used = _decode_bits(table, bits, None)
+        mask = sum(1 << p for _, p in codes)
+        assert int(ctab[v]) == (mask | (used << 12) if codes else 0), (v, bits)
+        codes3, used3 = _decode_bits(table, bits, 3)
+        e = int(dtab[v])
+        if not codes3:
+            assert e == 0
+            continue
+        assert (e >> 24) & 3 == len(codes3)
+        assert e >> 26 == used3
+        for k, (sym, _) in enumerate(codes3):
+            assert (e >> (8 * k)) & 0xFF == sym
