@@ -60,6 +60,7 @@ extern "C" {
 #define DF11_WINDOW_BYTES 8
 #define DF11_MAX_CODE_LEN 32
 #define DF11_MAX_SEGMENTS 64
+#define DF11_STATIC_MAX_ELEMS (1ull << 28) /* limit of df11_compress_encode_static */
 
 typedef enum {
     DF11_OK = 0,
@@ -153,6 +154,29 @@ df11_status df11_compress_encode(const void* const* d_segs, const df11_header* h
                                  void* d_workspace, uint64_t workspace_bytes, uint8_t* d_exp,
                                  uint8_t* d_sm, uint8_t* d_gaps, uint32_t* d_block_off,
                                  void* d_lut, void* stream);
+
+/* Compress, step 2 of 2, without allocating: the pages have no counterpart
+ * to this entry point.  It writes exactly what df11_compress_encode writes,
+ * but keeps its scratch (per-chunk bit totals and start bits) in a fixed
+ * array inside the library instead of a caller workspace.  It is for callers
+ * that cannot allocate device memory at compress time: serving engines that
+ * hand all of HBM to their own pools at start-up and forbid later cudaMalloc
+ * calls, and code running inside an allocator (an out-of-memory handler, for
+ * instance) where allocating would recurse.  It calls no cudaMalloc/cudaFree.
+ *   - At most DF11_STATIC_MAX_ELEMS (2^28) elements per call; larger streams
+ *     get DF11_ERR_TOO_LARGE (use df11_compress_encode with a workspace).
+ *   - The scratch is 786,432 bytes of device memory that every GPU loading
+ *     the library holds until exit.
+ *   - The first call on a device looks up the scratch's device address (with
+ *     that device current); make that first call before any stream capture.
+ *   - All calls share the one scratch array and every call overwrites all of
+ *     it that it reads, so no clearing is needed; calls whose work overlaps
+ *     on the GPU (other streams, other host threads) race on it and must be
+ *     serialised by the caller.
+ * Arguments as for df11_compress_encode, minus the workspace. */
+df11_status df11_compress_encode_static(const void* const* d_segs, const df11_header* hdr,
+                                        uint8_t* d_exp, uint8_t* d_sm, uint8_t* d_gaps,
+                                        uint32_t* d_block_off, void* d_lut, void* stream);
 
 /* Decompress one stream -- every matrix of a transformer block -- in one
  * kernel launch ("Descompressao por bloco de transformer"; two-phase kernel of

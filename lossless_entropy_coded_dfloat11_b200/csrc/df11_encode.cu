@@ -10,7 +10,9 @@
 // position per thread block).
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstring>
+#include <mutex>
 #include <vector>
 
 #include "df11_internal.h"
@@ -426,6 +428,122 @@ extern "C" df11_status df11_compress_encode(const void* const* d_segs, const df1
     uint32_t log2_bb = 6;
     while ((1u << (log2_bb - 6)) < hdr->threads_per_block) log2_bb++;
     pack_kernel<<<unsigned(chunks), kEncThreads, 0, s>>>(sg, ct, n, log2_bb, w.chunk_start,
+                                                         reinterpret_cast<uint32_t*>(d_exp), d_sm,
+                                                         reinterpret_cast<uint32_t*>(d_gaps), d_block_off,
+                                                         hdr->n_blocks);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail("encode launch", e);
+    return DF11_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Encode without any allocation: the same kernels as df11_compress_encode,
+// with their scratch (per-chunk bit totals and chunk start bits) in a
+// fixed-size array that lives in the library's own device memory.  For
+// callers that cannot allocate device memory when they compress: serving
+// engines that hand all of HBM to their own pools at start-up and forbid
+// later cudaMalloc calls, and code running inside an allocator (an
+// out-of-memory handler, say) where allocating would recurse.
+// ---------------------------------------------------------------------------
+namespace df11 {
+namespace {
+
+constexpr uint64_t kStaticChunks = DF11_STATIC_MAX_ELEMS / kEncChunk;
+constexpr uint64_t kStaticBitsBytes = 4 * kStaticChunks;
+constexpr uint64_t kStaticScratchBytes = kStaticBitsBytes + 8 * kStaticChunks;
+static_assert(DF11_STATIC_MAX_ELEMS % kEncChunk == 0, "whole chunks");
+
+// Loaded with the library on every GPU that uses it and held until exit.
+// Every call overwrites all of the scratch it reads, so nothing has to be
+// cleared between calls; two calls that overlap on the GPU share it and race.
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+// Device address of the scratch, looked up once per device with that device
+// current (host code cannot use the symbol itself as a device pointer).
+constexpr int kMaxDevices = 64;
+std::atomic<void*> g_static_scratch_addr[kMaxDevices];
+std::mutex g_static_scratch_mu;
+
+df11_status static_scratch_address(void** out) {
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail("cudaGetDevice", e);
+    if (dev < 0 || dev >= kMaxDevices) return fail(DF11_ERR_INVALID, "device ordinal %d above %d", dev, kMaxDevices);
+    void* p = g_static_scratch_addr[dev].load(std::memory_order_acquire);
+    if (!p) {
+        std::lock_guard<std::mutex> lock(g_static_scratch_mu);
+        p = g_static_scratch_addr[dev].load(std::memory_order_relaxed);
+        if (!p) {
+            e = cudaGetSymbolAddress(&p, g_static_scratch);
+            if (e != cudaSuccess) return cuda_fail("cudaGetSymbolAddress(static scratch)", e);
+            g_static_scratch_addr[dev].store(p, std::memory_order_release);
+        }
+    }
+    *out = p;
+    return DF11_OK;
+}
+
+}  // namespace
+}  // namespace df11
+
+extern "C" df11_status df11_compress_encode_static(const void* const* d_segs, const df11_header* hdr,
+                                                   uint8_t* d_exp, uint8_t* d_sm, uint8_t* d_gaps,
+                                                   uint32_t* d_block_off, void* d_lut, void* stream) {
+    df11_status st = check_header(hdr);
+    if (st != DF11_OK) return st;
+    if (hdr->n_elems > DF11_STATIC_MAX_ELEMS)
+        return fail(DF11_ERR_TOO_LARGE,
+                    "df11_compress_encode_static: %llu elements, its fixed scratch holds at most %llu; "
+                    "use df11_compress_encode with a workspace",
+                    (unsigned long long)hdr->n_elems, (unsigned long long)DF11_STATIC_MAX_ELEMS);
+    uint64_t counts[DF11_MAX_SEGMENTS];
+    if (hdr->n_segments < 1 || hdr->n_segments > DF11_MAX_SEGMENTS)
+        return fail(DF11_ERR_INVALID, "header n_segments %u", hdr->n_segments);
+    for (uint32_t k = 0; k < hdr->n_segments; k++) counts[k] = hdr->seg_elem_off[k + 1] - hdr->seg_elem_off[k];
+    SegTable sg;
+    uint64_t n = 0;
+    st = build_segtable(d_segs, counts, hdr->n_segments, &sg, &n);
+    if (st != DF11_OK) return st;
+    if (n != hdr->n_elems) return fail(DF11_ERR_INVALID, "segments disagree with header n_elems");
+    if (!d_exp || !d_sm || !d_gaps || !d_block_off || !d_lut)
+        return fail(DF11_ERR_INVALID, "df11_compress_encode_static: null output pointer");
+    if (!aligned16(d_exp) || !aligned16(d_sm) || !aligned16(d_gaps) || !aligned16(d_block_off) ||
+        !aligned16(d_lut))
+        return fail(DF11_ERR_INVALID, "df11_compress_encode_static: outputs must be 16-byte aligned");
+    void* scratch = nullptr;
+    st = static_scratch_address(&scratch);
+    if (st != DF11_OK) return st;
+    uint32_t* chunk_bits = static_cast<uint32_t*>(scratch);
+    unsigned long long* chunk_start =
+        reinterpret_cast<unsigned long long*>(static_cast<unsigned char*>(scratch) + kStaticBitsBytes);
+
+    CodeTable ct;
+    std::memcpy(ct.len, hdr->code_len, 256);
+    if (!canonical_codes(hdr->code_len, ct.code)) return fail(DF11_ERR_INVALID, "code lengths overflow");
+    // decode tables are built in this thread's own host buffer (no heap)
+    static thread_local unsigned char lut[kLutBytes];
+    st = df11_build_lut(hdr, lut, sizeof(lut));
+    if (st != DF11_OK) return st;
+
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    if ((e = cudaMemcpyAsync(d_lut, lut, kLutBytes, cudaMemcpyHostToDevice, s)) != cudaSuccess)
+        return cuda_fail("table upload", e);
+    if ((e = cudaMemsetAsync(d_exp, 0, hdr->bytes_exp, s)) != cudaSuccess) return cuda_fail("clear exp", e);
+    if ((e = cudaMemsetAsync(d_gaps, 0, hdr->bytes_gaps, s)) != cudaSuccess) return cuda_fail("clear gaps", e);
+    if ((e = cudaMemsetAsync(d_block_off, 0, hdr->bytes_off, s)) != cudaSuccess) return cuda_fail("clear off", e);
+    const uint64_t sm_tail = n & ~uint64_t(15);
+    if (hdr->bytes_sm > sm_tail &&
+        (e = cudaMemsetAsync(d_sm + sm_tail, 0, hdr->bytes_sm - sm_tail, s)) != cudaSuccess)
+        return cuda_fail("clear sm tail", e);
+    if (n == 0) return DF11_OK;
+
+    const uint64_t chunks = (n + kEncChunk - 1) / kEncChunk;
+    chunk_bits_kernel<<<unsigned(chunks), kEncThreads, 0, s>>>(sg, ct, n, chunk_bits);
+    chunk_scan_kernel<<<1, kScanThreads, 0, s>>>(chunk_bits, chunks, chunk_start);
+    uint32_t log2_bb = 6;
+    while ((1u << (log2_bb - 6)) < hdr->threads_per_block) log2_bb++;
+    pack_kernel<<<unsigned(chunks), kEncThreads, 0, s>>>(sg, ct, n, log2_bb, chunk_start,
                                                          reinterpret_cast<uint32_t*>(d_exp), d_sm,
                                                          reinterpret_cast<uint32_t*>(d_gaps), d_block_off,
                                                          hdr->n_blocks);
