@@ -5,10 +5,10 @@ builder behind the C ABI of include/df11.h); this package allocates
 caller-owned buffers with PyTorch and passes pointers.  Importing it does not
 load the library; the first call does, and raises if it is missing.
 """
-from .codec import (CompressedStream, HostStream, build_lut, code_lengths, compress, decompress,
+from .codec import (DEFAULT_THREADS_PER_BLOCK, CompressedStream, HostStream, build_lut, code_lengths, compress, decompress,
                     from_arrays, make_header, to_host, workspace_bytes)
 from ._binding import DF11Error, EXPORTED, load as load_library, library_path
 
-__all__ = ["CompressedStream", "HostStream", "build_lut", "code_lengths", "compress", "decompress",
+__all__ = ["DEFAULT_THREADS_PER_BLOCK", "CompressedStream", "HostStream", "build_lut", "code_lengths", "compress", "decompress",
            "from_arrays", "make_header", "to_host", "workspace_bytes", "DF11Error", "EXPORTED",
            "load_library", "library_path"]

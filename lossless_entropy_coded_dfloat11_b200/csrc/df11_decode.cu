@@ -1,26 +1,35 @@
-// DF11 decompression kernel for sm_100a.
+// DF11 decompression kernels for sm_100a.
 //
 // Follows the two-phase design of "DFloat11: compressao sem perda para
 // inferencia em GPU que reduz LLMs para 70% do tamanho", section "Kernel de
 // GPU em 2 etapas e metadados auxiliares": every thread owns one 8-byte
 // window of EncodedExponent and decodes the codes that start in it, beginning
-// at its 5-bit gap; phase 1 counts them, a block-wide prefix sum turns counts
-// into output positions (added to the thread block's stored position), and
-// phase 2 decodes again into an on-chip buffer that is written to HBM with
-// coalesced stores.  One launch covers a whole stream, i.e. every matrix of a
-// transformer block ("Descompressao por bloco de transformer").
+// at its 5-bit gap; phase 1 counts them, a prefix sum over the thread block
+// turns counts into output positions (added to the block's stored position),
+// and phase 2 decodes again into an on-chip buffer that is written to HBM
+// with coalesced stores.  One launch covers a whole stream, i.e. every matrix
+// of a transformer block ("Descompressao por bloco de transformer").
 //
 // B200 specifics:
-//   * persistent grid (resident CTAs x SMs): the decode tables are copied to
-//     shared memory once per CTA and reused for every thread block of the
-//     stream;
-//   * multi-symbol level-1 tables: the count table gives the start mask of
-//     every complete code in the next 12 bits, the decode table up to three
-//     symbols per lookup; codes longer than 12 bits use the canonical
-//     comparison ladder (level 2);
-//   * the merge of exponent and sign+mantissa works on 16 elements per
-//     thread: one 16-byte shared load, one 16-byte streaming global load, two
-//     16-byte streaming global stores.
+//   * persistent grid: the 57 KB of decode tables are copied to shared memory
+//     once per CTA and serve every thread block of the stream;
+//   * thread blocks of 32 threads (T = 32) are decoded by one warp each, with
+//     no CTA barrier at all: the prefix sum is five shuffles and the staging
+//     buffer is the warp's own; larger T use a block-wide scan;
+//   * software pipelining: the next block's window, gap and output positions
+//     are loaded while the current one is decoded, and the current block's
+//     sign+mantissa bytes are requested before its decode starts;
+//   * the decode loops keep (bit position << 16 | counter) in one register
+//     and advance both with one add; the loops run separately over the first
+//     and second 32 bits of the window so each peek is one funnel shift; codes
+//     longer than the 12-bit tables leave through an escape value that pushes
+//     the bit position out of the window, so the fast loops have one test;
+//   * phase 2 gathers symbols in registers and stores aligned 32-bit words;
+//     a thread's first word, shared with the previous thread, is filled
+//     byte-wise after a warp barrier;
+//   * the merge handles 16 elements per thread with one 16-byte shared load,
+//     one 16-byte streaming load, 24 logic/permute operations and two 16-byte
+//     streaming stores.
 #include <cuda_runtime.h>
 
 #include <atomic>
@@ -45,219 +54,467 @@ struct DecodeArgs {
     uint64_t n_blocks;
 };
 
+struct Tables {
+    const uint32_t* ctab;             // count table
+    const uint16_t* mtab;             // start-mask table
+    const uint2* dtab;                // decode table
+    const unsigned long long* lj_end; // level 2
+    const uint32_t* delta;
+    const uint8_t* syms;
+};
+
+__device__ __forceinline__ Tables tables_at(const uint8_t* s_lut) {
+    Tables t;
+    t.ctab = reinterpret_cast<const uint32_t*>(s_lut + kLutOffCount);
+    t.mtab = reinterpret_cast<const uint16_t*>(s_lut + kLutOffMask);
+    t.dtab = reinterpret_cast<const uint2*>(s_lut + kLutOffDecode);
+    t.lj_end = reinterpret_cast<const unsigned long long*>(s_lut + kLutOffLjEnd);
+    t.delta = reinterpret_cast<const uint32_t*>(s_lut + kLutOffDelta);
+    t.syms = s_lut + kLutOffSyms;
+    return t;
+}
+
 __device__ __forceinline__ uint32_t bswap32(uint32_t x) { return __byte_perm(x, 0, 0x0123); }
 
 // 32 stream bits starting at bit `pos` (0 <= pos < 64) of the 96-bit window
 // w0:w1:w2 (MSB first).
-__device__ __forceinline__ uint32_t peek32(uint32_t w0, uint32_t w1, uint32_t w2, int pos) {
+__device__ __forceinline__ uint32_t peek32(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t pos) {
     const uint32_t hi = pos < 32 ? w0 : w1;
     const uint32_t lo = pos < 32 ? w1 : w2;
-    return __funnelshift_l(lo, hi, uint32_t(pos));
+    return __funnelshift_l(lo, hi, pos);
 }
 
-// Length of the canonical code at the top of `peek` (level 2); 0 if no code
-// matches (only possible in a corrupt stream).
-__device__ __forceinline__ int code_length(const unsigned long long* lj_end, uint32_t peek) {
-    for (int l = 1; l <= 32; l++)
+// Level 2: length of the canonical code at the top of `peek`, 0 if none.
+// Codes shorter than `from` bits are known not to match.
+__device__ __forceinline__ int code_length(const unsigned long long* lj_end, uint32_t peek, int from = 1) {
+    for (int l = from; l <= 32; l++)
         if ((unsigned long long)peek < lj_end[l]) return l;
     return 0;
 }
 
-// Two BF16 results from exponent bytes and sign+mantissa bytes picked by
-// `sel` (0x4140: bytes 0 and 1, 0x4342: bytes 2 and 3):
-// bf16 = (sm & 0x80) << 8 | e << 7 | (sm & 0x7F).
-__device__ __forceinline__ uint32_t merge_pair(uint32_t e4, uint32_t s4, uint32_t sel) {
-    const uint32_t x = __byte_perm(s4, 0, sel);
-    const uint32_t e = __byte_perm(e4, 0, sel);
-    return (x & 0x007F007Fu) | ((x & 0x00800080u) << 8) | (e << 7);
+__device__ __forceinline__ uint32_t code_symbol(const Tables& t, uint32_t peek, int l) {
+    return t.syms[((peek >> (32 - l)) + t.delta[l]) & 0xFFu];
 }
 
-template <int T>
-__global__ void __launch_bounds__(T) decode_kernel(const DecodeArgs a) {
+// Raw loads of one thread's window, issued early and finished later.
+struct RawWindow {
+    uint2 v;        // the 8-byte window
+    uint32_t v2;    // 4-byte lookahead
+    uint32_t glo, ghi;
+};
+
+struct Window {
+    uint32_t w0, w1, w2;  // 96 stream bits, MSB first
+    uint32_t start;       // first code start in the window (the gap)
+    uint32_t wend;        // end of the window inside the stream, 0..64
+};
+
+__device__ __forceinline__ RawWindow load_window(const DecodeArgs& a, uint64_t tg) {
+    RawWindow r;
+    if (tg < a.n_threads) {
+        r.v = __ldg(reinterpret_cast<const uint2*>(a.exp) + tg);
+        r.v2 = __ldg(reinterpret_cast<const uint32_t*>(a.exp) + 2 * tg + 2);
+        const uint64_t gw = (5 * tg) >> 5;
+        r.glo = __ldg(a.gaps + gw);
+        r.ghi = __ldg(a.gaps + gw + 1);
+    } else {
+        r.v = make_uint2(0, 0);
+        r.v2 = r.glo = r.ghi = 0;
+    }
+    return r;
+}
+
+__device__ __forceinline__ Window finish_window(const DecodeArgs& a, const RawWindow& r, uint64_t tg) {
+    Window w;
+    w.w0 = bswap32(r.v.x);
+    w.w1 = bswap32(r.v.y);
+    w.w2 = bswap32(r.v2);
+    w.start = __funnelshift_r(r.glo, r.ghi, uint32_t(5 * tg)) & 31u;
+    if (tg < a.n_threads) {
+        const uint64_t rem = a.total_bits - 64 * tg;
+        w.wend = rem < 64 ? uint32_t(rem) : 64u;
+    } else {
+        w.wend = 0;
+    }
+    return w;
+}
+
+// Phase 1: number of codes that start in [start, wend).  Sets `bad` if a
+// bit pattern matches no code (corrupt stream).
+__device__ __forceinline__ uint32_t count_codes(const Window& w, const Tables& t, bool& bad) {
+    const uint32_t lim1 = min(w.wend, 32u) << 16;
+    const uint32_t lim2 = w.wend << 16;
+    uint32_t acc = w.start << 16;  // bit position << 16 | codes counted
+    uint32_t e = 0, idx = 0;
+    for (;;) {
+        while (acc < lim1) {
+            idx = __funnelshift_l(w.w1, w.w0, acc >> 16) >> (32 - kPeekBits);
+            e = t.ctab[idx];
+            acc += e;
+        }
+        while (acc < lim2) {
+            idx = __funnelshift_l(w.w2, w.w1, acc >> 16) >> (32 - kPeekBits);
+            e = t.ctab[idx];
+            acc += e;
+        }
+        if (acc < (kEscape << 16)) break;
+        // a code longer than the table: undo the escape, take it from level 2
+        acc -= kEscape << 16;
+        const int l = code_length(t.lj_end, peek32(w.w0, w.w1, w.w2, acc >> 16), kPeekBits + 1);
+        if (!l) {
+            bad = true;
+            return 0;
+        }
+        acc += (uint32_t(l) << 16) | 1u;
+        e = 0;
+    }
+    uint32_t cnt = acc & 0xFFFFu;
+    if (e) {  // the last table step may hold codes starting at or past wend
+        const uint32_t s = w.wend - ((acc >> 16) - (e >> 16));
+        if (s < uint32_t(kPeekBits)) cnt -= __popc(uint32_t(t.mtab[idx]) >> s);
+    }
+    return cnt;
+}
+
+// Phase 2: decode the same codes into staging bytes [pos0, pos0 + cnt).
+// Symbols collect in a 64-bit register pair and leave as aligned 32-bit
+// words.  The thread's first word is skipped when it starts mid-word (it is
+// shared with the previous thread; write_head fills those bytes after a
+// barrier).  A word holding the thread's last symbols may also carry up to
+// three bytes decoded past the window end; those positions are head bytes of
+// the following threads (which start mid-word), rewritten by write_head.
+__device__ __forceinline__ void decode_codes(const Window& w, const Tables& t, uint32_t* stage32, uint32_t pos0,
+                                             uint32_t cnt) {
+    if (cnt == 0) return;
+    const uint32_t lim1 = min(w.wend, 32u) << 16;
+    const uint32_t lim2 = w.wend << 16;
+    const uint32_t last_word = (pos0 + cnt - 1) >> 2;
+    const uint32_t skip_word = (pos0 & 3u) ? (pos0 >> 2) : 0xFFFFFFFFu;
+    uint32_t wi = pos0 >> 2;  // word the pending bytes belong to
+    uint32_t lo = 0, hi = 0;  // pending bytes, byte k = staging position 4*wi + k
+    uint32_t acc = (w.start << 16) | (pos0 & 3u);  // bit position << 16 | bytes pending
+    auto put = [&](uint32_t x, uint32_t y) {
+        const uint32_t sh = (acc << 3) & 24u;
+        lo |= x << sh;
+        hi = __funnelshift_l(x, 0u, sh);
+        acc += y;
+        if (acc & 4u) {  // a word is complete
+            if (wi != skip_word) stage32[wi] = lo;
+            wi++;
+            lo = hi;
+            acc -= 4u;
+        }
+    };
+    for (;;) {
+        while (acc < lim1) {
+            const uint2 e = t.dtab[__funnelshift_l(w.w1, w.w0, acc >> 16) >> (32 - kPeekBits)];
+            put(e.x, e.y);
+        }
+        while (acc < lim2) {
+            const uint2 e = t.dtab[__funnelshift_l(w.w2, w.w1, acc >> 16) >> (32 - kPeekBits)];
+            put(e.x, e.y);
+        }
+        if (acc < (kEscape << 16)) break;
+        acc -= kEscape << 16;
+        const uint32_t pk = peek32(w.w0, w.w1, w.w2, acc >> 16);
+        int l = code_length(t.lj_end, pk, kPeekBits + 1);
+        l = l ? l : 1;
+        put(code_symbol(t, pk, l), (uint32_t(l) << 16) | 1u);
+    }
+    if ((acc & 3u) && wi <= last_word && wi != skip_word) stage32[wi] = lo;
+}
+
+// After a barrier: bytes of this thread's first word when it starts mid-word
+// (positions pos0 .. the next word boundary, at most three symbols).
+__device__ __forceinline__ void write_head(const Window& w, const Tables& t, uint8_t* stage, uint32_t pos0,
+                                           uint32_t cnt) {
+    const uint32_t room = (4u - (pos0 & 3u)) & 3u;
+    const uint32_t k = cnt < room ? cnt : room;
+    if (k == 0) return;
+    uint8_t* base = stage + pos0;
+    const uint2 e = t.dtab[peek32(w.w0, w.w1, w.w2, w.start) >> (32 - kPeekBits)];
+    if ((e.y & 0xFFFFu) >= k) {
+        base[0] = uint8_t(e.x);
+        if (k > 1) base[1] = uint8_t(e.x >> 8);
+        if (k > 2) base[2] = uint8_t(e.x >> 16);
+    } else {  // one of the first codes is longer than the table
+        uint32_t p = w.start;
+        for (uint32_t j = 0; j < k; j++) {
+            const uint32_t q = peek32(w.w0, w.w1, w.w2, p);
+            int l = code_length(t.lj_end, q);
+            l = l ? l : 1;
+            base[j] = uint8_t(code_symbol(t, q, l));
+            p += uint32_t(l);
+        }
+    }
+}
+
+// Four BF16 values from four exponent bytes e4 and four sign+mantissa bytes
+// s4 (bf16 = sign << 15 | e << 7 | mantissa): the high output byte is
+// sign | e >> 1, the low one (e & 1) << 7 | mantissa.
+__device__ __forceinline__ void merge4(uint32_t e4, uint32_t s4, uint32_t& o01, uint32_t& o23) {
+    const uint32_t hi = (s4 & 0x80808080u) | ((e4 >> 1) & 0x7F7F7F7Fu);
+    const uint32_t lo = ((e4 << 7) & 0x80808080u) | (s4 & 0x7F7F7F7Fu);
+    o01 = __byte_perm(lo, hi, 0x5140);
+    o23 = __byte_perm(lo, hi, 0x7362);
+}
+
+// Merge and store chunk c (elements 16c..16c+15) of the range [lo, hi).
+__device__ __forceinline__ void merge_chunk(const uint4 ev, const uint4 sv, uint64_t c, uint32_t lo, uint32_t hi,
+                                            uint16_t* __restrict__ out) {
+    uint4 o0, o1;
+    merge4(ev.x, sv.x, o0.x, o0.y);
+    merge4(ev.y, sv.y, o0.z, o0.w);
+    merge4(ev.z, sv.z, o1.x, o1.y);
+    merge4(ev.w, sv.w, o1.z, o1.w);
+    const uint64_t i0 = 16 * c;
+    uint16_t* dst = out + i0;
+    if (i0 >= lo && i0 + 16 <= hi) {
+        __stcs(reinterpret_cast<uint4*>(dst), o0);
+        __stcs(reinterpret_cast<uint4*>(dst) + 1, o1);
+    } else {
+        const uint32_t words[8] = {o0.x, o0.y, o0.z, o0.w, o1.x, o1.y, o1.z, o1.w};
+#pragma unroll
+        for (int k = 0; k < 16; k++) {
+            const uint64_t i = i0 + k;
+            if (i >= lo && i < hi) dst[k] = uint16_t(words[k >> 1] >> (16 * (k & 1)));
+        }
+    }
+}
+
+__device__ __forceinline__ void copy_tables(uint8_t* s_lut, const uint4* g_lut, int nthreads) {
+    for (int i = threadIdx.x; i < int(kLutBytes / 16); i += nthreads)
+        reinterpret_cast<uint4*>(s_lut)[i] = __ldg(g_lut + i);
+}
+
+__device__ __forceinline__ bool block_consistent(uint32_t off0, uint32_t off1, uint32_t total, uint64_t n) {
+    return off0 <= off1 && uint64_t(off1) <= n && total == off1 - off0;
+}
+
+// ---------------------------------------------------------------------------
+// T = 32: one warp decodes one thread block at a time; no CTA barrier after
+// the table copy.  Each warp takes a contiguous run of thread blocks, so the
+// 16-element chunk that straddles two consecutive blocks is stored once, as a
+// whole, by the later block: the earlier block leaves it in the staging
+// buffer, the warp carries its bytes over, and only the first and last chunk
+// of a run need element-wise stores.  Staging per warp: 32 windows x 64
+// symbols + head (15) + spill (3), rounded up.
+// ---------------------------------------------------------------------------
+constexpr uint32_t kWarpStage = 32 * 64 + 64;
+
+template <int WARPS>
+__global__ void __launch_bounds__(WARPS * 32) decode_warp_kernel(const DecodeArgs a) {
     extern __shared__ __align__(16) uint8_t smem[];
-    uint8_t* s_lut = smem;
-    uint8_t* s_stage = smem + kLutBytes;                                    // 64*T + 64 bytes
-    uint32_t* s_warp = reinterpret_cast<uint32_t*>(s_stage + 64 * T + 64);  // T/32 words
-
-    for (int i = threadIdx.x; i < int(kLutBytes / 16); i += T)
-        reinterpret_cast<uint4*>(s_lut)[i] = a.lut[i];
+    copy_tables(smem, a.lut, WARPS * 32);
     __syncthreads();
-    const uint16_t* ctab = reinterpret_cast<const uint16_t*>(s_lut + kLutOffCount);
-    const uint32_t* dtab = reinterpret_cast<const uint32_t*>(s_lut + kLutOffDecode);
-    const unsigned long long* lj_end = reinterpret_cast<const unsigned long long*>(s_lut + kLutOffLjEnd);
-    const uint32_t* delta = reinterpret_cast<const uint32_t*>(s_lut + kLutOffDelta);
-    const uint8_t* syms = s_lut + kLutOffSyms;
-    const int lane = threadIdx.x & 31;
-    const int warp = threadIdx.x >> 5;
+    const Tables t = tables_at(smem);
+    const uint32_t lane = threadIdx.x & 31u;
+    const uint32_t warp = threadIdx.x >> 5;
+    uint8_t* stage = smem + kLutBytes + warp * kWarpStage;
 
-    for (uint64_t b = blockIdx.x; b < a.n_blocks; b += gridDim.x) {
-        const uint64_t tg = b * T + threadIdx.x;
-        uint32_t w0 = 0, w1 = 0, w2 = 0;
-        int start = 0, wend = 0;
-        if (tg < a.n_threads) {
-            const uint2 v = __ldg(reinterpret_cast<const uint2*>(a.exp) + tg);
-            const uint32_t v2 = __ldg(reinterpret_cast<const uint32_t*>(a.exp) + 2 * tg + 2);
-            w0 = bswap32(v.x);
-            w1 = bswap32(v.y);
-            w2 = bswap32(v2);
-            const uint64_t gbit = 5 * tg;
-            const uint32_t glo = __ldg(a.gaps + (gbit >> 5));
-            const uint32_t ghi = __ldg(a.gaps + (gbit >> 5) + 1);
-            start = int(__funnelshift_r(glo, ghi, uint32_t(gbit)) & 31u);
-            const uint64_t rem = a.total_bits - 64 * tg;
-            wend = rem < 64 ? int(rem) : 64;
+    // this warp's run of thread blocks [b, b_end)
+    const uint64_t nw = uint64_t(gridDim.x) * WARPS;
+    const uint64_t g = uint64_t(blockIdx.x) * WARPS + warp;
+    const uint64_t per = a.n_blocks / nw, extra = a.n_blocks % nw;
+    uint64_t b = g * per + (g < extra ? g : extra);
+    const uint64_t b_end = b + per + (g < extra ? 1 : 0);
+
+    RawWindow nraw{};
+    uint32_t noff0 = 0, noff1 = 0;
+    if (b < b_end) {
+        nraw = load_window(a, 32 * b + lane);
+        noff0 = __ldg(a.off + b);
+        noff1 = __ldg(a.off + b + 1);
+    }
+    uint4 carry = make_uint4(0, 0, 0, 0);  // staging bytes of the chunk left by the previous block
+    bool have_carry = false;
+    while (b < b_end) {
+        const RawWindow raw = nraw;
+        const uint32_t off0 = noff0, off1 = noff1;
+        const bool more = b + 1 < b_end;
+        if (more) {  // prefetch the next block (its first position is off1)
+            nraw = load_window(a, 32 * (b + 1) + lane);
+            noff0 = off1;
+            noff1 = __ldg(a.off + b + 2);
         }
-        const uint32_t off_b = __ldg(a.off + b);
-        const uint32_t off_b1 = __ldg(a.off + b + 1);
+        const bool offs_ok = off0 <= off1 && uint64_t(off1) <= a.n_elems;
+        const uint32_t head = off0 & 15u;
+        // chunks to store: the head chunk (completed by the carried bytes
+        // unless this block starts the run), up to the tail chunk, which is
+        // left to the next block when that block exists and shares it
+        const uint32_t c0 = off0 >> 4;
+        const uint32_t c1 = offs_ok ? (off1 + 15) >> 4 : c0;
+        const bool keep_tail = more && (off1 & 15u) != 0;
+        const uint32_t cw = keep_tail && c1 > c0 ? c1 - 1 : c1;
+        const bool use_carry = have_carry && head != 0;
+        const uint32_t lo = use_carry ? (off0 & ~15u) : off0;
+        uint4 s0 = make_uint4(0, 0, 0, 0), s1 = s0;
+        if (c0 + lane < cw) s0 = __ldcs(a.sm + c0 + lane);
+        if (c0 + lane + 32 < cw) s1 = __ldcs(a.sm + c0 + lane + 32);
 
-        // ---- phase 1: count the codes that start in the window ----------
-        uint32_t cnt = 0;
+        const Window w = finish_window(a, raw, 32 * b + lane);
         bool bad = false;
-        for (int p = start; p < wend;) {
-            const uint32_t pk = peek32(w0, w1, w2, p);
-            const uint32_t e = ctab[pk >> (32 - kCountBits)];
-            if (e) {
-                uint32_t m = e & 0xFFFu;
-                const int lim = wend - p;
-                if (lim < kCountBits) m &= (1u << lim) - 1u;
-                cnt += __popc(m);
-                p += int(e >> 12);
-            } else {
-                const int l = code_length(lj_end, pk);
-                if (!l) {
-                    bad = true;
-                    break;
-                }
-                cnt += 1;
-                p += l;
-            }
-        }
-
-        // ---- block-wide exclusive scan of the counts --------------------
+        const uint32_t cnt = count_codes(w, t, bad);
         uint32_t incl = cnt;
 #pragma unroll
         for (int d = 1; d < 32; d <<= 1) {
             const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, d);
-            if (lane >= d) incl += y;
+            if (lane >= uint32_t(d)) incl += y;
+        }
+        const uint32_t total = __shfl_sync(0xFFFFFFFFu, incl, 31);
+        if (__any_sync(0xFFFFFFFFu, bad) || !block_consistent(off0, off1, total, a.n_elems)) {
+            if (lane == 0 && a.status) atomicOr(a.status, uint32_t(DF11_ERR_CORRUPT));
+            have_carry = false;
+        } else {
+            if (lane == 0 && use_carry) *reinterpret_cast<uint4*>(stage) = carry;
+            __syncwarp();
+            const uint32_t pos0 = head + (incl - cnt);
+            decode_codes(w, t, reinterpret_cast<uint32_t*>(stage), pos0, cnt);
+            __syncwarp();
+            write_head(w, t, stage, pos0, cnt);
+            __syncwarp();
+            uint32_t k = lane;
+            for (int j = 0; c0 + k < cw; k += 32, j++) {
+                const uint4 sv = j == 0 ? s0 : (j == 1 ? s1 : __ldcs(a.sm + c0 + k));
+                const uint4 ev = *reinterpret_cast<const uint4*>(stage + 16 * k);
+                merge_chunk(ev, sv, c0 + k, lo, off1, a.out);
+            }
+            if (keep_tail) carry = *reinterpret_cast<const uint4*>(stage + 16 * (c1 - 1 - c0));
+            have_carry = keep_tail;
+        }
+        __syncwarp();
+        b++;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// T >= 64: one CTA of T threads decodes one thread block per iteration, with
+// a block-wide scan.
+// ---------------------------------------------------------------------------
+template <int T>
+constexpr size_t block_stage_bytes() {
+    return 64 * T + 64;
+}
+
+template <int T>
+__global__ void __launch_bounds__(T) decode_block_kernel(const DecodeArgs a) {
+    extern __shared__ __align__(16) uint8_t smem[];
+    copy_tables(smem, a.lut, T);
+    uint8_t* stage = smem + kLutBytes;
+    uint32_t* s_warp = reinterpret_cast<uint32_t*>(stage + block_stage_bytes<T>());
+    __syncthreads();
+    const Tables t = tables_at(smem);
+    const uint32_t lane = threadIdx.x & 31u;
+    const uint32_t warp = threadIdx.x >> 5;
+
+    uint64_t b = blockIdx.x;
+    RawWindow nraw{};
+    uint32_t noff0 = 0, noff1 = 0;
+    if (b < a.n_blocks) {
+        nraw = load_window(a, uint64_t(T) * b + threadIdx.x);
+        noff0 = __ldg(a.off + b);
+        noff1 = __ldg(a.off + b + 1);
+    }
+    while (b < a.n_blocks) {
+        const RawWindow raw = nraw;
+        const uint32_t off0 = noff0, off1 = noff1;
+        const uint64_t bn = b + gridDim.x;
+        if (bn < a.n_blocks) {
+            nraw = load_window(a, uint64_t(T) * bn + threadIdx.x);
+            noff0 = __ldg(a.off + bn);
+            noff1 = __ldg(a.off + bn + 1);
+        }
+        const bool offs_ok = off0 <= off1 && uint64_t(off1) <= a.n_elems;
+        const uint32_t c0 = off0 >> 4;
+        const uint32_t c1 = offs_ok ? (off1 + 15) >> 4 : c0;
+        uint4 s0 = make_uint4(0, 0, 0, 0);
+        if (c0 + threadIdx.x < c1) s0 = __ldcs(a.sm + c0 + threadIdx.x);
+
+        const Window w = finish_window(a, raw, uint64_t(T) * b + threadIdx.x);
+        bool bad = false;
+        const uint32_t cnt = count_codes(w, t, bad);
+        uint32_t incl = cnt;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+            if (lane >= uint32_t(d)) incl += y;
         }
         if (lane == 31) s_warp[warp] = incl;
         const int any_bad = __syncthreads_or(bad);
         uint32_t before = 0, total = 0;
 #pragma unroll
-        for (int w = 0; w < T / 32; w++) {
-            const uint32_t v = s_warp[w];
+        for (int k = 0; k < T / 32; k++) {
+            const uint32_t v = s_warp[k];
             total += v;
-            before += (w < warp) ? v : 0u;
+            before += (uint32_t(k) < warp) ? v : 0u;
         }
-        const uint32_t excl = before + incl - cnt;
-        if (any_bad || off_b1 < off_b || total != off_b1 - off_b || uint64_t(off_b1) > a.n_elems) {
+        if (any_bad || !block_consistent(off0, off1, total, a.n_elems)) {
             if (threadIdx.x == 0 && a.status) atomicOr(a.status, uint32_t(DF11_ERR_CORRUPT));
+        } else {
+            const uint32_t pos0 = (off0 & 15u) + before + incl - cnt;
+            decode_codes(w, t, reinterpret_cast<uint32_t*>(stage), pos0, cnt);
             __syncthreads();
-            continue;
-        }
-
-        // ---- phase 2: decode again into the staging buffer ---------------
-        // staging byte 0 holds element off_b rounded down to 16
-        const uint32_t head = off_b & 15u;
-        uint8_t* st = s_stage + head + excl;
-        {
-            int p = start;
-            for (uint32_t w = 0; w < cnt;) {
-                const uint32_t pk = peek32(w0, w1, w2, p);
-                const uint32_t e = dtab[pk >> (32 - kDecodeBits)];
-                uint32_t n = (e >> 24) & 3u;
-                uint32_t s3 = e;
-                if (n) {
-                    p += int(e >> 26);
-                } else {
-                    int l = code_length(lj_end, pk);
-                    l = l ? l : 1;
-                    s3 = syms[((pk >> (32 - l)) + delta[l]) & 0xFFu];
-                    n = 1;
-                    p += l;
-                }
-                const uint32_t r = cnt - w;
-                n = n < r ? n : r;
-                st[w] = uint8_t(s3);
-                if (n > 1) st[w + 1] = uint8_t(s3 >> 8);
-                if (n > 2) st[w + 2] = uint8_t(s3 >> 16);
-                w += n;
+            write_head(w, t, stage, pos0, cnt);
+            __syncthreads();
+            uint32_t k = threadIdx.x;
+            for (int j = 0; c0 + k < c1; k += T, j++) {
+                const uint4 sv = j == 0 ? s0 : __ldcs(a.sm + c0 + k);
+                const uint4 ev = *reinterpret_cast<const uint4*>(stage + 16 * k);
+                merge_chunk(ev, sv, c0 + k, off0, off1, a.out);
             }
         }
         __syncthreads();
-
-        // ---- merge with sign+mantissa, 16 elements per thread ------------
-        const uint64_t c0 = off_b >> 4;
-        const uint64_t c1 = (uint64_t(off_b1) + 15) >> 4;
-        for (uint64_t c = c0 + threadIdx.x; c < c1; c += T) {
-            const uint4 ev = *reinterpret_cast<const uint4*>(s_stage + 16 * (c - c0));
-            const uint4 sv = __ldcs(a.sm + c);
-            uint4 o0, o1;
-            o0.x = merge_pair(ev.x, sv.x, 0x4140);
-            o0.y = merge_pair(ev.x, sv.x, 0x4342);
-            o0.z = merge_pair(ev.y, sv.y, 0x4140);
-            o0.w = merge_pair(ev.y, sv.y, 0x4342);
-            o1.x = merge_pair(ev.z, sv.z, 0x4140);
-            o1.y = merge_pair(ev.z, sv.z, 0x4342);
-            o1.z = merge_pair(ev.w, sv.w, 0x4140);
-            o1.w = merge_pair(ev.w, sv.w, 0x4342);
-            const uint64_t i0 = 16 * c;
-            uint16_t* dst = a.out + i0;
-            if (i0 >= off_b && i0 + 16 <= off_b1) {
-                __stcs(reinterpret_cast<uint4*>(dst), o0);
-                __stcs(reinterpret_cast<uint4*>(dst) + 1, o1);
-            } else {
-                const uint32_t words[8] = {o0.x, o0.y, o0.z, o0.w, o1.x, o1.y, o1.z, o1.w};
-#pragma unroll
-                for (int k = 0; k < 16; k++) {
-                    const uint64_t i = i0 + k;
-                    if (i >= off_b && i < off_b1) dst[k] = uint16_t(words[k >> 1] >> (16 * (k & 1)));
-                }
-            }
-        }
-        __syncthreads();
+        b = bn;
     }
-}
-
-template <int T>
-constexpr size_t decode_smem_bytes() {
-    return kLutBytes + 64 * T + 64 + 4 * (T / 32);
 }
 
 struct LaunchInfo {
     std::atomic<int> ready{0};
-    int grid_per_sm = 0;
+    int per_sm = 0;
     int sms = 0;
 };
-LaunchInfo g_info[16][5];  // [device][log2(T) - 6]
+constexpr int kMaxDev = 64;
+LaunchInfo g_info[kMaxDev][6];  // [device][log2(T) - 5]
 
-template <int T>
-df11_status launch_decode(const DecodeArgs& a, cudaStream_t stream) {
+constexpr int kWarpsPerCta = 16;
+
+template <typename Kernel>
+df11_status launch_persistent(Kernel kernel, int slot, int threads, size_t smem, uint64_t work_units,
+                              const DecodeArgs& a, cudaStream_t stream) {
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 16)
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev)
         return fail(DF11_ERR_CUDA, "cudaGetDevice failed");
-    constexpr int slot = (T == 64) ? 0 : (T == 128) ? 1 : (T == 256) ? 2 : (T == 512) ? 3 : 4;
     LaunchInfo& li = g_info[dev][slot];
-    const size_t smem = decode_smem_bytes<T>();
     if (!li.ready.load(std::memory_order_acquire)) {
-        cudaError_t e = cudaFuncSetAttribute(decode_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             int(smem));
+        cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
         if (e != cudaSuccess) return fail(DF11_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
         int per_sm = 0, sms = 0;
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_kernel<T>, T, smem);
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, smem);
         if (e != cudaSuccess) return fail(DF11_ERR_CUDA, "occupancy query: %s", cudaGetErrorString(e));
         e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
         if (e != cudaSuccess) return fail(DF11_ERR_CUDA, "SM count: %s", cudaGetErrorString(e));
-        li.grid_per_sm = per_sm > 0 ? per_sm : 1;
+        li.per_sm = per_sm > 0 ? per_sm : 1;
         li.sms = sms;
         li.ready.store(1, std::memory_order_release);
     }
-    const uint64_t want = uint64_t(li.grid_per_sm) * uint64_t(li.sms);
-    const unsigned grid = unsigned(a.n_blocks < want ? a.n_blocks : want);
-    decode_kernel<T><<<grid, T, smem, stream>>>(a);
+    const uint64_t want = uint64_t(li.per_sm) * uint64_t(li.sms);
+    const unsigned grid = unsigned(work_units < want ? work_units : want);
+    kernel<<<grid, threads, smem, stream>>>(a);
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return fail(DF11_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
     return DF11_OK;
+}
+
+template <int T>
+df11_status launch_block(const DecodeArgs& a, cudaStream_t s, int slot) {
+    const size_t smem = kLutBytes + block_stage_bytes<T>() + 4 * (T / 32);
+    return launch_persistent(decode_block_kernel<T>, slot, T, smem, a.n_blocks, a, s);
+}
+
+df11_status launch_warp(const DecodeArgs& a, cudaStream_t s) {
+    const size_t smem = kLutBytes + size_t(kWarpsPerCta) * kWarpStage;
+    const uint64_t ctas = (a.n_blocks + kWarpsPerCta - 1) / kWarpsPerCta;
+    return launch_persistent(decode_warp_kernel<kWarpsPerCta>, 0, kWarpsPerCta * 32, smem, ctas, a, s);
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -271,7 +528,7 @@ df11_status check_header(const df11_header* h) {
     if (h->version != DF11_VERSION) return fail(DF11_ERR_INVALID, "header version %u", h->version);
     if (h->window_bytes != DF11_WINDOW_BYTES) return fail(DF11_ERR_INVALID, "window_bytes %u", h->window_bytes);
     const uint32_t T = h->threads_per_block;
-    if (T < 64 || T > 1024 || (T & (T - 1))) return fail(DF11_ERR_INVALID, "threads_per_block %u", T);
+    if (T < 32 || T > 1024 || (T & (T - 1))) return fail(DF11_ERR_INVALID, "threads_per_block %u", T);
     if (h->n_elems >= (uint64_t(1) << 32)) return fail(DF11_ERR_TOO_LARGE, "n_elems >= 2^32");
     df11_header ref = *h;
     fill_sizes(&ref);
@@ -314,11 +571,12 @@ extern "C" df11_status df11_decompress(const df11_header* hdr, const uint8_t* d_
     a.n_blocks = hdr->n_blocks;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     switch (hdr->threads_per_block) {
-        case 64: return launch_decode<64>(a, s);
-        case 128: return launch_decode<128>(a, s);
-        case 256: return launch_decode<256>(a, s);
-        case 512: return launch_decode<512>(a, s);
-        case 1024: return launch_decode<1024>(a, s);
+        case 32: return launch_warp(a, s);
+        case 64: return launch_block<64>(a, s, 1);
+        case 128: return launch_block<128>(a, s, 2);
+        case 256: return launch_block<256>(a, s, 3);
+        case 512: return launch_block<512>(a, s, 4);
+        case 1024: return launch_block<1024>(a, s, 5);
         default: return fail(DF11_ERR_INVALID, "threads_per_block %u", hdr->threads_per_block);
     }
 }

@@ -155,8 +155,8 @@ df11_status df11_header_init(df11_header* hdr, const uint8_t* code_len, uint64_t
                              uint32_t n_segs) {
     if (!hdr || !code_len) return fail(DF11_ERR_INVALID, "df11_header_init: null pointer");
     const uint32_t T = threads_per_block;
-    if (T < 64 || T > 1024 || (T & (T - 1)))
-        return fail(DF11_ERR_INVALID, "threads_per_block %u is not a power of two in 64..1024", T);
+    if (T < 32 || T > 1024 || (T & (T - 1)))
+        return fail(DF11_ERR_INVALID, "threads_per_block %u is not a power of two in 32..1024", T);
     if (max_code_len < 1 || max_code_len > 32)
         return fail(DF11_ERR_INVALID, "max_code_len %u outside 1..32", max_code_len);
     if (n_elems >= (uint64_t(1) << 32))
@@ -214,8 +214,8 @@ df11_status df11_build_lut(const df11_header* hdr, void* h_lut, uint64_t cap) {
     std::memset(blob, 0, kLutBytes);
     LutHeader lh{};
     lh.magic = kLutMagic;
-    lh.count_bits = kCountBits;
-    lh.decode_bits = kDecodeBits;
+    lh.peek_bits = kPeekBits;
+    lh.escape = kEscape;
 
     // per-length counts and first codes
     uint64_t count[34] = {0}, first[34] = {0};
@@ -255,34 +255,31 @@ df11_status df11_build_lut(const df11_header* hdr, void* h_lut, uint64_t cap) {
         return 0;
     };
 
-    uint16_t* ctab = reinterpret_cast<uint16_t*>(blob + kLutOffCount);
-    for (uint32_t v = 0; v < (1u << kCountBits); v++) {
-        uint32_t mask = 0;
+    // level 1: walk the complete codes at the front of every 12-bit peek
+    uint32_t* ctab = reinterpret_cast<uint32_t*>(blob + kLutOffCount);
+    uint16_t* mtab = reinterpret_cast<uint16_t*>(blob + kLutOffMask);
+    uint32_t* dtab = reinterpret_cast<uint32_t*>(blob + kLutOffDecode);  // pairs (x, y)
+    for (uint32_t v = 0; v < kLutEntries; v++) {
+        uint32_t mask = 0, count = 0, syms4 = 0, n4 = 0, used4 = 0;
         int pos = 0;
-        while (pos < kCountBits) {
-            uint64_t peek = (uint64_t(v) << (32 - kCountBits + pos)) & 0xFFFFFFFFull;
-            int l = code_length(peek);
-            if (l == 0 || pos + l > kCountBits) break;
+        while (pos < kPeekBits) {
+            const uint64_t peek = (uint64_t(v) << (32 - kPeekBits + pos)) & 0xFFFFFFFFull;
+            const int l = code_length(peek);
+            if (l == 0 || pos + l > kPeekBits) break;
             mask |= 1u << pos;
+            count++;
+            if (n4 < kDecodeSyms) {
+                const uint32_t value = uint32_t(peek >> (32 - l));
+                syms4 |= uint32_t(syms[(value + delta[l]) & 0xFFu]) << (8 * n4);
+                n4++;
+                used4 = uint32_t(pos + l);
+            }
             pos += l;
         }
-        ctab[v] = uint16_t(mask | (uint32_t(pos) << 12));
-    }
-    uint32_t* dtab = reinterpret_cast<uint32_t*>(blob + kLutOffDecode);
-    for (uint32_t v = 0; v < (1u << kDecodeBits); v++) {
-        uint32_t entry = 0, nsym = 0;
-        int pos = 0;
-        while (nsym < 3 && pos < kDecodeBits) {
-            uint64_t peek = (uint64_t(v) << (32 - kDecodeBits + pos)) & 0xFFFFFFFFull;
-            int l = code_length(peek);
-            if (l == 0 || pos + l > kDecodeBits) break;
-            uint32_t value = uint32_t(peek >> (32 - l));
-            uint32_t s = syms[(value + delta[l]) & 0xFFu];
-            entry |= s << (8 * nsym);
-            nsym++;
-            pos += l;
-        }
-        dtab[v] = nsym ? (entry | (nsym << 24) | (uint32_t(pos) << 26)) : 0u;
+        ctab[v] = count ? ((uint32_t(pos) << 16) | count) : (kEscape << 16);
+        mtab[v] = uint16_t(mask);
+        dtab[2 * v] = n4 ? syms4 : 0u;
+        dtab[2 * v + 1] = n4 ? ((used4 << 16) | n4) : (kEscape << 16);
     }
     std::memcpy(blob, &lh, sizeof(lh));
     return DF11_OK;

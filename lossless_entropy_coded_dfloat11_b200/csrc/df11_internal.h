@@ -11,35 +11,42 @@ namespace df11 {
 // ---------------------------------------------------------------------------
 // Decode tables ("Decodificacao com LUT hierarquica" in the DFloat11 summary:
 // lookup tables small enough for on-chip memory instead of a bit-level tree
-// walk).  Two levels:
+// walk).  Two levels.
 //
-//   level 1, indexed by the next K stream bits
-//     count table  (K = kCountBits):  uint16 = start mask | consumed << 12.
-//         Bit j of the 12-bit mask is set when a complete code starts at
-//         offset j of the peek; `consumed` is the number of bits the complete
-//         codes use.  0 = the first code is longer than K bits.
-//     decode table (K = kDecodeBits): uint32 = up to three symbols (bits
-//         0..23, first symbol lowest) | n << 24 | consumed << 26.
-//         n = number of complete codes decoded (<= 3); 0 = first code longer
-//         than K bits.
-//   level 2, for codes longer than K: canonical codes of one length are
-//     consecutive integers, so a code's length is the smallest l with
-//     peek32 < lj_end[l] (lj_end[l] = end of the length-l codes, shifted to
-//     the top of 32 bits), and its symbol is syms[(peek32 >> (32 - l)) +
-//     delta[l]] with syms sorted by (length, value).
+// Level 1 is indexed by the next K = 12 stream bits:
+//   count table  uint32 = consumed << 16 | count
+//       count    = complete codes at the front of the peek (0..12)
+//       consumed = bits those codes use (1..12)
+//       The kernel keeps (bit position << 16 | code count) in one register,
+//       so one add advances both.
+//   mask table   uint16, bit j set when a complete code starts at offset j
+//       (used once per window, to drop codes that start past its end).
+//   decode table uint2: x = up to four symbols (first in bits 0..7, unused
+//       bytes zero); y = consumed << 16 | n, n = codes decoded (1..4).  The
+//       kernel keeps (bit position << 16 | output offset) in one register.
+//   A peek whose first code is longer than K bits (or matches no code) holds
+//   the escape value kEscape << 16 (count 0, n 0, symbols 0): adding it
+//   pushes the bit position past every window end, so the fast loops need
+//   no escape test; the slow path undoes it.
+// Level 2, for codes longer than K: canonical codes of one length are
+//   consecutive integers, so a code's length is the smallest l with
+//   peek32 < lj_end[l] (lj_end[l] = end of the length-l codes, shifted to the
+//   top of 32 bits), and its symbol is syms[(peek32 >> (32 - l)) + delta[l]]
+//   with syms sorted by (length, value).
 //
 // The pages cut the tree into 8-bit-high subtrees with 256-entry tables and
 // re-use exponent values 240..255 as pointers; here every exponent value
 // must stay representable, so level 2 is the comparison ladder instead.
 // ---------------------------------------------------------------------------
 constexpr uint32_t kLutMagic = 0x31314644u;  // "DF11"
-constexpr int kCountBits = 12;
-constexpr int kDecodeBits = 12;
+constexpr int kPeekBits = 12;
+constexpr uint32_t kEscape = 128;            // > any bit position inside a window + K
+constexpr uint32_t kDecodeSyms = 4;          // symbols per decode-table entry
 
 struct LutHeader {
     uint32_t magic;
-    uint32_t count_bits;
-    uint32_t decode_bits;
+    uint32_t peek_bits;
+    uint32_t escape;
     uint32_t n_syms;
     uint32_t min_len;
     uint32_t max_len;
@@ -48,12 +55,14 @@ struct LutHeader {
 static_assert(sizeof(LutHeader) == 64, "LutHeader is 64 bytes");
 
 constexpr uint64_t align16(uint64_t v) { return (v + 15) & ~uint64_t(15); }
+constexpr uint64_t kLutEntries = uint64_t(1) << kPeekBits;
 constexpr uint64_t kLutOffLjEnd = 64;                                       // uint64[33]
 constexpr uint64_t kLutOffDelta = align16(kLutOffLjEnd + 33 * 8);           // uint32[33]
 constexpr uint64_t kLutOffSyms = align16(kLutOffDelta + 33 * 4);            // uint8[256]
-constexpr uint64_t kLutOffCount = align16(kLutOffSyms + 256);               // uint16[2^K]
-constexpr uint64_t kLutOffDecode = align16(kLutOffCount + (2ull << kCountBits));  // uint32[2^K]
-constexpr uint64_t kLutBytes = align16(kLutOffDecode + (4ull << kDecodeBits));
+constexpr uint64_t kLutOffCount = align16(kLutOffSyms + 256);               // uint32[2^K]
+constexpr uint64_t kLutOffMask = align16(kLutOffCount + 4 * kLutEntries);   // uint16[2^K]
+constexpr uint64_t kLutOffDecode = align16(kLutOffMask + 2 * kLutEntries);  // uint2[2^K]
+constexpr uint64_t kLutBytes = align16(kLutOffDecode + 8 * kLutEntries);
 
 // Canonical code per value (DEFLATE-style construction); false if the
 // lengths overflow the code space.

@@ -6,7 +6,8 @@ Both directions on the same seeded inputs:
     lengths, codes, bit packing, Gaps and block offsets) and the oracle
     decodes them back to the input.
 Sizes span many thread blocks and ragged tails; the full-size workloads run in
-the launch configuration the benchmark times (T = 256, one launch per stream).
+the launch configuration the benchmark times (the default T, one launch per
+stream).
 """
 import numpy as np
 import pytest
@@ -51,7 +52,7 @@ def assert_same_stream(cs: df11.CompressedStream, s: oracle.Stream):
     np.testing.assert_array_equal(h["block_off"], s.block_off)
 
 
-def both_directions(w: inputs.Workload, T=256, L=32, windowed=True):
+def both_directions(w: inputs.Workload, T=df11.DEFAULT_THREADS_PER_BLOCK, L=32):
     x = w.flat_u16()
     s = oracle.encode(x, threads_per_block=T, max_len=L)
     # oracle stream -> library kernel
@@ -76,7 +77,7 @@ def test_matrix_1k():
     both_directions(inputs.matrix_1k())
 
 
-@pytest.mark.parametrize("T", [64, 128, 512, 1024])
+@pytest.mark.parametrize("T", [32, 64, 128, 256, 512, 1024])
 def test_threads_per_block_variants(T):
     both_directions(inputs.matrix_1k(), T=T)
     both_directions(inputs.edge_case(65537, "zipf", 515), T=T)
@@ -127,7 +128,7 @@ def test_llama8b_block_single_launch():
     """One Llama-3.1-8B-shaped block, one shared table, one launch."""
     w = inputs.llama_block()
     assert w.n_elems == 218_112_000
-    cs, s = both_directions(w, windowed=False)
+    cs, s = both_directions(w)
     out = df11.decompress(cs)
     torch.cuda.synchronize()
     for name, v, t in zip(w.names, cs.views(out), w.tensors):
@@ -153,7 +154,7 @@ def test_llama70b_block_reused_buffer():
     assert np.array_equal(u16(out), x)
     lib = df11.to_host(cs)
     ls = oracle.Stream(code_len=lib["code_len"], n_elems=lib["n_elems"], total_bits=lib["total_bits"],
-                       threads_per_block=256, n_threads=lib["n_threads"], n_blocks=lib["n_blocks"],
+                       threads_per_block=cs.threads_per_block, n_threads=lib["n_threads"], n_blocks=lib["n_blocks"],
                        exp=lib["exp"], sm=lib["sm"], gaps=lib["gaps"], block_off=lib["block_off"])
     rng = np.random.default_rng(70)
     for b in list(rng.integers(0, ls.n_blocks, size=48)) + [0, ls.n_blocks - 1]:
@@ -186,12 +187,13 @@ def test_empty_and_single_element():
 
 def test_corrupt_block_offsets_are_reported_not_trapped():
     x = inputs.matrix_1k().flat_u16()
-    s = oracle.encode(x)
+    T = df11.DEFAULT_THREADS_PER_BLOCK
+    s = oracle.encode(x, threads_per_block=T)
     guard = 4096
     for b, delta in ((5, 1), (100, -3), (s.n_blocks, 1000)):
         off = s.block_off.copy()
         off[b] = np.uint32(int(off[b]) + delta)
-        cs = df11.from_arrays(s.code_len, s.n_elems, s.total_bits, 256, s.exp, s.sm, s.gaps, off)
+        cs = df11.from_arrays(s.code_len, s.n_elems, s.total_bits, T, s.exp, s.sm, s.gaps, off)
         buf = torch.full((s.n_elems + guard,), 7.0, dtype=torch.bfloat16, device="cuda")
         status = torch.zeros(1, dtype=torch.int32, device="cuda")
         df11.decompress(cs, out=buf[: s.n_elems], status=status)
@@ -202,10 +204,11 @@ def test_corrupt_block_offsets_are_reported_not_trapped():
 
 def test_corrupt_gaps_and_bits_terminate():
     x = inputs.matrix_outliers(512, 512, seed=5).flat_u16()
-    s = oracle.encode(x)
+    T = df11.DEFAULT_THREADS_PER_BLOCK
+    s = oracle.encode(x, threads_per_block=T)
     gaps = s.gaps.copy()
     gaps[40] ^= 0x1F
-    cs = df11.from_arrays(s.code_len, s.n_elems, s.total_bits, 256, s.exp, s.sm, gaps, s.block_off)
+    cs = df11.from_arrays(s.code_len, s.n_elems, s.total_bits, T, s.exp, s.sm, gaps, s.block_off)
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     df11.decompress(cs, status=status)
     torch.cuda.synchronize()
@@ -215,7 +218,7 @@ def test_corrupt_gaps_and_bits_terminate():
         exp = s.exp.copy()
         idx = rng.integers(0, (s.total_bits + 7) // 8, size=16)
         exp[idx] ^= rng.integers(1, 256, size=16).astype(np.uint8)
-        cs = df11.from_arrays(s.code_len, s.n_elems, s.total_bits, 256, exp, s.sm, s.gaps, s.block_off)
+        cs = df11.from_arrays(s.code_len, s.n_elems, s.total_bits, T, exp, s.sm, s.gaps, s.block_off)
         status.zero_()
         out = df11.decompress(cs, status=status)
         torch.cuda.synchronize()
@@ -224,7 +227,7 @@ def test_corrupt_gaps_and_bits_terminate():
 
 
 def test_host_side_argument_checks():
-    s = oracle.encode(inputs.matrix_1k().flat_u16())
+    s = oracle.encode(inputs.matrix_1k().flat_u16(), threads_per_block=df11.DEFAULT_THREADS_PER_BLOCK)
     cs = lib_stream_from_oracle(s)
     out = torch.empty(s.n_elems + 8, dtype=torch.bfloat16, device="cuda")
     with pytest.raises(df11.DF11Error) as e:

@@ -128,10 +128,14 @@ def test_header_validation():
         df11.make_header(one, 3, 6, 64)
 
 
-LUT_COUNT_BITS = 12
-LUT_DECODE_BITS = 12
-OFF_COUNT = 736          # after the 64-byte header, lj_end[33], delta[33], syms[256]
-OFF_DECODE = OFF_COUNT + 2 * 4096
+PEEK_BITS = 12
+ESCAPE = 128
+# table offsets: 64-byte header, lj_end u64[33], delta u32[33], syms u8[256],
+# then count u32[4096], mask u16[4096], decode (u32, u32)[4096]
+OFF_COUNT = 736
+OFF_MASK = OFF_COUNT + 4 * 4096
+OFF_DECODE = OFF_MASK + 2 * 4096
+LUT_BYTES = OFF_DECODE + 8 * 4096
 
 
 def _oracle_prefix_decoder(code_len):
@@ -170,22 +174,25 @@ def test_decode_tables_agree_with_oracle_codes(source):
     s = oracle.encode(x)
     hdr = df11.make_header(s.code_len, s.n_elems, s.total_bits, 256)
     lut = df11.build_lut(hdr)
+    assert lut.size == LUT_BYTES == int(hdr.bytes_lut)
     assert lut[:4].tobytes() == b"DF11"
-    ctab = lut[OFF_COUNT:OFF_COUNT + 2 * 4096].view(np.uint16)
-    dtab = lut[OFF_DECODE:OFF_DECODE + 4 * 4096].view(np.uint32)
+    ctab = lut[OFF_COUNT:OFF_MASK].view(np.uint32)
+    mtab = lut[OFF_MASK:OFF_DECODE].view(np.uint16)
+    dtab = lut[OFF_DECODE:LUT_BYTES].view(np.uint32).reshape(-1, 2)
     table = _oracle_prefix_decoder(s.code_len)
     rng = np.random.default_rng(3)
     for v in list(range(64)) + list(rng.integers(0, 4096, size=400)) + list(range(4032, 4096)):
         bits = format(int(v), "012b")
         codes, used = _decode_bits(table, bits, None)
         mask = sum(1 << p for _, p in codes)
-        assert int(ctab[v]) == (mask | (used << 12) if codes else 0), (v, bits)
-        codes3, used3 = _decode_bits(table, bits, 3)
-        e = int(dtab[v])
-        if not codes3:
-            assert e == 0
+        assert int(mtab[v]) == mask, (v, bits)
+        assert int(ctab[v]) == ((used << 16) | len(codes) if codes else ESCAPE << 16), (v, bits)
+        codes4, used4 = _decode_bits(table, bits, 4)
+        x, y = int(dtab[v, 0]), int(dtab[v, 1])
+        if not codes4:
+            assert (x, y) == (0, ESCAPE << 16)
             continue
-        assert (e >> 24) & 3 == len(codes3)
-        assert e >> 26 == used3
-        for k, (sym, _) in enumerate(codes3):
-            assert (e >> (8 * k)) & 0xFF == sym
+        assert y == (used4 << 16) | len(codes4)
+        assert len(codes4) == 4 or x >> (8 * len(codes4)) == 0   # unused symbol bytes are zero
+        for k, (sym, _) in enumerate(codes4):
+            assert (x >> (8 * k)) & 0xFF == sym
