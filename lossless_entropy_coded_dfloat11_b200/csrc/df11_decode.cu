@@ -24,12 +24,14 @@
 //     and second 32 bits of the window so each peek is one funnel shift; codes
 //     longer than the 12-bit tables leave through an escape value that pushes
 //     the bit position out of the window, so the fast loops have one test;
-//   * phase 2 gathers symbols in registers and stores aligned 32-bit words;
-//     a thread's first word, shared with the previous thread, is filled
-//     byte-wise after a warp barrier;
+//   * phase 2 gathers symbols in a register pair and stores aligned 32-bit
+//     words; a thread's first word, shared with the previous thread, is kept
+//     in a register and written byte-wise after a barrier;
 //   * the merge handles 16 elements per thread with one 16-byte shared load,
 //     one 16-byte streaming load, 24 logic/permute operations and two 16-byte
 //     streaming stores.
+// Indices are 32-bit: n_elems < 2^32 and codes of at most 32 bits keep the
+// window count below 2^31.
 #include <cuda_runtime.h>
 
 #include <atomic>
@@ -48,10 +50,10 @@ struct DecodeArgs {
     const uint4* lut;
     uint16_t* out;
     uint32_t* status;
-    uint64_t n_elems;
-    uint64_t total_bits;
-    uint64_t n_threads;
-    uint64_t n_blocks;
+    uint32_t n_elems;
+    uint32_t n_threads;
+    uint32_t n_blocks;
+    uint32_t last_wend;  // bits of the last window inside the stream, 1..64
 };
 
 struct Tables {
@@ -86,7 +88,7 @@ __device__ __forceinline__ uint32_t peek32(uint32_t w0, uint32_t w1, uint32_t w2
 
 // Level 2: length of the canonical code at the top of `peek`, 0 if none.
 // Codes shorter than `from` bits are known not to match.
-__device__ __forceinline__ int code_length(const unsigned long long* lj_end, uint32_t peek, int from = 1) {
+__device__ __forceinline__ int code_length(const unsigned long long* lj_end, uint32_t peek, int from) {
     for (int l = from; l <= 32; l++)
         if ((unsigned long long)peek < lj_end[l]) return l;
     return 0;
@@ -109,14 +111,14 @@ struct Window {
     uint32_t wend;        // end of the window inside the stream, 0..64
 };
 
-__device__ __forceinline__ RawWindow load_window(const DecodeArgs& a, uint64_t tg) {
+// tg = window index; its gap field sits in gap words gword, gword + 1.
+__device__ __forceinline__ RawWindow load_window(const DecodeArgs& a, uint32_t tg, uint32_t gword) {
     RawWindow r;
     if (tg < a.n_threads) {
         r.v = __ldg(reinterpret_cast<const uint2*>(a.exp) + tg);
         r.v2 = __ldg(reinterpret_cast<const uint32_t*>(a.exp) + 2 * tg + 2);
-        const uint64_t gw = (5 * tg) >> 5;
-        r.glo = __ldg(a.gaps + gw);
-        r.ghi = __ldg(a.gaps + gw + 1);
+        r.glo = __ldg(a.gaps + gword);
+        r.ghi = __ldg(a.gaps + gword + 1);
     } else {
         r.v = make_uint2(0, 0);
         r.v2 = r.glo = r.ghi = 0;
@@ -124,18 +126,15 @@ __device__ __forceinline__ RawWindow load_window(const DecodeArgs& a, uint64_t t
     return r;
 }
 
-__device__ __forceinline__ Window finish_window(const DecodeArgs& a, const RawWindow& r, uint64_t tg) {
+__device__ __forceinline__ Window finish_window(const DecodeArgs& a, const RawWindow& r, uint32_t tg,
+                                                uint32_t gshift) {
     Window w;
     w.w0 = bswap32(r.v.x);
     w.w1 = bswap32(r.v.y);
     w.w2 = bswap32(r.v2);
-    w.start = __funnelshift_r(r.glo, r.ghi, uint32_t(5 * tg)) & 31u;
-    if (tg < a.n_threads) {
-        const uint64_t rem = a.total_bits - 64 * tg;
-        w.wend = rem < 64 ? uint32_t(rem) : 64u;
-    } else {
-        w.wend = 0;
-    }
+    w.start = __funnelshift_r(r.glo, r.ghi, gshift) & 31u;
+    const uint32_t last = a.n_threads - 1;
+    w.wend = tg < last ? 64u : (tg == last ? a.last_wend : 0u);
     return w;
 }
 
@@ -177,32 +176,33 @@ __device__ __forceinline__ uint32_t count_codes(const Window& w, const Tables& t
 }
 
 // Phase 2: decode the same codes into staging bytes [pos0, pos0 + cnt).
-// Symbols collect in a 64-bit register pair and leave as aligned 32-bit
-// words.  The thread's first word is skipped when it starts mid-word (it is
-// shared with the previous thread; write_head fills those bytes after a
-// barrier).  A word holding the thread's last symbols may also carry up to
-// three bytes decoded past the window end; those positions are head bytes of
-// the following threads (which start mid-word), rewritten by write_head.
-__device__ __forceinline__ void decode_codes(const Window& w, const Tables& t, uint32_t* stage32, uint32_t pos0,
-                                             uint32_t cnt) {
-    if (cnt == 0) return;
+// Symbols collect in a register pair and leave as aligned 32-bit words.  The
+// thread's first word is not stored when it starts mid-word (it is shared
+// with the previous thread): it is returned, for write_head after a barrier.
+// A stored word holding the thread's last symbols may carry up to three
+// bytes decoded past the window end; those positions are head bytes of the
+// following threads (which start mid-word) and are rewritten by them.
+__device__ __forceinline__ uint32_t decode_codes(const Window& w, const Tables& t, uint32_t* stage32,
+                                                 uint32_t pos0, uint32_t cnt) {
+    if (cnt == 0) return 0;
     const uint32_t lim1 = min(w.wend, 32u) << 16;
     const uint32_t lim2 = w.wend << 16;
     const uint32_t last_word = (pos0 + cnt - 1) >> 2;
     const uint32_t skip_word = (pos0 & 3u) ? (pos0 >> 2) : 0xFFFFFFFFu;
     uint32_t wi = pos0 >> 2;  // word the pending bytes belong to
-    uint32_t lo = 0, hi = 0;  // pending bytes, byte k = staging position 4*wi + k
-    uint32_t acc = (w.start << 16) | (pos0 & 3u);  // bit position << 16 | bytes pending
+    uint32_t lo = 0, head = 0;
+    // bit position << 16 | 8 x bytes pending: the low five bits are the shift
+    // that places the next symbols in `lo`
+    uint32_t acc = (w.start << 16) | ((pos0 & 3u) << 3);
     auto put = [&](uint32_t x, uint32_t y) {
-        const uint32_t sh = (acc << 3) & 24u;
-        lo |= x << sh;
-        hi = __funnelshift_l(x, 0u, sh);
+        lo |= __funnelshift_l(0u, x, acc);                // x << (acc & 31)
+        const uint32_t hi = __funnelshift_l(x, 0u, acc);  // bytes spilling past lo
         acc += y;
-        if (acc & 4u) {  // a word is complete
-            if (wi != skip_word) stage32[wi] = lo;
+        if (acc & 32u) {  // a word is complete
+            if (wi != skip_word) stage32[wi] = lo; else head = lo;
             wi++;
             lo = hi;
-            acc -= 4u;
+            acc -= 32u;
         }
     };
     for (;;) {
@@ -219,34 +219,25 @@ __device__ __forceinline__ void decode_codes(const Window& w, const Tables& t, u
         const uint32_t pk = peek32(w.w0, w.w1, w.w2, acc >> 16);
         int l = code_length(t.lj_end, pk, kPeekBits + 1);
         l = l ? l : 1;
-        put(code_symbol(t, pk, l), (uint32_t(l) << 16) | 1u);
+        put(code_symbol(t, pk, l), (uint32_t(l) << 16) | 8u);
     }
-    if ((acc & 3u) && wi <= last_word && wi != skip_word) stage32[wi] = lo;
+    if (acc & 31u) {
+        if (wi == skip_word) head = lo;
+        else if (wi <= last_word) stage32[wi] = lo;
+    }
+    return head;
 }
 
-// After a barrier: bytes of this thread's first word when it starts mid-word
-// (positions pos0 .. the next word boundary, at most three symbols).
-__device__ __forceinline__ void write_head(const Window& w, const Tables& t, uint8_t* stage, uint32_t pos0,
-                                           uint32_t cnt) {
-    const uint32_t room = (4u - (pos0 & 3u)) & 3u;
+// After a barrier: the bytes of this thread's first word when it starts
+// mid-word, from the word phase 2 kept back.
+__device__ __forceinline__ void write_head(uint8_t* stage, uint32_t pos0, uint32_t cnt, uint32_t head) {
+    const uint32_t b0 = pos0 & 3u;
+    const uint32_t room = (4u - b0) & 3u;
     const uint32_t k = cnt < room ? cnt : room;
-    if (k == 0) return;
-    uint8_t* base = stage + pos0;
-    const uint2 e = t.dtab[peek32(w.w0, w.w1, w.w2, w.start) >> (32 - kPeekBits)];
-    if ((e.y & 0xFFFFu) >= k) {
-        base[0] = uint8_t(e.x);
-        if (k > 1) base[1] = uint8_t(e.x >> 8);
-        if (k > 2) base[2] = uint8_t(e.x >> 16);
-    } else {  // one of the first codes is longer than the table
-        uint32_t p = w.start;
-        for (uint32_t j = 0; j < k; j++) {
-            const uint32_t q = peek32(w.w0, w.w1, w.w2, p);
-            int l = code_length(t.lj_end, q);
-            l = l ? l : 1;
-            base[j] = uint8_t(code_symbol(t, q, l));
-            p += uint32_t(l);
-        }
-    }
+    uint8_t* d = stage + pos0;
+    if (k > 0) d[0] = uint8_t(head >> (8 * b0));
+    if (k > 1) d[1] = uint8_t(head >> (8 * b0 + 8));
+    if (k > 2) d[2] = uint8_t(head >> 24);
 }
 
 // Four BF16 values from four exponent bytes e4 and four sign+mantissa bytes
@@ -260,24 +251,25 @@ __device__ __forceinline__ void merge4(uint32_t e4, uint32_t s4, uint32_t& o01, 
 }
 
 // Merge and store chunk c (elements 16c..16c+15) of the range [lo, hi).
-__device__ __forceinline__ void merge_chunk(const uint4 ev, const uint4 sv, uint64_t c, uint32_t lo, uint32_t hi,
+__device__ __forceinline__ void merge_chunk(const uint4 ev, const uint4 sv, uint32_t c, uint32_t lo, uint32_t hi,
                                             uint16_t* __restrict__ out) {
     uint4 o0, o1;
     merge4(ev.x, sv.x, o0.x, o0.y);
     merge4(ev.y, sv.y, o0.z, o0.w);
     merge4(ev.z, sv.z, o1.x, o1.y);
     merge4(ev.w, sv.w, o1.z, o1.w);
-    const uint64_t i0 = 16 * c;
-    uint16_t* dst = out + i0;
+    uint4* dst = reinterpret_cast<uint4*>(out) + 2 * size_t(c);
+    const uint32_t i0 = 16 * c;
     if (i0 >= lo && i0 + 16 <= hi) {
-        __stcs(reinterpret_cast<uint4*>(dst), o0);
-        __stcs(reinterpret_cast<uint4*>(dst) + 1, o1);
+        __stcs(dst, o0);
+        __stcs(dst + 1, o1);
     } else {
         const uint32_t words[8] = {o0.x, o0.y, o0.z, o0.w, o1.x, o1.y, o1.z, o1.w};
+        uint16_t* d16 = reinterpret_cast<uint16_t*>(dst);
 #pragma unroll
         for (int k = 0; k < 16; k++) {
-            const uint64_t i = i0 + k;
-            if (i >= lo && i < hi) dst[k] = uint16_t(words[k >> 1] >> (16 * (k & 1)));
+            const uint32_t i = i0 + k;
+            if (i >= lo && i < hi) d16[k] = uint16_t(words[k >> 1] >> (16 * (k & 1)));
         }
     }
 }
@@ -287,8 +279,8 @@ __device__ __forceinline__ void copy_tables(uint8_t* s_lut, const uint4* g_lut, 
         reinterpret_cast<uint4*>(s_lut)[i] = __ldg(g_lut + i);
 }
 
-__device__ __forceinline__ bool block_consistent(uint32_t off0, uint32_t off1, uint32_t total, uint64_t n) {
-    return off0 <= off1 && uint64_t(off1) <= n && total == off1 - off0;
+__device__ __forceinline__ bool block_consistent(uint32_t off0, uint32_t off1, uint32_t total, uint32_t n) {
+    return off0 <= off1 && off1 <= n && total == off1 - off0;
 }
 
 // ---------------------------------------------------------------------------
@@ -311,18 +303,21 @@ __global__ void __launch_bounds__(WARPS * 32) decode_warp_kernel(const DecodeArg
     const uint32_t lane = threadIdx.x & 31u;
     const uint32_t warp = threadIdx.x >> 5;
     uint8_t* stage = smem + kLutBytes + warp * kWarpStage;
+    // the gap field of window 32b + lane lies in the block's five gap words
+    const uint32_t lane_gword = (5 * lane) >> 5;
+    const uint32_t lane_gshift = (5 * lane) & 31u;
 
     // this warp's run of thread blocks [b, b_end)
-    const uint64_t nw = uint64_t(gridDim.x) * WARPS;
-    const uint64_t g = uint64_t(blockIdx.x) * WARPS + warp;
-    const uint64_t per = a.n_blocks / nw, extra = a.n_blocks % nw;
-    uint64_t b = g * per + (g < extra ? g : extra);
-    const uint64_t b_end = b + per + (g < extra ? 1 : 0);
+    const uint32_t nw = gridDim.x * WARPS;
+    const uint32_t g = blockIdx.x * WARPS + warp;
+    const uint32_t per = a.n_blocks / nw, extra = a.n_blocks % nw;
+    uint32_t b = g * per + (g < extra ? g : extra);
+    const uint32_t b_end = b + per + (g < extra ? 1u : 0u);
 
     RawWindow nraw{};
     uint32_t noff0 = 0, noff1 = 0;
     if (b < b_end) {
-        nraw = load_window(a, 32 * b + lane);
+        nraw = load_window(a, 32 * b + lane, 5 * b + lane_gword);
         noff0 = __ldg(a.off + b);
         noff1 = __ldg(a.off + b + 1);
     }
@@ -333,11 +328,11 @@ __global__ void __launch_bounds__(WARPS * 32) decode_warp_kernel(const DecodeArg
         const uint32_t off0 = noff0, off1 = noff1;
         const bool more = b + 1 < b_end;
         if (more) {  // prefetch the next block (its first position is off1)
-            nraw = load_window(a, 32 * (b + 1) + lane);
+            nraw = load_window(a, 32 * (b + 1) + lane, 5 * (b + 1) + lane_gword);
             noff0 = off1;
             noff1 = __ldg(a.off + b + 2);
         }
-        const bool offs_ok = off0 <= off1 && uint64_t(off1) <= a.n_elems;
+        const bool offs_ok = off0 <= off1 && off1 <= a.n_elems;
         const uint32_t head = off0 & 15u;
         // chunks to store: the head chunk (completed by the carried bytes
         // unless this block starts the run), up to the tail chunk, which is
@@ -352,7 +347,7 @@ __global__ void __launch_bounds__(WARPS * 32) decode_warp_kernel(const DecodeArg
         if (c0 + lane < cw) s0 = __ldcs(a.sm + c0 + lane);
         if (c0 + lane + 32 < cw) s1 = __ldcs(a.sm + c0 + lane + 32);
 
-        const Window w = finish_window(a, raw, 32 * b + lane);
+        const Window w = finish_window(a, raw, 32 * b + lane, lane_gshift);
         bool bad = false;
         const uint32_t cnt = count_codes(w, t, bad);
         uint32_t incl = cnt;
@@ -369,17 +364,16 @@ __global__ void __launch_bounds__(WARPS * 32) decode_warp_kernel(const DecodeArg
             if (lane == 0 && use_carry) *reinterpret_cast<uint4*>(stage) = carry;
             __syncwarp();
             const uint32_t pos0 = head + (incl - cnt);
-            decode_codes(w, t, reinterpret_cast<uint32_t*>(stage), pos0, cnt);
+            const uint32_t hword = decode_codes(w, t, reinterpret_cast<uint32_t*>(stage), pos0, cnt);
             __syncwarp();
-            write_head(w, t, stage, pos0, cnt);
+            write_head(stage, pos0, cnt, hword);
             __syncwarp();
-            uint32_t k = lane;
-            for (int j = 0; c0 + k < cw; k += 32, j++) {
-                const uint4 sv = j == 0 ? s0 : (j == 1 ? s1 : __ldcs(a.sm + c0 + k));
-                const uint4 ev = *reinterpret_cast<const uint4*>(stage + 16 * k);
-                merge_chunk(ev, sv, c0 + k, lo, off1, a.out);
-            }
-            if (keep_tail) carry = *reinterpret_cast<const uint4*>(stage + 16 * (c1 - 1 - c0));
+            const uint4* ev = reinterpret_cast<const uint4*>(stage);
+            if (c0 + lane < cw) merge_chunk(ev[lane], s0, c0 + lane, lo, off1, a.out);
+            if (c0 + lane + 32 < cw) merge_chunk(ev[lane + 32], s1, c0 + lane + 32, lo, off1, a.out);
+            for (uint32_t k = lane + 64; c0 + k < cw; k += 32)
+                merge_chunk(ev[k], __ldcs(a.sm + c0 + k), c0 + k, lo, off1, a.out);
+            if (keep_tail) carry = ev[c1 - 1 - c0];
             have_carry = keep_tail;
         }
         __syncwarp();
@@ -406,31 +400,34 @@ __global__ void __launch_bounds__(T) decode_block_kernel(const DecodeArgs a) {
     const Tables t = tables_at(smem);
     const uint32_t lane = threadIdx.x & 31u;
     const uint32_t warp = threadIdx.x >> 5;
+    const uint32_t my_gword = (5 * threadIdx.x) >> 5;
+    const uint32_t my_gshift = (5 * threadIdx.x) & 31u;
+    constexpr uint32_t kGwordsPerBlock = 5 * T / 32;
 
-    uint64_t b = blockIdx.x;
+    uint32_t b = blockIdx.x;
     RawWindow nraw{};
     uint32_t noff0 = 0, noff1 = 0;
     if (b < a.n_blocks) {
-        nraw = load_window(a, uint64_t(T) * b + threadIdx.x);
+        nraw = load_window(a, T * b + threadIdx.x, kGwordsPerBlock * b + my_gword);
         noff0 = __ldg(a.off + b);
         noff1 = __ldg(a.off + b + 1);
     }
     while (b < a.n_blocks) {
         const RawWindow raw = nraw;
         const uint32_t off0 = noff0, off1 = noff1;
-        const uint64_t bn = b + gridDim.x;
+        const uint32_t bn = b + gridDim.x;
         if (bn < a.n_blocks) {
-            nraw = load_window(a, uint64_t(T) * bn + threadIdx.x);
+            nraw = load_window(a, T * bn + threadIdx.x, kGwordsPerBlock * bn + my_gword);
             noff0 = __ldg(a.off + bn);
             noff1 = __ldg(a.off + bn + 1);
         }
-        const bool offs_ok = off0 <= off1 && uint64_t(off1) <= a.n_elems;
+        const bool offs_ok = off0 <= off1 && off1 <= a.n_elems;
         const uint32_t c0 = off0 >> 4;
         const uint32_t c1 = offs_ok ? (off1 + 15) >> 4 : c0;
         uint4 s0 = make_uint4(0, 0, 0, 0);
         if (c0 + threadIdx.x < c1) s0 = __ldcs(a.sm + c0 + threadIdx.x);
 
-        const Window w = finish_window(a, raw, uint64_t(T) * b + threadIdx.x);
+        const Window w = finish_window(a, raw, T * b + threadIdx.x, my_gshift);
         bool bad = false;
         const uint32_t cnt = count_codes(w, t, bad);
         uint32_t incl = cnt;
@@ -452,16 +449,14 @@ __global__ void __launch_bounds__(T) decode_block_kernel(const DecodeArgs a) {
             if (threadIdx.x == 0 && a.status) atomicOr(a.status, uint32_t(DF11_ERR_CORRUPT));
         } else {
             const uint32_t pos0 = (off0 & 15u) + before + incl - cnt;
-            decode_codes(w, t, reinterpret_cast<uint32_t*>(stage), pos0, cnt);
+            const uint32_t hword = decode_codes(w, t, reinterpret_cast<uint32_t*>(stage), pos0, cnt);
             __syncthreads();
-            write_head(w, t, stage, pos0, cnt);
+            write_head(stage, pos0, cnt, hword);
             __syncthreads();
-            uint32_t k = threadIdx.x;
-            for (int j = 0; c0 + k < c1; k += T, j++) {
-                const uint4 sv = j == 0 ? s0 : __ldcs(a.sm + c0 + k);
-                const uint4 ev = *reinterpret_cast<const uint4*>(stage + 16 * k);
-                merge_chunk(ev, sv, c0 + k, off0, off1, a.out);
-            }
+            const uint4* ev = reinterpret_cast<const uint4*>(stage);
+            if (c0 + threadIdx.x < c1) merge_chunk(ev[threadIdx.x], s0, c0 + threadIdx.x, off0, off1, a.out);
+            for (uint32_t k = threadIdx.x + T; c0 + k < c1; k += T)
+                merge_chunk(ev[k], __ldcs(a.sm + c0 + k), c0 + k, off0, off1, a.out);
         }
         __syncthreads();
         b = bn;
@@ -513,7 +508,7 @@ df11_status launch_block(const DecodeArgs& a, cudaStream_t s, int slot) {
 
 df11_status launch_warp(const DecodeArgs& a, cudaStream_t s) {
     const size_t smem = kLutBytes + size_t(kWarpsPerCta) * kWarpStage;
-    const uint64_t ctas = (a.n_blocks + kWarpsPerCta - 1) / kWarpsPerCta;
+    const uint64_t ctas = (uint64_t(a.n_blocks) + kWarpsPerCta - 1) / kWarpsPerCta;
     return launch_persistent(decode_warp_kernel<kWarpsPerCta>, 0, kWarpsPerCta * 32, smem, ctas, a, s);
 }
 
@@ -565,10 +560,10 @@ extern "C" df11_status df11_decompress(const df11_header* hdr, const uint8_t* d_
     a.lut = reinterpret_cast<const uint4*>(d_lut);
     a.out = d_out;
     a.status = d_status;
-    a.n_elems = hdr->n_elems;
-    a.total_bits = hdr->total_bits;
-    a.n_threads = hdr->n_threads;
-    a.n_blocks = hdr->n_blocks;
+    a.n_elems = uint32_t(hdr->n_elems);
+    a.n_threads = uint32_t(hdr->n_threads);
+    a.n_blocks = uint32_t(hdr->n_blocks);
+    a.last_wend = uint32_t(hdr->total_bits - 64 * (hdr->n_threads - 1));
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     switch (hdr->threads_per_block) {
         case 32: return launch_warp(a, s);

@@ -279,7 +279,7 @@ df11_status df11_build_lut(const df11_header* hdr, void* h_lut, uint64_t cap) {
         ctab[v] = count ? ((uint32_t(pos) << 16) | count) : (kEscape << 16);
         mtab[v] = uint16_t(mask);
         dtab[2 * v] = n4 ? syms4 : 0u;
-        dtab[2 * v + 1] = n4 ? ((used4 << 16) | n4) : (kEscape << 16);
+        dtab[2 * v + 1] = n4 ? ((used4 << 16) | (8 * n4)) : (kEscape << 16);
     }
     std::memcpy(blob, &lh, sizeof(lh));
     return DF11_OK;

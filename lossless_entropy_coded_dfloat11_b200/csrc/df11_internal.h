@@ -22,8 +22,10 @@ namespace df11 {
 //   mask table   uint16, bit j set when a complete code starts at offset j
 //       (used once per window, to drop codes that start past its end).
 //   decode table uint2: x = up to four symbols (first in bits 0..7, unused
-//       bytes zero); y = consumed << 16 | n, n = codes decoded (1..4).  The
-//       kernel keeps (bit position << 16 | output offset) in one register.
+//       bytes zero); y = consumed << 16 | 8n, n = codes decoded (1..4).  The
+//       kernel keeps (bit position << 16 | 8 x bytes pending) in one
+//       register, whose low five bits then are the shift that places the
+//       next symbols.
 //   A peek whose first code is longer than K bits (or matches no code) holds
 //   the escape value kEscape << 16 (count 0, n 0, symbols 0): adding it
 //   pushes the bit position past every window end, so the fast loops need

@@ -192,7 +192,7 @@ def test_decode_tables_agree_with_oracle_codes(source):
         if not codes4:
             assert (x, y) == (0, ESCAPE << 16)
             continue
-        assert y == (used4 << 16) | len(codes4)
+        assert y == (used4 << 16) | (8 * len(codes4))
         assert len(codes4) == 4 or x >> (8 * len(codes4)) == 0   # unused symbol bytes are zero
         for k, (sym, _) in enumerate(codes4):
             assert (x >> (8 * k)) & 0xFF == sym
