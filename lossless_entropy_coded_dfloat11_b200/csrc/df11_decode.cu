@@ -11,8 +11,8 @@
 // of a transformer block ("Descompressao por bloco de transformer").
 //
 // B200 specifics:
-//   * persistent grid: the 57 KB of decode tables are copied to shared memory
-//     once per CTA and serve every thread block of the stream;
+//   * persistent grid: the decode tables are copied to shared memory once
+//     per CTA and serve every thread block of the stream;
 //   * thread blocks of 32 threads (T = 32) are decoded by one warp each, with
 //     no CTA barrier at all: the prefix sum is five shuffles and the staging
 //     buffer is the warp's own; larger T use a block-wide scan;
@@ -285,24 +285,165 @@ __device__ __forceinline__ bool block_consistent(uint32_t off0, uint32_t off1, u
 
 // ---------------------------------------------------------------------------
 // T = 32: one warp decodes one thread block at a time; no CTA barrier after
-// the table copy.  Each warp takes a contiguous run of thread blocks, so the
-// 16-element chunk that straddles two consecutive blocks is stored once, as a
-// whole, by the later block: the earlier block leaves it in the staging
-// buffer, the warp carries its bytes over, and only the first and last chunk
-// of a run need element-wise stores.  Staging per warp: 32 windows x 64
-// symbols + head (15) + spill (3), rounded up.
+// the table copy.
+//
+// Decode once: each thread decodes its window a single time into a private
+// 68-byte slot (an odd number of words apart, so lanes writing the same slot
+// word hit different banks) and learns its count from the bytes it wrote,
+// corrected for codes of the last table step that start past the window end.
+// After the warp's prefix sum the slots are copied, one aligned word at a
+// time, into the block's contiguous staging buffer; the first word of a slot
+// range that starts mid-word is written byte-wise after a warp barrier, and a
+// last word's bytes past the thread's range belong to such heads, so they are
+// overwritten then.  The level-1 count table is not needed here.
+//
+// Each warp takes a contiguous run of thread blocks, so the 16-element chunk
+// that straddles two consecutive blocks is stored once, as a whole, by the
+// later block: the earlier block leaves it in the staging buffer and the warp
+// carries its bytes over; only the first and last chunk of a run need
+// element-wise stores.
 // ---------------------------------------------------------------------------
-constexpr uint32_t kWarpStage = 32 * 64 + 64;
+constexpr uint32_t kSlotWords = 17;                 // 64 symbols + 3 spilled, odd stride
+constexpr uint32_t kWarpSlots = 32 * kSlotWords * 4;
+constexpr uint32_t kWarpStage = 32 * 64 + 64;       // 32 windows x 64 symbols + head + spill
+constexpr uint32_t kWarpBytes = kWarpSlots + kWarpStage;
+// shared-memory copy of the tables this kernel uses: ladder, deltas and
+// symbols, then the mask and decode tables
+constexpr uint32_t kCompactSmall = uint32_t(kLutOffCount);
+constexpr uint32_t kCompactMask = kCompactSmall;
+constexpr uint32_t kCompactDecode = kCompactMask + uint32_t(kLutOffDecode - kLutOffMask);
+constexpr uint32_t kCompactBytes = kCompactDecode + uint32_t(kLutBytes - kLutOffDecode);
+
+__device__ __forceinline__ void copy_compact_tables(uint8_t* s, const uint4* g, int nthreads) {
+    for (int i = threadIdx.x; i < int(kCompactSmall / 16); i += nthreads)
+        reinterpret_cast<uint4*>(s)[i] = __ldg(g + i);
+    const uint4* g2 = g + kLutOffMask / 16;
+    uint4* s2 = reinterpret_cast<uint4*>(s + kCompactMask);
+    for (int i = threadIdx.x; i < int((kLutBytes - kLutOffMask) / 16); i += nthreads) s2[i] = __ldg(g2 + i);
+}
+
+// One half of the window (bit positions below lim, peeking at hi:lo) through
+// the decode table, in hand-scheduled PTX: 17 instructions per step.  Keeps
+// the pending symbol bytes in `pend`, stores completed words at `wad` (a
+// shared-window address), and leaves the last entry's index and y word for
+// the end-of-window correction.
+__device__ __forceinline__ void decode_half(uint32_t& acc, uint32_t& pend, uint32_t& wad, uint32_t& idx,
+                                            uint32_t& ylast, uint32_t hi, uint32_t lo, uint32_t lim,
+                                            uint32_t dtab_s) {
+    asm volatile(
+        "{\n\t"
+        ".reg .pred p, q;\n\t"
+        ".reg .u32 sh, pk, ad, x, t1, spill, zero;\n\t"
+        "mov.u32 zero, 0;\n\t"
+        "setp.ge.u32 p, %0, %7;\n\t"
+        "@p bra DONE;\n\t"
+        "LOOP:\n\t"
+        "shr.u32 sh, %0, 16;\n\t"
+        "shf.l.wrap.b32 pk, %6, %5, sh;\n\t"
+        "shr.u32 %3, pk, 20;\n\t"
+        "mad.lo.u32 ad, %3, 8, %8;\n\t"
+        "ld.shared.v2.u32 {x, %4}, [ad];\n\t"
+        "shf.l.wrap.b32 t1, zero, x, %0;\n\t"
+        "or.b32 %1, %1, t1;\n\t"
+        "shf.l.wrap.b32 spill, x, zero, %0;\n\t"
+        "add.u32 %0, %0, %4;\n\t"
+        "and.b32 t1, %0, 32;\n\t"
+        "setp.ne.u32 q, t1, 0;\n\t"
+        "@q st.shared.u32 [%2], %1;\n\t"
+        "@q add.u32 %2, %2, 4;\n\t"
+        "@q mov.b32 %1, spill;\n\t"
+        "@q sub.u32 %0, %0, 32;\n\t"
+        "setp.lt.u32 p, %0, %7;\n\t"
+        "@p bra LOOP;\n\t"
+        "DONE:\n\t"
+        "}"
+        : "+r"(acc), "+r"(pend), "+r"(wad), "+r"(idx), "+r"(ylast)
+        : "r"(hi), "r"(lo), "r"(lim), "r"(dtab_s)
+        : "memory");
+}
+
+// Decode the window into the slot at shared address slot_s; returns the
+// number of codes that start in the window.
+__device__ __forceinline__ uint32_t decode_window_once(const Window& w, const Tables& t, uint32_t dtab_s,
+                                                       uint32_t slot_s, bool& bad) {
+    const uint32_t lim1 = min(w.wend, 32u) << 16;
+    const uint32_t lim2 = w.wend << 16;
+    // bit position << 16 | 8 x bytes pending; low five bits = placement shift
+    uint32_t acc = w.start << 16;
+    uint32_t pend = 0, wad = slot_s, idx = 0, ylast = 0;
+    for (;;) {
+        decode_half(acc, pend, wad, idx, ylast, w.w0, w.w1, lim1, dtab_s);
+        decode_half(acc, pend, wad, idx, ylast, w.w1, w.w2, lim2, dtab_s);
+        if (acc < (kEscape << 16)) break;
+        // a code longer than the table: undo the escape, take it from level 2
+        acc -= kEscape << 16;
+        const uint32_t pk = peek32(w.w0, w.w1, w.w2, acc >> 16);
+        const int l = code_length(t.lj_end, pk, kPeekBits + 1);
+        if (!l) {
+            bad = true;
+            return 0;
+        }
+        pend |= code_symbol(t, pk, l) << (acc & 31u);
+        acc += (uint32_t(l) << 16) | 8u;
+        if (acc & 32u) {
+            asm volatile("st.shared.u32 [%0], %1;" ::"r"(wad), "r"(pend) : "memory");
+            wad += 4;
+            pend = 0;
+            acc -= 32u;
+        }
+        ylast = 0;
+    }
+    if (acc & 31u) asm volatile("st.shared.u32 [%0], %1;" ::"r"(wad), "r"(pend) : "memory");
+    uint32_t cnt = (wad - slot_s) + ((acc & 31u) >> 3);
+    if (ylast) {  // codes of the last table step that start at or past wend
+        const uint32_t s = w.wend - ((acc >> 16) - (ylast >> 16));
+        if (s < uint32_t(kPeekBits)) {
+            const uint32_t n = (ylast & 0xFFu) >> 3;
+            const uint32_t before = __popc(uint32_t(t.mtab[idx]) & ((1u << s) - 1u));
+            cnt -= n - min(n, before);
+        }
+    }
+    return cnt;
+}
+
+// Copy slot bytes [0, cnt) to staging bytes [pos0, pos0 + cnt): whole words
+// from the first word boundary on; returns the slot's first word, whose
+// leading bytes go to the positions before that boundary (write_head).
+__device__ __forceinline__ uint32_t copy_slot(const uint32_t* slot, uint32_t* stage32, uint32_t pos0, uint32_t cnt) {
+    if (cnt == 0) return 0;
+    const uint32_t r = (4u - (pos0 & 3u)) & 3u;  // slot byte landing on the first word boundary
+    const uint32_t fw = (pos0 + 3) >> 2;
+    const uint32_t lw = (pos0 + cnt - 1) >> 2;
+    const uint32_t first = slot[0];
+    uint32_t cur = first;
+    uint32_t k = 1;
+    for (uint32_t j = fw; j <= lw; j++, k++) {
+        const uint32_t nxt = slot[k];
+        stage32[j] = __funnelshift_r(cur, nxt, 8 * r);
+        cur = nxt;
+    }
+    return first;
+}
 
 template <int WARPS>
 __global__ void __launch_bounds__(WARPS * 32) decode_warp_kernel(const DecodeArgs a) {
     extern __shared__ __align__(16) uint8_t smem[];
-    copy_tables(smem, a.lut, WARPS * 32);
+    copy_compact_tables(smem, a.lut, WARPS * 32);
     __syncthreads();
-    const Tables t = tables_at(smem);
+    Tables t;
+    t.ctab = nullptr;
+    t.mtab = reinterpret_cast<const uint16_t*>(smem + kCompactMask);
+    t.dtab = reinterpret_cast<const uint2*>(smem + kCompactDecode);
+    t.lj_end = reinterpret_cast<const unsigned long long*>(smem + kLutOffLjEnd);
+    t.delta = reinterpret_cast<const uint32_t*>(smem + kLutOffDelta);
+    t.syms = smem + kLutOffSyms;
+    const uint32_t dtab_s = uint32_t(__cvta_generic_to_shared(t.dtab));
     const uint32_t lane = threadIdx.x & 31u;
     const uint32_t warp = threadIdx.x >> 5;
-    uint8_t* stage = smem + kLutBytes + warp * kWarpStage;
+    uint8_t* wbase = smem + kCompactBytes + warp * kWarpBytes;
+    uint32_t* slot = reinterpret_cast<uint32_t*>(wbase) + lane * kSlotWords;
+    const uint32_t slot_s = uint32_t(__cvta_generic_to_shared(slot));
+    uint8_t* stage = wbase + kWarpSlots;
     // the gap field of window 32b + lane lies in the block's five gap words
     const uint32_t lane_gword = (5 * lane) >> 5;
     const uint32_t lane_gshift = (5 * lane) & 31u;
@@ -349,7 +490,7 @@ __global__ void __launch_bounds__(WARPS * 32) decode_warp_kernel(const DecodeArg
 
         const Window w = finish_window(a, raw, 32 * b + lane, lane_gshift);
         bool bad = false;
-        const uint32_t cnt = count_codes(w, t, bad);
+        const uint32_t cnt = decode_window_once(w, t, dtab_s, slot_s, bad);
         uint32_t incl = cnt;
 #pragma unroll
         for (int d = 1; d < 32; d <<= 1) {
@@ -364,9 +505,16 @@ __global__ void __launch_bounds__(WARPS * 32) decode_warp_kernel(const DecodeArg
             if (lane == 0 && use_carry) *reinterpret_cast<uint4*>(stage) = carry;
             __syncwarp();
             const uint32_t pos0 = head + (incl - cnt);
-            const uint32_t hword = decode_codes(w, t, reinterpret_cast<uint32_t*>(stage), pos0, cnt);
+            const uint32_t hword = copy_slot(slot, reinterpret_cast<uint32_t*>(stage), pos0, cnt);
             __syncwarp();
-            write_head(stage, pos0, cnt, hword);
+            {  // bytes before this thread's first word boundary
+                const uint32_t room = (4u - (pos0 & 3u)) & 3u;
+                const uint32_t k = cnt < room ? cnt : room;
+                uint8_t* d = stage + pos0;
+                if (k > 0) d[0] = uint8_t(hword);
+                if (k > 1) d[1] = uint8_t(hword >> 8);
+                if (k > 2) d[2] = uint8_t(hword >> 16);
+            }
             __syncwarp();
             const uint4* ev = reinterpret_cast<const uint4*>(stage);
             if (c0 + lane < cw) merge_chunk(ev[lane], s0, c0 + lane, lo, off1, a.out);
@@ -507,7 +655,7 @@ df11_status launch_block(const DecodeArgs& a, cudaStream_t s, int slot) {
 }
 
 df11_status launch_warp(const DecodeArgs& a, cudaStream_t s) {
-    const size_t smem = kLutBytes + size_t(kWarpsPerCta) * kWarpStage;
+    const size_t smem = kCompactBytes + size_t(kWarpsPerCta) * kWarpBytes;
     const uint64_t ctas = (uint64_t(a.n_blocks) + kWarpsPerCta - 1) / kWarpsPerCta;
     return launch_persistent(decode_warp_kernel<kWarpsPerCta>, 0, kWarpsPerCta * 32, smem, ctas, a, s);
 }
