@@ -27,9 +27,10 @@
 //   * phase 2 gathers symbols in a register pair and stores aligned 32-bit
 //     words; a thread's first word, shared with the previous thread, is kept
 //     in a register and written byte-wise after a barrier;
-//   * the merge handles 16 elements per thread with one 16-byte shared load,
-//     one 16-byte streaming load, 24 logic/permute operations and two 16-byte
-//     streaming stores.
+//   * exponents are staged rotated right by one bit, so the merge is two
+//     bit-selects and two byte-permutes per four elements: 16 elements per
+//     thread with one 16-byte shared load, one 16-byte streaming load and two
+//     16-byte streaming stores.
 // Indices are 32-bit: n_elems < 2^32 and codes of at most 32 bits keep the
 // window count below 2^31.
 #include <cuda_runtime.h>
@@ -115,10 +116,12 @@ struct Window {
 __device__ __forceinline__ RawWindow load_window(const DecodeArgs& a, uint32_t tg, uint32_t gword) {
     RawWindow r;
     if (tg < a.n_threads) {
-        r.v = __ldg(reinterpret_cast<const uint2*>(a.exp) + tg);
-        r.v2 = __ldg(reinterpret_cast<const uint32_t*>(a.exp) + 2 * tg + 2);
-        r.glo = __ldg(a.gaps + gword);
-        r.ghi = __ldg(a.gaps + gword + 1);
+        const uint8_t* base = a.exp + 8 * size_t(tg);
+        r.v = __ldg(reinterpret_cast<const uint2*>(base));
+        r.v2 = __ldg(reinterpret_cast<const uint32_t*>(base + 8));
+        const uint32_t* gp = a.gaps + gword;
+        r.glo = __ldg(gp);
+        r.ghi = __ldg(gp + 1);
     } else {
         r.v = make_uint2(0, 0);
         r.v2 = r.glo = r.ghi = 0;
@@ -240,12 +243,12 @@ __device__ __forceinline__ void write_head(uint8_t* stage, uint32_t pos0, uint32
     if (k > 2) d[2] = uint8_t(head >> 24);
 }
 
-// Four BF16 values from four exponent bytes e4 and four sign+mantissa bytes
-// s4 (bf16 = sign << 15 | e << 7 | mantissa): the high output byte is
-// sign | e >> 1, the low one (e & 1) << 7 | mantissa.
-__device__ __forceinline__ void merge4(uint32_t e4, uint32_t s4, uint32_t& o01, uint32_t& o23) {
-    const uint32_t hi = (s4 & 0x80808080u) | ((e4 >> 1) & 0x7F7F7F7Fu);
-    const uint32_t lo = ((e4 << 7) & 0x80808080u) | (s4 & 0x7F7F7F7Fu);
+// Four BF16 values from four staged (rotated) exponent bytes r4 and four
+// sign+mantissa bytes s4: the high output byte is sign | e >> 1 and the low
+// one (e & 1) << 7 | mantissa, i.e. two bit-selects between r4 and s4.
+__device__ __forceinline__ void merge4(uint32_t r4, uint32_t s4, uint32_t& o01, uint32_t& o23) {
+    const uint32_t hi = (s4 & 0x80808080u) | (r4 & 0x7F7F7F7Fu);
+    const uint32_t lo = (r4 & 0x80808080u) | (s4 & 0x7F7F7F7Fu);
     o01 = __byte_perm(lo, hi, 0x5140);
     o23 = __byte_perm(lo, hi, 0x7362);
 }
@@ -414,14 +417,18 @@ __device__ __forceinline__ uint32_t copy_slot(const uint32_t* slot, uint32_t* st
     const uint32_t r = (4u - (pos0 & 3u)) & 3u;  // slot byte landing on the first word boundary
     const uint32_t fw = (pos0 + 3) >> 2;
     const uint32_t lw = (pos0 + cnt - 1) >> 2;
+    const uint32_t sh = 8 * r;
     const uint32_t first = slot[0];
     uint32_t cur = first;
-    uint32_t k = 1;
-    for (uint32_t j = fw; j <= lw; j++, k++) {
-        const uint32_t nxt = slot[k];
-        stage32[j] = __funnelshift_r(cur, nxt, 8 * r);
-        cur = nxt;
+    uint32_t j = fw;
+    const uint32_t* src = slot + 1;
+    for (; j + 1 <= lw; j += 2, src += 2) {
+        const uint32_t n1 = src[0], n2 = src[1];
+        stage32[j] = __funnelshift_r(cur, n1, sh);
+        stage32[j + 1] = __funnelshift_r(n1, n2, sh);
+        cur = n2;
     }
+    if (j <= lw) stage32[j] = __funnelshift_r(cur, src[0], sh);
     return first;
 }
 

@@ -80,6 +80,12 @@ static bool kraft_units(const uint8_t* len, uint64_t* units, int* n_present) {
 
 using namespace df11;
 
+// Decoded exponents are staged rotated right by one bit (bit 0 moves to bit
+// 7): the two bytes of a BF16 value are then bit-selects of the rotated
+// exponent and the sign+mantissa byte (high: sign | e >> 1, low:
+// (e & 1) << 7 | mantissa).
+static uint8_t rotate_symbol(uint8_t e) { return uint8_t((e >> 1) | (e << 7)); }
+
 extern "C" {
 
 int df11_version(void) { return DF11_VERSION; }
@@ -235,7 +241,7 @@ df11_status df11_build_lut(const df11_header* hdr, void* h_lut, uint64_t cap) {
     for (int l = 1; l <= 32; l++) {
         base[l] = uint32_t(n);
         for (int s = 0; s < 256; s++)
-            if (len[s] == l) syms[n++] = uint8_t(s);
+            if (len[s] == l) syms[n++] = rotate_symbol(uint8_t(s));
         if (count[l] && !lh.min_len) lh.min_len = l;
         if (count[l]) lh.max_len = l;
     }

@@ -22,7 +22,8 @@ namespace df11 {
 //   mask table   uint16, bit j set when a complete code starts at offset j
 //       (used once per window, to drop codes that start past its end).
 //   decode table uint2: x = up to four symbols (first in bits 0..7, unused
-//       bytes zero); y = consumed << 16 | 8n, n = codes decoded (1..4).  The
+//       bytes zero), each an exponent rotated right by one bit (bit 0 moved
+//       to bit 7) so that the merge needs only bit-selects; y = consumed << 16 | 8n, n = codes decoded (1..4).  The
 //       kernel keeps (bit position << 16 | 8 x bytes pending) in one
 //       register, whose low five bits then are the shift that places the
 //       next symbols.
@@ -34,7 +35,7 @@ namespace df11 {
 //   consecutive integers, so a code's length is the smallest l with
 //   peek32 < lj_end[l] (lj_end[l] = end of the length-l codes, shifted to the
 //   top of 32 bits), and its symbol is syms[(peek32 >> (32 - l)) + delta[l]]
-//   with syms sorted by (length, value).
+//   with syms sorted by (length, value) (stored rotated, as above).
 //
 // The pages cut the tree into 8-bit-high subtrees with 256-entry tables and
 // re-use exponent values 240..255 as pointers; here every exponent value

@@ -194,5 +194,5 @@ def test_decode_tables_agree_with_oracle_codes(source):
             continue
         assert y == (used4 << 16) | (8 * len(codes4))
         assert len(codes4) == 4 or x >> (8 * len(codes4)) == 0   # unused symbol bytes are zero
-        for k, (sym, _) in enumerate(codes4):
-            assert (x >> (8 * k)) & 0xFF == sym
+        for k, (sym, _) in enumerate(codes4):   # staged rotated right by one bit
+            assert (x >> (8 * k)) & 0xFF == ((sym >> 1) | (sym << 7)) & 0xFF
