@@ -306,10 +306,17 @@ __device__ __forceinline__ bool block_consistent(uint32_t off0, uint32_t off1, u
 // carries its bytes over; only the first and last chunk of a run need
 // element-wise stores.
 // ---------------------------------------------------------------------------
-constexpr uint32_t kSlotWords = 17;                 // 64 symbols + 3 spilled, odd stride
-constexpr uint32_t kWarpSlots = 32 * kSlotWords * 4;
-constexpr uint32_t kWarpStage = 32 * 64 + 64;       // 32 windows x 64 symbols + head + spill
-constexpr uint32_t kWarpBytes = kWarpSlots + kWarpStage;
+// Per-warp buffers depend on the shortest code length: a 64-bit window
+// holds at most 64 / min_len code starts, plus up to three symbols decoded
+// past its end.  Slots are an odd number of words apart.
+template <int MIN_LEN>
+struct WarpLayout {
+    static constexpr uint32_t kMaxCodes = 64 / MIN_LEN;
+    static constexpr uint32_t kSlotWords = ((kMaxCodes + 3 + 3) / 4) | 1u;
+    static constexpr uint32_t kSlots = 32 * kSlotWords * 4;
+    static constexpr uint32_t kStage = 32 * kMaxCodes + 64;  // + head (15) + spill, rounded
+    static constexpr uint32_t kBytes = kSlots + kStage;
+};
 // shared-memory copy of the tables this kernel uses: ladder, deltas and
 // symbols, then the mask and decode tables
 constexpr uint32_t kCompactSmall = uint32_t(kLutOffCount);
@@ -432,8 +439,9 @@ __device__ __forceinline__ uint32_t copy_slot(const uint32_t* slot, uint32_t* st
     return first;
 }
 
-template <int WARPS>
-__global__ void __launch_bounds__(WARPS * 32) decode_warp_kernel(const DecodeArgs a) {
+template <int WARPS, int MIN_LEN>
+__global__ void __launch_bounds__(WARPS * 32, 2) decode_warp_kernel(const DecodeArgs a) {
+    using L = WarpLayout<MIN_LEN>;
     extern __shared__ __align__(16) uint8_t smem[];
     copy_compact_tables(smem, a.lut, WARPS * 32);
     __syncthreads();
@@ -447,10 +455,10 @@ __global__ void __launch_bounds__(WARPS * 32) decode_warp_kernel(const DecodeArg
     const uint32_t dtab_s = uint32_t(__cvta_generic_to_shared(t.dtab));
     const uint32_t lane = threadIdx.x & 31u;
     const uint32_t warp = threadIdx.x >> 5;
-    uint8_t* wbase = smem + kCompactBytes + warp * kWarpBytes;
-    uint32_t* slot = reinterpret_cast<uint32_t*>(wbase) + lane * kSlotWords;
+    uint8_t* wbase = smem + kCompactBytes + warp * L::kBytes;
+    uint32_t* slot = reinterpret_cast<uint32_t*>(wbase) + lane * L::kSlotWords;
     const uint32_t slot_s = uint32_t(__cvta_generic_to_shared(slot));
-    uint8_t* stage = wbase + kWarpSlots;
+    uint8_t* stage = wbase + L::kSlots;
     // the gap field of window 32b + lane lies in the block's five gap words
     const uint32_t lane_gword = (5 * lane) >> 5;
     const uint32_t lane_gshift = (5 * lane) & 31u;
@@ -624,9 +632,12 @@ struct LaunchInfo {
     int sms = 0;
 };
 constexpr int kMaxDev = 64;
-LaunchInfo g_info[kMaxDev][6];  // [device][log2(T) - 5]
+LaunchInfo g_info[kMaxDev][7];  // [device][variant]
 
-constexpr int kWarpsPerCta = 16;
+// Warps per CTA for each variant: all warps of an SM share one copy of the
+// tables per CTA, two CTAs per SM.
+constexpr int kWarpsLong = 16;   // some code is 1 bit long
+constexpr int kWarpsShort = 20;  // every code has 2 bits or more
 
 template <typename Kernel>
 df11_status launch_persistent(Kernel kernel, int slot, int threads, size_t smem, uint64_t work_units,
@@ -661,10 +672,16 @@ df11_status launch_block(const DecodeArgs& a, cudaStream_t s, int slot) {
     return launch_persistent(decode_block_kernel<T>, slot, T, smem, a.n_blocks, a, s);
 }
 
-df11_status launch_warp(const DecodeArgs& a, cudaStream_t s) {
-    const size_t smem = kCompactBytes + size_t(kWarpsPerCta) * kWarpBytes;
-    const uint64_t ctas = (uint64_t(a.n_blocks) + kWarpsPerCta - 1) / kWarpsPerCta;
-    return launch_persistent(decode_warp_kernel<kWarpsPerCta>, 0, kWarpsPerCta * 32, smem, ctas, a, s);
+template <int WARPS, int MIN_LEN>
+df11_status launch_warp_variant(const DecodeArgs& a, cudaStream_t s, int slot) {
+    const size_t smem = kCompactBytes + size_t(WARPS) * WarpLayout<MIN_LEN>::kBytes;
+    const uint64_t ctas = (uint64_t(a.n_blocks) + WARPS - 1) / WARPS;
+    return launch_persistent(decode_warp_kernel<WARPS, MIN_LEN>, slot, WARPS * 32, smem, ctas, a, s);
+}
+
+df11_status launch_warp(const DecodeArgs& a, cudaStream_t s, uint32_t min_len) {
+    if (min_len >= 2) return launch_warp_variant<kWarpsShort, 2>(a, s, 6);
+    return launch_warp_variant<kWarpsLong, 1>(a, s, 0);
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -721,7 +738,12 @@ extern "C" df11_status df11_decompress(const df11_header* hdr, const uint8_t* d_
     a.last_wend = uint32_t(hdr->total_bits - 64 * (hdr->n_threads - 1));
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     switch (hdr->threads_per_block) {
-        case 32: return launch_warp(a, s);
+        case 32: {
+            uint32_t min_len = 32;
+            for (int v = 0; v < 256; v++)
+                if (hdr->code_len[v] && hdr->code_len[v] < min_len) min_len = hdr->code_len[v];
+            return launch_warp(a, s, min_len);
+        }
         case 64: return launch_block<64>(a, s, 1);
         case 128: return launch_block<128>(a, s, 2);
         case 256: return launch_block<256>(a, s, 3);
