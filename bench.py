@@ -58,6 +58,30 @@ def aggregate(per_rank_elapsed_ms: list[float], bytes_per_rank_step: int, steps:
     return {"ms": t, "gbs": total / (t * 1e-3) / 1e9, "ms_per_step": t / steps}
 
 
+def max_over_ranks(value: float, device) -> float:
+    """The largest value over all ranks (the slowest rank's time); a no-op
+    without a process group.  `device` is where the reduction tensor lives:
+    the rank's GPU under NCCL, the CPU under gloo."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return value
+    t = torch.tensor([value], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def min_over_ranks(flag: bool, device) -> bool:
+    """True only if every rank reports True."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return flag
+    t = torch.tensor([1 if flag else 0], device=device, dtype=torch.int32)
+    dist.all_reduce(t, op=dist.ReduceOp.MIN)
+    return bool(t.item())
+
+
 def rank_seed_offset(rank: int) -> int:
     """Each rank draws its own block (seeds shifted by 1000 per rank)."""
     return 1000 * rank
@@ -311,14 +335,8 @@ def run_native(args, rank: int, world: int, local_rank: int) -> None:
                 exact &= bool(torch.equal(v.reshape(-1).view(torch.int16)[:: 4093], f))
     torch.cuda.synchronize()
 
-    per_rank = [elapsed]
-    if world > 1:
-        t = torch.tensor([elapsed], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        per_rank = [float(t.item())] * world
-        e = torch.tensor([1 if exact else 0], device=dev, dtype=torch.int32)
-        dist.all_reduce(e, op=dist.ReduceOp.MIN)
-        exact = bool(e.item())
+    per_rank = [max_over_ranks(elapsed, dev)] * world
+    exact = min_over_ranks(exact, dev)
     agg = aggregate(per_rank, out_bytes, args.steps)
 
     # ---- end to end: host buffers through the public API --------------------
@@ -338,11 +356,7 @@ def run_native(args, rank: int, world: int, local_rank: int) -> None:
             res = hs.run(stream)
         e1.record(stream)
         torch.cuda.synchronize()
-        ems = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([ems], device=dev, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ems = float(t.item())
+        ems = max_over_ranks(e0.elapsed_time(e1), dev)
         e2e_exact = bool(torch.equal(res.view(torch.int16), originals[0].cpu()))
         e2e = {"value": 2 * streams[0].n_elems * k * world / (ems * 1e-3) / 1e9, "unit": UNIT,
                "h2d_bytes_per_step": hs.h2d_bytes(), "d2h_bytes_per_step": hs.d2h_bytes(),
