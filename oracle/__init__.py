@@ -45,7 +45,9 @@ def _load():
     global _lib
     if _lib is not None:
         return _lib
-    lib = ctypes.CDLL(build())
+    # a test may point at a deliberately broken build of the oracle to show
+    # that the pins catch it
+    lib = ctypes.CDLL(os.environ.get("DF11_ORACLE_LIB") or build())
     u8p = ctypes.POINTER(ctypes.c_uint8)
     u16p = ctypes.POINTER(ctypes.c_uint16)
     u32p = ctypes.POINTER(ctypes.c_uint32)

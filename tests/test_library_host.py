@@ -82,6 +82,19 @@ def test_code_lengths_fibonacci_and_workloads():
         np.testing.assert_array_equal(df11.code_lengths(h, 32), oracle.code_lengths(h, 32))
 
 
+def test_code_lengths_tie_rule_golden(golden_dir):
+    """The hand-worked tie case (tests/golden, example C)."""
+    from tests.conftest import parse_golden
+    g = parse_golden(os.path.join(golden_dir, "df11_tiny_stream.txt"))
+    h = np.zeros(256, dtype=np.uint64)
+    for item in g["C.counts"].split():
+        k, v = item.split("=")
+        h[int(k)] = int(v)
+    ln = df11.code_lengths(h, int(g["C.max_len"]))
+    want = {int(k): int(v) for k, v in (i.split("=") for i in g["C.code_len"].split())}
+    assert {s: int(ln[s]) for s in np.nonzero(ln)[0]} == want
+
+
 def test_code_lengths_rejects_bad_limits():
     h = hist_of([1] * 5, range(5))
     with pytest.raises(df11.DF11Error):

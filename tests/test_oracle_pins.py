@@ -299,6 +299,16 @@ def test_single_and_empty_alphabets():
     assert (oracle.code_lengths(np.zeros(256, dtype=np.uint64)) == 0).all()
 
 
+def test_tie_rule_leaf_before_package_golden(golden_dir):
+    """Hand-worked example C: on a leaf/package tie the leaf comes first."""
+    g = _golden(golden_dir)
+    h = np.zeros(256, dtype=np.uint64)
+    for sym, cnt in _kv(g["C.counts"]).items():
+        h[sym] = cnt
+    ln = oracle.code_lengths(h, int(g["C.max_len"]))
+    assert {s: int(ln[s]) for s in np.nonzero(ln)[0]} == _kv(g["C.code_len"])
+
+
 def test_tie_rule_orders_equal_counts_by_value():
     # three equal weights: one symbol gets 1 bit, two get 2 bits.  The tie
     # rule orders leaves by (count, value), so among equal counts the lower
