@@ -253,6 +253,38 @@ __device__ __forceinline__ void merge4(uint32_t r4, uint32_t s4, uint32_t& o01, 
     o23 = __byte_perm(lo, hi, 0x7362);
 }
 
+// Merge 16 elements and store them as two 16-byte streaming stores:
+// staged (rotated) exponents at shared address ev_s, sign+mantissa bytes sv.
+__device__ __forceinline__ void merge_store16(uint32_t ev_s, const uint4 sv, uint4* dst) {
+    asm volatile(
+        "{\n\t"
+        ".reg .b32 e0, e1, e2, e3, h, l, m, o0, o1, o2, o3, o4, o5, o6, o7;\n\t"
+        "mov.b32 m, 0x80808080;\n\t"
+        "ld.shared.v4.u32 {e0, e1, e2, e3}, [%0];\n\t"
+        "lop3.b32 h, %1, e0, m, 0xE4;\n\t"
+        "lop3.b32 l, e0, %1, m, 0xE4;\n\t"
+        "prmt.b32 o0, l, h, 0x5140;\n\t"
+        "prmt.b32 o1, l, h, 0x7362;\n\t"
+        "lop3.b32 h, %2, e1, m, 0xE4;\n\t"
+        "lop3.b32 l, e1, %2, m, 0xE4;\n\t"
+        "prmt.b32 o2, l, h, 0x5140;\n\t"
+        "prmt.b32 o3, l, h, 0x7362;\n\t"
+        "lop3.b32 h, %3, e2, m, 0xE4;\n\t"
+        "lop3.b32 l, e2, %3, m, 0xE4;\n\t"
+        "prmt.b32 o4, l, h, 0x5140;\n\t"
+        "prmt.b32 o5, l, h, 0x7362;\n\t"
+        "lop3.b32 h, %4, e3, m, 0xE4;\n\t"
+        "lop3.b32 l, e3, %4, m, 0xE4;\n\t"
+        "prmt.b32 o6, l, h, 0x5140;\n\t"
+        "prmt.b32 o7, l, h, 0x7362;\n\t"
+        "st.global.cs.v4.u32 [%5], {o0, o1, o2, o3};\n\t"
+        "st.global.cs.v4.u32 [%5 + 16], {o4, o5, o6, o7};\n\t"
+        "}"
+        :
+        : "r"(ev_s), "r"(sv.x), "r"(sv.y), "r"(sv.z), "r"(sv.w), "l"(dst)
+        : "memory");
+}
+
 // Merge and store chunk c (elements 16c..16c+15) of the range [lo, hi).
 __device__ __forceinline__ void merge_chunk(const uint4 ev, const uint4 sv, uint32_t c, uint32_t lo, uint32_t hi,
                                             uint16_t* __restrict__ out) {
@@ -322,6 +354,7 @@ struct WarpLayout {
 constexpr uint32_t kCompactSmall = uint32_t(kLutOffCount);
 constexpr uint32_t kCompactMask = kCompactSmall;
 constexpr uint32_t kCompactDecode = kCompactMask + uint32_t(kLutOffDecode - kLutOffMask);
+constexpr uint32_t kCompactLong = kCompactDecode + uint32_t(kLutOffLong - kLutOffDecode);
 constexpr uint32_t kCompactBytes = kCompactDecode + uint32_t(kLutBytes - kLutOffDecode);
 
 __device__ __forceinline__ void copy_compact_tables(uint8_t* s, const uint4* g, int nthreads) {
@@ -375,7 +408,8 @@ __device__ __forceinline__ void decode_half(uint32_t& acc, uint32_t& pend, uint3
 // Decode the window into the slot at shared address slot_s; returns the
 // number of codes that start in the window.
 __device__ __forceinline__ uint32_t decode_window_once(const Window& w, const Tables& t, uint32_t dtab_s,
-                                                       uint32_t slot_s, bool& bad) {
+                                                       uint32_t slot_s, const uint16_t* ltab, uint32_t long_base,
+                                                       uint32_t long_count, bool& bad) {
     const uint32_t lim1 = min(w.wend, 32u) << 16;
     const uint32_t lim2 = w.wend << 16;
     // bit position << 16 | 8 x bytes pending; low five bits = placement shift
@@ -388,12 +422,22 @@ __device__ __forceinline__ uint32_t decode_window_once(const Window& w, const Ta
         // a code longer than the table: undo the escape, take it from level 2
         acc -= kEscape << 16;
         const uint32_t pk = peek32(w.w0, w.w1, w.w2, acc >> 16);
-        const int l = code_length(t.lj_end, pk, kPeekBits + 1);
-        if (!l) {
-            bad = true;
-            return 0;
+        const uint32_t li = (pk >> (32 - kLongBits)) - long_base;
+        const uint32_t le = li < long_count ? uint32_t(ltab[li]) : 0u;
+        int l;
+        uint32_t sym;
+        if (le) {
+            l = int(le >> 8);
+            sym = le & 0xFFu;
+        } else {
+            l = code_length(t.lj_end, pk, kPeekBits + 1);
+            if (!l) {
+                bad = true;
+                return 0;
+            }
+            sym = code_symbol(t, pk, l);
         }
-        pend |= code_symbol(t, pk, l) << (acc & 31u);
+        pend |= sym << (acc & 31u);
         acc += (uint32_t(l) << 16) | 8u;
         if (acc & 32u) {
             asm volatile("st.shared.u32 [%0], %1;" ::"r"(wad), "r"(pend) : "memory");
@@ -440,7 +484,7 @@ __device__ __forceinline__ uint32_t copy_slot(const uint32_t* slot, uint32_t* st
 }
 
 template <int WARPS, int MIN_LEN>
-__global__ void __launch_bounds__(WARPS * 32, 2) decode_warp_kernel(const DecodeArgs a) {
+__global__ void __launch_bounds__(WARPS * 32, 1) decode_warp_kernel(const DecodeArgs a) {
     using L = WarpLayout<MIN_LEN>;
     extern __shared__ __align__(16) uint8_t smem[];
     copy_compact_tables(smem, a.lut, WARPS * 32);
@@ -453,6 +497,9 @@ __global__ void __launch_bounds__(WARPS * 32, 2) decode_warp_kernel(const Decode
     t.delta = reinterpret_cast<const uint32_t*>(smem + kLutOffDelta);
     t.syms = smem + kLutOffSyms;
     const uint32_t dtab_s = uint32_t(__cvta_generic_to_shared(t.dtab));
+    const uint16_t* ltab = reinterpret_cast<const uint16_t*>(smem + kCompactLong);
+    const uint32_t long_base = reinterpret_cast<const LutHeader*>(smem)->long_base;
+    const uint32_t long_count = reinterpret_cast<const LutHeader*>(smem)->long_count;
     const uint32_t lane = threadIdx.x & 31u;
     const uint32_t warp = threadIdx.x >> 5;
     uint8_t* wbase = smem + kCompactBytes + warp * L::kBytes;
@@ -505,7 +552,7 @@ __global__ void __launch_bounds__(WARPS * 32, 2) decode_warp_kernel(const Decode
 
         const Window w = finish_window(a, raw, 32 * b + lane, lane_gshift);
         bool bad = false;
-        const uint32_t cnt = decode_window_once(w, t, dtab_s, slot_s, bad);
+        const uint32_t cnt = decode_window_once(w, t, dtab_s, slot_s, ltab, long_base, long_count, bad);
         uint32_t incl = cnt;
 #pragma unroll
         for (int d = 1; d < 32; d <<= 1) {
@@ -532,10 +579,18 @@ __global__ void __launch_bounds__(WARPS * 32, 2) decode_warp_kernel(const Decode
             }
             __syncwarp();
             const uint4* ev = reinterpret_cast<const uint4*>(stage);
-            if (c0 + lane < cw) merge_chunk(ev[lane], s0, c0 + lane, lo, off1, a.out);
-            if (c0 + lane + 32 < cw) merge_chunk(ev[lane + 32], s1, c0 + lane + 32, lo, off1, a.out);
-            for (uint32_t k = lane + 64; c0 + k < cw; k += 32)
-                merge_chunk(ev[k], __ldcs(a.sm + c0 + k), c0 + k, lo, off1, a.out);
+            const uint32_t stage_s = uint32_t(__cvta_generic_to_shared(stage));
+            const uint32_t cf = (lo + 15) >> 4, cl = off1 >> 4;  // whole chunks: [cf, cl)
+            auto chunk = [&](uint32_t k, const uint4 sv) {
+                const uint32_t c = c0 + k;
+                if (c >= cf && c < cl)
+                    merge_store16(stage_s + 16 * k, sv, reinterpret_cast<uint4*>(a.out) + 2 * size_t(c));
+                else
+                    merge_chunk(ev[k], sv, c, lo, off1, a.out);
+            };
+            if (c0 + lane < cw) chunk(lane, s0);
+            if (c0 + lane + 32 < cw) chunk(lane + 32, s1);
+            for (uint32_t k = lane + 64; c0 + k < cw; k += 32) chunk(k, __ldcs(a.sm + c0 + k));
             if (keep_tail) carry = ev[c1 - 1 - c0];
             have_carry = keep_tail;
         }
@@ -634,10 +689,11 @@ struct LaunchInfo {
 constexpr int kMaxDev = 64;
 LaunchInfo g_info[kMaxDev][7];  // [device][variant]
 
-// Warps per CTA for each variant: all warps of an SM share one copy of the
-// tables per CTA, two CTAs per SM.
-constexpr int kWarpsLong = 16;   // some code is 1 bit long
-constexpr int kWarpsShort = 20;  // every code has 2 bits or more
+// One CTA of 32 warps per SM: all warps share one copy of the tables, and
+// the register budget (64 per thread) leaves the decode loop unconstrained;
+// this measured faster than two CTAs of 20 warps at 48 registers.
+constexpr int kWarpsLong = 32;   // some code is 1 bit long
+constexpr int kWarpsShort = 32;  // every code has 2 bits or more
 
 template <typename Kernel>
 df11_status launch_persistent(Kernel kernel, int slot, int threads, size_t smem, uint64_t work_units,

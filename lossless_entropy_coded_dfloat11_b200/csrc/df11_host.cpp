@@ -287,6 +287,20 @@ df11_status df11_build_lut(const df11_header* hdr, void* h_lut, uint64_t cap) {
         dtab[2 * v] = n4 ? syms4 : 0u;
         dtab[2 * v + 1] = n4 ? ((used4 << 16) | (8 * n4)) : (kEscape << 16);
     }
+    // level 2: long codes of up to kLongBits bits by their 20-bit prefix
+    uint16_t* ltab = reinterpret_cast<uint16_t*>(blob + kLutOffLong);
+    const uint64_t region = (uint64_t(1) << 32) - lj_end[kPeekBits];  // code space of long codes
+    const uint64_t n_long = (region + (uint64_t(1) << (32 - kLongBits)) - 1) >> (32 - kLongBits);
+    lh.long_base = uint32_t(lj_end[kPeekBits] >> (32 - kLongBits));
+    lh.long_count = (lj_end[kPeekBits] < (uint64_t(1) << 32) && n_long <= kLongEntries) ? uint32_t(n_long) : 0u;
+    for (uint32_t i = 0; i < lh.long_count; i++) {
+        const uint64_t peek = uint64_t(lh.long_base + i) << (32 - kLongBits);
+        const int l = code_length(peek);
+        if (l > kPeekBits && l <= int(kLongBits)) {
+            const uint32_t value = uint32_t(peek >> (32 - l));
+            ltab[i] = uint16_t(syms[(value + delta[l]) & 0xFFu] | (uint32_t(l) << 8));
+        }
+    }
     std::memcpy(blob, &lh, sizeof(lh));
     return DF11_OK;
 }

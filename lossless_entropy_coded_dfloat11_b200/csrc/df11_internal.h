@@ -31,11 +31,16 @@ namespace df11 {
 //   the escape value kEscape << 16 (count 0, n 0, symbols 0): adding it
 //   pushes the bit position past every window end, so the fast loops need
 //   no escape test; the slow path undoes it.
-// Level 2, for codes longer than K: canonical codes of one length are
-//   consecutive integers, so a code's length is the smallest l with
-//   peek32 < lj_end[l] (lj_end[l] = end of the length-l codes, shifted to the
-//   top of 32 bits), and its symbol is syms[(peek32 >> (32 - l)) + delta[l]]
-//   with syms sorted by (length, value) (stored rotated, as above).
+// Level 2, for codes longer than K.  Canonical codes put every code longer
+//   than K bits at the top of the code space, from lj_end[K] up (lj_end[l] =
+//   end of the codes of length <= l, shifted to the top of 32 bits).
+//   * long table uint16[<= 4096]: entry i describes the 20-bit prefix
+//     (lj_end[K] >> 12) + i: rotated symbol | length << 8 when the code has
+//     at most 20 bits, else 0.  Built only when the long codes fit in 4096
+//     such prefixes (LutHeader::long_count, 0 otherwise).
+//   * ladder: a code's length is the smallest l with peek32 < lj_end[l], its
+//     symbol syms[(peek32 >> (32 - l)) + delta[l]] with syms sorted by
+//     (length, value) (stored rotated, as above).
 //
 // The pages cut the tree into 8-bit-high subtrees with 256-entry tables and
 // re-use exponent values 240..255 as pointers; here every exponent value
@@ -53,7 +58,9 @@ struct LutHeader {
     uint32_t n_syms;
     uint32_t min_len;
     uint32_t max_len;
-    uint32_t pad[10];
+    uint32_t long_base;   // (lj_end[K] >> 12): 20-bit prefix of the first long code
+    uint32_t long_count;  // entries of the long table, 0 = ladder only
+    uint32_t pad[8];
 };
 static_assert(sizeof(LutHeader) == 64, "LutHeader is 64 bytes");
 
@@ -65,7 +72,10 @@ constexpr uint64_t kLutOffSyms = align16(kLutOffDelta + 33 * 4);            // u
 constexpr uint64_t kLutOffCount = align16(kLutOffSyms + 256);               // uint32[2^K]
 constexpr uint64_t kLutOffMask = align16(kLutOffCount + 4 * kLutEntries);   // uint16[2^K]
 constexpr uint64_t kLutOffDecode = align16(kLutOffMask + 2 * kLutEntries);  // uint2[2^K]
-constexpr uint64_t kLutBytes = align16(kLutOffDecode + 8 * kLutEntries);
+constexpr uint32_t kLongEntries = 4096;
+constexpr uint32_t kLongBits = 20;                                          // long-table resolution
+constexpr uint64_t kLutOffLong = align16(kLutOffDecode + 8 * kLutEntries);  // uint16[kLongEntries]
+constexpr uint64_t kLutBytes = align16(kLutOffLong + 2 * kLongEntries);
 
 // Canonical code per value (DEFLATE-style construction); false if the
 // lengths overflow the code space.

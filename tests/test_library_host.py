@@ -148,7 +148,8 @@ ESCAPE = 128
 OFF_COUNT = 736
 OFF_MASK = OFF_COUNT + 4 * 4096
 OFF_DECODE = OFF_MASK + 2 * 4096
-LUT_BYTES = OFF_DECODE + 8 * 4096
+OFF_LONG = OFF_DECODE + 8 * 4096
+LUT_BYTES = OFF_LONG + 2 * 4096
 
 
 def _oracle_prefix_decoder(code_len):
@@ -191,7 +192,7 @@ def test_decode_tables_agree_with_oracle_codes(source):
     assert lut[:4].tobytes() == b"DF11"
     ctab = lut[OFF_COUNT:OFF_MASK].view(np.uint32)
     mtab = lut[OFF_MASK:OFF_DECODE].view(np.uint16)
-    dtab = lut[OFF_DECODE:LUT_BYTES].view(np.uint32).reshape(-1, 2)
+    dtab = lut[OFF_DECODE:OFF_LONG].view(np.uint32).reshape(-1, 2)
     table = _oracle_prefix_decoder(s.code_len)
     rng = np.random.default_rng(3)
     for v in list(range(64)) + list(rng.integers(0, 4096, size=400)) + list(range(4032, 4096)):
@@ -209,3 +210,36 @@ def test_decode_tables_agree_with_oracle_codes(source):
         assert len(codes4) == 4 or x >> (8 * len(codes4)) == 0   # unused symbol bytes are zero
         for k, (sym, _) in enumerate(codes4):   # staged rotated right by one bit
             assert (x >> (8 * k)) & 0xFF == ((sym >> 1) | (sym << 7)) & 0xFF
+
+
+@pytest.mark.parametrize("source", ["outliers", "fibonacci", "matrix_1k"])
+def test_long_code_table_agrees_with_oracle_codes(source):
+    """Level 2: entry i of the long table describes the code at the top of the
+    20-bit prefix long_base + i (rotated symbol | length << 8, 0 if longer)."""
+    if source == "outliers":
+        x = inputs.matrix_outliers(1024, 1024, seed=21).flat_u16()
+    elif source == "fibonacci":
+        x = inputs.fibonacci().flat_u16()
+    else:
+        x = inputs.matrix_1k().flat_u16()
+    s = oracle.encode(x)
+    hdr = df11.make_header(s.code_len, s.n_elems, s.total_bits, 32)
+    lut = df11.build_lut(hdr)
+    long_base, long_count = (int(v) for v in lut[24:32].view(np.uint32))
+    assert 0 < long_count <= 4096
+    ltab = lut[OFF_LONG:LUT_BYTES].view(np.uint16)
+    table = _oracle_prefix_decoder(s.code_len)
+    # the first long prefix is where the codes of more than 12 bits begin
+    short_space = sum(1 << (32 - int(l)) for l in s.code_len if 0 < l <= 12)
+    assert long_base == short_space >> 12
+    for i in range(long_count):
+        bits = format(long_base + i, "020b")
+        codes, _ = _decode_bits(table, bits, 1)
+        e = int(ltab[i])
+        if not codes:
+            assert e == 0                       # longer than 20 bits: ladder
+            continue
+        sym, _ = codes[0]
+        length = next(len(k) for k, v in table.items() if v == sym)
+        assert length > 12
+        assert e == (((sym >> 1) | (sym << 7)) & 0xFF) | (length << 8)
