@@ -253,38 +253,6 @@ __device__ __forceinline__ void merge4(uint32_t r4, uint32_t s4, uint32_t& o01, 
     o23 = __byte_perm(lo, hi, 0x7362);
 }
 
-// Merge 16 elements and store them as two 16-byte streaming stores:
-// staged (rotated) exponents at shared address ev_s, sign+mantissa bytes sv.
-__device__ __forceinline__ void merge_store16(uint32_t ev_s, const uint4 sv, uint4* dst) {
-    asm volatile(
-        "{\n\t"
-        ".reg .b32 e0, e1, e2, e3, h, l, m, o0, o1, o2, o3, o4, o5, o6, o7;\n\t"
-        "mov.b32 m, 0x80808080;\n\t"
-        "ld.shared.v4.u32 {e0, e1, e2, e3}, [%0];\n\t"
-        "lop3.b32 h, %1, e0, m, 0xE4;\n\t"
-        "lop3.b32 l, e0, %1, m, 0xE4;\n\t"
-        "prmt.b32 o0, l, h, 0x5140;\n\t"
-        "prmt.b32 o1, l, h, 0x7362;\n\t"
-        "lop3.b32 h, %2, e1, m, 0xE4;\n\t"
-        "lop3.b32 l, e1, %2, m, 0xE4;\n\t"
-        "prmt.b32 o2, l, h, 0x5140;\n\t"
-        "prmt.b32 o3, l, h, 0x7362;\n\t"
-        "lop3.b32 h, %3, e2, m, 0xE4;\n\t"
-        "lop3.b32 l, e2, %3, m, 0xE4;\n\t"
-        "prmt.b32 o4, l, h, 0x5140;\n\t"
-        "prmt.b32 o5, l, h, 0x7362;\n\t"
-        "lop3.b32 h, %4, e3, m, 0xE4;\n\t"
-        "lop3.b32 l, e3, %4, m, 0xE4;\n\t"
-        "prmt.b32 o6, l, h, 0x5140;\n\t"
-        "prmt.b32 o7, l, h, 0x7362;\n\t"
-        "st.global.cs.v4.u32 [%5], {o0, o1, o2, o3};\n\t"
-        "st.global.cs.v4.u32 [%5 + 16], {o4, o5, o6, o7};\n\t"
-        "}"
-        :
-        : "r"(ev_s), "r"(sv.x), "r"(sv.y), "r"(sv.z), "r"(sv.w), "l"(dst)
-        : "memory");
-}
-
 // Merge and store chunk c (elements 16c..16c+15) of the range [lo, hi).
 __device__ __forceinline__ void merge_chunk(const uint4 ev, const uint4 sv, uint32_t c, uint32_t lo, uint32_t hi,
                                             uint16_t* __restrict__ out) {
@@ -309,6 +277,51 @@ __device__ __forceinline__ void merge_chunk(const uint4 ev, const uint4 sv, uint
     }
 }
 
+// Merge 8 elements and store them as one 16-byte streaming store: staged
+// (rotated) exponents at shared address ev_s, sign+mantissa bytes sv.  A
+// warp storing units 32 apart per instruction writes 512 contiguous bytes.
+__device__ __forceinline__ void merge_store8(uint32_t ev_s, const uint2 sv, uint4* dst) {
+    asm volatile(
+        "{\n\t"
+        ".reg .b32 e0, e1, h, l, m, o0, o1, o2, o3;\n\t"
+        "mov.b32 m, 0x80808080;\n\t"
+        "ld.shared.v2.u32 {e0, e1}, [%0];\n\t"
+        "lop3.b32 h, %1, e0, m, 0xE4;\n\t"
+        "lop3.b32 l, e0, %1, m, 0xE4;\n\t"
+        "prmt.b32 o0, l, h, 0x5140;\n\t"
+        "prmt.b32 o1, l, h, 0x7362;\n\t"
+        "lop3.b32 h, %2, e1, m, 0xE4;\n\t"
+        "lop3.b32 l, e1, %2, m, 0xE4;\n\t"
+        "prmt.b32 o2, l, h, 0x5140;\n\t"
+        "prmt.b32 o3, l, h, 0x7362;\n\t"
+        "st.global.cs.v4.u32 [%3], {o0, o1, o2, o3};\n\t"
+        "}"
+        :
+        : "r"(ev_s), "r"(sv.x), "r"(sv.y), "l"(dst)
+        : "memory");
+}
+
+// Merge and store unit u (elements 8u..8u+7) of the range [lo, hi).
+__device__ __forceinline__ void merge_unit(const uint2 ev, const uint2 sv, uint32_t u, uint32_t lo, uint32_t hi,
+                                           uint16_t* __restrict__ out) {
+    uint4 o;
+    merge4(ev.x, sv.x, o.x, o.y);
+    merge4(ev.y, sv.y, o.z, o.w);
+    uint4* dst = reinterpret_cast<uint4*>(out) + size_t(u);
+    const uint32_t i0 = 8 * u;
+    if (i0 >= lo && i0 + 8 <= hi) {
+        __stcs(dst, o);
+    } else {
+        const uint32_t words[4] = {o.x, o.y, o.z, o.w};
+        uint16_t* d16 = reinterpret_cast<uint16_t*>(dst);
+#pragma unroll
+        for (int k = 0; k < 8; k++) {
+            const uint32_t i = i0 + k;
+            if (i >= lo && i < hi) d16[k] = uint16_t(words[k >> 1] >> (16 * (k & 1)));
+        }
+    }
+}
+
 __device__ __forceinline__ void copy_tables(uint8_t* s_lut, const uint4* g_lut, int nthreads) {
     for (int i = threadIdx.x; i < int(kLutBytes / 16); i += nthreads)
         reinterpret_cast<uint4*>(s_lut)[i] = __ldg(g_lut + i);
@@ -323,8 +336,7 @@ __device__ __forceinline__ bool block_consistent(uint32_t off0, uint32_t off1, u
 // the table copy.
 //
 // Decode once: each thread decodes its window a single time into a private
-// 68-byte slot (an odd number of words apart, so lanes writing the same slot
-// word hit different banks) and learns its count from the bytes it wrote,
+// slot of shared memory and learns its count from the bytes it wrote,
 // corrected for codes of the last table step that start past the window end.
 // After the warp's prefix sum the slots are copied, one aligned word at a
 // time, into the block's contiguous staging buffer; the first word of a slot
@@ -332,25 +344,30 @@ __device__ __forceinline__ bool block_consistent(uint32_t off0, uint32_t off1, u
 // last word's bytes past the thread's range belong to such heads, so they are
 // overwritten then.  The level-1 count table is not needed here.
 //
-// Each warp takes a contiguous run of thread blocks, so the 16-element chunk
-// that straddles two consecutive blocks is stored once, as a whole, by the
-// later block: the earlier block leaves it in the staging buffer and the warp
-// carries its bytes over; only the first and last chunk of a run need
-// element-wise stores.
+// The merge works on 8-element units (8 sign+mantissa bytes in, one 16-byte
+// store out); lane L takes units L, L + 32, ..., so each store instruction
+// of the warp covers 512 contiguous bytes.  Each warp takes a contiguous run
+// of thread blocks, so the unit that straddles two consecutive blocks is
+// stored once, as a whole, by the later block: the earlier block leaves it
+// in the staging buffer and the warp carries its bytes over; only the first
+// and last unit of a run need element-wise stores.
 // ---------------------------------------------------------------------------
 // Per-warp buffers depend on the shortest code length: a 64-bit window
 // holds at most 64 / min_len code starts, plus up to three symbols decoded
-// past its end.  Slots are an odd number of words apart.
+// past its end.  The slots are stored transposed (word k of lane L at word
+// 32k + L), so each lane always uses the same bank: the decode loop's
+// stores, which happen at a different word offset in every lane, and the
+// copy's loads are free of bank conflicts.
 template <int MIN_LEN>
 struct WarpLayout {
     static constexpr uint32_t kMaxCodes = 64 / MIN_LEN;
-    static constexpr uint32_t kSlotWords = ((kMaxCodes + 3 + 3) / 4) | 1u;
+    static constexpr uint32_t kSlotWords = (kMaxCodes + 3 + 3) / 4;
     static constexpr uint32_t kSlots = 32 * kSlotWords * 4;
     static constexpr uint32_t kStage = 32 * kMaxCodes + 64;  // + head (15) + spill, rounded
     static constexpr uint32_t kBytes = kSlots + kStage;
 };
 // shared-memory copy of the tables this kernel uses: ladder, deltas and
-// symbols, then the mask and decode tables
+// symbols, then the mask, decode and long tables
 constexpr uint32_t kCompactSmall = uint32_t(kLutOffCount);
 constexpr uint32_t kCompactMask = kCompactSmall;
 constexpr uint32_t kCompactDecode = kCompactMask + uint32_t(kLutOffDecode - kLutOffMask);
@@ -393,7 +410,7 @@ __device__ __forceinline__ void decode_half(uint32_t& acc, uint32_t& pend, uint3
         "and.b32 t1, %0, 32;\n\t"
         "setp.ne.u32 q, t1, 0;\n\t"
         "@q st.shared.u32 [%2], %1;\n\t"
-        "@q add.u32 %2, %2, 4;\n\t"
+        "@q add.u32 %2, %2, 128;\n\t"
         "@q mov.b32 %1, spill;\n\t"
         "@q sub.u32 %0, %0, 32;\n\t"
         "setp.lt.u32 p, %0, %7;\n\t"
@@ -405,8 +422,8 @@ __device__ __forceinline__ void decode_half(uint32_t& acc, uint32_t& pend, uint3
         : "memory");
 }
 
-// Decode the window into the slot at shared address slot_s; returns the
-// number of codes that start in the window.
+// Decode the window into the (transposed) slot at shared address slot_s;
+// returns the number of codes that start in the window.
 __device__ __forceinline__ uint32_t decode_window_once(const Window& w, const Tables& t, uint32_t dtab_s,
                                                        uint32_t slot_s, const uint16_t* ltab, uint32_t long_base,
                                                        uint32_t long_count, bool& bad) {
@@ -441,14 +458,14 @@ __device__ __forceinline__ uint32_t decode_window_once(const Window& w, const Ta
         acc += (uint32_t(l) << 16) | 8u;
         if (acc & 32u) {
             asm volatile("st.shared.u32 [%0], %1;" ::"r"(wad), "r"(pend) : "memory");
-            wad += 4;
+            wad += 128;
             pend = 0;
             acc -= 32u;
         }
         ylast = 0;
     }
     if (acc & 31u) asm volatile("st.shared.u32 [%0], %1;" ::"r"(wad), "r"(pend) : "memory");
-    uint32_t cnt = (wad - slot_s) + ((acc & 31u) >> 3);
+    uint32_t cnt = ((wad - slot_s) >> 5) + ((acc & 31u) >> 3);
     if (ylast) {  // codes of the last table step that start at or past wend
         const uint32_t s = w.wend - ((acc >> 16) - (ylast >> 16));
         if (s < uint32_t(kPeekBits)) {
@@ -462,7 +479,8 @@ __device__ __forceinline__ uint32_t decode_window_once(const Window& w, const Ta
 
 // Copy slot bytes [0, cnt) to staging bytes [pos0, pos0 + cnt): whole words
 // from the first word boundary on; returns the slot's first word, whose
-// leading bytes go to the positions before that boundary (write_head).
+// leading bytes go to the positions before that boundary (write_head).  The
+// slot is transposed: its words are 32 words apart.
 __device__ __forceinline__ uint32_t copy_slot(const uint32_t* slot, uint32_t* stage32, uint32_t pos0, uint32_t cnt) {
     if (cnt == 0) return 0;
     const uint32_t r = (4u - (pos0 & 3u)) & 3u;  // slot byte landing on the first word boundary
@@ -472,9 +490,9 @@ __device__ __forceinline__ uint32_t copy_slot(const uint32_t* slot, uint32_t* st
     const uint32_t first = slot[0];
     uint32_t cur = first;
     uint32_t j = fw;
-    const uint32_t* src = slot + 1;
-    for (; j + 1 <= lw; j += 2, src += 2) {
-        const uint32_t n1 = src[0], n2 = src[1];
+    const uint32_t* src = slot + 32;
+    for (; j + 1 <= lw; j += 2, src += 64) {
+        const uint32_t n1 = src[0], n2 = src[32];
         stage32[j] = __funnelshift_r(cur, n1, sh);
         stage32[j + 1] = __funnelshift_r(n1, n2, sh);
         cur = n2;
@@ -503,7 +521,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_warp_kernel(const Decode
     const uint32_t lane = threadIdx.x & 31u;
     const uint32_t warp = threadIdx.x >> 5;
     uint8_t* wbase = smem + kCompactBytes + warp * L::kBytes;
-    uint32_t* slot = reinterpret_cast<uint32_t*>(wbase) + lane * L::kSlotWords;
+    uint32_t* slot = reinterpret_cast<uint32_t*>(wbase) + lane;
     const uint32_t slot_s = uint32_t(__cvta_generic_to_shared(slot));
     uint8_t* stage = wbase + L::kSlots;
     // the gap field of window 32b + lane lies in the block's five gap words
@@ -524,7 +542,8 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_warp_kernel(const Decode
         noff0 = __ldg(a.off + b);
         noff1 = __ldg(a.off + b + 1);
     }
-    uint4 carry = make_uint4(0, 0, 0, 0);  // staging bytes of the chunk left by the previous block
+    const uint2* sm8 = reinterpret_cast<const uint2*>(a.sm);
+    uint2 carry = make_uint2(0, 0);  // staging bytes of the unit left by the previous block
     bool have_carry = false;
     while (b < b_end) {
         const RawWindow raw = nraw;
@@ -536,19 +555,20 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_warp_kernel(const Decode
             noff1 = __ldg(a.off + b + 2);
         }
         const bool offs_ok = off0 <= off1 && off1 <= a.n_elems;
-        const uint32_t head = off0 & 15u;
-        // chunks to store: the head chunk (completed by the carried bytes
-        // unless this block starts the run), up to the tail chunk, which is
+        const uint32_t head = off0 & 7u;
+        // units to store: the head unit (completed by the carried bytes
+        // unless this block starts the run), up to the tail unit, which is
         // left to the next block when that block exists and shares it
-        const uint32_t c0 = off0 >> 4;
-        const uint32_t c1 = offs_ok ? (off1 + 15) >> 4 : c0;
-        const bool keep_tail = more && (off1 & 15u) != 0;
-        const uint32_t cw = keep_tail && c1 > c0 ? c1 - 1 : c1;
+        const uint32_t u0 = off0 >> 3;
+        const uint32_t u1 = offs_ok ? (off1 + 7) >> 3 : u0;
+        const bool keep_tail = more && (off1 & 7u) != 0;
+        const uint32_t uw = keep_tail && u1 > u0 ? u1 - 1 : u1;
         const bool use_carry = have_carry && head != 0;
-        const uint32_t lo = use_carry ? (off0 & ~15u) : off0;
-        uint4 s0 = make_uint4(0, 0, 0, 0), s1 = s0;
-        if (c0 + lane < cw) s0 = __ldcs(a.sm + c0 + lane);
-        if (c0 + lane + 32 < cw) s1 = __ldcs(a.sm + c0 + lane + 32);
+        const uint32_t lo = use_carry ? (off0 & ~7u) : off0;
+        uint2 sv[4];
+#pragma unroll
+        for (int r = 0; r < 4; r++)
+            sv[r] = u0 + lane + 32 * r < uw ? __ldcs(sm8 + u0 + lane + 32 * r) : make_uint2(0, 0);
 
         const Window w = finish_window(a, raw, 32 * b + lane, lane_gshift);
         bool bad = false;
@@ -564,7 +584,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_warp_kernel(const Decode
             if (lane == 0 && a.status) atomicOr(a.status, uint32_t(DF11_ERR_CORRUPT));
             have_carry = false;
         } else {
-            if (lane == 0 && use_carry) *reinterpret_cast<uint4*>(stage) = carry;
+            if (lane == 0 && use_carry) *reinterpret_cast<uint2*>(stage) = carry;
             __syncwarp();
             const uint32_t pos0 = head + (incl - cnt);
             const uint32_t hword = copy_slot(slot, reinterpret_cast<uint32_t*>(stage), pos0, cnt);
@@ -578,20 +598,21 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_warp_kernel(const Decode
                 if (k > 2) d[2] = uint8_t(hword >> 16);
             }
             __syncwarp();
-            const uint4* ev = reinterpret_cast<const uint4*>(stage);
+            const uint2* ev = reinterpret_cast<const uint2*>(stage);
             const uint32_t stage_s = uint32_t(__cvta_generic_to_shared(stage));
-            const uint32_t cf = (lo + 15) >> 4, cl = off1 >> 4;  // whole chunks: [cf, cl)
-            auto chunk = [&](uint32_t k, const uint4 sv) {
-                const uint32_t c = c0 + k;
-                if (c >= cf && c < cl)
-                    merge_store16(stage_s + 16 * k, sv, reinterpret_cast<uint4*>(a.out) + 2 * size_t(c));
+            const uint32_t uf = (lo + 7) >> 3, ul = off1 >> 3;  // whole units: [uf, ul)
+            auto unit = [&](uint32_t k, const uint2 s8) {
+                const uint32_t u = u0 + k;
+                if (u >= uf && u < ul)
+                    merge_store8(stage_s + 8 * k, s8, reinterpret_cast<uint4*>(a.out) + u);
                 else
-                    merge_chunk(ev[k], sv, c, lo, off1, a.out);
+                    merge_unit(ev[k], s8, u, lo, off1, a.out);
             };
-            if (c0 + lane < cw) chunk(lane, s0);
-            if (c0 + lane + 32 < cw) chunk(lane + 32, s1);
-            for (uint32_t k = lane + 64; c0 + k < cw; k += 32) chunk(k, __ldcs(a.sm + c0 + k));
-            if (keep_tail) carry = ev[c1 - 1 - c0];
+#pragma unroll
+            for (int r = 0; r < 4; r++)
+                if (u0 + lane + 32 * r < uw) unit(lane + 32 * r, sv[r]);
+            for (uint32_t k = lane + 128; u0 + k < uw; k += 32) unit(k, __ldcs(sm8 + u0 + k));
+            if (keep_tail) carry = ev[u1 - 1 - u0];
             have_carry = keep_tail;
         }
         __syncwarp();
@@ -730,7 +751,8 @@ df11_status launch_block(const DecodeArgs& a, cudaStream_t s, int slot) {
 
 template <int WARPS, int MIN_LEN>
 df11_status launch_warp_variant(const DecodeArgs& a, cudaStream_t s, int slot) {
-    const size_t smem = kCompactBytes + size_t(WARPS) * WarpLayout<MIN_LEN>::kBytes;
+    constexpr size_t smem = kCompactBytes + size_t(WARPS) * WarpLayout<MIN_LEN>::kBytes;
+    static_assert(smem <= 227 * 1024, "shared memory per CTA");
     const uint64_t ctas = (uint64_t(a.n_blocks) + WARPS - 1) / WARPS;
     return launch_persistent(decode_warp_kernel<WARPS, MIN_LEN>, slot, WARPS * 32, smem, ctas, a, s);
 }
