@@ -278,26 +278,27 @@ __device__ __forceinline__ void merge_chunk(const uint4 ev, const uint4 sv, uint
 }
 
 // Merge 8 elements and store them as one 16-byte streaming store: staged
-// (rotated) exponents at shared address ev_s, sign+mantissa bytes sv.  A
-// warp storing units 32 apart per instruction writes 512 contiguous bytes.
-__device__ __forceinline__ void merge_store8(uint32_t ev_s, const uint2 sv, uint4* dst) {
+// (rotated) exponents at shared address ev_s + EV_OFF, sign+mantissa bytes
+// sv, destination dst + DST_OFF bytes; m = 0x80808080.  A warp storing
+// units 32 apart per instruction writes 512 contiguous bytes.
+template <int EV_OFF = 0, int DST_OFF = 0>
+__device__ __forceinline__ void merge_store8(uint32_t ev_s, const uint2 sv, uint4* dst, uint32_t m) {
     asm volatile(
         "{\n\t"
-        ".reg .b32 e0, e1, h, l, m, o0, o1, o2, o3;\n\t"
-        "mov.b32 m, 0x80808080;\n\t"
-        "ld.shared.v2.u32 {e0, e1}, [%0];\n\t"
-        "lop3.b32 h, %1, e0, m, 0xE4;\n\t"
-        "lop3.b32 l, e0, %1, m, 0xE4;\n\t"
+        ".reg .b32 e0, e1, h, l, o0, o1, o2, o3;\n\t"
+        "ld.shared.v2.u32 {e0, e1}, [%0+%5];\n\t"
+        "lop3.b32 h, %1, e0, %4, 0xE4;\n\t"
+        "lop3.b32 l, e0, %1, %4, 0xE4;\n\t"
         "prmt.b32 o0, l, h, 0x5140;\n\t"
         "prmt.b32 o1, l, h, 0x7362;\n\t"
-        "lop3.b32 h, %2, e1, m, 0xE4;\n\t"
-        "lop3.b32 l, e1, %2, m, 0xE4;\n\t"
+        "lop3.b32 h, %2, e1, %4, 0xE4;\n\t"
+        "lop3.b32 l, e1, %2, %4, 0xE4;\n\t"
         "prmt.b32 o2, l, h, 0x5140;\n\t"
         "prmt.b32 o3, l, h, 0x7362;\n\t"
-        "st.global.cs.v4.u32 [%3], {o0, o1, o2, o3};\n\t"
+        "st.global.cs.v4.u32 [%3+%6], {o0, o1, o2, o3};\n\t"
         "}"
         :
-        : "r"(ev_s), "r"(sv.x), "r"(sv.y), "l"(dst)
+        : "r"(ev_s), "r"(sv.x), "r"(sv.y), "l"(dst), "r"(m), "n"(EV_OFF), "n"(DST_OFF)
         : "memory");
 }
 
@@ -579,8 +580,9 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_warp_kernel(const Decode
             const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, d);
             if (lane >= uint32_t(d)) incl += y;
         }
-        const uint32_t total = __shfl_sync(0xFFFFFFFFu, incl, 31);
-        if (__any_sync(0xFFFFFFFFu, bad) || !block_consistent(off0, off1, total, a.n_elems)) {
+        // the block's codes must fill exactly its range of output positions
+        const bool ok = !bad && offs_ok && (lane != 31 || incl == off1 - off0);
+        if (!__all_sync(0xFFFFFFFFu, ok)) {
             if (lane == 0 && a.status) atomicOr(a.status, uint32_t(DF11_ERR_CORRUPT));
             have_carry = false;
         } else {
@@ -600,18 +602,32 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_warp_kernel(const Decode
             __syncwarp();
             const uint2* ev = reinterpret_cast<const uint2*>(stage);
             const uint32_t stage_s = uint32_t(__cvta_generic_to_shared(stage));
-            const uint32_t uf = (lo + 7) >> 3, ul = off1 >> 3;  // whole units: [uf, ul)
-            auto unit = [&](uint32_t k, const uint2 s8) {
-                const uint32_t u = u0 + k;
-                if (u >= uf && u < ul)
-                    merge_store8(stage_s + 8 * k, s8, reinterpret_cast<uint4*>(a.out) + u);
-                else
-                    merge_unit(ev[k], s8, u, lo, off1, a.out);
-            };
+            const uint32_t nu = uw - u0;  // units this block stores
+            const uint32_t m = 0x80808080u;
+            if (lo == 8 * u0 && (keep_tail || (off1 & 7u) == 0)) {
+                // every unit is whole (all but the first and last block of a run)
+                const uint32_t ev_s = stage_s + 8 * lane;
+                uint4* dst = reinterpret_cast<uint4*>(a.out) + u0 + lane;
+                if (lane < nu) merge_store8<0, 0>(ev_s, sv[0], dst, m);
+                if (lane + 32 < nu) merge_store8<256, 512>(ev_s, sv[1], dst, m);
+                if (lane + 64 < nu) merge_store8<512, 1024>(ev_s, sv[2], dst, m);
+                if (lane + 96 < nu) merge_store8<768, 1536>(ev_s, sv[3], dst, m);
+                for (uint32_t k = 128; lane + k < nu; k += 32)
+                    merge_store8(ev_s + 8 * k, __ldcs(sm8 + u0 + lane + k), dst + k, m);
+            } else {
+                const uint32_t uf = (lo + 7) >> 3, ul = off1 >> 3;  // whole units: [uf, ul)
+                auto unit = [&](uint32_t k, const uint2 s8) {
+                    const uint32_t u = u0 + k;
+                    if (u >= uf && u < ul)
+                        merge_store8(stage_s + 8 * k, s8, reinterpret_cast<uint4*>(a.out) + u, m);
+                    else
+                        merge_unit(ev[k], s8, u, lo, off1, a.out);
+                };
 #pragma unroll
-            for (int r = 0; r < 4; r++)
-                if (u0 + lane + 32 * r < uw) unit(lane + 32 * r, sv[r]);
-            for (uint32_t k = lane + 128; u0 + k < uw; k += 32) unit(k, __ldcs(sm8 + u0 + k));
+                for (int r = 0; r < 4; r++)
+                    if (lane + 32 * r < nu) unit(lane + 32 * r, sv[r]);
+                for (uint32_t k = lane + 128; k < nu; k += 32) unit(k, __ldcs(sm8 + u0 + k));
+            }
             if (keep_tail) carry = ev[u1 - 1 - u0];
             have_carry = keep_tail;
         }
