@@ -384,43 +384,56 @@ __device__ __forceinline__ void copy_compact_tables(uint8_t* s, const uint4* g, 
 }
 
 // One half of the window (bit positions below lim, peeking at hi:lo) through
-// the decode table, in hand-scheduled PTX: 17 instructions per step.  Keeps
-// the pending symbol bytes in `pend`, stores completed words at `wad` (a
-// shared-window address), and leaves the last entry's index and y word for
-// the end-of-window correction.
+// the decode table, in hand-written PTX: 16 instructions per step, with no
+// branch but the loop's own.  `acc` is (bit position << 16 | 8 x bytes
+// produced so far); its low five bits place the next symbols in `pend`, and a
+// word is complete when bit 5 of acc flips.  The completed word is stored at
+// `wad` (a shared-window address, stepping 128 bytes in the transposed slot)
+// and `pend` becomes the spilled bytes through one clamped funnel shift.  The
+// loop is unrolled twice with acc alternating between two registers.  The
+// last entry's index and y word stay behind for the end-of-window correction.
 __device__ __forceinline__ void decode_half(uint32_t& acc, uint32_t& pend, uint32_t& wad, uint32_t& idx,
                                             uint32_t& ylast, uint32_t hi, uint32_t lo, uint32_t lim,
                                             uint32_t dtab_s) {
+#define DF11_STEP(A, B)                                  \
+    "shr.u32 sh, " A ", 16;\n\t"                          \
+    "shf.l.wrap.b32 pk, %6, %5, sh;\n\t"                  \
+    "shr.u32 %3, pk, 20;\n\t"                             \
+    "mad.lo.u32 ad, %3, 8, %8;\n\t"                       \
+    "ld.shared.v2.u32 {x, %4}, [ad];\n\t"                 \
+    "shf.l.wrap.b32 t1, zero, x, " A ";\n\t"              \
+    "or.b32 %1, %1, t1;\n\t"                              \
+    "shf.l.wrap.b32 spill, x, zero, " A ";\n\t"           \
+    "add.u32 " B ", " A ", %4;\n\t"                       \
+    "lop3.b32 t1, " B ", " A ", c32, 0x28;\n\t"           \
+    "setp.ne.u32 q, t1, 0;\n\t"                           \
+    "@q st.shared.u32 [%2], %1;\n\t"                      \
+    "mad.lo.u32 %2, t1, 4, %2;\n\t"                       \
+    "shf.r.clamp.b32 %1, %1, spill, t1;\n\t"
     asm volatile(
         "{\n\t"
         ".reg .pred p, q;\n\t"
-        ".reg .u32 sh, pk, ad, x, t1, spill, zero;\n\t"
+        ".reg .u32 sh, pk, ad, x, t1, spill, zero, c32, b;\n\t"
         "mov.u32 zero, 0;\n\t"
+        "mov.u32 c32, 32;\n\t"
         "setp.ge.u32 p, %0, %7;\n\t"
         "@p bra DONE;\n\t"
         "LOOP:\n\t"
-        "shr.u32 sh, %0, 16;\n\t"
-        "shf.l.wrap.b32 pk, %6, %5, sh;\n\t"
-        "shr.u32 %3, pk, 20;\n\t"
-        "mad.lo.u32 ad, %3, 8, %8;\n\t"
-        "ld.shared.v2.u32 {x, %4}, [ad];\n\t"
-        "shf.l.wrap.b32 t1, zero, x, %0;\n\t"
-        "or.b32 %1, %1, t1;\n\t"
-        "shf.l.wrap.b32 spill, x, zero, %0;\n\t"
-        "add.u32 %0, %0, %4;\n\t"
-        "and.b32 t1, %0, 32;\n\t"
-        "setp.ne.u32 q, t1, 0;\n\t"
-        "@q st.shared.u32 [%2], %1;\n\t"
-        "@q add.u32 %2, %2, 128;\n\t"
-        "@q mov.b32 %1, spill;\n\t"
-        "@q sub.u32 %0, %0, 32;\n\t"
+        DF11_STEP("%0", "b")
+        "setp.ge.u32 p, b, %7;\n\t"
+        "@p bra DONE_B;\n\t"
+        DF11_STEP("b", "%0")
         "setp.lt.u32 p, %0, %7;\n\t"
         "@p bra LOOP;\n\t"
+        "bra.uni DONE;\n\t"
+        "DONE_B:\n\t"
+        "mov.u32 %0, b;\n\t"
         "DONE:\n\t"
         "}"
         : "+r"(acc), "+r"(pend), "+r"(wad), "+r"(idx), "+r"(ylast)
         : "r"(hi), "r"(lo), "r"(lim), "r"(dtab_s)
         : "memory");
+#undef DF11_STEP
 }
 
 // Decode the window into the (transposed) slot at shared address slot_s;
@@ -430,7 +443,7 @@ __device__ __forceinline__ uint32_t decode_window_once(const Window& w, const Ta
                                                        uint32_t long_count, bool& bad) {
     const uint32_t lim1 = min(w.wend, 32u) << 16;
     const uint32_t lim2 = w.wend << 16;
-    // bit position << 16 | 8 x bytes pending; low five bits = placement shift
+    // bit position << 16 | 8 x bytes produced; low five bits = placement shift
     uint32_t acc = w.start << 16;
     uint32_t pend = 0, wad = slot_s, idx = 0, ylast = 0;
     for (;;) {
@@ -456,17 +469,17 @@ __device__ __forceinline__ uint32_t decode_window_once(const Window& w, const Ta
             sym = code_symbol(t, pk, l);
         }
         pend |= sym << (acc & 31u);
+        const uint32_t before_sym = acc;
         acc += (uint32_t(l) << 16) | 8u;
-        if (acc & 32u) {
+        if ((acc ^ before_sym) & 32u) {  // the word is complete
             asm volatile("st.shared.u32 [%0], %1;" ::"r"(wad), "r"(pend) : "memory");
             wad += 128;
             pend = 0;
-            acc -= 32u;
         }
         ylast = 0;
     }
     if (acc & 31u) asm volatile("st.shared.u32 [%0], %1;" ::"r"(wad), "r"(pend) : "memory");
-    uint32_t cnt = ((wad - slot_s) >> 5) + ((acc & 31u) >> 3);
+    uint32_t cnt = (acc & 0xFFFFu) >> 3;
     if (ylast) {  // codes of the last table step that start at or past wend
         const uint32_t s = w.wend - ((acc >> 16) - (ylast >> 16));
         if (s < uint32_t(kPeekBits)) {
