@@ -24,13 +24,17 @@
 //     and second 32 bits of the window so each peek is one funnel shift; codes
 //     longer than the 12-bit tables leave through an escape value that pushes
 //     the bit position out of the window, so the fast loops have one test;
-//   * phase 2 gathers symbols in a register pair and stores aligned 32-bit
-//     words; a thread's first word, shared with the previous thread, is kept
-//     in a register and written byte-wise after a barrier;
+//   * symbols are gathered in a register pair and leave as aligned 32-bit
+//     words; a thread's first word, shared with the previous thread, is
+//     written byte-wise after a barrier.  The T = 32 kernel decodes each
+//     window only once, into a per-thread shared-memory slot, and copies the
+//     slot into place after the scan; larger T decode twice (count, then
+//     decode into place);
 //   * exponents are staged rotated right by one bit, so the merge is two
-//     bit-selects and two byte-permutes per four elements: 16 elements per
-//     thread with one 16-byte shared load, one 16-byte streaming load and two
-//     16-byte streaming stores.
+//     bit-selects and two byte-permutes per four elements.  The T = 32
+//     kernel merges 8-element units (8-byte shared load, 8-byte streaming
+//     load, one 16-byte streaming store; one store instruction of a warp
+//     covers 512 contiguous bytes), larger T merge 16-element chunks.
 // Indices are 32-bit: n_elems < 2^32 and codes of at most 32 bits keep the
 // window count below 2^31.
 #include <cuda_runtime.h>

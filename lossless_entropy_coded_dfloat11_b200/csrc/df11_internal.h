@@ -23,10 +23,10 @@ namespace df11 {
 //       (used once per window, to drop codes that start past its end).
 //   decode table uint2: x = up to four symbols (first in bits 0..7, unused
 //       bytes zero), each an exponent rotated right by one bit (bit 0 moved
-//       to bit 7) so that the merge needs only bit-selects; y = consumed << 16 | 8n, n = codes decoded (1..4).  The
-//       kernel keeps (bit position << 16 | 8 x bytes pending) in one
-//       register, whose low five bits then are the shift that places the
-//       next symbols.
+//       to bit 7) so that the merge needs only bit-selects;
+//       y = consumed << 16 | 8n, n = codes decoded (1..4).  The kernels keep
+//       (bit position << 16 | 8 x bytes produced) in one register, whose
+//       low five bits then are the shift that places the next symbols.
 //   A peek whose first code is longer than K bits (or matches no code) holds
 //   the escape value kEscape << 16 (count 0, n 0, symbols 0): adding it
 //   pushes the bit position past every window end, so the fast loops need
