@@ -273,6 +273,29 @@ def run_reference(args, rank: int, world: int) -> None:
     print(json.dumps(line), flush=True)
 
 
+def time_compress(df11, w, repeats: int) -> dict:
+    """Wall-clock time of the public compress call on device-resident BF16
+    tensors (histogram kernel, host code build, table upload, bit-pack
+    kernels), synchronised on both sides; the median of `repeats` calls after
+    one untimed call."""
+    import torch
+    times = []
+    for r in range(repeats + 1):
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        cs = df11.compress(w.tensors, names=w.names)
+        torch.cuda.synchronize()
+        if r:
+            times.append(time.perf_counter() - t0)
+        del cs
+    t = sorted(times)[len(times) // 2]
+    in_bytes = sum(2 * x.numel() for x in w.tensors)
+    return {"value": in_bytes / t / 1e9, "unit": "GB/s of BF16 input", "ms": t * 1e3,
+            "repeats": repeats, "elements": in_bytes // 2,
+            "what": "df11.compress on device-resident BF16: histogram kernel, host package-merge and "
+                    "table build, bit-pack kernels; median wall clock, synchronised"}
+
+
 def run_native(args, rank: int, world: int, local_rank: int) -> None:
     import numpy as np
     import torch
@@ -286,7 +309,10 @@ def run_native(args, rank: int, world: int, local_rank: int) -> None:
     # ---- build the compressed workload on this GPU ------------------------
     workloads = make_workloads(args.config, rank, "cuda")
     streams, originals = [], []
+    compress = None
     for w in workloads:
+        if compress is None and not args.no_compress:
+            compress = time_compress(df11, w, args.compress_repeats)
         cs = df11.compress(w.tensors, names=w.names)
         streams.append(cs)
         originals.append(torch.cat([t.reshape(-1) for t in w.tensors]).view(torch.int16)
@@ -423,6 +449,7 @@ def run_native(args, rank: int, world: int, local_rank: int) -> None:
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": args.steps * launches_per_step,
+        "compress": compress,
         "clocks": sampler.record(),
         "when": datetime.datetime.now(datetime.timezone.utc).isoformat(timespec="seconds"),
     }
@@ -443,6 +470,8 @@ def main(argv=None):
                     help="elements per step in the reference arm")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-compress", action="store_true", help="skip timing the compress call")
+    ap.add_argument("--compress-repeats", type=int, default=5)
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("at least 3 warm-up steps")

@@ -13,6 +13,7 @@
 #include <atomic>
 #include <cstring>
 #include <mutex>
+#include <type_traits>
 #include <vector>
 
 #include "df11_internal.h"
@@ -131,155 +132,335 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* s
 }
 
 // ---------------------------------------------------------------------------
-// Bits of code per chunk of kEncChunk elements.
+// The encode kernels are persistent: each CTA stages the code table in shared
+// memory once and then walks chunks of kEncChunk elements in grid-stride
+// order, loading the next chunk's elements while it works on the current one.
+// (Indexing the table in the kernel's parameter space with a different
+// exponent in every lane would serialise in the constant cache.)
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(kEncThreads) chunk_bits_kernel(const __grid_constant__ SegTable sg,
-                                                                 const __grid_constant__ CodeTable ct,
-                                                                 uint64_t n, uint32_t* __restrict__ chunk_bits) {
-    __shared__ uint32_t s_warp[kEncThreads / 32];
-    const uint64_t i0 = uint64_t(blockIdx.x) * kEncChunk + uint64_t(threadIdx.x) * kEncPerThread;
-    uint32_t bits = 0;
+struct SharedCodes {
+    uint2 e[256];  // x = code left-aligned in 32 bits, y = its length (0 = absent)
+};
+
+__device__ __forceinline__ void stage_codes(SharedCodes& sc, const CodeTable& ct) {
+    for (int v = threadIdx.x; v < 256; v += blockDim.x) {
+        const uint32_t l = ct.len[v];
+        sc.e[v] = make_uint2(l ? ct.code[v] << (32u - l) : 0u, l);
+    }
+}
+
+// One thread's kEncPerThread elements as eight words (element 2j in the low
+// half of word j), loaded ahead of use: 32 aligned bytes when they lie in one
+// segment, else gathered element by element when used.
+struct RawElems {
+    uint4 a, b;
+    bool direct;
+};
+
+// c0 = the chunk's first element: its segment is looked up once (the same
+// for every thread), a thread whose elements lie in a later segment looks
+// up its own.
+__device__ __forceinline__ RawElems load_raw(const SegTable& sg, uint64_t c0, uint64_t i0, uint64_t n) {
+    RawElems r;
+    r.direct = false;
     if (i0 < n) {
+        uint32_t seg = find_seg(sg, c0);
+        if (i0 >= sg.start[seg + 1]) seg = find_seg(sg, i0);
+        const uint16_t* p = sg.ptr[seg] + (i0 - sg.start[seg]);
+        if (i0 + kEncPerThread <= sg.start[seg + 1] && (reinterpret_cast<uintptr_t>(p) & 15u) == 0) {
+            r.a = __ldcs(reinterpret_cast<const uint4*>(p));
+            r.b = __ldcs(reinterpret_cast<const uint4*>(p) + 1);
+            r.direct = true;
+        }
+    }
+    return r;
+}
+
+__device__ __forceinline__ void raw_words(const SegTable& sg, const RawElems& r, uint64_t i0, uint64_t n,
+                                          uint32_t (&w)[kEncPerThread / 2]) {
+    if (r.direct) {
+        w[0] = r.a.x; w[1] = r.a.y; w[2] = r.a.z; w[3] = r.a.w;
+        w[4] = r.b.x; w[5] = r.b.y; w[6] = r.b.z; w[7] = r.b.w;
+    } else {
         uint16_t x[kEncPerThread];
         load_chunk(sg, i0, n, x);
 #pragma unroll
-        for (int k = 0; k < int(kEncPerThread); k++)
-            if (i0 + k < n) bits += ct.len[(x[k] >> 7) & 0xFFu];
+        for (int j = 0; j < int(kEncPerThread / 2); j++) w[j] = x[2 * j] | (uint32_t(x[2 * j + 1]) << 16);
     }
-    uint32_t total;
-    block_exclusive_scan<kEncThreads>(bits, s_warp, total);
-    if (threadIdx.x == 0) chunk_bits[blockIdx.x] = total;
 }
 
-// Exclusive prefix sum of the chunk totals (one CTA; a few thousand chunks
-// per stream at most a million).
+__device__ __forceinline__ uint32_t elem(const uint32_t (&w)[kEncPerThread / 2], int k) {
+    return (w[k >> 1] >> (16 * (k & 1))) & 0xFFFFu;
+}
+
+// Code bits of this thread's elements (those past n count 0).
+__device__ __forceinline__ uint32_t thread_bits(const SharedCodes& sc, const uint32_t (&w)[kEncPerThread / 2],
+                                                uint32_t valid) {
+    uint32_t bits = 0;
+    if (valid == kEncPerThread) {
+#pragma unroll
+        for (int k = 0; k < int(kEncPerThread); k++) bits += sc.e[(elem(w, k) >> 7) & 0xFFu].y;
+    } else {
+#pragma unroll
+        for (int k = 0; k < int(kEncPerThread); k++)
+            if (uint32_t(k) < valid) bits += sc.e[(elem(w, k) >> 7) & 0xFFu].y;
+    }
+    return bits;
+}
+
+// Bits of code per chunk.
+__global__ void __launch_bounds__(kEncThreads) chunk_bits_kernel(const __grid_constant__ SegTable sg,
+                                                                 const __grid_constant__ CodeTable ct,
+                                                                 uint64_t n, uint64_t n_chunks,
+                                                                 uint32_t* __restrict__ chunk_bits) {
+    __shared__ SharedCodes sc;
+    __shared__ uint32_t s_warp[kEncThreads / 32];
+    stage_codes(sc, ct);
+    __syncthreads();
+    const uint64_t tofs = uint64_t(threadIdx.x) * kEncPerThread;
+    uint64_t c = blockIdx.x;
+    RawElems next = load_raw(sg, c * kEncChunk, c * kEncChunk + tofs, n);
+    for (; c < n_chunks; c += gridDim.x) {
+        const RawElems cur = next;
+        const uint64_t i0 = c * kEncChunk + tofs;
+        if (c + gridDim.x < n_chunks)
+            next = load_raw(sg, (c + gridDim.x) * kEncChunk, (c + gridDim.x) * kEncChunk + tofs, n);
+        uint32_t bits = 0;
+        if (i0 < n) {
+            uint32_t w[kEncPerThread / 2];
+            raw_words(sg, cur, i0, n, w);
+            const uint64_t left = n - i0;
+            bits = thread_bits(sc, w, left < kEncPerThread ? uint32_t(left) : kEncPerThread);
+        }
+        uint32_t total;
+        block_exclusive_scan<kEncThreads>(bits, s_warp, total);
+        if (threadIdx.x == 0) chunk_bits[c] = total;
+        __syncthreads();  // s_warp is reused by the next chunk
+    }
+}
+
+// Exclusive prefix sum of the chunk totals in one CTA, 4096 chunks per tile
+// (four per thread, 16-byte loads), the next tile's loads issued before the
+// current tile is scanned.
 constexpr int kScanThreads = 1024;
 __global__ void __launch_bounds__(kScanThreads) chunk_scan_kernel(const uint32_t* __restrict__ chunk_bits,
                                                                   uint64_t n_chunks,
                                                                   unsigned long long* __restrict__ chunk_start) {
-    __shared__ unsigned long long s_part[kScanThreads];
-    const uint64_t per = (n_chunks + kScanThreads - 1) / kScanThreads;
-    const uint64_t lo = per * threadIdx.x;
-    const uint64_t hi = lo + per < n_chunks ? lo + per : n_chunks;
-    unsigned long long sum = 0;
-    for (uint64_t c = lo; c < hi; c++) sum += chunk_bits[c];
-    s_part[threadIdx.x] = sum;
-    __syncthreads();
-    // Hillis-Steele over 1024 partial sums
-    for (int d = 1; d < kScanThreads; d <<= 1) {
-        const unsigned long long y = threadIdx.x >= d ? s_part[threadIdx.x - d] : 0ull;
+    __shared__ unsigned long long s_warp[kScanThreads / 32];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    constexpr uint64_t kTile = 4 * kScanThreads;
+    auto load4 = [&](uint64_t base) {
+        const uint64_t c = base + 4 * uint64_t(threadIdx.x);
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (c + 4 <= n_chunks) {
+            v = __ldg(reinterpret_cast<const uint4*>(chunk_bits + c));
+        } else {
+            if (c < n_chunks) v.x = chunk_bits[c];
+            if (c + 1 < n_chunks) v.y = chunk_bits[c + 1];
+            if (c + 2 < n_chunks) v.z = chunk_bits[c + 2];
+            if (c + 3 < n_chunks) v.w = chunk_bits[c + 3];
+        }
+        return v;
+    };
+    unsigned long long carry = 0;
+    uint4 v = load4(0);
+    for (uint64_t base = 0; base < n_chunks; base += kTile) {
+        const uint4 cur = v;
+        if (base + kTile < n_chunks) v = load4(base + kTile);
+        const unsigned long long own = (unsigned long long)cur.x + cur.y + cur.z + cur.w;
+        unsigned long long incl = own;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const unsigned long long y = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+            if (lane >= d) incl += y;
+        }
+        if (lane == 31) s_warp[warp] = incl;
         __syncthreads();
-        s_part[threadIdx.x] += y;
-        __syncthreads();
-    }
-    unsigned long long run = s_part[threadIdx.x] - sum;
-    for (uint64_t c = lo; c < hi; c++) {
-        chunk_start[c] = run;
-        run += chunk_bits[c];
+        unsigned long long before = 0, total = 0;
+        for (int w = 0; w < kScanThreads / 32; w++) {
+            const unsigned long long t = s_warp[w];
+            total += t;
+            before += w < warp ? t : 0ull;
+        }
+        __syncthreads();  // s_warp is rewritten by the next tile
+        unsigned long long run = carry + before + incl - own;
+        const uint64_t c = base + 4 * uint64_t(threadIdx.x);
+        const uint32_t e[4] = {cur.x, cur.y, cur.z, cur.w};
+#pragma unroll
+        for (int k = 0; k < 4; k++) {
+            if (c + k < n_chunks) chunk_start[c + k] = run;
+            run += e[k];
+        }
+        carry += total;
     }
 }
 
 // ---------------------------------------------------------------------------
-// Bit-pack: codes are OR-ed into a shared-memory image of the chunk's words,
-// interior words are stored, the two boundary words (shared with the
-// neighbouring chunks) are OR-ed into global memory.  The same pass writes
-// the sign+mantissa bytes, each window's gap and each thread block's output
-// position, using only the element's own start bit s and length l:
+// Bit-pack.  Each thread appends its codes to a register word with funnel
+// shifts; its first word (which it may share with the previous thread) and
+// its last, partial word (shared with the next) are OR-ed into a
+// shared-memory image of the chunk, the words in between are stored.  The
+// image's interior words are then stored to EncodedExponent and its two
+// boundary words, shared with the neighbouring chunks, are OR-ed into global
+// memory.  The same pass writes the sign+mantissa bytes, each window's gap
+// and each thread block's output position from the element's own start bit
+// s and length l:
 //   * a code that starts inside window w-1 and runs into window w sets
 //     gap[w] = s + l - 64w (gaps of windows that begin exactly at a code start
 //     stay 0);
 //   * a code that starts exactly at bit 64*T*b sets off[b] = i, one that runs
 //     over that bit sets off[b] = i + 1.
+// Positions are kept 32-bit relative to the chunk's first bit rounded down to
+// a thread-block boundary; a code covers a window boundary exactly when
+// (u >> 6) changes across it, u = relative start + 63, which is one test per
+// element.
 // ---------------------------------------------------------------------------
 constexpr int kPackWords = kEncChunk + 4;  // 32 bits per element at most, plus the misalignment
+// windows a thread's codes can reach into: 16 codes of at most 32 bits
+constexpr int kMaxEvents = (int(kEncPerThread) * 32) / 64 + 1;
+static_assert(kPackWords % 4 == 0, "image cleared in 16-byte stores");
 
 __global__ void __launch_bounds__(kEncThreads) pack_kernel(const __grid_constant__ SegTable sg,
                                                            const __grid_constant__ CodeTable ct, uint64_t n,
-                                                           uint32_t log2_block_bits,
+                                                           uint64_t n_chunks, uint32_t log2_block_bits,
                                                            const unsigned long long* __restrict__ chunk_start,
                                                            uint32_t* __restrict__ exp32, uint8_t* __restrict__ sm,
                                                            uint32_t* __restrict__ gaps32,
                                                            uint32_t* __restrict__ block_off, uint64_t n_blocks) {
-    __shared__ uint32_t s_words[kPackWords];
+    __shared__ SharedCodes sc;
+    __shared__ __align__(16) uint32_t s_words[kPackWords];
+    __shared__ uint32_t s_ev[kMaxEvents][kEncThreads];
     __shared__ uint32_t s_warp[kEncThreads / 32];
-    const uint64_t i0 = uint64_t(blockIdx.x) * kEncChunk + uint64_t(threadIdx.x) * kEncPerThread;
-    uint16_t x[kEncPerThread];
-    uint32_t bits = 0;
-    if (i0 < n) {
-        load_chunk(sg, i0, n, x);
-#pragma unroll
-        for (int k = 0; k < int(kEncPerThread); k++)
-            if (i0 + k < n) bits += ct.len[(x[k] >> 7) & 0xFFu];
-    }
-    for (int j = threadIdx.x; j < kPackWords; j += kEncThreads) s_words[j] = 0;
-    uint32_t chunk_total;
-    const uint32_t my_off = block_exclusive_scan<kEncThreads>(bits, s_warp, chunk_total);
-    const uint64_t S = chunk_start[blockIdx.x];
-    const uint32_t lead = uint32_t(S & 31u);
-
-    if (i0 < n) {
-        uint32_t q = lead + my_off;  // bit position relative to word S/32
-        uint8_t smb[kEncPerThread];
-#pragma unroll
-        for (int k = 0; k < int(kEncPerThread); k++) {
-            const uint64_t i = i0 + k;
-            const uint32_t xv = x[k];
-            smb[k] = uint8_t(((xv >> 8) & 0x80u) | (xv & 0x7Fu));
-            if (i >= n) continue;
-            const uint32_t e = (xv >> 7) & 0xFFu;
-            const uint32_t l = ct.len[e];
-            const uint32_t code = ct.code[e];
-            const uint32_t o = q & 31u;
-            if (o + l <= 32) {
-                atomicOr(&s_words[q >> 5], code << (32 - o - l));
-            } else {
-                atomicOr(&s_words[q >> 5], code >> (o + l - 32));
-                atomicOr(&s_words[(q >> 5) + 1], code << (64 - o - l));
-            }
-            // gaps and block offsets from the absolute start bit
-            const uint64_t s = (S & ~uint64_t(31)) + q;
-            const uint64_t last = s + l - 1;
-            if ((s & 63) != 0 && (s >> 6) != (last >> 6)) {
-                const uint64_t w = (s >> 6) + 1;
-                const uint32_t g = uint32_t(s + l - 64 * w);
-                const uint64_t gb = 5 * w;
+    stage_codes(sc, ct);
+    __syncthreads();
+    const uint64_t block_mask = (uint64_t(1) << log2_block_bits) - 1;
+    const uint64_t tofs = uint64_t(threadIdx.x) * kEncPerThread;
+    uint64_t c = blockIdx.x;
+    RawElems next = load_raw(sg, c * kEncChunk, c * kEncChunk + tofs, n);
+    for (; c < n_chunks; c += gridDim.x) {
+        const RawElems cur = next;
+        const uint64_t i0 = c * kEncChunk + tofs;
+        if (c + gridDim.x < n_chunks)
+            next = load_raw(sg, (c + gridDim.x) * kEncChunk, (c + gridDim.x) * kEncChunk + tofs, n);
+        uint32_t w8[kEncPerThread / 2];
+        uint32_t valid = 0, bits = 0;
+        if (i0 < n) {
+            raw_words(sg, cur, i0, n, w8);
+            const uint64_t left = n - i0;
+            valid = left < kEncPerThread ? uint32_t(left) : kEncPerThread;
+            bits = thread_bits(sc, w8, valid);
+        }
+        for (int j = threadIdx.x; j < kPackWords / 4; j += kEncThreads)
+            reinterpret_cast<uint4*>(s_words)[j] = make_uint4(0, 0, 0, 0);
+        uint32_t chunk_total;
+        const uint32_t my_off = block_exclusive_scan<kEncThreads>(bits, s_warp, chunk_total);
+        const uint64_t S = chunk_start[c];
+        const uint32_t lead = uint32_t(S & 31u);
+        const uint64_t Sb = S & ~block_mask;  // a thread-block (and window) boundary
+        // gap and output position for a code at relative start r (bits from
+        // Sb) of length l, element i, that covers a window boundary
+        const uint64_t gap_base = 5 * (Sb >> 6);
+        const uint64_t blk_base = Sb >> log2_block_bits;
+        auto window_event = [&](uint32_t r, uint32_t l, uint64_t i) {
+            if (r & 63u) {
+                const uint32_t wr = (r >> 6) + 1;
+                const uint32_t g = r + l - 64 * wr;
+                const uint64_t gb = gap_base + 5 * uint64_t(wr);
                 const uint32_t sh = uint32_t(gb & 31);
                 atomicOr(gaps32 + (gb >> 5), g << sh);
                 if (sh > 27) atomicOr(gaps32 + (gb >> 5) + 1, g >> (32 - sh));
             }
-            const uint64_t bb = s >> log2_block_bits;
-            if ((s & ((uint64_t(1) << log2_block_bits) - 1)) == 0) {
-                block_off[bb] = uint32_t(i);
-            } else if ((last >> log2_block_bits) != bb) {
-                block_off[bb + 1] = uint32_t(i + 1);
+            const uint32_t br = r >> log2_block_bits;
+            if ((r & uint32_t(block_mask)) == 0) {
+                block_off[blk_base + br] = uint32_t(i);
+            } else if (((r + l - 1) >> log2_block_bits) != br) {
+                block_off[blk_base + br + 1] = uint32_t(i + 1);
             }
-            if (i == n - 1) block_off[n_blocks] = uint32_t(n);
-            q += l;
+        };
+        // Append this thread's codes to the image.  A completed word is OR-ed
+        // in (the first may be shared with the previous thread).  Codes that
+        // cover a window boundary (at most 9 for 16 codes of <= 32 bits) are
+        // only noted in the thread's column of s_ev and handled after the
+        // loop, so the warp does not run that handler on every element.
+        auto pack_codes = [&](auto full_tag) {
+            constexpr bool kFull = decltype(full_tag)::value;  // all kEncPerThread elements valid
+            const uint32_t q = lead + my_off;  // bit position in the chunk image
+            uint32_t w = q >> 5, fill = q & 31u, cur_word = 0;
+            uint32_t u = uint32_t(S - Sb) + my_off + 63u;  // relative start + 63
+            uint32_t ne = 0;
+#pragma unroll
+            for (int k = 0; k < int(kEncPerThread); k++) {
+                if (!kFull && uint32_t(k) >= valid) break;
+                const uint2 ce = sc.e[(elem(w8, k) >> 7) & 0xFFu];
+                const uint32_t t = ce.x, l = ce.y;
+                cur_word |= t >> fill;
+                const uint32_t spill = __funnelshift_r(0u, t, fill);  // bits that did not fit
+                fill += l;
+                if (fill >= 32u) {
+                    atomicOr(&s_words[w], cur_word);
+                    w++;
+                    cur_word = spill;
+                    fill -= 32u;
+                }
+                const uint32_t nu = u + l;
+                if ((u ^ nu) >= 64u) s_ev[ne++][threadIdx.x] = (u << 10) | (l << 4) | uint32_t(k);
+                u = nu;
+            }
+            if (fill) atomicOr(&s_words[w], cur_word);
+            for (uint32_t j = 0; j < ne; j++) {
+                const uint32_t e = s_ev[j][threadIdx.x];
+                window_event((e >> 10) - 63u, (e >> 4) & 63u, i0 + (e & 15u));
+            }
+        };
+        if (valid == kEncPerThread)
+            pack_codes(std::true_type{});
+        else if (valid)
+            pack_codes(std::false_type{});
+        if (valid) {
+            if (n - i0 <= kEncPerThread) block_off[n_blocks] = uint32_t(n);
+            // sign+mantissa bytes: sign (bit 15) to bit 7, mantissa bits 6..0
+            uint32_t smw[kEncPerThread / 4];
+#pragma unroll
+            for (int j = 0; j < int(kEncPerThread / 4); j++) {
+                const uint32_t a = w8[2 * j], b = w8[2 * j + 1];
+                const uint32_t pa = ((a >> 8) & 0x00800080u) | (a & 0x007F007Fu);  // bytes 0 and 2
+                const uint32_t pb = ((b >> 8) & 0x00800080u) | (b & 0x007F007Fu);
+                smw[j] = __byte_perm(pa, pb, 0x6420);
+            }
+            if (valid == kEncPerThread) {
+                __stcs(reinterpret_cast<uint4*>(sm + i0), make_uint4(smw[0], smw[1], smw[2], smw[3]));
+            } else {
+#pragma unroll
+                for (int k = 0; k < int(kEncPerThread); k++)
+                    if (uint32_t(k) < valid) sm[i0 + k] = uint8_t(smw[k >> 2] >> (8 * (k & 3)));
+            }
         }
-        // sign+mantissa bytes
-        if (i0 + kEncPerThread <= n) {
-            uint4 v;
-            v.x = smb[0] | (smb[1] << 8) | (smb[2] << 16) | (uint32_t(smb[3]) << 24);
-            v.y = smb[4] | (smb[5] << 8) | (smb[6] << 16) | (uint32_t(smb[7]) << 24);
-            v.z = smb[8] | (smb[9] << 8) | (smb[10] << 16) | (uint32_t(smb[11]) << 24);
-            v.w = smb[12] | (smb[13] << 8) | (smb[14] << 16) | (uint32_t(smb[15]) << 24);
-            *reinterpret_cast<uint4*>(sm + i0) = v;
-        } else {
-            for (int k = 0; k < int(kEncPerThread); k++)
-                if (i0 + k < n) sm[i0 + k] = smb[k];
+        __syncthreads();
+        const uint32_t nwords = (lead + chunk_total + 31) >> 5;
+        const uint64_t W0 = S >> 5;
+        for (uint32_t j = threadIdx.x; j < nwords; j += kEncThreads) {
+            const uint32_t v = __byte_perm(s_words[j], 0, 0x0123);  // MSB-first bytes
+            if (j == 0 || j == nwords - 1) {
+                if (v) atomicOr(exp32 + W0 + j, v);
+            } else {
+                exp32[W0 + j] = v;
+            }
         }
+        __syncthreads();  // s_words and s_warp are reused by the next chunk
     }
-    __syncthreads();
-    const uint32_t nwords = (lead + chunk_total + 31) >> 5;
-    const uint64_t W0 = S >> 5;
-    for (uint32_t j = threadIdx.x; j < nwords; j += kEncThreads) {
-        const uint32_t v = __byte_perm(s_words[j], 0, 0x0123);  // MSB-first bytes
-        if (j == 0 || j == nwords - 1) {
-            if (v) atomicOr(exp32 + W0 + j, v);
-        } else {
-            exp32[W0 + j] = v;
-        }
-    }
+}
+
+// Persistent grid for an encode kernel: as many CTAs as can be resident on
+// every SM at once.
+template <typename Kernel>
+unsigned encode_grid(Kernel kernel, uint64_t chunks) {
+    int dev = 0, sms = 148, per_sm = 1;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kEncThreads, 0) != cudaSuccess || per_sm < 1)
+        per_sm = 1;
+    const uint64_t want = uint64_t(sms) * uint64_t(per_sm);
+    return unsigned(chunks < want ? chunks : want);
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -423,11 +604,11 @@ extern "C" df11_status df11_compress_encode(const void* const* d_segs, const df1
 
     const uint64_t chunks = (n + kEncChunk - 1) / kEncChunk;
     if (chunks >= (uint64_t(1) << 31)) return fail(DF11_ERR_TOO_LARGE, "too many chunks");
-    chunk_bits_kernel<<<unsigned(chunks), kEncThreads, 0, s>>>(sg, ct, n, w.chunk_bits);
+    chunk_bits_kernel<<<encode_grid(chunk_bits_kernel, chunks), kEncThreads, 0, s>>>(sg, ct, n, chunks, w.chunk_bits);
     chunk_scan_kernel<<<1, kScanThreads, 0, s>>>(w.chunk_bits, chunks, w.chunk_start);
     uint32_t log2_bb = 6;
     while ((1u << (log2_bb - 6)) < hdr->threads_per_block) log2_bb++;
-    pack_kernel<<<unsigned(chunks), kEncThreads, 0, s>>>(sg, ct, n, log2_bb, w.chunk_start,
+    pack_kernel<<<encode_grid(pack_kernel, chunks), kEncThreads, 0, s>>>(sg, ct, n, chunks, log2_bb, w.chunk_start,
                                                          reinterpret_cast<uint32_t*>(d_exp), d_sm,
                                                          reinterpret_cast<uint32_t*>(d_gaps), d_block_off,
                                                          hdr->n_blocks);
@@ -539,11 +720,11 @@ extern "C" df11_status df11_compress_encode_static(const void* const* d_segs, co
     if (n == 0) return DF11_OK;
 
     const uint64_t chunks = (n + kEncChunk - 1) / kEncChunk;
-    chunk_bits_kernel<<<unsigned(chunks), kEncThreads, 0, s>>>(sg, ct, n, chunk_bits);
+    chunk_bits_kernel<<<encode_grid(chunk_bits_kernel, chunks), kEncThreads, 0, s>>>(sg, ct, n, chunks, chunk_bits);
     chunk_scan_kernel<<<1, kScanThreads, 0, s>>>(chunk_bits, chunks, chunk_start);
     uint32_t log2_bb = 6;
     while ((1u << (log2_bb - 6)) < hdr->threads_per_block) log2_bb++;
-    pack_kernel<<<unsigned(chunks), kEncThreads, 0, s>>>(sg, ct, n, log2_bb, chunk_start,
+    pack_kernel<<<encode_grid(pack_kernel, chunks), kEncThreads, 0, s>>>(sg, ct, n, chunks, log2_bb, chunk_start,
                                                          reinterpret_cast<uint32_t*>(d_exp), d_sm,
                                                          reinterpret_cast<uint32_t*>(d_gaps), d_block_off,
                                                          hdr->n_blocks);
