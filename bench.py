@@ -456,6 +456,72 @@ def run_native(args, rank: int, world: int, local_rank: int) -> None:
     print(json.dumps(line), flush=True)
 
 
+def run_pipeline(args, local_rank: int) -> None:
+    """Decompress-into-consumer: Llama-3.1-70B-shaped blocks, each block's
+    matrices multiplied by a [tokens, in] BF16 activation (torch matmul) as
+    the consumer.  Times, per block: the consumer alone, the decode alone,
+    decode then consumer on one stream, and BlockPrefetcher (next block
+    decoded on a side stream, optionally on capped SMs).  Prints one JSON
+    line."""
+    import torch
+    import lossless_entropy_coded_dfloat11_b200 as df11
+    from lossless_entropy_coded_dfloat11_b200 import inputs as I
+
+    torch.cuda.set_device(local_rank)
+    df11.load_library()
+    streams = []
+    for b in range(args.pipeline_blocks):
+        w = I.llama_block(I.LLAMA_70B, seed_base=100 + 16 * b, device="cuda")
+        streams.append(df11.compress(w.tensors, names=w.names))
+        del w
+    n_max = max(cs.n_elems for cs in streams)
+    buf = torch.empty(n_max, dtype=torch.bfloat16, device="cuda")
+    act = torch.randn(args.tokens, I.LLAMA_70B["intermediate"], device="cuda").to(torch.bfloat16)
+    stream = torch.cuda.current_stream()
+
+    def consume(views):
+        for v in views:
+            if v.dim() == 2:
+                torch.matmul(act[:, : v.shape[1]], v.t())
+
+    def timed(fn, reps=3):
+        fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / (reps * len(streams))
+
+    first = streams[0].views(df11.decompress(streams[0], out=buf[: streams[0].n_elems]))
+    res = {"consumer_only": timed(lambda: [consume(first) for _ in streams]),
+           "decode_only": timed(lambda: [df11.decompress(cs, out=buf[: cs.n_elems]) for cs in streams])}
+
+    def serial():
+        for cs in streams:
+            consume(cs.views(df11.decompress(cs, out=buf[: cs.n_elems])))
+    res["serial"] = timed(serial)
+    for cap in [None] + args.pipeline_sms:
+        pf = df11.BlockPrefetcher(streams, max_sms=cap)
+        res["prefetch_all_sms" if cap is None else f"prefetch_{cap}_sms"] = timed(
+            lambda: [consume(views) for _, views in pf])
+    best = min(v for k, v in res.items() if k.startswith("prefetch"))
+    hidden = (res["serial"] - best) / min(res["decode_only"], res["consumer_only"])
+    flops = 2 * args.tokens * sum(cs.n_elems for cs in streams) / len(streams)
+    line = {"metric": "decompress-into-consumer, ms per transformer block", "unit": "ms",
+            "higher_is_better": False, "n_gpus": 1, "data": "synthetic",
+            "config": {"workload": "llama3.1-70b-blocks (855,654,400 weights each), consumer: "
+                                   f"[{args.tokens}, in] x [in, out] BF16 matmul per matrix",
+                       "blocks": len(streams), "tokens": args.tokens},
+            "ms_per_block": res, "best_prefetch_ms": best,
+            "decode_hidden_frac": hidden,
+            "consumer_tflops": flops / (res["consumer_only"] * 1e-3) / 1e12,
+            "when": datetime.datetime.now(datetime.timezone.utc).isoformat(timespec="seconds")}
+    print(json.dumps(line), flush=True)
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -472,6 +538,11 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-compress", action="store_true", help="skip timing the compress call")
     ap.add_argument("--compress-repeats", type=int, default=5)
+    ap.add_argument("--pipeline", action="store_true",
+                    help="time decompress-into-consumer (BlockPrefetcher) instead of the decode alone")
+    ap.add_argument("--pipeline-blocks", type=int, default=4)
+    ap.add_argument("--tokens", type=int, default=1024, help="consumer activation rows (--pipeline)")
+    ap.add_argument("--pipeline-sms", type=int, nargs="*", default=[16, 32, 64])
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("at least 3 warm-up steps")
@@ -481,6 +552,10 @@ def main(argv=None):
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         run_reference(args, rank, world)
+        return
+    if args.pipeline:
+        if world == 1:
+            run_pipeline(args, local_rank)
         return
     if world > 1:
         import torch

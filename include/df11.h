@@ -195,6 +195,22 @@ df11_status df11_decompress(const df11_header* hdr, const uint8_t* d_exp, const 
                             const void* d_lut, uint16_t* d_out, uint32_t* d_status,
                             void* stream);
 
+/* df11_decompress on at most max_sms SMs.  The pages decompress a
+ * transformer block's matrices as one batch right before that block's
+ * forward pass and drop the BF16 copy after the matrix multiplications
+ * ("Descompressao adaptada para inferencia em GPU", "Descompressao por bloco
+ * de transformer"); decoding block i+1 while block i computes on another
+ * CUDA stream is our extension of that pattern, and this entry point lets
+ * the decode leave the remaining SMs to the computation (the decode kernel
+ * keeps one CTA resident per SM for the whole launch, using all of that SM's
+ * registers).  Same arguments, result and asynchrony as df11_decompress;
+ * max_sms above the device's SM count means all SMs; max_sms = 0 is
+ * DF11_ERR_INVALID. */
+df11_status df11_decompress_sms(const df11_header* hdr, const uint8_t* d_exp, const uint8_t* d_sm,
+                                const uint8_t* d_gaps, const uint32_t* d_block_off,
+                                const void* d_lut, uint16_t* d_out, uint32_t* d_status,
+                                uint32_t max_sms, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -198,19 +198,24 @@ def to_host(cs: CompressedStream) -> dict:
 
 
 def decompress(cs: CompressedStream, out: torch.Tensor | None = None, status: torch.Tensor | None = None,
-               stream=None) -> torch.Tensor:
+               stream=None, max_sms: int | None = None) -> torch.Tensor:
     """One kernel launch rebuilding all n_elems BF16 values of the stream.
     Asynchronous; `out` (bfloat16, n_elems, contiguous) may be reused across
     calls.  `status` (int32 device word, zeroed by the caller) receives
-    DF11_ERR_CORRUPT if the stream disagrees with its metadata."""
+    DF11_ERR_CORRUPT if the stream disagrees with its metadata.  `max_sms`
+    caps the SMs the decode occupies (df11_decompress_sms), leaving the rest
+    to kernels on other streams."""
     n = cs.n_elems
     if out is None:
         out = torch.empty(max(n, 1), dtype=torch.bfloat16, device=cs.exp.device)[:n]
     if out.dtype != torch.bfloat16 or not out.is_contiguous() or out.numel() < n:
         raise ValueError("out must be a contiguous bfloat16 tensor with n_elems elements")
-    B.call("df11_decompress", ctypes.byref(cs.header), _ptr(cs.exp), _ptr(cs.sm), _ptr(cs.gaps),
-           _ptr(cs.block_off), _ptr(cs.lut), _ptr(out),
-           _ptr(status) if status is not None else ctypes.c_void_p(0), _stream_handle(stream))
+    args = (ctypes.byref(cs.header), _ptr(cs.exp), _ptr(cs.sm), _ptr(cs.gaps), _ptr(cs.block_off),
+            _ptr(cs.lut), _ptr(out), _ptr(status) if status is not None else ctypes.c_void_p(0))
+    if max_sms is None:
+        B.call("df11_decompress", *args, _stream_handle(stream))
+    else:
+        B.call("df11_decompress_sms", *args, ctypes.c_uint32(max_sms), _stream_handle(stream))
     return out
 
 

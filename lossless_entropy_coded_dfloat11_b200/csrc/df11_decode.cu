@@ -751,7 +751,7 @@ constexpr int kWarpsShort = 32;  // every code has 2 bits or more
 
 template <typename Kernel>
 df11_status launch_persistent(Kernel kernel, int slot, int threads, size_t smem, uint64_t work_units,
-                              const DecodeArgs& a, cudaStream_t stream) {
+                              uint32_t max_sms, const DecodeArgs& a, cudaStream_t stream) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev)
         return fail(DF11_ERR_CUDA, "cudaGetDevice failed");
@@ -768,7 +768,8 @@ df11_status launch_persistent(Kernel kernel, int slot, int threads, size_t smem,
         li.sms = sms;
         li.ready.store(1, std::memory_order_release);
     }
-    const uint64_t want = uint64_t(li.per_sm) * uint64_t(li.sms);
+    const uint64_t sms = max_sms < uint32_t(li.sms) ? max_sms : uint32_t(li.sms);
+    const uint64_t want = uint64_t(li.per_sm) * sms;
     const unsigned grid = unsigned(work_units < want ? work_units : want);
     kernel<<<grid, threads, smem, stream>>>(a);
     const cudaError_t e = cudaGetLastError();
@@ -777,22 +778,22 @@ df11_status launch_persistent(Kernel kernel, int slot, int threads, size_t smem,
 }
 
 template <int T>
-df11_status launch_block(const DecodeArgs& a, cudaStream_t s, int slot) {
+df11_status launch_block(const DecodeArgs& a, cudaStream_t s, int slot, uint32_t max_sms) {
     const size_t smem = kLutBytes + block_stage_bytes<T>() + 4 * (T / 32);
-    return launch_persistent(decode_block_kernel<T>, slot, T, smem, a.n_blocks, a, s);
+    return launch_persistent(decode_block_kernel<T>, slot, T, smem, a.n_blocks, max_sms, a, s);
 }
 
 template <int WARPS, int MIN_LEN>
-df11_status launch_warp_variant(const DecodeArgs& a, cudaStream_t s, int slot) {
+df11_status launch_warp_variant(const DecodeArgs& a, cudaStream_t s, int slot, uint32_t max_sms) {
     constexpr size_t smem = kCompactBytes + size_t(WARPS) * WarpLayout<MIN_LEN>::kBytes;
     static_assert(smem <= 227 * 1024, "shared memory per CTA");
     const uint64_t ctas = (uint64_t(a.n_blocks) + WARPS - 1) / WARPS;
-    return launch_persistent(decode_warp_kernel<WARPS, MIN_LEN>, slot, WARPS * 32, smem, ctas, a, s);
+    return launch_persistent(decode_warp_kernel<WARPS, MIN_LEN>, slot, WARPS * 32, smem, ctas, max_sms, a, s);
 }
 
-df11_status launch_warp(const DecodeArgs& a, cudaStream_t s, uint32_t min_len) {
-    if (min_len >= 2) return launch_warp_variant<kWarpsShort, 2>(a, s, 6);
-    return launch_warp_variant<kWarpsLong, 1>(a, s, 0);
+df11_status launch_warp(const DecodeArgs& a, cudaStream_t s, uint32_t min_len, uint32_t max_sms) {
+    if (min_len >= 2) return launch_warp_variant<kWarpsShort, 2>(a, s, 6, max_sms);
+    return launch_warp_variant<kWarpsLong, 1>(a, s, 0, max_sms);
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -823,10 +824,12 @@ df11_status check_header(const df11_header* h) {
 
 using namespace df11;
 
-extern "C" df11_status df11_decompress(const df11_header* hdr, const uint8_t* d_exp, const uint8_t* d_sm,
-                                       const uint8_t* d_gaps, const uint32_t* d_block_off,
-                                       const void* d_lut, uint16_t* d_out, uint32_t* d_status,
-                                       void* stream) {
+namespace df11 {
+namespace {
+
+df11_status decompress_on(const df11_header* hdr, const uint8_t* d_exp, const uint8_t* d_sm,
+                          const uint8_t* d_gaps, const uint32_t* d_block_off, const void* d_lut,
+                          uint16_t* d_out, uint32_t* d_status, uint32_t max_sms, void* stream) {
     df11_status st = check_header(hdr);
     if (st != DF11_OK) return st;
     if (hdr->n_elems == 0) return DF11_OK;
@@ -853,13 +856,31 @@ extern "C" df11_status df11_decompress(const df11_header* hdr, const uint8_t* d_
             uint32_t min_len = 32;
             for (int v = 0; v < 256; v++)
                 if (hdr->code_len[v] && hdr->code_len[v] < min_len) min_len = hdr->code_len[v];
-            return launch_warp(a, s, min_len);
+            return launch_warp(a, s, min_len, max_sms);
         }
-        case 64: return launch_block<64>(a, s, 1);
-        case 128: return launch_block<128>(a, s, 2);
-        case 256: return launch_block<256>(a, s, 3);
-        case 512: return launch_block<512>(a, s, 4);
-        case 1024: return launch_block<1024>(a, s, 5);
+        case 64: return launch_block<64>(a, s, 1, max_sms);
+        case 128: return launch_block<128>(a, s, 2, max_sms);
+        case 256: return launch_block<256>(a, s, 3, max_sms);
+        case 512: return launch_block<512>(a, s, 4, max_sms);
+        case 1024: return launch_block<1024>(a, s, 5, max_sms);
         default: return fail(DF11_ERR_INVALID, "threads_per_block %u", hdr->threads_per_block);
     }
+}
+
+}  // namespace
+}  // namespace df11
+
+extern "C" df11_status df11_decompress(const df11_header* hdr, const uint8_t* d_exp, const uint8_t* d_sm,
+                                       const uint8_t* d_gaps, const uint32_t* d_block_off,
+                                       const void* d_lut, uint16_t* d_out, uint32_t* d_status,
+                                       void* stream) {
+    return decompress_on(hdr, d_exp, d_sm, d_gaps, d_block_off, d_lut, d_out, d_status, UINT32_MAX, stream);
+}
+
+extern "C" df11_status df11_decompress_sms(const df11_header* hdr, const uint8_t* d_exp, const uint8_t* d_sm,
+                                           const uint8_t* d_gaps, const uint32_t* d_block_off,
+                                           const void* d_lut, uint16_t* d_out, uint32_t* d_status,
+                                           uint32_t max_sms, void* stream) {
+    if (max_sms == 0) return fail(DF11_ERR_INVALID, "df11_decompress_sms: max_sms must be at least 1");
+    return decompress_on(hdr, d_exp, d_sm, d_gaps, d_block_off, d_lut, d_out, d_status, max_sms, stream);
 }
