@@ -18,7 +18,7 @@ from . import _binding as B
 
 # Thread blocks of one warp: the decode kernel then needs no CTA-wide barrier
 # (the block offsets cost 4 bytes per 32 windows, ~0.2% of the stream).
-DEFAULT_THREADS_PER_BLOCK = 32
+DEFAULT_THREADS_PER_BLOCK = 64
 
 
 def _stream_handle(stream) -> ctypes.c_void_p:

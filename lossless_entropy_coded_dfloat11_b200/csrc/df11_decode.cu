@@ -357,15 +357,15 @@ __device__ __forceinline__ bool block_consistent(uint32_t off0, uint32_t off1, u
 // in the staging buffer and the warp carries its bytes over; only the first
 // and last unit of a run need element-wise stores.
 // ---------------------------------------------------------------------------
-// Per-warp buffers depend on the shortest code length: a 64-bit window
-// holds at most 64 / min_len code starts, plus up to three symbols decoded
-// past its end.  The slots are stored transposed (word k of lane L at word
+// Per-warp buffers depend on the shortest code length and the windows per
+// lane: a lane's 64 WPL bits hold at most 64 WPL / min_len code starts, plus
+// up to three symbols decoded past their end.  The slots are stored transposed (word k of lane L at word
 // 32k + L), so each lane always uses the same bank: the decode loop's
 // stores, which happen at a different word offset in every lane, and the
 // copy's loads are free of bank conflicts.
-template <int MIN_LEN>
+template <int MIN_LEN, int WPL>
 struct WarpLayout {
-    static constexpr uint32_t kMaxCodes = 64 / MIN_LEN;
+    static constexpr uint32_t kMaxCodes = 64 * WPL / MIN_LEN;
     static constexpr uint32_t kSlotWords = (kMaxCodes + 3 + 3) / 4;
     static constexpr uint32_t kSlots = 32 * kSlotWords * 4;
     static constexpr uint32_t kStage = 32 * kMaxCodes + 64;  // + head (15) + spill, rounded
@@ -440,23 +440,101 @@ __device__ __forceinline__ void decode_half(uint32_t& acc, uint32_t& pend, uint3
 #undef DF11_STEP
 }
 
-// Decode the window into the (transposed) slot at shared address slot_s;
-// returns the number of codes that start in the window.
-__device__ __forceinline__ uint32_t decode_window_once(const Window& w, const Tables& t, uint32_t dtab_s,
-                                                       uint32_t slot_s, const uint16_t* ltab, uint32_t long_base,
-                                                       uint32_t long_count, bool& bad) {
-    const uint32_t lim1 = min(w.wend, 32u) << 16;
-    const uint32_t lim2 = w.wend << 16;
+// The bits one lane of the warp kernel decodes: WPL consecutive 8-byte
+// windows read as one run of 64 WPL bits, from the gap of the first window.
+// The codes that start in the later windows are exactly the ones the run
+// reaches, so their gaps are not needed.
+template <int WPL>
+struct LaneWindow {
+    uint32_t w[2 * WPL + 1];  // 64 WPL stream bits and a 32-bit lookahead, MSB first
+    uint32_t start;           // first code start (the first window's gap)
+    uint32_t wend;            // end of the run inside the stream, 0..64 WPL
+};
+
+template <int WPL>
+struct RawLane {
+    uint32_t v[2 * WPL];
+    uint32_t look;  // lookahead word (WPL = 2: loaded by lane 31 only)
+    uint32_t glo, ghi;
+};
+
+// tg0 = the lane's first window; its gap field sits in gap words gword, gword + 1.
+template <int WPL>
+__device__ __forceinline__ RawLane<WPL> load_lane(const DecodeArgs& a, uint32_t tg0, uint32_t gword,
+                                                  uint32_t lane) {
+    RawLane<WPL> r;
+    if (tg0 < a.n_threads) {
+        const uint8_t* base = a.exp + 8 * size_t(tg0);
+        if constexpr (WPL == 2) {
+            const uint4 q = __ldg(reinterpret_cast<const uint4*>(base));
+            r.v[0] = q.x; r.v[1] = q.y; r.v[2] = q.z; r.v[3] = q.w;
+            r.look = lane == 31 ? __ldg(reinterpret_cast<const uint32_t*>(base + 16)) : 0u;
+        } else {
+            const uint2 q = __ldg(reinterpret_cast<const uint2*>(base));
+            r.v[0] = q.x; r.v[1] = q.y;
+            r.look = __ldg(reinterpret_cast<const uint32_t*>(base + 8));
+        }
+        r.glo = __ldg(a.gaps + gword);
+        r.ghi = __ldg(a.gaps + gword + 1);
+    } else {
+#pragma unroll
+        for (int k = 0; k < 2 * WPL; k++) r.v[k] = 0;
+        r.look = r.glo = r.ghi = 0;
+    }
+    return r;
+}
+
+// Called by all 32 lanes of the warp together.
+template <int WPL>
+__device__ __forceinline__ LaneWindow<WPL> finish_lane(const DecodeArgs& a, const RawLane<WPL>& r, uint32_t tg0,
+                                                       uint32_t gshift, uint32_t lane) {
+    LaneWindow<WPL> w;
+#pragma unroll
+    for (int k = 0; k < 2 * WPL; k++) w.w[k] = bswap32(r.v[k]);
+    if constexpr (WPL == 2) {
+        const uint32_t next = __shfl_down_sync(0xFFFFFFFFu, r.v[0], 1);  // the next lane's first word
+        w.w[2 * WPL] = bswap32(lane == 31 ? r.look : next);
+    } else {
+        w.w[2 * WPL] = bswap32(r.look);
+    }
+    w.start = __funnelshift_r(r.glo, r.ghi, gshift) & 31u;
+    // every window but the stream's last is whole
+    const uint32_t last = a.n_threads - 1;
+    const uint32_t whole = tg0 < last ? min(uint32_t(WPL), last - tg0) : 0u;
+    const bool has_last = tg0 <= last && last < tg0 + WPL;
+    w.wend = 64 * whole + (has_last ? a.last_wend : 0u);
+    return w;
+}
+
+// Decode the lane's run into its (transposed) slot at shared address slot_s;
+// returns the number of codes that start in the run.
+template <int WPL>
+__device__ __forceinline__ uint32_t decode_lane_once(const LaneWindow<WPL>& w, const Tables& t, uint32_t dtab_s,
+                                                     uint32_t slot_s, const uint16_t* ltab, uint32_t long_base,
+                                                     uint32_t long_count, bool& bad) {
     // bit position << 16 | 8 x bytes produced; low five bits = placement shift
     uint32_t acc = w.start << 16;
     uint32_t pend = 0, wad = slot_s, idx = 0, ylast = 0;
     for (;;) {
-        decode_half(acc, pend, wad, idx, ylast, w.w0, w.w1, lim1, dtab_s);
-        decode_half(acc, pend, wad, idx, ylast, w.w1, w.w2, lim2, dtab_s);
+#pragma unroll
+        for (int k = 0; k < 2 * WPL; k++)  // one loop per 32 bits, each peeking at one word pair
+            decode_half(acc, pend, wad, idx, ylast, w.w[k], w.w[k + 1], min(w.wend, 32u * (k + 1)) << 16,
+                        dtab_s);
         if (acc < (kEscape << 16)) break;
         // a code longer than the table: undo the escape, take it from level 2
         acc -= kEscape << 16;
-        const uint32_t pk = peek32(w.w0, w.w1, w.w2, acc >> 16);
+        const uint32_t pos = acc >> 16;
+        // the word pair holding bit pos, by selects (an indexed pick would
+        // put the window in local memory)
+        const bool odd = (pos >> 5) & 1u;
+        uint32_t hi = odd ? w.w[1] : w.w[0], lo = odd ? w.w[2] : w.w[1];
+        if constexpr (WPL == 2) {
+            if ((pos >> 5) & 2u) {
+                hi = odd ? w.w[3] : w.w[2];
+                lo = odd ? w.w[4] : w.w[3];
+            }
+        }
+        const uint32_t pk = __funnelshift_l(lo, hi, pos);
         const uint32_t li = (pk >> (32 - kLongBits)) - long_base;
         const uint32_t le = li < long_count ? uint32_t(ltab[li]) : 0u;
         int l;
@@ -519,9 +597,9 @@ __device__ __forceinline__ uint32_t copy_slot(const uint32_t* slot, uint32_t* st
     return first;
 }
 
-template <int WARPS, int MIN_LEN>
+template <int WARPS, int MIN_LEN, int WPL>
 __global__ void __launch_bounds__(WARPS * 32, 1) decode_warp_kernel(const DecodeArgs a) {
-    using L = WarpLayout<MIN_LEN>;
+    using L = WarpLayout<MIN_LEN, WPL>;
     extern __shared__ __align__(16) uint8_t smem[];
     copy_compact_tables(smem, a.lut, WARPS * 32);
     __syncthreads();
@@ -542,9 +620,10 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_warp_kernel(const Decode
     uint32_t* slot = reinterpret_cast<uint32_t*>(wbase) + lane;
     const uint32_t slot_s = uint32_t(__cvta_generic_to_shared(slot));
     uint8_t* stage = wbase + L::kSlots;
-    // the gap field of window 32b + lane lies in the block's five gap words
-    const uint32_t lane_gword = (5 * lane) >> 5;
-    const uint32_t lane_gshift = (5 * lane) & 31u;
+    // the gap field of the lane's first window, WPL (32b + lane), lies in the
+    // block's 5 WPL gap words
+    const uint32_t lane_gword = (5 * WPL * lane) >> 5;
+    const uint32_t lane_gshift = (5 * WPL * lane) & 31u;
 
     // this warp's run of thread blocks [b, b_end)
     const uint32_t nw = gridDim.x * WARPS;
@@ -553,10 +632,10 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_warp_kernel(const Decode
     uint32_t b = g * per + (g < extra ? g : extra);
     const uint32_t b_end = b + per + (g < extra ? 1u : 0u);
 
-    RawWindow nraw{};
+    RawLane<WPL> nraw{};
     uint32_t noff0 = 0, noff1 = 0;
     if (b < b_end) {
-        nraw = load_window(a, 32 * b + lane, 5 * b + lane_gword);
+        nraw = load_lane<WPL>(a, WPL * (32 * b + lane), 5 * WPL * b + lane_gword, lane);
         noff0 = __ldg(a.off + b);
         noff1 = __ldg(a.off + b + 1);
     }
@@ -564,11 +643,11 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_warp_kernel(const Decode
     uint2 carry = make_uint2(0, 0);  // staging bytes of the unit left by the previous block
     bool have_carry = false;
     while (b < b_end) {
-        const RawWindow raw = nraw;
+        const RawLane<WPL> raw = nraw;
         const uint32_t off0 = noff0, off1 = noff1;
         const bool more = b + 1 < b_end;
         if (more) {  // prefetch the next block (its first position is off1)
-            nraw = load_window(a, 32 * (b + 1) + lane, 5 * (b + 1) + lane_gword);
+            nraw = load_lane<WPL>(a, WPL * (32 * (b + 1) + lane), 5 * WPL * (b + 1) + lane_gword, lane);
             noff0 = off1;
             noff1 = __ldg(a.off + b + 2);
         }
@@ -583,14 +662,17 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_warp_kernel(const Decode
         const uint32_t uw = keep_tail && u1 > u0 ? u1 - 1 : u1;
         const bool use_carry = have_carry && head != 0;
         const uint32_t lo = use_carry ? (off0 & ~7u) : off0;
-        uint2 sv[4];
+        // sign+mantissa units requested before the decode: 4 rounds of 32
+        // (a 32-window block has ~100 units), 7 for two windows per lane
+        constexpr int kPre = WPL == 1 ? 4 : 7;
+        uint2 sv[kPre];
 #pragma unroll
-        for (int r = 0; r < 4; r++)
+        for (int r = 0; r < kPre; r++)
             sv[r] = u0 + lane + 32 * r < uw ? __ldcs(sm8 + u0 + lane + 32 * r) : make_uint2(0, 0);
 
-        const Window w = finish_window(a, raw, 32 * b + lane, lane_gshift);
+        const LaneWindow<WPL> w = finish_lane<WPL>(a, raw, WPL * (32 * b + lane), lane_gshift, lane);
         bool bad = false;
-        const uint32_t cnt = decode_window_once(w, t, dtab_s, slot_s, ltab, long_base, long_count, bad);
+        const uint32_t cnt = decode_lane_once<WPL>(w, t, dtab_s, slot_s, ltab, long_base, long_count, bad);
         uint32_t incl = cnt;
 #pragma unroll
         for (int d = 1; d < 32; d <<= 1) {
@@ -629,7 +711,12 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_warp_kernel(const Decode
                 if (lane + 32 < nu) merge_store8<256, 512>(ev_s, sv[1], dst, m);
                 if (lane + 64 < nu) merge_store8<512, 1024>(ev_s, sv[2], dst, m);
                 if (lane + 96 < nu) merge_store8<768, 1536>(ev_s, sv[3], dst, m);
-                for (uint32_t k = 128; lane + k < nu; k += 32)
+                if constexpr (kPre == 7) {
+                    if (lane + 128 < nu) merge_store8<1024, 2048>(ev_s, sv[4], dst, m);
+                    if (lane + 160 < nu) merge_store8<1280, 2560>(ev_s, sv[5], dst, m);
+                    if (lane + 192 < nu) merge_store8<1536, 3072>(ev_s, sv[6], dst, m);
+                }
+                for (uint32_t k = 32 * kPre; lane + k < nu; k += 32)
                     merge_store8(ev_s + 8 * k, __ldcs(sm8 + u0 + lane + k), dst + k, m);
             } else {
                 const uint32_t uf = (lo + 7) >> 3, ul = off1 >> 3;  // whole units: [uf, ul)
@@ -641,9 +728,9 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_warp_kernel(const Decode
                         merge_unit(ev[k], s8, u, lo, off1, a.out);
                 };
 #pragma unroll
-                for (int r = 0; r < 4; r++)
+                for (int r = 0; r < kPre; r++)
                     if (lane + 32 * r < nu) unit(lane + 32 * r, sv[r]);
-                for (uint32_t k = lane + 128; k < nu; k += 32) unit(k, __ldcs(sm8 + u0 + k));
+                for (uint32_t k = lane + 32 * kPre; k < nu; k += 32) unit(k, __ldcs(sm8 + u0 + k));
             }
             if (keep_tail) carry = ev[u1 - 1 - u0];
             have_carry = keep_tail;
@@ -741,7 +828,7 @@ struct LaunchInfo {
     int sms = 0;
 };
 constexpr int kMaxDev = 64;
-LaunchInfo g_info[kMaxDev][7];  // [device][variant]
+LaunchInfo g_info[kMaxDev][8];  // [device][variant]
 
 // One CTA of 32 warps per SM: all warps share one copy of the tables, and
 // the register budget (64 per thread) leaves the decode loop unconstrained;
@@ -783,17 +870,18 @@ df11_status launch_block(const DecodeArgs& a, cudaStream_t s, int slot, uint32_t
     return launch_persistent(decode_block_kernel<T>, slot, T, smem, a.n_blocks, max_sms, a, s);
 }
 
-template <int WARPS, int MIN_LEN>
+template <int WARPS, int MIN_LEN, int WPL>
 df11_status launch_warp_variant(const DecodeArgs& a, cudaStream_t s, int slot, uint32_t max_sms) {
-    constexpr size_t smem = kCompactBytes + size_t(WARPS) * WarpLayout<MIN_LEN>::kBytes;
+    constexpr size_t smem = kCompactBytes + size_t(WARPS) * WarpLayout<MIN_LEN, WPL>::kBytes;
     static_assert(smem <= 227 * 1024, "shared memory per CTA");
     const uint64_t ctas = (uint64_t(a.n_blocks) + WARPS - 1) / WARPS;
-    return launch_persistent(decode_warp_kernel<WARPS, MIN_LEN>, slot, WARPS * 32, smem, ctas, max_sms, a, s);
+    return launch_persistent(decode_warp_kernel<WARPS, MIN_LEN, WPL>, slot, WARPS * 32, smem, ctas, max_sms, a, s);
 }
 
+// T = 32: one window per lane.
 df11_status launch_warp(const DecodeArgs& a, cudaStream_t s, uint32_t min_len, uint32_t max_sms) {
-    if (min_len >= 2) return launch_warp_variant<kWarpsShort, 2>(a, s, 6, max_sms);
-    return launch_warp_variant<kWarpsLong, 1>(a, s, 0, max_sms);
+    if (min_len >= 2) return launch_warp_variant<kWarpsShort, 2, 1>(a, s, 6, max_sms);
+    return launch_warp_variant<kWarpsLong, 1, 1>(a, s, 0, max_sms);
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -851,14 +939,14 @@ df11_status decompress_on(const df11_header* hdr, const uint8_t* d_exp, const ui
     a.n_blocks = uint32_t(hdr->n_blocks);
     a.last_wend = uint32_t(hdr->total_bits - 64 * (hdr->n_threads - 1));
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint32_t min_len = 32;
+    for (int v = 0; v < 256; v++)
+        if (hdr->code_len[v] && hdr->code_len[v] < min_len) min_len = hdr->code_len[v];
     switch (hdr->threads_per_block) {
-        case 32: {
-            uint32_t min_len = 32;
-            for (int v = 0; v < 256; v++)
-                if (hdr->code_len[v] && hdr->code_len[v] < min_len) min_len = hdr->code_len[v];
-            return launch_warp(a, s, min_len, max_sms);
-        }
-        case 64: return launch_block<64>(a, s, 1, max_sms);
+        case 32: return launch_warp(a, s, min_len, max_sms);
+        case 64:  // two windows per lane when every code has 2 bits or more (the slots then fit)
+            if (min_len >= 2) return launch_warp_variant<kWarpsShort, 2, 2>(a, s, 7, max_sms);
+            return launch_block<64>(a, s, 1, max_sms);
         case 128: return launch_block<128>(a, s, 2, max_sms);
         case 256: return launch_block<256>(a, s, 3, max_sms);
         case 512: return launch_block<512>(a, s, 4, max_sms);

@@ -48,7 +48,7 @@ namespace df11 {
 // ---------------------------------------------------------------------------
 constexpr uint32_t kLutMagic = 0x31314644u;  // "DF11"
 constexpr int kPeekBits = 12;
-constexpr uint32_t kEscape = 128;            // > any bit position inside a window + K
+constexpr uint32_t kEscape = 256;            // > any bit position a thread decodes (<= 128) + K
 constexpr uint32_t kDecodeSyms = 4;          // symbols per decode-table entry
 
 struct LutHeader {

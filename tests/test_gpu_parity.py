@@ -90,6 +90,16 @@ def test_edge_sweep(idx, dist):
     both_directions(inputs.edge_case(n, dist, 500 + idx))
 
 
+@pytest.mark.parametrize("dist", inputs.EDGE_DISTS)
+@pytest.mark.parametrize("n", [1, 33, 127, 4097, 65537, (1 << 20) + 7])
+def test_edge_cases_one_window_per_lane(n, dist):
+    # the sweep above runs the default T = 64 (two windows per lane when every
+    # code has 2 bits or more, the block kernel when a code is 1 bit long);
+    # T = 32 streams take the one-window warp kernel, whose 1-bit-code variant
+    # the 99.9%-one-exponent distribution reaches
+    both_directions(inputs.edge_case(n, dist, 900 + n % 97), T=32)
+
+
 def test_all_bf16_patterns():
     both_directions(inputs.all_patterns())
 

@@ -142,7 +142,7 @@ def test_header_validation():
 
 
 PEEK_BITS = 12
-ESCAPE = 128
+ESCAPE = 256
 # table offsets: 64-byte header, lj_end u64[33], delta u32[33], syms u8[256],
 # then count u32[4096], mask u16[4096], decode (u32, u32)[4096]
 OFF_COUNT = 736
