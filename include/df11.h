@@ -76,7 +76,7 @@ typedef enum {
 typedef struct {
     uint32_t version;            /* DF11_VERSION                               */
     uint32_t window_bytes;       /* 8                                          */
-    uint32_t threads_per_block;  /* T: 64, 128, 256, 512 or 1024               */
+    uint32_t threads_per_block;  /* T: 32, 64, ..., 1024 (library default 64) */
     uint32_t max_code_len;       /* L used to build the code, 1..32            */
     uint64_t n_elems;            /* BF16 elements, < 2^32                      */
     uint64_t total_bits;         /* bits in EncodedExponent                    */
@@ -114,7 +114,7 @@ df11_status df11_code_lengths(const uint64_t* hist, uint32_t max_code_len, uint8
  *   code_len[256]       in: lengths; must form a prefix code (Kraft <= 1,
  *                           equality required for >= 2 present values)
  *   n_elems, total_bits in: element count (< 2^32) and stream length in bits
- *   threads_per_block   in: T (64..1024, power of two)
+ *   threads_per_block   in: T (32..1024, power of two)
  *   seg_counts[n_segs]  in: elements per segment, summing to n_elems; NULL
  *                           with n_segs = 1 means one segment
  * Validates and fills every size field, including bytes_lut. */

@@ -13,28 +13,31 @@
 // B200 specifics:
 //   * persistent grid: the decode tables are copied to shared memory once
 //     per CTA and serve every thread block of the stream;
-//   * thread blocks of 32 threads (T = 32) are decoded by one warp each, with
-//     no CTA barrier at all: the prefix sum is five shuffles and the staging
-//     buffer is the warp's own; larger T use a block-wide scan;
+//   * thread blocks of T = 32 or 64 threads are decoded by one warp each,
+//     with no CTA barrier at all: the prefix sum is five shuffles and the
+//     staging buffer is the warp's own; for T = 64 each lane decodes its two
+//     windows as one 128-bit run from the first window's gap (the second
+//     window's codes are the ones the run reaches); larger T use a
+//     block-wide scan;
 //   * software pipelining: the next block's window, gap and output positions
 //     are loaded while the current one is decoded, and the current block's
 //     sign+mantissa bytes are requested before its decode starts;
 //   * the decode loops keep (bit position << 16 | counter) in one register
-//     and advance both with one add; the loops run separately over the first
-//     and second 32 bits of the window so each peek is one funnel shift; codes
+//     and advance both with one add; one loop runs per 32 bits of the run so
+//     each peek is one funnel shift of a word pair; codes
 //     longer than the 12-bit tables leave through an escape value that pushes
 //     the bit position out of the window, so the fast loops have one test;
 //   * symbols are gathered in a register pair and leave as aligned 32-bit
 //     words; a thread's first word, shared with the previous thread, is
-//     written byte-wise after a barrier.  The T = 32 kernel decodes each
+//     written byte-wise after a barrier.  The warp kernel decodes each
 //     window only once, into a per-thread shared-memory slot, and copies the
-//     slot into place after the scan; larger T decode twice (count, then
-//     decode into place);
+//     slot into place after the scan; the block kernel decodes twice (count,
+//     then decode into place);
 //   * exponents are staged rotated right by one bit, so the merge is two
-//     bit-selects and two byte-permutes per four elements.  The T = 32
-//     kernel merges 8-element units (8-byte shared load, 8-byte streaming
-//     load, one 16-byte streaming store; one store instruction of a warp
-//     covers 512 contiguous bytes), larger T merge 16-element chunks.
+//     bit-selects and two byte-permutes per four elements.  The warp kernel
+//     merges 8-element units (8-byte shared load, 8-byte streaming load, one
+//     16-byte streaming store; one store instruction of a warp covers 512
+//     contiguous bytes), the block kernel 16-element chunks.
 // Indices are 32-bit: n_elems < 2^32 and codes of at most 32 bits keep the
 // window count below 2^31.
 #include <cuda_runtime.h>
@@ -337,12 +340,12 @@ __device__ __forceinline__ bool block_consistent(uint32_t off0, uint32_t off1, u
 }
 
 // ---------------------------------------------------------------------------
-// T = 32: one warp decodes one thread block at a time; no CTA barrier after
-// the table copy.
+// T = 32 and T = 64: one warp decodes one thread block at a time, each lane
+// WPL = T / 32 consecutive windows; no CTA barrier after the table copy.
 //
-// Decode once: each thread decodes its window a single time into a private
+// Decode once: each thread decodes its windows a single time into a private
 // slot of shared memory and learns its count from the bytes it wrote,
-// corrected for codes of the last table step that start past the window end.
+// corrected for codes of the last table step that start past the run's end.
 // After the warp's prefix sum the slots are copied, one aligned word at a
 // time, into the block's contiguous staging buffer; the first word of a slot
 // range that starts mid-word is written byte-wise after a warp barrier, and a
@@ -878,7 +881,7 @@ df11_status launch_warp_variant(const DecodeArgs& a, cudaStream_t s, int slot, u
     return launch_persistent(decode_warp_kernel<WARPS, MIN_LEN, WPL>, slot, WARPS * 32, smem, ctas, max_sms, a, s);
 }
 
-// T = 32: one window per lane.
+// T = 32: one window per lane (T = 64 streams: two, see df11_decompress).
 df11_status launch_warp(const DecodeArgs& a, cudaStream_t s, uint32_t min_len, uint32_t max_sms) {
     if (min_len >= 2) return launch_warp_variant<kWarpsShort, 2, 1>(a, s, 6, max_sms);
     return launch_warp_variant<kWarpsLong, 1, 1>(a, s, 0, max_sms);
