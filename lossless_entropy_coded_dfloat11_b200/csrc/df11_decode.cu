@@ -628,9 +628,11 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_warp_kernel(const Decode
     const uint32_t lane_gword = (5 * WPL * lane) >> 5;
     const uint32_t lane_gshift = (5 * WPL * lane) & 31u;
 
-    // this warp's run of thread blocks [b, b_end)
+    // this warp's run of thread blocks [b, b_end); warps are numbered across
+    // the CTAs first, so the runs one block longer than the rest (the first
+    // n_blocks mod nw) fall at most one per SM instead of filling a few SMs
     const uint32_t nw = gridDim.x * WARPS;
-    const uint32_t g = blockIdx.x * WARPS + warp;
+    const uint32_t g = warp * gridDim.x + blockIdx.x;
     const uint32_t per = a.n_blocks / nw, extra = a.n_blocks % nw;
     uint32_t b = g * per + (g < extra ? g : extra);
     const uint32_t b_end = b + per + (g < extra ? 1u : 0u);
@@ -833,11 +835,14 @@ struct LaunchInfo {
 constexpr int kMaxDev = 64;
 LaunchInfo g_info[kMaxDev][8];  // [device][variant]
 
-// One CTA of 32 warps per SM: all warps share one copy of the tables, and
-// the register budget (64 per thread) leaves the decode loop unconstrained;
-// this measured faster than two CTAs of 20 warps at 48 registers.
+// One CTA per SM: all warps share one copy of the tables.  With one window
+// per lane, 32 warps at 64 registers measured faster than two CTAs of 20
+// warps at 48 registers.
 constexpr int kWarpsLong = 32;   // some code is 1 bit long
 constexpr int kWarpsShort = 32;  // every code has 2 bits or more
+// two windows per lane: 28 warps leave 72 registers per thread (the merge's
+// seven prefetched rounds fit) and measured faster than 24, 26, 30 or 32
+constexpr int kWarpsTwoWindows = 28;
 
 template <typename Kernel>
 df11_status launch_persistent(Kernel kernel, int slot, int threads, size_t smem, uint64_t work_units,
@@ -948,7 +953,7 @@ df11_status decompress_on(const df11_header* hdr, const uint8_t* d_exp, const ui
     switch (hdr->threads_per_block) {
         case 32: return launch_warp(a, s, min_len, max_sms);
         case 64:  // two windows per lane when every code has 2 bits or more (the slots then fit)
-            if (min_len >= 2) return launch_warp_variant<kWarpsShort, 2, 2>(a, s, 7, max_sms);
+            if (min_len >= 2) return launch_warp_variant<kWarpsTwoWindows, 2, 2>(a, s, 7, max_sms);
             return launch_block<64>(a, s, 1, max_sms);
         case 128: return launch_block<128>(a, s, 2, max_sms);
         case 256: return launch_block<256>(a, s, 3, max_sms);
