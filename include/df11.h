@@ -211,6 +211,28 @@ df11_status df11_decompress_sms(const df11_header* hdr, const uint8_t* d_exp, co
                                 const void* d_lut, uint16_t* d_out, uint32_t* d_status,
                                 uint32_t max_sms, void* stream);
 
+/* Streams of 8-bit symbols coded whole: the codec of "EntroLLM: Compressao
+ * de Pesos Codificada por Entropia para Inferencia Eficiente de Modelos de
+ * Linguagem Grandes em Dispositivos de Borda" (section "Metodologia", items 2
+ * and 3: Huffman coding of the quantized integer weights, decoded in
+ * parallel) on this library's container.  The symbol of each element is its
+ * whole byte (e.g. a per-tensor quantized weight) and there is no
+ * PackedSignMantissa array; EncodedExponent, Gaps, block offsets, the code
+ * table, the header and its sizes are as for BF16 streams (bytes_sm is not
+ * used).  Arguments as for the BF16 calls, with segments of n bytes.
+ * T must be 32, or 64 when no code is 1 bit long (df11_decompress_u8
+ * returns DF11_ERR_INVALID otherwise). */
+df11_status df11_compress_plan_u8(const void* const* d_segs, const uint64_t* seg_counts, uint32_t n_segs,
+                                  uint32_t threads_per_block, uint32_t max_code_len, void* d_workspace,
+                                  uint64_t workspace_bytes, df11_header* hdr, void* stream);
+df11_status df11_compress_encode_u8(const void* const* d_segs, const df11_header* hdr, void* d_workspace,
+                                    uint64_t workspace_bytes, uint8_t* d_exp, uint8_t* d_gaps,
+                                    uint32_t* d_block_off, void* d_lut, void* stream);
+/* d_out: n_elems bytes, 16-byte aligned; asynchronous, no allocation. */
+df11_status df11_decompress_u8(const df11_header* hdr, const uint8_t* d_exp, const uint8_t* d_gaps,
+                               const uint32_t* d_block_off, const void* d_lut, uint8_t* d_out,
+                               uint32_t* d_status, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -6,10 +6,11 @@ caller-owned buffers with PyTorch and passes pointers.  Importing it does not
 load the library; the first call does, and raises if it is missing.
 """
 from .codec import (DEFAULT_THREADS_PER_BLOCK, CompressedStream, HostStream, build_lut, code_lengths, compress, decompress,
-                    from_arrays, make_header, to_host, workspace_bytes)
+                    compress_u8, decompress_u8, from_arrays, make_header, to_host, workspace_bytes)
 from ._binding import DF11Error, EXPORTED, load as load_library, library_path
 from .prefetch import BlockPrefetcher
 
 __all__ = ["DEFAULT_THREADS_PER_BLOCK", "CompressedStream", "HostStream", "build_lut", "code_lengths", "compress", "decompress",
+           "compress_u8", "decompress_u8",
            "from_arrays", "make_header", "to_host", "workspace_bytes", "DF11Error", "EXPORTED",
            "load_library", "library_path", "BlockPrefetcher"]

@@ -47,6 +47,7 @@ class CompressedStream:
     lut: torch.Tensor        # uint8  decode tables (df11_build_lut)
     names: list = field(default_factory=list)
     shapes: list = field(default_factory=list)
+    symbols: str = "bf16"    # "bf16": BF16 weights; "u8": 8-bit symbols coded whole (no sm array)
 
     @property
     def n_elems(self) -> int:
@@ -69,14 +70,16 @@ class CompressedStream:
         per element, 5 bits per thread, 4 bytes per thread-block position and
         the 256-byte code-length table."""
         h = self.header
-        return ((h.total_bits + 7) // 8 + h.n_elems + (5 * h.n_threads + 7) // 8
+        side = h.n_elems if self.symbols == "bf16" else 0
+        return ((h.total_bits + 7) // 8 + side + (5 * h.n_threads + 7) // 8
                 + 4 * (h.n_blocks + 1) + 256)
 
     def read_bytes(self) -> int:
         """Bytes one decompress reads from HBM (the format's arrays as the
         kernel fetches them, plus the decode tables once per CTA from L2)."""
         h = self.header
-        return (h.total_bits + 7) // 8 + h.n_elems + (5 * h.n_threads + 7) // 8 + 4 * (h.n_blocks + 1)
+        side = h.n_elems if self.symbols == "bf16" else 0
+        return (h.total_bits + 7) // 8 + side + (5 * h.n_threads + 7) // 8 + 4 * (h.n_blocks + 1)
 
     def views(self, flat: torch.Tensor) -> list[torch.Tensor]:
         """Per-matrix views of a decompressed flat buffer."""
@@ -120,13 +123,13 @@ def workspace_bytes(n_elems: int) -> int:
     return int(v.value)
 
 
-def _as_segments(tensors):
+def _as_segments(tensors, dtype=torch.bfloat16):
     if isinstance(tensors, torch.Tensor):
         tensors = [tensors]
     segs = []
     for t in tensors:
-        if t.dtype != torch.bfloat16:
-            raise TypeError(f"DF11 compresses bfloat16 tensors, got {t.dtype}")
+        if t.dtype != dtype:
+            raise TypeError(f"expected {dtype} tensors, got {t.dtype}")
         if not t.is_cuda:
             raise ValueError("compress expects CUDA tensors")
         segs.append(t.contiguous())
@@ -163,12 +166,18 @@ def compress(tensors, names=None, threads_per_block: int = DEFAULT_THREADS_PER_B
 
 
 def from_arrays(code_len: np.ndarray, n_elems: int, total_bits: int, threads_per_block: int,
-                exp: np.ndarray, sm: np.ndarray, gaps: np.ndarray, block_off: np.ndarray,
-                max_code_len: int = 32, seg_counts=None, shapes=None, device="cuda") -> CompressedStream:
-    """Upload a stream made elsewhere (another encoder, a file)."""
+                exp: np.ndarray, sm: np.ndarray | None, gaps: np.ndarray, block_off: np.ndarray,
+                max_code_len: int = 32, seg_counts=None, shapes=None, device="cuda",
+                symbols: str = "bf16") -> CompressedStream:
+    """Upload a stream made elsewhere (another encoder, a file); streams of
+    8-bit symbols (symbols="u8") have no sm array."""
     hdr = make_header(code_len, n_elems, total_bits, threads_per_block, max_code_len, seg_counts)
-    for name, arr, need in (("exp", exp, hdr.bytes_exp), ("sm", sm, hdr.bytes_sm),
-                            ("gaps", gaps, hdr.bytes_gaps), ("block_off", block_off, hdr.n_blocks + 1)):
+    if symbols == "u8":
+        sm = np.zeros(0, dtype=np.uint8)
+    arrays = [("exp", exp, hdr.bytes_exp), ("gaps", gaps, hdr.bytes_gaps), ("block_off", block_off, hdr.n_blocks + 1)]
+    if symbols == "bf16":
+        arrays.append(("sm", sm, hdr.bytes_sm))
+    for name, arr, need in arrays:
         if arr.size < need:
             raise ValueError(f"{name}: {arr.size} entries, header needs {need}")
     lut = build_lut(hdr)
@@ -182,7 +191,7 @@ def from_arrays(code_len: np.ndarray, n_elems: int, total_bits: int, threads_per
     shapes = shapes or [(int(c),) for c in (seg_counts or [n_elems])]
     return CompressedStream(hdr, up(exp), up(sm), up(gaps),
                             up(np.ascontiguousarray(block_off, dtype=np.uint32), torch.int32), up(lut),
-                            names=[f"t{k}" for k in range(len(shapes))], shapes=shapes)
+                            names=[f"t{k}" for k in range(len(shapes))], shapes=shapes, symbols=symbols)
 
 
 def to_host(cs: CompressedStream) -> dict:
@@ -192,7 +201,7 @@ def to_host(cs: CompressedStream) -> dict:
                 threads_per_block=int(h.threads_per_block), n_threads=int(h.n_threads),
                 n_blocks=int(h.n_blocks),
                 exp=cs.exp.cpu().numpy()[: int(h.bytes_exp)],
-                sm=cs.sm.cpu().numpy()[: int(h.bytes_sm)],
+                sm=cs.sm.cpu().numpy()[: int(h.bytes_sm)] if cs.symbols == "bf16" else np.zeros(0, np.uint8),
                 gaps=cs.gaps.cpu().numpy()[: int(h.bytes_gaps)],
                 block_off=cs.block_off.cpu().numpy().view(np.uint32)[: int(h.n_blocks) + 1])
 
@@ -247,3 +256,53 @@ class HostStream:
             decompress(self.dev_stream, self.out_dev, stream=s)
             self.out_host.copy_(self.out_dev, non_blocking=True)
         return self.out_host
+
+
+def compress_u8(tensors, names=None, threads_per_block: int = DEFAULT_THREADS_PER_BLOCK, max_code_len: int = 32,
+                stream=None) -> CompressedStream:
+    """Compress one uint8 tensor (e.g. per-tensor quantized weights), or a
+    list, coding each byte whole with one shared table; no side array.  T = 64
+    falls back to T = 32 when the code has a 1-bit symbol (the two-window
+    decoder needs codes of 2 bits or more)."""
+    segs = _as_segments(tensors, torch.uint8)
+    device = segs[0].device
+    n = sum(t.numel() for t in segs)
+    ws = torch.empty(max(workspace_bytes(n), 16), dtype=torch.uint8, device=device)
+    ptrs = (ctypes.c_void_p * len(segs))(*[int(t.data_ptr()) for t in segs])
+    counts = (ctypes.c_uint64 * len(segs))(*[t.numel() for t in segs])
+    hdr = B.Header()
+    sh = _stream_handle(stream)
+    B.call("df11_compress_plan_u8", ptrs, counts, len(segs), threads_per_block, max_code_len, _ptr(ws),
+           ws.numel(), ctypes.byref(hdr), sh)
+    ln = np.frombuffer(bytes(hdr.code_len), dtype=np.uint8)
+    if threads_per_block == 64 and n and ln[ln > 0].min() == 1:
+        hdr = make_header(ln, int(hdr.n_elems), int(hdr.total_bits), 32, max_code_len,
+                          [t.numel() for t in segs])
+    exp = torch.empty(int(hdr.bytes_exp), dtype=torch.uint8, device=device)
+    gaps = torch.empty(int(hdr.bytes_gaps), dtype=torch.uint8, device=device)
+    off = torch.empty(int(hdr.n_blocks) + 1, dtype=torch.int32, device=device)
+    lut = torch.empty(int(hdr.bytes_lut), dtype=torch.uint8, device=device)
+    B.call("df11_compress_encode_u8", ptrs, ctypes.byref(hdr), _ptr(ws), ws.numel(), _ptr(exp), _ptr(gaps),
+           _ptr(off), _ptr(lut), sh)
+    (stream or torch.cuda.current_stream()).synchronize()
+    return CompressedStream(hdr, exp, torch.zeros(16, dtype=torch.uint8, device=device), gaps, off, lut,
+                            names=list(names) if names else [f"t{k}" for k in range(len(segs))],
+                            shapes=[tuple(t.shape) for t in segs], symbols="u8")
+
+
+def decompress_u8(cs: CompressedStream, out: torch.Tensor | None = None, status: torch.Tensor | None = None,
+                  stream=None) -> torch.Tensor:
+    """One kernel launch rebuilding all n_elems bytes of a stream of 8-bit
+    symbols.  Asynchronous; `out` (uint8, n_elems, contiguous, 16-byte
+    aligned) may be reused."""
+    if cs.symbols != "u8":
+        raise ValueError("decompress_u8 takes streams of 8-bit symbols (compress_u8)")
+    n = cs.n_elems
+    if out is None:
+        out = torch.empty(max(n, 16), dtype=torch.uint8, device=cs.exp.device)[:n]
+    if out.dtype != torch.uint8 or not out.is_contiguous() or out.numel() < n:
+        raise ValueError("out must be a contiguous uint8 tensor with n_elems elements")
+    B.call("df11_decompress_u8", ctypes.byref(cs.header), _ptr(cs.exp), _ptr(cs.gaps), _ptr(cs.block_off),
+           _ptr(cs.lut), _ptr(out), _ptr(status) if status is not None else ctypes.c_void_p(0),
+           _stream_handle(stream))
+    return out

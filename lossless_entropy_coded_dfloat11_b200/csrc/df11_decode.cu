@@ -56,7 +56,8 @@ struct DecodeArgs {
     const uint32_t* gaps;
     const uint32_t* off;
     const uint4* lut;
-    uint16_t* out;
+    uint16_t* out;        // BF16 output (streams of BF16 weights)
+    uint8_t* out8;        // symbol output (streams of 8-bit symbols)
     uint32_t* status;
     uint32_t n_elems;
     uint32_t n_threads;
@@ -330,6 +331,14 @@ __device__ __forceinline__ void merge_unit(const uint2 ev, const uint2 sv, uint3
     }
 }
 
+// Sixteen staged symbols rotated back: the tables hold each symbol rotated
+// right by one bit (for the BF16 merge); an 8-bit symbol is its byte rotated
+// left by one.
+__device__ __forceinline__ uint4 unrotate16(const uint4 r) {
+    auto rol1 = [](uint32_t w) { return ((w << 1) & 0xFEFEFEFEu) | ((w >> 7) & 0x01010101u); };
+    return make_uint4(rol1(r.x), rol1(r.y), rol1(r.z), rol1(r.w));
+}
+
 __device__ __forceinline__ void copy_tables(uint8_t* s_lut, const uint4* g_lut, int nthreads) {
     for (int i = threadIdx.x; i < int(kLutBytes / 16); i += nthreads)
         reinterpret_cast<uint4*>(s_lut)[i] = __ldg(g_lut + i);
@@ -600,9 +609,11 @@ __device__ __forceinline__ uint32_t copy_slot(const uint32_t* slot, uint32_t* st
     return first;
 }
 
-template <int WARPS, int MIN_LEN, int WPL>
+template <int WARPS, int MIN_LEN, int WPL, bool U8>
 __global__ void __launch_bounds__(WARPS * 32, 1) decode_warp_kernel(const DecodeArgs a) {
     using L = WarpLayout<MIN_LEN, WPL>;
+    // elements per merge unit, 16 output bytes either way
+    constexpr uint32_t kUnit = U8 ? 16u : 8u;
     extern __shared__ __align__(16) uint8_t smem[];
     copy_compact_tables(smem, a.lut, WARPS * 32);
     __syncthreads();
@@ -645,7 +656,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_warp_kernel(const Decode
         noff1 = __ldg(a.off + b + 1);
     }
     const uint2* sm8 = reinterpret_cast<const uint2*>(a.sm);
-    uint2 carry = make_uint2(0, 0);  // staging bytes of the unit left by the previous block
+    uint4 carry = make_uint4(0, 0, 0, 0);  // staging bytes of the unit left by the previous block
     bool have_carry = false;
     while (b < b_end) {
         const RawLane<WPL> raw = nraw;
@@ -657,23 +668,25 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_warp_kernel(const Decode
             noff1 = __ldg(a.off + b + 2);
         }
         const bool offs_ok = off0 <= off1 && off1 <= a.n_elems;
-        const uint32_t head = off0 & 7u;
+        const uint32_t head = off0 & (kUnit - 1);
         // units to store: the head unit (completed by the carried bytes
         // unless this block starts the run), up to the tail unit, which is
         // left to the next block when that block exists and shares it
-        const uint32_t u0 = off0 >> 3;
-        const uint32_t u1 = offs_ok ? (off1 + 7) >> 3 : u0;
-        const bool keep_tail = more && (off1 & 7u) != 0;
+        const uint32_t u0 = off0 / kUnit;
+        const uint32_t u1 = offs_ok ? (off1 + kUnit - 1) / kUnit : u0;
+        const bool keep_tail = more && (off1 & (kUnit - 1)) != 0;
         const uint32_t uw = keep_tail && u1 > u0 ? u1 - 1 : u1;
         const bool use_carry = have_carry && head != 0;
-        const uint32_t lo = use_carry ? (off0 & ~7u) : off0;
+        const uint32_t lo = use_carry ? (off0 & ~(kUnit - 1)) : off0;
         // sign+mantissa units requested before the decode: 4 rounds of 32
         // (a 32-window block has ~100 units), 7 for two windows per lane
         constexpr int kPre = WPL == 1 ? 4 : 7;
         uint2 sv[kPre];
+        if constexpr (!U8) {
 #pragma unroll
-        for (int r = 0; r < kPre; r++)
-            sv[r] = u0 + lane + 32 * r < uw ? __ldcs(sm8 + u0 + lane + 32 * r) : make_uint2(0, 0);
+            for (int r = 0; r < kPre; r++)
+                sv[r] = u0 + lane + 32 * r < uw ? __ldcs(sm8 + u0 + lane + 32 * r) : make_uint2(0, 0);
+        }
 
         const LaneWindow<WPL> w = finish_lane<WPL>(a, raw, WPL * (32 * b + lane), lane_gshift, lane);
         bool bad = false;
@@ -690,7 +703,10 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_warp_kernel(const Decode
             if (lane == 0 && a.status) atomicOr(a.status, uint32_t(DF11_ERR_CORRUPT));
             have_carry = false;
         } else {
-            if (lane == 0 && use_carry) *reinterpret_cast<uint2*>(stage) = carry;
+            if (lane == 0 && use_carry) {
+                if constexpr (U8) *reinterpret_cast<uint4*>(stage) = carry;
+                else *reinterpret_cast<uint2*>(stage) = make_uint2(carry.x, carry.y);
+            }
             __syncwarp();
             const uint32_t pos0 = head + (incl - cnt);
             const uint32_t hword = copy_slot(slot, reinterpret_cast<uint32_t*>(stage), pos0, cnt);
@@ -704,40 +720,68 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_warp_kernel(const Decode
                 if (k > 2) d[2] = uint8_t(hword >> 16);
             }
             __syncwarp();
-            const uint2* ev = reinterpret_cast<const uint2*>(stage);
-            const uint32_t stage_s = uint32_t(__cvta_generic_to_shared(stage));
-            const uint32_t nu = uw - u0;  // units this block stores
-            const uint32_t m = 0x80808080u;
-            if (lo == 8 * u0 && (keep_tail || (off1 & 7u) == 0)) {
-                // every unit is whole (all but the first and last block of a run)
-                const uint32_t ev_s = stage_s + 8 * lane;
-                uint4* dst = reinterpret_cast<uint4*>(a.out) + u0 + lane;
-                if (lane < nu) merge_store8<0, 0>(ev_s, sv[0], dst, m);
-                if (lane + 32 < nu) merge_store8<256, 512>(ev_s, sv[1], dst, m);
-                if (lane + 64 < nu) merge_store8<512, 1024>(ev_s, sv[2], dst, m);
-                if (lane + 96 < nu) merge_store8<768, 1536>(ev_s, sv[3], dst, m);
-                if constexpr (kPre == 7) {
-                    if (lane + 128 < nu) merge_store8<1024, 2048>(ev_s, sv[4], dst, m);
-                    if (lane + 160 < nu) merge_store8<1280, 2560>(ev_s, sv[5], dst, m);
-                    if (lane + 192 < nu) merge_store8<1536, 3072>(ev_s, sv[6], dst, m);
+            if constexpr (!U8) {
+                const uint2* ev = reinterpret_cast<const uint2*>(stage);
+                const uint32_t stage_s = uint32_t(__cvta_generic_to_shared(stage));
+                const uint32_t nu = uw - u0;  // units this block stores
+                const uint32_t m = 0x80808080u;
+                if (lo == 8 * u0 && (keep_tail || (off1 & 7u) == 0)) {
+                    // every unit is whole (all but the first and last block of a run)
+                    const uint32_t ev_s = stage_s + 8 * lane;
+                    uint4* dst = reinterpret_cast<uint4*>(a.out) + u0 + lane;
+                    if (lane < nu) merge_store8<0, 0>(ev_s, sv[0], dst, m);
+                    if (lane + 32 < nu) merge_store8<256, 512>(ev_s, sv[1], dst, m);
+                    if (lane + 64 < nu) merge_store8<512, 1024>(ev_s, sv[2], dst, m);
+                    if (lane + 96 < nu) merge_store8<768, 1536>(ev_s, sv[3], dst, m);
+                    if constexpr (kPre == 7) {
+                        if (lane + 128 < nu) merge_store8<1024, 2048>(ev_s, sv[4], dst, m);
+                        if (lane + 160 < nu) merge_store8<1280, 2560>(ev_s, sv[5], dst, m);
+                        if (lane + 192 < nu) merge_store8<1536, 3072>(ev_s, sv[6], dst, m);
+                    }
+                    for (uint32_t k = 32 * kPre; lane + k < nu; k += 32)
+                        merge_store8(ev_s + 8 * k, __ldcs(sm8 + u0 + lane + k), dst + k, m);
+                } else {
+                    const uint32_t uf = (lo + 7) >> 3, ul = off1 >> 3;  // whole units: [uf, ul)
+                    auto unit = [&](uint32_t k, const uint2 s8) {
+                        const uint32_t u = u0 + k;
+                        if (u >= uf && u < ul)
+                            merge_store8(stage_s + 8 * k, s8, reinterpret_cast<uint4*>(a.out) + u, m);
+                        else
+                            merge_unit(ev[k], s8, u, lo, off1, a.out);
+                    };
+    #pragma unroll
+                    for (int r = 0; r < kPre; r++)
+                        if (lane + 32 * r < nu) unit(lane + 32 * r, sv[r]);
+                    for (uint32_t k = lane + 32 * kPre; k < nu; k += 32) unit(k, __ldcs(sm8 + u0 + k));
                 }
-                for (uint32_t k = 32 * kPre; lane + k < nu; k += 32)
-                    merge_store8(ev_s + 8 * k, __ldcs(sm8 + u0 + lane + k), dst + k, m);
+                if (keep_tail) {
+                    const uint2 c = ev[u1 - 1 - u0];
+                    carry = make_uint4(c.x, c.y, 0, 0);
+                }
             } else {
-                const uint32_t uf = (lo + 7) >> 3, ul = off1 >> 3;  // whole units: [uf, ul)
-                auto unit = [&](uint32_t k, const uint2 s8) {
-                    const uint32_t u = u0 + k;
-                    if (u >= uf && u < ul)
-                        merge_store8(stage_s + 8 * k, s8, reinterpret_cast<uint4*>(a.out) + u, m);
-                    else
-                        merge_unit(ev[k], s8, u, lo, off1, a.out);
-                };
+                // 8-bit symbols: the staged bytes themselves, rotated back
+                const uint4* ev16 = reinterpret_cast<const uint4*>(stage);
+                const uint32_t nu = uw - u0;  // units this block stores
+                uint4* out16 = reinterpret_cast<uint4*>(a.out8);
+                if (lo == kUnit * u0 && (keep_tail || (off1 & (kUnit - 1)) == 0)) {
+                    for (uint32_t k = lane; k < nu; k += 32) __stcs(out16 + u0 + k, unrotate16(ev16[k]));
+                } else {
+                    for (uint32_t k = lane; k < nu; k += 32) {
+                        const uint32_t u = u0 + k;
+                        const uint4 v = unrotate16(ev16[k]);
+                        const uint32_t i0 = kUnit * u;
+                        if (i0 >= lo && i0 + kUnit <= off1) {
+                            __stcs(out16 + u, v);
+                        } else {
+                            const uint32_t words[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-                for (int r = 0; r < kPre; r++)
-                    if (lane + 32 * r < nu) unit(lane + 32 * r, sv[r]);
-                for (uint32_t k = lane + 32 * kPre; k < nu; k += 32) unit(k, __ldcs(sm8 + u0 + k));
+                            for (int q = 0; q < 16; q++)
+                                if (i0 + q >= lo && i0 + q < off1) a.out8[i0 + q] = uint8_t(words[q >> 2] >> (8 * (q & 3)));
+                        }
+                    }
+                }
+                if (keep_tail) carry = ev16[u1 - 1 - u0];
             }
-            if (keep_tail) carry = ev[u1 - 1 - u0];
             have_carry = keep_tail;
         }
         __syncwarp();
@@ -833,7 +877,7 @@ struct LaunchInfo {
     int sms = 0;
 };
 constexpr int kMaxDev = 64;
-LaunchInfo g_info[kMaxDev][8];  // [device][variant]
+LaunchInfo g_info[kMaxDev][16];  // [device][variant]: BF16 0..7, 8-bit symbols 8..15
 
 // One CTA per SM: all warps share one copy of the tables.  With one window
 // per lane, 32 warps at 64 registers measured faster than two CTAs of 20
@@ -878,18 +922,20 @@ df11_status launch_block(const DecodeArgs& a, cudaStream_t s, int slot, uint32_t
     return launch_persistent(decode_block_kernel<T>, slot, T, smem, a.n_blocks, max_sms, a, s);
 }
 
-template <int WARPS, int MIN_LEN, int WPL>
+template <int WARPS, int MIN_LEN, int WPL, bool U8>
 df11_status launch_warp_variant(const DecodeArgs& a, cudaStream_t s, int slot, uint32_t max_sms) {
     constexpr size_t smem = kCompactBytes + size_t(WARPS) * WarpLayout<MIN_LEN, WPL>::kBytes;
     static_assert(smem <= 227 * 1024, "shared memory per CTA");
     const uint64_t ctas = (uint64_t(a.n_blocks) + WARPS - 1) / WARPS;
-    return launch_persistent(decode_warp_kernel<WARPS, MIN_LEN, WPL>, slot, WARPS * 32, smem, ctas, max_sms, a, s);
+    return launch_persistent(decode_warp_kernel<WARPS, MIN_LEN, WPL, U8>, slot + (U8 ? 8 : 0), WARPS * 32, smem,
+                             ctas, max_sms, a, s);
 }
 
-// T = 32: one window per lane (T = 64 streams: two, see df11_decompress).
+// T = 32: one window per lane (T = 64 streams: two, see decompress_on).
+template <bool U8>
 df11_status launch_warp(const DecodeArgs& a, cudaStream_t s, uint32_t min_len, uint32_t max_sms) {
-    if (min_len >= 2) return launch_warp_variant<kWarpsShort, 2, 1>(a, s, 6, max_sms);
-    return launch_warp_variant<kWarpsLong, 1, 1>(a, s, 0, max_sms);
+    if (min_len >= 2) return launch_warp_variant<kWarpsShort, 2, 1, U8>(a, s, 6, max_sms);
+    return launch_warp_variant<kWarpsLong, 1, 1, U8>(a, s, 0, max_sms);
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -923,24 +969,27 @@ using namespace df11;
 namespace df11 {
 namespace {
 
-df11_status decompress_on(const df11_header* hdr, const uint8_t* d_exp, const uint8_t* d_sm,
-                          const uint8_t* d_gaps, const uint32_t* d_block_off, const void* d_lut,
-                          uint16_t* d_out, uint32_t* d_status, uint32_t max_sms, void* stream) {
+// BF16 streams (u8 = false): d_sm read, d_out holds n_elems uint16; streams
+// of 8-bit symbols (u8 = true): no d_sm, d_out holds n_elems bytes.
+df11_status decompress_on(const char* fn, bool u8, const df11_header* hdr, const uint8_t* d_exp,
+                          const uint8_t* d_sm, const uint8_t* d_gaps, const uint32_t* d_block_off,
+                          const void* d_lut, void* d_out, uint32_t* d_status, uint32_t max_sms, void* stream) {
     df11_status st = check_header(hdr);
     if (st != DF11_OK) return st;
     if (hdr->n_elems == 0) return DF11_OK;
-    if (!d_exp || !d_sm || !d_gaps || !d_block_off || !d_lut || !d_out)
-        return fail(DF11_ERR_INVALID, "df11_decompress: null device pointer");
-    if (!aligned16(d_exp) || !aligned16(d_sm) || !aligned16(d_gaps) || !aligned16(d_block_off) ||
+    if (!d_exp || (!u8 && !d_sm) || !d_gaps || !d_block_off || !d_lut || !d_out)
+        return fail(DF11_ERR_INVALID, "%s: null device pointer", fn);
+    if (!aligned16(d_exp) || (!u8 && !aligned16(d_sm)) || !aligned16(d_gaps) || !aligned16(d_block_off) ||
         !aligned16(d_lut) || !aligned16(d_out))
-        return fail(DF11_ERR_INVALID, "df11_decompress: device pointers must be 16-byte aligned");
+        return fail(DF11_ERR_INVALID, "%s: device pointers must be 16-byte aligned", fn);
     DecodeArgs a;
     a.exp = d_exp;
     a.sm = reinterpret_cast<const uint4*>(d_sm);
     a.gaps = reinterpret_cast<const uint32_t*>(d_gaps);
     a.off = d_block_off;
     a.lut = reinterpret_cast<const uint4*>(d_lut);
-    a.out = d_out;
+    a.out = u8 ? nullptr : static_cast<uint16_t*>(d_out);
+    a.out8 = u8 ? static_cast<uint8_t*>(d_out) : nullptr;
     a.status = d_status;
     a.n_elems = uint32_t(hdr->n_elems);
     a.n_threads = uint32_t(hdr->n_threads);
@@ -950,10 +999,17 @@ df11_status decompress_on(const df11_header* hdr, const uint8_t* d_exp, const ui
     uint32_t min_len = 32;
     for (int v = 0; v < 256; v++)
         if (hdr->code_len[v] && hdr->code_len[v] < min_len) min_len = hdr->code_len[v];
+    if (u8) {  // the warp kernel only
+        if (hdr->threads_per_block == 32) return launch_warp<true>(a, s, min_len, max_sms);
+        if (hdr->threads_per_block == 64 && min_len >= 2)
+            return launch_warp_variant<kWarpsTwoWindows, 2, 2, true>(a, s, 7, max_sms);
+        return fail(DF11_ERR_INVALID,
+                    "%s: streams of 8-bit symbols decode with T = 32, or T = 64 when no code is 1 bit long", fn);
+    }
     switch (hdr->threads_per_block) {
-        case 32: return launch_warp(a, s, min_len, max_sms);
+        case 32: return launch_warp<false>(a, s, min_len, max_sms);
         case 64:  // two windows per lane when every code has 2 bits or more (the slots then fit)
-            if (min_len >= 2) return launch_warp_variant<kWarpsTwoWindows, 2, 2>(a, s, 7, max_sms);
+            if (min_len >= 2) return launch_warp_variant<kWarpsTwoWindows, 2, 2, false>(a, s, 7, max_sms);
             return launch_block<64>(a, s, 1, max_sms);
         case 128: return launch_block<128>(a, s, 2, max_sms);
         case 256: return launch_block<256>(a, s, 3, max_sms);
@@ -970,7 +1026,8 @@ extern "C" df11_status df11_decompress(const df11_header* hdr, const uint8_t* d_
                                        const uint8_t* d_gaps, const uint32_t* d_block_off,
                                        const void* d_lut, uint16_t* d_out, uint32_t* d_status,
                                        void* stream) {
-    return decompress_on(hdr, d_exp, d_sm, d_gaps, d_block_off, d_lut, d_out, d_status, UINT32_MAX, stream);
+    return decompress_on("df11_decompress", false, hdr, d_exp, d_sm, d_gaps, d_block_off, d_lut, d_out, d_status,
+                         UINT32_MAX, stream);
 }
 
 extern "C" df11_status df11_decompress_sms(const df11_header* hdr, const uint8_t* d_exp, const uint8_t* d_sm,
@@ -978,5 +1035,13 @@ extern "C" df11_status df11_decompress_sms(const df11_header* hdr, const uint8_t
                                            const void* d_lut, uint16_t* d_out, uint32_t* d_status,
                                            uint32_t max_sms, void* stream) {
     if (max_sms == 0) return fail(DF11_ERR_INVALID, "df11_decompress_sms: max_sms must be at least 1");
-    return decompress_on(hdr, d_exp, d_sm, d_gaps, d_block_off, d_lut, d_out, d_status, max_sms, stream);
+    return decompress_on("df11_decompress_sms", false, hdr, d_exp, d_sm, d_gaps, d_block_off, d_lut, d_out,
+                         d_status, max_sms, stream);
+}
+
+extern "C" df11_status df11_decompress_u8(const df11_header* hdr, const uint8_t* d_exp, const uint8_t* d_gaps,
+                                          const uint32_t* d_block_off, const void* d_lut, uint8_t* d_out,
+                                          uint32_t* d_status, void* stream) {
+    return decompress_on("df11_decompress_u8", true, hdr, d_exp, nullptr, d_gaps, d_block_off, d_lut, d_out,
+                         d_status, UINT32_MAX, stream);
 }

@@ -24,8 +24,10 @@ df11_status check_header(const df11_header* h);
 
 namespace {
 
+// Segments of the input, in elements of ES bytes: ES = 2 for BF16 weights
+// (the symbol is the exponent field), ES = 1 for 8-bit symbols coded whole.
 struct SegTable {
-    const uint16_t* ptr[DF11_MAX_SEGMENTS];
+    const uint8_t* ptr[DF11_MAX_SEGMENTS];
     uint64_t start[DF11_MAX_SEGMENTS + 1];
     uint32_t n;
 };
@@ -36,10 +38,36 @@ struct CodeTable {
 };
 
 // ---------------------------------------------------------------------------
-// Histogram of the exponent field of one segment; per-warp shared-memory
-// histograms, flushed into 64-bit global counters.
+// Histogram of the symbols of one segment (the exponent field of BF16
+// elements, or 8-bit symbols); per-warp shared-memory histograms, flushed
+// into 64-bit global counters.
 // ---------------------------------------------------------------------------
 constexpr int kHistThreads = 256;
+
+__global__ void __launch_bounds__(kHistThreads) histogram_u8_kernel(const uint8_t* __restrict__ x, uint64_t n,
+                                                                    unsigned long long* __restrict__ hist) {
+    __shared__ uint32_t sh[kHistThreads / 32][256];
+    uint32_t* mine = sh[threadIdx.x >> 5];
+    for (int i = threadIdx.x; i < (kHistThreads / 32) * 256; i += kHistThreads) (&sh[0][0])[i] = 0;
+    __syncthreads();
+    const uint64_t nvec = n / 16;
+    const uint4* xv = reinterpret_cast<const uint4*>(x);
+    const uint64_t stride = uint64_t(gridDim.x) * kHistThreads;
+    for (uint64_t v = uint64_t(blockIdx.x) * kHistThreads + threadIdx.x; v < nvec; v += stride) {
+        const uint4 q = __ldcs(xv + v);
+        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+        for (int k = 0; k < 16; k++) atomicAdd(&mine[(w[k >> 2] >> (8 * (k & 3))) & 0xFFu], 1u);
+    }
+    for (uint64_t i = nvec * 16 + uint64_t(blockIdx.x) * kHistThreads + threadIdx.x; i < n; i += stride)
+        atomicAdd(&mine[x[i]], 1u);
+    __syncthreads();
+    for (int s = threadIdx.x; s < 256; s += kHistThreads) {
+        uint64_t t = 0;
+        for (int w = 0; w < kHistThreads / 32; w++) t += sh[w][s];
+        if (t) atomicAdd(hist + s, (unsigned long long)t);
+    }
+}
 
 __global__ void __launch_bounds__(kHistThreads) histogram_kernel(const uint16_t* __restrict__ x, uint64_t n,
                                                                  unsigned long long* __restrict__ hist) {
@@ -70,9 +98,12 @@ __global__ void __launch_bounds__(kHistThreads) histogram_kernel(const uint16_t*
 }
 
 // Element i of the concatenated segments.
+template <int ES>
 __device__ __forceinline__ uint16_t load_elem(const SegTable& sg, uint64_t i, uint32_t& seg) {
     while (seg + 1 < sg.n && i >= sg.start[seg + 1]) seg++;
-    return sg.ptr[seg][i - sg.start[seg]];
+    const uint64_t rel = i - sg.start[seg];
+    if constexpr (ES == 2) return reinterpret_cast<const uint16_t*>(sg.ptr[seg])[rel];
+    else return sg.ptr[seg][rel];
 }
 
 __device__ __forceinline__ uint32_t find_seg(const SegTable& sg, uint64_t i) {
@@ -84,27 +115,16 @@ __device__ __forceinline__ uint32_t find_seg(const SegTable& sg, uint64_t i) {
     return lo;
 }
 
-// Loads the kEncPerThread elements of this thread (those past n read as 0).
+// The kEncPerThread elements of this thread gathered one by one (those past
+// n read as 0): threads whose elements straddle segments or are unaligned.
+template <int ES>
 __device__ __forceinline__ void load_chunk(const SegTable& sg, uint64_t i0, uint64_t n,
                                            uint16_t (&x)[kEncPerThread]) {
     uint32_t seg = find_seg(sg, i0 < n ? i0 : n - 1);
-    const uint64_t rel = i0 - sg.start[seg];
-    const uint16_t* p = sg.ptr[seg] + rel;
-    if (i0 + kEncPerThread <= sg.start[seg + 1] && (reinterpret_cast<uintptr_t>(p) & 15u) == 0) {
-        const uint4 a = __ldcs(reinterpret_cast<const uint4*>(p));
-        const uint4 b = __ldcs(reinterpret_cast<const uint4*>(p) + 1);
-        const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
-        for (int k = 0; k < 8; k++) {
-            x[2 * k] = uint16_t(w[k]);
-            x[2 * k + 1] = uint16_t(w[k] >> 16);
-        }
-    } else {
-#pragma unroll
-        for (int k = 0; k < int(kEncPerThread); k++) {
-            const uint64_t i = i0 + k;
-            x[k] = i < n ? load_elem(sg, i, seg) : uint16_t(0);
-        }
+    for (int k = 0; k < int(kEncPerThread); k++) {
+        const uint64_t i = i0 + k;
+        x[k] = i < n ? load_elem<ES>(sg, i, seg) : uint16_t(0);
     }
 }
 
@@ -149,66 +169,85 @@ __device__ __forceinline__ void stage_codes(SharedCodes& sc, const CodeTable& ct
     }
 }
 
-// One thread's kEncPerThread elements as eight words (element 2j in the low
-// half of word j), loaded ahead of use: 32 aligned bytes when they lie in one
-// segment, else gathered element by element when used.
+// One thread's kEncPerThread elements packed in words (ES = 2: element 2j
+// in the low half of word j; ES = 1: element 4j + q in byte q of word j),
+// loaded ahead of use: 16 ES aligned bytes when they lie in one segment,
+// else gathered element by element when used.
+template <int ES>
+constexpr int kWords = int(kEncPerThread) * ES / 4;
+
 struct RawElems {
-    uint4 a, b;
+    uint4 a, b;  // b unused when ES = 1
     bool direct;
 };
 
 // c0 = the chunk's first element: its segment is looked up once (the same
 // for every thread), a thread whose elements lie in a later segment looks
 // up its own.
+template <int ES>
 __device__ __forceinline__ RawElems load_raw(const SegTable& sg, uint64_t c0, uint64_t i0, uint64_t n) {
     RawElems r;
     r.direct = false;
     if (i0 < n) {
         uint32_t seg = find_seg(sg, c0);
         if (i0 >= sg.start[seg + 1]) seg = find_seg(sg, i0);
-        const uint16_t* p = sg.ptr[seg] + (i0 - sg.start[seg]);
+        const uint8_t* p = sg.ptr[seg] + ES * (i0 - sg.start[seg]);
         if (i0 + kEncPerThread <= sg.start[seg + 1] && (reinterpret_cast<uintptr_t>(p) & 15u) == 0) {
             r.a = __ldcs(reinterpret_cast<const uint4*>(p));
-            r.b = __ldcs(reinterpret_cast<const uint4*>(p) + 1);
+            if constexpr (ES == 2) r.b = __ldcs(reinterpret_cast<const uint4*>(p) + 1);
             r.direct = true;
         }
     }
     return r;
 }
 
+template <int ES>
 __device__ __forceinline__ void raw_words(const SegTable& sg, const RawElems& r, uint64_t i0, uint64_t n,
-                                          uint32_t (&w)[kEncPerThread / 2]) {
+                                          uint32_t (&w)[kWords<ES>]) {
     if (r.direct) {
         w[0] = r.a.x; w[1] = r.a.y; w[2] = r.a.z; w[3] = r.a.w;
-        w[4] = r.b.x; w[5] = r.b.y; w[6] = r.b.z; w[7] = r.b.w;
+        if constexpr (ES == 2) {
+            w[4] = r.b.x; w[5] = r.b.y; w[6] = r.b.z; w[7] = r.b.w;
+        }
     } else {
         uint16_t x[kEncPerThread];
-        load_chunk(sg, i0, n, x);
+        load_chunk<ES>(sg, i0, n, x);
 #pragma unroll
-        for (int j = 0; j < int(kEncPerThread / 2); j++) w[j] = x[2 * j] | (uint32_t(x[2 * j + 1]) << 16);
+        for (int j = 0; j < kWords<ES>; j++) {
+            if constexpr (ES == 2)
+                w[j] = x[2 * j] | (uint32_t(x[2 * j + 1]) << 16);
+            else
+                w[j] = x[4 * j] | (uint32_t(x[4 * j + 1]) << 8) | (uint32_t(x[4 * j + 2]) << 16) |
+                       (uint32_t(x[4 * j + 3]) << 24);
+        }
     }
 }
 
-__device__ __forceinline__ uint32_t elem(const uint32_t (&w)[kEncPerThread / 2], int k) {
-    return (w[k >> 1] >> (16 * (k & 1))) & 0xFFFFu;
+// The symbol of element k: the exponent field of a BF16 element, or the byte.
+template <int ES>
+__device__ __forceinline__ uint32_t symbol(const uint32_t (&w)[kWords<ES>], int k) {
+    if constexpr (ES == 2) return (w[k >> 1] >> (16 * (k & 1) + 7)) & 0xFFu;
+    else return (w[k >> 2] >> (8 * (k & 3))) & 0xFFu;
 }
 
 // Code bits of this thread's elements (those past n count 0).
-__device__ __forceinline__ uint32_t thread_bits(const SharedCodes& sc, const uint32_t (&w)[kEncPerThread / 2],
+template <int ES>
+__device__ __forceinline__ uint32_t thread_bits(const SharedCodes& sc, const uint32_t (&w)[kWords<ES>],
                                                 uint32_t valid) {
     uint32_t bits = 0;
     if (valid == kEncPerThread) {
 #pragma unroll
-        for (int k = 0; k < int(kEncPerThread); k++) bits += sc.e[(elem(w, k) >> 7) & 0xFFu].y;
+        for (int k = 0; k < int(kEncPerThread); k++) bits += sc.e[symbol<ES>(w, k)].y;
     } else {
 #pragma unroll
         for (int k = 0; k < int(kEncPerThread); k++)
-            if (uint32_t(k) < valid) bits += sc.e[(elem(w, k) >> 7) & 0xFFu].y;
+            if (uint32_t(k) < valid) bits += sc.e[symbol<ES>(w, k)].y;
     }
     return bits;
 }
 
 // Bits of code per chunk.
+template <int ES>
 __global__ void __launch_bounds__(kEncThreads) chunk_bits_kernel(const __grid_constant__ SegTable sg,
                                                                  const __grid_constant__ CodeTable ct,
                                                                  uint64_t n, uint64_t n_chunks,
@@ -219,18 +258,18 @@ __global__ void __launch_bounds__(kEncThreads) chunk_bits_kernel(const __grid_co
     __syncthreads();
     const uint64_t tofs = uint64_t(threadIdx.x) * kEncPerThread;
     uint64_t c = blockIdx.x;
-    RawElems next = load_raw(sg, c * kEncChunk, c * kEncChunk + tofs, n);
+    RawElems next = load_raw<ES>(sg, c * kEncChunk, c * kEncChunk + tofs, n);
     for (; c < n_chunks; c += gridDim.x) {
         const RawElems cur = next;
         const uint64_t i0 = c * kEncChunk + tofs;
         if (c + gridDim.x < n_chunks)
-            next = load_raw(sg, (c + gridDim.x) * kEncChunk, (c + gridDim.x) * kEncChunk + tofs, n);
+            next = load_raw<ES>(sg, (c + gridDim.x) * kEncChunk, (c + gridDim.x) * kEncChunk + tofs, n);
         uint32_t bits = 0;
         if (i0 < n) {
-            uint32_t w[kEncPerThread / 2];
-            raw_words(sg, cur, i0, n, w);
+            uint32_t w[kWords<ES>];
+            raw_words<ES>(sg, cur, i0, n, w);
             const uint64_t left = n - i0;
-            bits = thread_bits(sc, w, left < kEncPerThread ? uint32_t(left) : kEncPerThread);
+            bits = thread_bits<ES>(sc, w, left < kEncPerThread ? uint32_t(left) : kEncPerThread);
         }
         uint32_t total;
         block_exclusive_scan<kEncThreads>(bits, s_warp, total);
@@ -320,6 +359,7 @@ constexpr int kPackWords = kEncChunk + 4;  // 32 bits per element at most, plus 
 constexpr int kMaxEvents = (int(kEncPerThread) * 32) / 64 + 1;
 static_assert(kPackWords % 4 == 0, "image cleared in 16-byte stores");
 
+template <int ES>
 __global__ void __launch_bounds__(kEncThreads) pack_kernel(const __grid_constant__ SegTable sg,
                                                            const __grid_constant__ CodeTable ct, uint64_t n,
                                                            uint64_t n_chunks, uint32_t log2_block_bits,
@@ -336,19 +376,19 @@ __global__ void __launch_bounds__(kEncThreads) pack_kernel(const __grid_constant
     const uint64_t block_mask = (uint64_t(1) << log2_block_bits) - 1;
     const uint64_t tofs = uint64_t(threadIdx.x) * kEncPerThread;
     uint64_t c = blockIdx.x;
-    RawElems next = load_raw(sg, c * kEncChunk, c * kEncChunk + tofs, n);
+    RawElems next = load_raw<ES>(sg, c * kEncChunk, c * kEncChunk + tofs, n);
     for (; c < n_chunks; c += gridDim.x) {
         const RawElems cur = next;
         const uint64_t i0 = c * kEncChunk + tofs;
         if (c + gridDim.x < n_chunks)
-            next = load_raw(sg, (c + gridDim.x) * kEncChunk, (c + gridDim.x) * kEncChunk + tofs, n);
-        uint32_t w8[kEncPerThread / 2];
+            next = load_raw<ES>(sg, (c + gridDim.x) * kEncChunk, (c + gridDim.x) * kEncChunk + tofs, n);
+        uint32_t w8[kWords<ES>];
         uint32_t valid = 0, bits = 0;
         if (i0 < n) {
-            raw_words(sg, cur, i0, n, w8);
+            raw_words<ES>(sg, cur, i0, n, w8);
             const uint64_t left = n - i0;
             valid = left < kEncPerThread ? uint32_t(left) : kEncPerThread;
-            bits = thread_bits(sc, w8, valid);
+            bits = thread_bits<ES>(sc, w8, valid);
         }
         for (int j = threadIdx.x; j < kPackWords / 4; j += kEncThreads)
             reinterpret_cast<uint4*>(s_words)[j] = make_uint4(0, 0, 0, 0);
@@ -391,7 +431,7 @@ __global__ void __launch_bounds__(kEncThreads) pack_kernel(const __grid_constant
 #pragma unroll
             for (int k = 0; k < int(kEncPerThread); k++) {
                 if (!kFull && uint32_t(k) >= valid) break;
-                const uint2 ce = sc.e[(elem(w8, k) >> 7) & 0xFFu];
+                const uint2 ce = sc.e[symbol<ES>(w8, k)];
                 const uint32_t t = ce.x, l = ce.y;
                 cur_word |= t >> fill;
                 const uint32_t spill = __funnelshift_r(0u, t, fill);  // bits that did not fit
@@ -416,8 +456,8 @@ __global__ void __launch_bounds__(kEncThreads) pack_kernel(const __grid_constant
             pack_codes(std::true_type{});
         else if (valid)
             pack_codes(std::false_type{});
-        if (valid) {
-            if (n - i0 <= kEncPerThread) block_off[n_blocks] = uint32_t(n);
+        if (valid && n - i0 <= kEncPerThread) block_off[n_blocks] = uint32_t(n);
+        if constexpr (ES == 2) if (valid) {
             // sign+mantissa bytes: sign (bit 15) to bit 7, mantissa bits 6..0
             uint32_t smw[kEncPerThread / 4];
 #pragma unroll
@@ -502,7 +542,7 @@ df11_status build_segtable(const void* const* d_segs, const uint64_t* counts, ui
         if (counts[k] && !d_segs[k]) return fail(DF11_ERR_INVALID, "null segment %u", k);
         if (counts[k] && !aligned16(d_segs[k]))
             return fail(DF11_ERR_INVALID, "segment %u is not 16-byte aligned", k);
-        sg->ptr[k] = static_cast<const uint16_t*>(d_segs[k]);
+        sg->ptr[k] = static_cast<const uint8_t*>(d_segs[k]);
         sg->start[k] = acc;
         acc += counts[k];
     }
@@ -513,20 +553,17 @@ df11_status build_segtable(const void* const* d_segs, const uint64_t* counts, ui
     return DF11_OK;
 }
 
-}  // namespace
-}  // namespace df11
-
-using namespace df11;
-
-extern "C" df11_status df11_compress_plan(const void* const* d_segs, const uint64_t* seg_counts, uint32_t n_segs,
-                                          uint32_t threads_per_block, uint32_t max_code_len, void* d_workspace,
-                                          uint64_t workspace_bytes, df11_header* hdr, void* stream) {
+// Histogram kernels (one launch per segment), host code builder, header.
+template <int ES>
+df11_status compress_plan(const void* const* d_segs, const uint64_t* seg_counts, uint32_t n_segs,
+                          uint32_t threads_per_block, uint32_t max_code_len, void* d_workspace,
+                          uint64_t workspace_bytes, df11_header* hdr, void* stream) {
     if (!hdr) return fail(DF11_ERR_INVALID, "null header");
     SegTable sg;
     uint64_t n = 0;
     df11_status st = build_segtable(d_segs, seg_counts, n_segs, &sg, &n);
     if (st != DF11_OK) return st;
-    Workspace w;
+    Workspace w{};
     st = carve(d_workspace, workspace_bytes, n, &w);
     if (st != DF11_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -538,10 +575,14 @@ extern "C" df11_status df11_compress_plan(const void* const* d_segs, const uint6
     for (uint32_t k = 0; k < n_segs; k++) {
         const uint64_t cnt = seg_counts[k];
         if (!cnt) continue;
-        const uint64_t vec_blocks = (cnt / 8 + kHistThreads - 1) / kHistThreads;
+        const uint64_t vec_blocks = (cnt / (16 / ES) + kHistThreads - 1) / kHistThreads;
         uint64_t grid = vec_blocks < uint64_t(4 * sms) ? vec_blocks : uint64_t(4 * sms);
         if (grid == 0) grid = 1;
-        histogram_kernel<<<unsigned(grid), kHistThreads, 0, s>>>(sg.ptr[k], cnt, w.hist);
+        if constexpr (ES == 2)
+            histogram_kernel<<<unsigned(grid), kHistThreads, 0, s>>>(
+                reinterpret_cast<const uint16_t*>(sg.ptr[k]), cnt, w.hist);
+        else
+            histogram_u8_kernel<<<unsigned(grid), kHistThreads, 0, s>>>(sg.ptr[k], cnt, w.hist);
     }
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail("histogram launch", e);
@@ -558,10 +599,12 @@ extern "C" df11_status df11_compress_plan(const void* const* d_segs, const uint6
     return df11_header_init(hdr, len, n, bits, threads_per_block, max_code_len, seg_counts, n_segs);
 }
 
-extern "C" df11_status df11_compress_encode(const void* const* d_segs, const df11_header* hdr, void* d_workspace,
-                                            uint64_t workspace_bytes, uint8_t* d_exp, uint8_t* d_sm,
-                                            uint8_t* d_gaps, uint32_t* d_block_off, void* d_lut,
-                                            void* stream) {
+// Table upload, clears, then the chunk-bits, scan and bit-pack kernels.
+// d_sm is written for BF16 input (ES = 2) only.
+template <int ES>
+df11_status compress_encode(const char* fn, const void* const* d_segs, const df11_header* hdr,
+                            uint32_t* chunk_bits, unsigned long long* chunk_start, uint8_t* d_exp, uint8_t* d_sm,
+                            uint8_t* d_gaps, uint32_t* d_block_off, void* d_lut, void* stream) {
     df11_status st = check_header(hdr);
     if (st != DF11_OK) return st;
     uint64_t counts[DF11_MAX_SEGMENTS];
@@ -573,48 +616,90 @@ extern "C" df11_status df11_compress_encode(const void* const* d_segs, const df1
     st = build_segtable(d_segs, counts, hdr->n_segments, &sg, &n);
     if (st != DF11_OK) return st;
     if (n != hdr->n_elems) return fail(DF11_ERR_INVALID, "segments disagree with header n_elems");
-    if (!d_exp || !d_sm || !d_gaps || !d_block_off || !d_lut)
-        return fail(DF11_ERR_INVALID, "df11_compress_encode: null output pointer");
-    if (!aligned16(d_exp) || !aligned16(d_sm) || !aligned16(d_gaps) || !aligned16(d_block_off) ||
+    if (!d_exp || (ES == 2 && !d_sm) || !d_gaps || !d_block_off || !d_lut)
+        return fail(DF11_ERR_INVALID, "%s: null output pointer", fn);
+    if (!aligned16(d_exp) || (ES == 2 && !aligned16(d_sm)) || !aligned16(d_gaps) || !aligned16(d_block_off) ||
         !aligned16(d_lut))
-        return fail(DF11_ERR_INVALID, "df11_compress_encode: outputs must be 16-byte aligned");
-    Workspace w;
-    st = carve(d_workspace, workspace_bytes, n, &w);
-    if (st != DF11_OK) return st;
+        return fail(DF11_ERR_INVALID, "%s: outputs must be 16-byte aligned", fn);
 
     CodeTable ct;
     std::memcpy(ct.len, hdr->code_len, 256);
     if (!canonical_codes(hdr->code_len, ct.code)) return fail(DF11_ERR_INVALID, "code lengths overflow");
-    std::vector<uint8_t> lut(kLutBytes);
-    st = df11_build_lut(hdr, lut.data(), lut.size());
+    // decode tables are built in this thread's own host buffer (no heap)
+    static thread_local unsigned char lut[kLutBytes];
+    st = df11_build_lut(hdr, lut, sizeof(lut));
     if (st != DF11_OK) return st;
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     cudaError_t e;
-    if ((e = cudaMemcpyAsync(d_lut, lut.data(), kLutBytes, cudaMemcpyHostToDevice, s)) != cudaSuccess)
+    if ((e = cudaMemcpyAsync(d_lut, lut, kLutBytes, cudaMemcpyHostToDevice, s)) != cudaSuccess)
         return cuda_fail("table upload", e);
     if ((e = cudaMemsetAsync(d_exp, 0, hdr->bytes_exp, s)) != cudaSuccess) return cuda_fail("clear exp", e);
     if ((e = cudaMemsetAsync(d_gaps, 0, hdr->bytes_gaps, s)) != cudaSuccess) return cuda_fail("clear gaps", e);
     if ((e = cudaMemsetAsync(d_block_off, 0, hdr->bytes_off, s)) != cudaSuccess) return cuda_fail("clear off", e);
-    const uint64_t sm_tail = n & ~uint64_t(15);
-    if (hdr->bytes_sm > sm_tail &&
-        (e = cudaMemsetAsync(d_sm + sm_tail, 0, hdr->bytes_sm - sm_tail, s)) != cudaSuccess)
-        return cuda_fail("clear sm tail", e);
+    if constexpr (ES == 2) {
+        const uint64_t sm_tail = n & ~uint64_t(15);
+        if (hdr->bytes_sm > sm_tail &&
+            (e = cudaMemsetAsync(d_sm + sm_tail, 0, hdr->bytes_sm - sm_tail, s)) != cudaSuccess)
+            return cuda_fail("clear sm tail", e);
+    }
     if (n == 0) return DF11_OK;
 
     const uint64_t chunks = (n + kEncChunk - 1) / kEncChunk;
     if (chunks >= (uint64_t(1) << 31)) return fail(DF11_ERR_TOO_LARGE, "too many chunks");
-    chunk_bits_kernel<<<encode_grid(chunk_bits_kernel, chunks), kEncThreads, 0, s>>>(sg, ct, n, chunks, w.chunk_bits);
-    chunk_scan_kernel<<<1, kScanThreads, 0, s>>>(w.chunk_bits, chunks, w.chunk_start);
+    chunk_bits_kernel<ES><<<encode_grid(chunk_bits_kernel<ES>, chunks), kEncThreads, 0, s>>>(sg, ct, n, chunks,
+                                                                                          chunk_bits);
+    chunk_scan_kernel<<<1, kScanThreads, 0, s>>>(chunk_bits, chunks, chunk_start);
     uint32_t log2_bb = 6;
     while ((1u << (log2_bb - 6)) < hdr->threads_per_block) log2_bb++;
-    pack_kernel<<<encode_grid(pack_kernel, chunks), kEncThreads, 0, s>>>(sg, ct, n, chunks, log2_bb, w.chunk_start,
-                                                         reinterpret_cast<uint32_t*>(d_exp), d_sm,
-                                                         reinterpret_cast<uint32_t*>(d_gaps), d_block_off,
-                                                         hdr->n_blocks);
+    pack_kernel<ES><<<encode_grid(pack_kernel<ES>, chunks), kEncThreads, 0, s>>>(
+        sg, ct, n, chunks, log2_bb, chunk_start, reinterpret_cast<uint32_t*>(d_exp), d_sm,
+        reinterpret_cast<uint32_t*>(d_gaps), d_block_off, hdr->n_blocks);
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail("encode launch", e);
     return DF11_OK;
+}
+
+}  // namespace
+}  // namespace df11
+
+using namespace df11;
+
+extern "C" df11_status df11_compress_plan(const void* const* d_segs, const uint64_t* seg_counts, uint32_t n_segs,
+                                          uint32_t threads_per_block, uint32_t max_code_len, void* d_workspace,
+                                          uint64_t workspace_bytes, df11_header* hdr, void* stream) {
+    return compress_plan<2>(d_segs, seg_counts, n_segs, threads_per_block, max_code_len, d_workspace,
+                            workspace_bytes, hdr, stream);
+}
+
+extern "C" df11_status df11_compress_encode(const void* const* d_segs, const df11_header* hdr, void* d_workspace,
+                                            uint64_t workspace_bytes, uint8_t* d_exp, uint8_t* d_sm,
+                                            uint8_t* d_gaps, uint32_t* d_block_off, void* d_lut,
+                                            void* stream) {
+    Workspace w{};
+    const df11_status st = carve(d_workspace, workspace_bytes, hdr ? hdr->n_elems : 0, &w);
+    if (st != DF11_OK) return st;
+    return compress_encode<2>("df11_compress_encode", d_segs, hdr, w.chunk_bits, w.chunk_start, d_exp, d_sm, d_gaps,
+                              d_block_off, d_lut, stream);
+}
+
+extern "C" df11_status df11_compress_plan_u8(const void* const* d_segs, const uint64_t* seg_counts,
+                                             uint32_t n_segs, uint32_t threads_per_block, uint32_t max_code_len,
+                                             void* d_workspace, uint64_t workspace_bytes, df11_header* hdr,
+                                             void* stream) {
+    return compress_plan<1>(d_segs, seg_counts, n_segs, threads_per_block, max_code_len, d_workspace,
+                            workspace_bytes, hdr, stream);
+}
+
+extern "C" df11_status df11_compress_encode_u8(const void* const* d_segs, const df11_header* hdr,
+                                               void* d_workspace, uint64_t workspace_bytes, uint8_t* d_exp,
+                                               uint8_t* d_gaps, uint32_t* d_block_off, void* d_lut,
+                                               void* stream) {
+    Workspace w{};
+    const df11_status st = carve(d_workspace, workspace_bytes, hdr ? hdr->n_elems : 0, &w);
+    if (st != DF11_OK) return st;
+    return compress_encode<1>("df11_compress_encode_u8", d_segs, hdr, w.chunk_bits, w.chunk_start, d_exp,
+                              nullptr, d_gaps, d_block_off, d_lut, stream);
 }
 
 // ---------------------------------------------------------------------------
@@ -677,58 +762,12 @@ extern "C" df11_status df11_compress_encode_static(const void* const* d_segs, co
                     "df11_compress_encode_static: %llu elements, its fixed scratch holds at most %llu; "
                     "use df11_compress_encode with a workspace",
                     (unsigned long long)hdr->n_elems, (unsigned long long)DF11_STATIC_MAX_ELEMS);
-    uint64_t counts[DF11_MAX_SEGMENTS];
-    if (hdr->n_segments < 1 || hdr->n_segments > DF11_MAX_SEGMENTS)
-        return fail(DF11_ERR_INVALID, "header n_segments %u", hdr->n_segments);
-    for (uint32_t k = 0; k < hdr->n_segments; k++) counts[k] = hdr->seg_elem_off[k + 1] - hdr->seg_elem_off[k];
-    SegTable sg;
-    uint64_t n = 0;
-    st = build_segtable(d_segs, counts, hdr->n_segments, &sg, &n);
-    if (st != DF11_OK) return st;
-    if (n != hdr->n_elems) return fail(DF11_ERR_INVALID, "segments disagree with header n_elems");
-    if (!d_exp || !d_sm || !d_gaps || !d_block_off || !d_lut)
-        return fail(DF11_ERR_INVALID, "df11_compress_encode_static: null output pointer");
-    if (!aligned16(d_exp) || !aligned16(d_sm) || !aligned16(d_gaps) || !aligned16(d_block_off) ||
-        !aligned16(d_lut))
-        return fail(DF11_ERR_INVALID, "df11_compress_encode_static: outputs must be 16-byte aligned");
     void* scratch = nullptr;
     st = static_scratch_address(&scratch);
     if (st != DF11_OK) return st;
     uint32_t* chunk_bits = static_cast<uint32_t*>(scratch);
     unsigned long long* chunk_start =
         reinterpret_cast<unsigned long long*>(static_cast<unsigned char*>(scratch) + kStaticBitsBytes);
-
-    CodeTable ct;
-    std::memcpy(ct.len, hdr->code_len, 256);
-    if (!canonical_codes(hdr->code_len, ct.code)) return fail(DF11_ERR_INVALID, "code lengths overflow");
-    // decode tables are built in this thread's own host buffer (no heap)
-    static thread_local unsigned char lut[kLutBytes];
-    st = df11_build_lut(hdr, lut, sizeof(lut));
-    if (st != DF11_OK) return st;
-
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    cudaError_t e;
-    if ((e = cudaMemcpyAsync(d_lut, lut, kLutBytes, cudaMemcpyHostToDevice, s)) != cudaSuccess)
-        return cuda_fail("table upload", e);
-    if ((e = cudaMemsetAsync(d_exp, 0, hdr->bytes_exp, s)) != cudaSuccess) return cuda_fail("clear exp", e);
-    if ((e = cudaMemsetAsync(d_gaps, 0, hdr->bytes_gaps, s)) != cudaSuccess) return cuda_fail("clear gaps", e);
-    if ((e = cudaMemsetAsync(d_block_off, 0, hdr->bytes_off, s)) != cudaSuccess) return cuda_fail("clear off", e);
-    const uint64_t sm_tail = n & ~uint64_t(15);
-    if (hdr->bytes_sm > sm_tail &&
-        (e = cudaMemsetAsync(d_sm + sm_tail, 0, hdr->bytes_sm - sm_tail, s)) != cudaSuccess)
-        return cuda_fail("clear sm tail", e);
-    if (n == 0) return DF11_OK;
-
-    const uint64_t chunks = (n + kEncChunk - 1) / kEncChunk;
-    chunk_bits_kernel<<<encode_grid(chunk_bits_kernel, chunks), kEncThreads, 0, s>>>(sg, ct, n, chunks, chunk_bits);
-    chunk_scan_kernel<<<1, kScanThreads, 0, s>>>(chunk_bits, chunks, chunk_start);
-    uint32_t log2_bb = 6;
-    while ((1u << (log2_bb - 6)) < hdr->threads_per_block) log2_bb++;
-    pack_kernel<<<encode_grid(pack_kernel, chunks), kEncThreads, 0, s>>>(sg, ct, n, chunks, log2_bb, chunk_start,
-                                                         reinterpret_cast<uint32_t*>(d_exp), d_sm,
-                                                         reinterpret_cast<uint32_t*>(d_gaps), d_block_off,
-                                                         hdr->n_blocks);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_fail("encode launch", e);
-    return DF11_OK;
+    return compress_encode<2>("df11_compress_encode_static", d_segs, hdr, chunk_bits, chunk_start, d_exp, d_sm,
+                              d_gaps, d_block_off, d_lut, stream);
 }

@@ -41,7 +41,7 @@ SIGMA_DEFAULT = 0.02
 class Workload:
     name: str
     names: list[str]          # one per matrix / vector
-    tensors: list[torch.Tensor]  # bfloat16, 1-D or 2-D, same device
+    tensors: list[torch.Tensor]  # bfloat16 (uint8 for 8-bit symbol workloads), 1-D or 2-D, same device
 
     @property
     def n_elems(self) -> int:
@@ -183,3 +183,31 @@ def fibonacci(k: int = 34, seed: int = 11, first_exponent: int = 100) -> Workloa
     e = e[torch.randperm(e.numel(), generator=g)]
     sm = torch.randint(0, 256, (e.numel(),), generator=g)
     return Workload(f"fibonacci_{k}", ["x"], [_bf16_from_fields(e, sm)])
+
+
+# --------------------------------------------------------------------------- #
+# 8-bit symbol streams                                                        #
+# --------------------------------------------------------------------------- #
+def quantize_u8(t: torch.Tensor) -> torch.Tensor:
+    """Per-tensor asymmetric 8-bit quantisation: the tensor's range [min, max]
+    mapped onto 0..255 (round to nearest).  Generates the kind of integer
+    symbols an entropy coder of quantized weights sees; the codec itself
+    takes the bytes as they are."""
+    x = t.float()
+    lo, hi = x.min(), x.max()
+    scale = (hi - lo).clamp_min(1e-30) / 255.0
+    return torch.round((x - lo) / scale).clamp_(0, 255).to(torch.uint8)
+
+
+def llama_block_u8(cfg: dict = LLAMA_8B, seed_base: int = 3, device: str = "cpu") -> Workload:
+    """The matrices of `llama_block` quantized per tensor to uint8."""
+    w = llama_block(cfg, seed_base, device)
+    return Workload(w.name + "-u8", list(w.names), [quantize_u8(t) for t in w.tensors])
+
+
+def edge_case_u8(n: int, dist: str, seed: int) -> Workload:
+    """n bytes with the symbol distribution of `edge_case` (uniform over
+    0..254, 99.9% one value, Zipf over a permuted alphabet)."""
+    w = edge_case(n, dist, seed)
+    x = w.tensors[0].view(torch.int16).to(torch.int32)
+    return Workload(f"edge_u8_{dist}_{n}", ["x"], [((x >> 7) & 0xFF).to(torch.uint8)])
