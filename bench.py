@@ -35,6 +35,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "decompressed BF16 GB/s on 1 B200 (bit-exact), % of HBM roofline"
+METRIC_U8 = "decompressed 8-bit symbols GB/s on 1 B200 (bit-exact), % of HBM roofline"
 UNIT = "GB/s"
 FALLBACK_HBM_GBS = 6650.0
 L2_BYTES = 126 * 2**20  # B200 L2 capacity
@@ -48,7 +49,10 @@ CONFIGS = {
           "2 RMSNorm 4096; 218,112,000 BF16 weights, one table, one launch",
     "c4": "8 llama3.1-70b-blocks: hidden 8192, intermediate 28672, kv 1024x8192; 855,654,400 weights "
           "per block, each block one launch into one reused buffer",
+    "c5": "llama3.1-8b-block quantized per tensor to uint8 (asymmetric, round to nearest); 218,112,000 "
+          "8-bit symbols coded whole with one table, no side array, one launch",
 }
+U8_CONFIGS = {"c5"}
 
 
 # --------------------------------------------------------------------------- #
@@ -205,6 +209,8 @@ def make_workloads(config: str, rank: int, device: str):
         return [I.llama_block(I.LLAMA_8B, seed_base=3 + off, device=device)]
     if config == "c4":
         return [I.llama_block(I.LLAMA_70B, seed_base=100 + 16 * b + off, device=device) for b in range(8)]
+    if config == "c5":
+        return [I.llama_block_u8(I.LLAMA_8B, seed_base=3 + off, device=device)]
     raise ValueError(config)
 
 
@@ -213,6 +219,11 @@ def reference_sample(config: str, n_target: int):
     workload's concatenated matrices, drawn with the CPU generator."""
     import numpy as np
     from lossless_entropy_coded_dfloat11_b200 import inputs as I
+    if config == "c5":
+        # the oracle codes byte v as the exponent field of the BF16 pattern v << 7
+        w = I.llama_block_u8(I.LLAMA_8B, seed_base=3)
+        v = np.concatenate([t.reshape(-1).numpy() for t in w.tensors])[:n_target]
+        return v.astype(np.uint16) << 7
     if config == "c4":
         cfg, base = I.LLAMA_70B, 100
     elif config == "c3":
@@ -257,9 +268,10 @@ def run_reference(args, rank: int, world: int) -> None:
     n_sample = args.ref_sample
     x = reference_sample(args.config, n_sample)
     dt, s = time_oracle_decode(x, args.steps, args.warmup)
-    value = 2 * x.size * args.steps / dt / 1e9
+    esize = 1 if args.config in U8_CONFIGS else 2  # output bytes per element
+    value = esize * x.size * args.steps / dt / 1e9
     line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "impl": "reference", "metric": METRIC_U8 if esize == 1 else METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u8",
         "data": "synthetic",
@@ -273,7 +285,7 @@ def run_reference(args, rank: int, world: int) -> None:
     print(json.dumps(line), flush=True)
 
 
-def time_compress(df11, w, repeats: int) -> dict:
+def time_compress(df11, w, repeats: int, u8: bool = False) -> dict:
     """Wall-clock time of the public compress call on device-resident BF16
     tensors (histogram kernel, host code build, table upload, bit-pack
     kernels), synchronised on both sides; the median of `repeats` calls after
@@ -283,16 +295,18 @@ def time_compress(df11, w, repeats: int) -> dict:
     for r in range(repeats + 1):
         torch.cuda.synchronize()
         t0 = time.perf_counter()
-        cs = df11.compress(w.tensors, names=w.names)
+        cs = (df11.compress_u8 if u8 else df11.compress)(w.tensors, names=w.names)
         torch.cuda.synchronize()
         if r:
             times.append(time.perf_counter() - t0)
         del cs
     t = sorted(times)[len(times) // 2]
-    in_bytes = sum(2 * x.numel() for x in w.tensors)
-    return {"value": in_bytes / t / 1e9, "unit": "GB/s of BF16 input", "ms": t * 1e3,
-            "repeats": repeats, "elements": in_bytes // 2,
-            "what": "df11.compress on device-resident BF16: histogram kernel, host package-merge and "
+    in_bytes = sum(x.numel() * x.element_size() for x in w.tensors)
+    return {"value": in_bytes / t / 1e9, "unit": "GB/s of uint8 input" if u8 else "GB/s of BF16 input",
+            "ms": t * 1e3,
+            "repeats": repeats, "elements": sum(x.numel() for x in w.tensors),
+            "what": f"df11.{'compress_u8' if u8 else 'compress'} on device-resident "
+                    f"{'uint8' if u8 else 'BF16'} tensors: histogram kernel, host package-merge and "
                     "table build, bit-pack kernels; median wall clock, synchronised"}
 
 
@@ -308,14 +322,17 @@ def run_native(args, rank: int, world: int, local_rank: int) -> None:
 
     # ---- build the compressed workload on this GPU ------------------------
     workloads = make_workloads(args.config, rank, "cuda")
+    u8 = args.config in U8_CONFIGS  # 8-bit symbols: uint8 out, no side array
+    esize = 1 if u8 else 2          # output bytes per element
+    bits16 = (lambda t: t) if u8 else (lambda t: t.view(torch.int16))
     streams, originals = [], []
     compress = None
     for w in workloads:
         if compress is None and not args.no_compress:
-            compress = time_compress(df11, w, args.compress_repeats)
-        cs = df11.compress(w.tensors, names=w.names)
+            compress = time_compress(df11, w, args.compress_repeats, u8)
+        cs = (df11.compress_u8 if u8 else df11.compress)(w.tensors, names=w.names)
         streams.append(cs)
-        originals.append(torch.cat([t.reshape(-1) for t in w.tensors]).view(torch.int16)
+        originals.append(bits16(torch.cat([t.reshape(-1) for t in w.tensors]))
                          if len(workloads) == 1 else None)
         if len(workloads) > 1:
             # keep a fingerprint per block instead of all 6.9B weights
@@ -323,15 +340,16 @@ def run_native(args, rank: int, world: int, local_rank: int) -> None:
         del w
     torch.cuda.synchronize()
     n_max = max(cs.n_elems for cs in streams)
-    out = torch.empty(n_max, dtype=torch.bfloat16, device=dev)
+    out = torch.empty(max(n_max, 16), dtype=torch.uint8 if u8 else torch.bfloat16, device=dev)
     stream = torch.cuda.current_stream()
-    out_bytes = sum(2 * cs.n_elems for cs in streams)
-    alg_bytes = sum(cs.read_bytes() + 2 * cs.n_elems for cs in streams)
+    out_bytes = sum(esize * cs.n_elems for cs in streams)
+    alg_bytes = sum(cs.read_bytes() + esize * cs.n_elems for cs in streams)
     launches_per_step = len(streams)
+    decode = df11.decompress_u8 if u8 else df11.decompress
 
     def step():
         for cs in streams:
-            df11.decompress(cs, out=out[: cs.n_elems], stream=stream)
+            decode(cs, out=out[: cs.n_elems], stream=stream)
 
     for _ in range(args.warmup):
         step()
@@ -370,7 +388,7 @@ def run_native(args, rank: int, world: int, local_rank: int) -> None:
     # ---- bit-exact check of the last step's output --------------------------
     exact = True
     if len(streams) == 1:
-        exact = bool(torch.equal(out[: streams[0].n_elems].view(torch.int16), originals[0]))
+        exact = bool(torch.equal(bits16(out[: streams[0].n_elems]), originals[0]))
     else:
         for cs, fp in zip(streams, originals):
             step_out = df11.decompress(cs, out=out[: cs.n_elems], stream=stream)
@@ -400,8 +418,8 @@ def run_native(args, rank: int, world: int, local_rank: int) -> None:
         e1.record(stream)
         torch.cuda.synchronize()
         ems = max_over_ranks(e0.elapsed_time(e1), dev)
-        e2e_exact = bool(torch.equal(res.view(torch.int16), originals[0].cpu()))
-        e2e = {"value": 2 * streams[0].n_elems * k * world / (ems * 1e-3) / 1e9, "unit": UNIT,
+        e2e_exact = bool(torch.equal(bits16(res), originals[0].cpu()))
+        e2e = {"value": esize * streams[0].n_elems * k * world / (ems * 1e-3) / 1e9, "unit": UNIT,
                "h2d_bytes_per_step": hs.h2d_bytes(), "d2h_bytes_per_step": hs.d2h_bytes(),
                "steps": k, "bit_exact": e2e_exact}
         del hs
@@ -411,11 +429,13 @@ def run_native(args, rank: int, world: int, local_rank: int) -> None:
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         n_sample = min(args.cpu_sample, streams[0].n_elems)
         if len(streams) == 1:
-            x = originals[0][:n_sample].cpu().numpy().view(np.uint16)
+            x = originals[0][:n_sample].cpu().numpy()
+            # the oracle codes byte v as the exponent field of the BF16 pattern v << 7
+            x = x.astype(np.uint16) << 7 if u8 else x.view(np.uint16)
         else:
             x = reference_sample(args.config, n_sample)
         dt, _ = time_oracle_decode(x, 1, 0)
-        cpu = {"value": 2 * x.size / dt / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
+        cpu = {"value": esize * x.size / dt / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
                "sample": f"first {x.size} elements of the workload, oracle bit-serial decode, one "
                          f"thread on {cpu_model()} ({os.cpu_count()} host cores present)",
                "seconds": dt}
@@ -428,18 +448,19 @@ def run_native(args, rank: int, world: int, local_rank: int) -> None:
     traffic = recorded_traffic() if args.config == "c3" else None
     cs0 = streams[0]
     line = {
-        "metric": METRIC, "value": agg["gbs"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "metric": METRIC_U8 if u8 else METRIC, "value": agg["gbs"], "unit": UNIT, "n_gpus": world,
+        "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": agg["ms_per_step"], "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "u8", "data": "synthetic",
         "config": {"workload": CONFIGS[args.config], "elements_per_step": sum(c.n_elems for c in streams),
                    "threads_per_block": cs0.threads_per_block, "launches_per_step": launches_per_step,
-                   "l2": ("no flush: compressed input + BF16 output per step exceed the 126 MB L2"
+                   "l2": ("no flush: compressed input + output per step exceed the 126 MB L2"
                           if flush is None else
                           f"flushed: a {2 * L2_BYTES >> 20} MiB buffer is written before each step; "
                           "per-step CUDA events time the decode alone"),
                    "parallelism": f"replicas x{world} (independent streams per rank)"},
         "bit_exact": exact,
-        "elements_per_s": agg["gbs"] * 1e9 / 2,
+        "elements_per_s": agg["gbs"] * 1e9 / esize,
         "compression_ratio": sum(c.compressed_bytes() for c in streams) / out_bytes,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic,

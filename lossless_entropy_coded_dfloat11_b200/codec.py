@@ -230,30 +230,36 @@ def decompress(cs: CompressedStream, out: torch.Tensor | None = None, status: to
 
 class HostStream:
     """A stream kept in pinned host memory, decompressed end to end: copy the
-    compressed arrays to the device, decode, copy the BF16 result back."""
+    compressed arrays to the device, decode, copy the result (BF16, or bytes
+    for a stream of 8-bit symbols) back."""
 
     def __init__(self, cs: CompressedStream):
         self.header = cs.header
-        self.host = {k: getattr(cs, k).cpu().pin_memory() for k in ("exp", "sm", "gaps", "block_off", "lut")}
+        self.u8 = cs.symbols == "u8"
+        keys = ("exp", "gaps", "block_off", "lut") if self.u8 else ("exp", "sm", "gaps", "block_off", "lut")
+        self.host = {k: getattr(cs, k).cpu().pin_memory() for k in keys}
         dev = cs.exp.device
         self.dev = {k: torch.empty_like(v, device=dev) for k, v in self.host.items()}
-        self.dev_stream = CompressedStream(cs.header, self.dev["exp"], self.dev["sm"], self.dev["gaps"],
-                                           self.dev["block_off"], self.dev["lut"], cs.names, cs.shapes)
-        self.out_dev = torch.empty(max(cs.n_elems, 1), dtype=torch.bfloat16, device=dev)[: cs.n_elems]
-        self.out_host = torch.empty(max(cs.n_elems, 1), dtype=torch.bfloat16).pin_memory()[: cs.n_elems]
+        self.dev_stream = CompressedStream(cs.header, self.dev["exp"], self.dev.get("sm", cs.sm), self.dev["gaps"],
+                                           self.dev["block_off"], self.dev["lut"], cs.names, cs.shapes,
+                                           symbols=cs.symbols)
+        dtype = torch.uint8 if self.u8 else torch.bfloat16
+        n = cs.n_elems
+        self.out_dev = torch.empty(max(n, 16), dtype=dtype, device=dev)[:n]
+        self.out_host = torch.empty(max(n, 16), dtype=dtype).pin_memory()[:n]
 
     def h2d_bytes(self) -> int:
         return sum(v.numel() * v.element_size() for v in self.host.values())
 
     def d2h_bytes(self) -> int:
-        return 2 * int(self.header.n_elems)
+        return self.out_host.element_size() * int(self.header.n_elems)
 
     def run(self, stream=None) -> torch.Tensor:
         s = stream or torch.cuda.current_stream()
         with torch.cuda.stream(s):
             for k, v in self.host.items():
                 self.dev[k].copy_(v, non_blocking=True)
-            decompress(self.dev_stream, self.out_dev, stream=s)
+            (decompress_u8 if self.u8 else decompress)(self.dev_stream, self.out_dev, stream=s)
             self.out_host.copy_(self.out_dev, non_blocking=True)
         return self.out_host
 
