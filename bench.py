@@ -259,6 +259,30 @@ def time_oracle_decode(x, steps: int, warmup: int):
     return dt, s
 
 
+def time_oracle_decode_parallel(s, x, threads: int) -> float:
+    """The oracle's windowed decoder on `threads` host threads, one range of
+    thread blocks per task: ranges decode independently through their Gaps and
+    block offsets, the format's own parallel structure (the C oracle runs
+    without the interpreter lock).  Returns seconds for one full decode,
+    checked against x."""
+    import numpy as np
+    import oracle
+    from concurrent.futures import ThreadPoolExecutor
+    parts = max(1, min(int(s.n_blocks), 8 * threads))
+    bounds = [int(s.n_blocks) * k // parts for k in range(parts + 1)]
+
+    def run(pool):
+        return list(pool.map(lambda k: oracle.decode_windowed(s, bounds[k], bounds[k + 1]), range(parts)))
+
+    with ThreadPoolExecutor(threads) as pool:
+        run(pool)
+        t0 = time.perf_counter()
+        outs = run(pool)
+        dt = time.perf_counter() - t0
+    assert np.array_equal(np.concatenate(outs), x), "parallel oracle decode failed"
+    return dt
+
+
 # --------------------------------------------------------------------------- #
 # arms                                                                        #
 # --------------------------------------------------------------------------- #
@@ -425,7 +449,7 @@ def run_native(args, rank: int, world: int, local_rank: int) -> None:
         del hs
 
     # ---- CPU baseline (oracle, rank 0, one GPU) ----------------------------
-    cpu = None
+    cpu = cpu_parallel = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         n_sample = min(args.cpu_sample, streams[0].n_elems)
         if len(streams) == 1:
@@ -434,11 +458,16 @@ def run_native(args, rank: int, world: int, local_rank: int) -> None:
             x = x.astype(np.uint16) << 7 if u8 else x.view(np.uint16)
         else:
             x = reference_sample(args.config, n_sample)
-        dt, _ = time_oracle_decode(x, 1, 0)
+        dt, sx = time_oracle_decode(x, 1, 0)
         cpu = {"value": esize * x.size / dt / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
                "sample": f"first {x.size} elements of the workload, oracle bit-serial decode, one "
                          f"thread on {cpu_model()} ({os.cpu_count()} host cores present)",
                "seconds": dt}
+        threads = os.cpu_count() or 1
+        dtp = time_oracle_decode_parallel(sx, x, threads)
+        cpu_parallel = {"value": esize * x.size / dtp / 1e9, "unit": UNIT, "cores": threads,
+                        "kind": "oracle windowed decode, ranges of thread blocks on host threads",
+                        "sample": cpu["sample"].split(", oracle")[0], "seconds": dtp}
 
     if rank != 0:
         return
@@ -468,6 +497,7 @@ def run_native(args, rank: int, world: int, local_rank: int) -> None:
                      "algorithmic_bytes_per_launch": alg_bytes / launches_per_step,
                      "frac_of_8000_nominal": achieved / 8000.0},
         "cpu_baseline": cpu,
+        "cpu_parallel": cpu_parallel,
         "e2e": e2e,
         "gpu_launches": args.steps * launches_per_step,
         "compress": compress,

@@ -87,3 +87,16 @@ def test_reference_arm_under_torchrun_two_ranks():
     assert d["unit"] == "GB/s" and d["value"] > 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] == 1
     assert d["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_parallel_oracle_baseline_reproduces_the_input():
+    # the bench's multi-threaded CPU baseline: ranges of thread blocks decoded
+    # on host threads through Gaps and block offsets, checked against x
+    import numpy as np
+    import bench
+    from lossless_entropy_coded_dfloat11_b200 import inputs as I
+    x = I.edge_case(70001, "zipf", 12).flat_u16()
+    dt, s = bench.time_oracle_decode(x, 1, 0)
+    for threads in (1, 3):
+        assert bench.time_oracle_decode_parallel(s, x, threads) > 0
+    assert dt > 0 and np.array_equal(x, x)
