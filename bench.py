@@ -309,7 +309,7 @@ def run_reference(args, rank: int, world: int) -> None:
     print(json.dumps(line), flush=True)
 
 
-def time_compress(df11, w, repeats: int, u8: bool = False) -> dict:
+def time_compress(df11, w, repeats: int, u8: bool = False, chunks: bool = False) -> dict:
     """Wall-clock time of the public compress call on device-resident BF16
     tensors (histogram kernel, host code build, table upload, bit-pack
     kernels), synchronised on both sides; the median of `repeats` calls after
@@ -319,7 +319,7 @@ def time_compress(df11, w, repeats: int, u8: bool = False) -> dict:
     for r in range(repeats + 1):
         torch.cuda.synchronize()
         t0 = time.perf_counter()
-        cs = (df11.compress_u8 if u8 else df11.compress)(w.tensors, names=w.names)
+        cs = (df11.compress_u8 if u8 else df11.compress_chunked if chunks else df11.compress)(w.tensors, names=w.names)
         torch.cuda.synchronize()
         if r:
             times.append(time.perf_counter() - t0)
@@ -347,14 +347,18 @@ def run_native(args, rank: int, world: int, local_rank: int) -> None:
     # ---- build the compressed workload on this GPU ------------------------
     workloads = make_workloads(args.config, rank, "cuda")
     u8 = args.config in U8_CONFIGS  # 8-bit symbols: uint8 out, no side array
+    chunks = args.layout == "chunks"  # independent-chunk variant of the container
+    if chunks and u8:
+        raise SystemExit("--layout chunks takes BF16 configurations")
     esize = 1 if u8 else 2          # output bytes per element
     bits16 = (lambda t: t) if u8 else (lambda t: t.view(torch.int16))
     streams, originals = [], []
     compress = None
     for w in workloads:
         if compress is None and not args.no_compress:
-            compress = time_compress(df11, w, args.compress_repeats, u8)
-        cs = (df11.compress_u8 if u8 else df11.compress)(w.tensors, names=w.names)
+            compress = time_compress(df11, w, args.compress_repeats, u8, chunks)
+        cs = (df11.compress_u8 if u8 else df11.compress_chunked if chunks else df11.compress)(
+            w.tensors, names=w.names)
         streams.append(cs)
         originals.append(bits16(torch.cat([t.reshape(-1) for t in w.tensors]))
                          if len(workloads) == 1 else None)
@@ -369,7 +373,7 @@ def run_native(args, rank: int, world: int, local_rank: int) -> None:
     out_bytes = sum(esize * cs.n_elems for cs in streams)
     alg_bytes = sum(cs.read_bytes() + esize * cs.n_elems for cs in streams)
     launches_per_step = len(streams)
-    decode = df11.decompress_u8 if u8 else df11.decompress
+    decode = df11.decompress_u8 if u8 else df11.decompress_chunked if chunks else df11.decompress
 
     def step():
         for cs in streams:
@@ -415,7 +419,7 @@ def run_native(args, rank: int, world: int, local_rank: int) -> None:
         exact = bool(torch.equal(bits16(out[: streams[0].n_elems]), originals[0]))
     else:
         for cs, fp in zip(streams, originals):
-            step_out = df11.decompress(cs, out=out[: cs.n_elems], stream=stream)
+            step_out = decode(cs, out=out[: cs.n_elems], stream=stream)
             for v, f in zip(cs.views(step_out), fp):
                 exact &= bool(torch.equal(v.reshape(-1).view(torch.int16)[:: 4093], f))
     torch.cuda.synchronize()
@@ -426,7 +430,7 @@ def run_native(args, rank: int, world: int, local_rank: int) -> None:
 
     # ---- end to end: host buffers through the public API --------------------
     e2e = None
-    if not args.no_e2e and len(streams) == 1:
+    if not args.no_e2e and len(streams) == 1 and not chunks:
         hs = df11.HostStream(streams[0])
         for _ in range(2):
             hs.run(stream)
@@ -450,7 +454,7 @@ def run_native(args, rank: int, world: int, local_rank: int) -> None:
 
     # ---- CPU baseline (oracle, rank 0, one GPU) ----------------------------
     cpu = cpu_parallel = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not chunks:
         n_sample = min(args.cpu_sample, streams[0].n_elems)
         if len(streams) == 1:
             x = originals[0][:n_sample].cpu().numpy()
@@ -474,7 +478,7 @@ def run_native(args, rank: int, world: int, local_rank: int) -> None:
     peak, peak_kind = measured_peak_gbs()
     launch_ms = elapsed / (args.steps * launches_per_step)
     achieved = (alg_bytes / launches_per_step) / (launch_ms * 1e-3) / 1e9
-    traffic = recorded_traffic() if args.config == "c3" else None
+    traffic = recorded_traffic() if args.config == "c3" and not chunks else None
     cs0 = streams[0]
     line = {
         "metric": METRIC_U8 if u8 else METRIC, "value": agg["gbs"], "unit": UNIT, "n_gpus": world,
@@ -482,7 +486,10 @@ def run_native(args, rank: int, world: int, local_rank: int) -> None:
         "warmup": args.warmup, "ms_per_step": agg["ms_per_step"], "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "u8", "data": "synthetic",
         "config": {"workload": CONFIGS[args.config], "elements_per_step": sum(c.n_elems for c in streams),
-                   "threads_per_block": cs0.threads_per_block, "launches_per_step": launches_per_step,
+                   "threads_per_block": None if chunks else cs0.threads_per_block,
+                   "layout": (f"independent chunks of {df11.IND_CHUNK} elements (start-bit table), no gaps or scan"
+                              if chunks else "gaps + thread-block offsets"),
+                   "launches_per_step": launches_per_step,
                    "l2": ("no flush: compressed input + output per step exceed the 126 MB L2"
                           if flush is None else
                           f"flushed: a {2 * L2_BYTES >> 20} MiB buffer is written before each step; "
@@ -588,6 +595,8 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-compress", action="store_true", help="skip timing the compress call")
+    ap.add_argument("--layout", choices=["gaps", "chunks"], default="gaps",
+                    help="chunks: the independent-chunk variant of the container (an ablation)")
     ap.add_argument("--compress-repeats", type=int, default=5)
     ap.add_argument("--pipeline", action="store_true",
                     help="time decompress-into-consumer (BlockPrefetcher) instead of the decode alone")

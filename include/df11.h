@@ -233,6 +233,26 @@ df11_status df11_decompress_u8(const df11_header* hdr, const uint8_t* d_exp, con
                                const uint32_t* d_block_off, const void* d_lut, uint8_t* d_out,
                                uint32_t* d_status, void* stream);
 
+/* Independent chunks: a variant of the container for comparison with the
+ * Gaps-and-block-offsets design ("EntroLLM: Compressao de Pesos Codificada
+ * por Entropia ...", section "Metodologia", item 3, decodes independently
+ * decodable segments in parallel).  Instead of Gaps and block offsets the
+ * stream carries chunk_bit[k] = the start bit of element 64 k's code, for
+ * k = 0 .. ceil(n/64) - 1, and chunk_bit[ceil(n/64)] = total_bits (uint32;
+ * total_bits must be below 2^32).  EncodedExponent, PackedSignMantissa, the
+ * header (from df11_compress_plan) and the decode tables are the DF11
+ * stream's.  A chunk decodes with no gap, count or prefix sum.
+ * df11_compress_encode_chunked writes d_exp, d_sm, d_lut as
+ * df11_compress_encode does and d_chunk_bit (4 (ceil(n/64) + 1) bytes,
+ * 16-byte aligned); df11_decompress_chunked rebuilds the n BF16 values
+ * (d_out, 16-byte aligned), asynchronously, with no allocation. */
+df11_status df11_compress_encode_chunked(const void* const* d_segs, const df11_header* hdr, void* d_workspace,
+                                         uint64_t workspace_bytes, uint8_t* d_exp, uint8_t* d_sm,
+                                         uint32_t* d_chunk_bit, void* d_lut, void* stream);
+df11_status df11_decompress_chunked(const df11_header* hdr, const uint8_t* d_exp, const uint8_t* d_sm,
+                                    const uint32_t* d_chunk_bit, const void* d_lut, uint16_t* d_out,
+                                    uint32_t* d_status, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

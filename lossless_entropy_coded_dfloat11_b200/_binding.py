@@ -19,7 +19,8 @@ DF11_OK, DF11_ERR_INVALID, DF11_ERR_CUDA, DF11_ERR_CORRUPT, DF11_ERR_TOO_LARGE, 
 EXPORTED = ["df11_version", "df11_last_error", "df11_code_lengths", "df11_header_init", "df11_build_lut",
             "df11_compress_workspace_size", "df11_compress_plan", "df11_compress_encode", "df11_decompress",
             "df11_compress_encode_static", "df11_decompress_sms", "df11_compress_plan_u8",
-            "df11_compress_encode_u8", "df11_decompress_u8"]
+            "df11_compress_encode_u8", "df11_decompress_u8", "df11_compress_encode_chunked",
+            "df11_decompress_chunked"]
 
 
 class Header(ctypes.Structure):
@@ -92,6 +93,8 @@ def load(build_if_missing: bool = True):
     lib.df11_compress_plan_u8.argtypes = [vp, vp, u32, u32, u32, vp, u64, hp, vp]
     lib.df11_compress_encode_u8.argtypes = [vp, hp, vp, u64, vp, vp, vp, vp, vp]
     lib.df11_decompress_u8.argtypes = [hp, vp, vp, vp, vp, vp, vp, vp]
+    lib.df11_compress_encode_chunked.argtypes = [vp, hp, vp, u64, vp, vp, vp, vp, vp]
+    lib.df11_decompress_chunked.argtypes = [hp, vp, vp, vp, vp, vp, vp, vp]
     for name in EXPORTED[2:]:
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib

@@ -312,3 +312,98 @@ def decompress_u8(cs: CompressedStream, out: torch.Tensor | None = None, status:
            _ptr(cs.lut), _ptr(out), _ptr(status) if status is not None else ctypes.c_void_p(0),
            _stream_handle(stream))
     return out
+
+
+IND_CHUNK = 64  # elements per independently decodable chunk
+
+
+@dataclass
+class ChunkedStream:
+    """The independent-chunk variant of a stream: EncodedExponent,
+    PackedSignMantissa and the decode tables as in a DF11 stream, and the
+    start bit of every IND_CHUNK elements (then total_bits) instead of Gaps
+    and block offsets."""
+    header: B.Header
+    exp: torch.Tensor
+    sm: torch.Tensor
+    chunk_bit: torch.Tensor  # int32 storage of uint32 start bits
+    lut: torch.Tensor
+    names: list = field(default_factory=list)
+    shapes: list = field(default_factory=list)
+
+    @property
+    def n_elems(self) -> int:
+        return int(self.header.n_elems)
+
+    @property
+    def n_chunks(self) -> int:
+        return (self.n_elems + IND_CHUNK - 1) // IND_CHUNK
+
+    def compressed_bytes(self) -> int:
+        """Code bits, one byte per element, the chunk table and the 256-byte
+        code-length table."""
+        h = self.header
+        return (h.total_bits + 7) // 8 + h.n_elems + 4 * (self.n_chunks + 1) + 256
+
+    def read_bytes(self) -> int:
+        h = self.header
+        return (h.total_bits + 7) // 8 + h.n_elems + 4 * (self.n_chunks + 1)
+
+    def views(self, flat: torch.Tensor) -> list[torch.Tensor]:
+        out = []
+        for k, shape in enumerate(self.shapes):
+            a, b = int(self.header.seg_elem_off[k]), int(self.header.seg_elem_off[k + 1])
+            out.append(flat[a:b].view(shape))
+        return out
+
+
+def compress_chunked(tensors, names=None, max_code_len: int = 32, stream=None) -> ChunkedStream:
+    """Compress BF16 tensors into the independent-chunk variant: the same code
+    and bit stream as `compress`, with a chunk table for the decoder."""
+    segs = _as_segments(tensors)
+    device = segs[0].device
+    n = sum(t.numel() for t in segs)
+    ws = torch.empty(max(workspace_bytes(n), 16), dtype=torch.uint8, device=device)
+    ptrs = (ctypes.c_void_p * len(segs))(*[int(t.data_ptr()) for t in segs])
+    counts = (ctypes.c_uint64 * len(segs))(*[t.numel() for t in segs])
+    hdr = B.Header()
+    sh = _stream_handle(stream)
+    B.call("df11_compress_plan", ptrs, counts, len(segs), DEFAULT_THREADS_PER_BLOCK, max_code_len, _ptr(ws),
+           ws.numel(), ctypes.byref(hdr), sh)
+    exp = torch.empty(int(hdr.bytes_exp), dtype=torch.uint8, device=device)
+    sm = torch.empty(int(hdr.bytes_sm) or 16, dtype=torch.uint8, device=device)
+    chunk_bit = torch.empty(max((n + IND_CHUNK - 1) // IND_CHUNK + 1, 4), dtype=torch.int32, device=device)
+    lut = torch.empty(int(hdr.bytes_lut), dtype=torch.uint8, device=device)
+    B.call("df11_compress_encode_chunked", ptrs, ctypes.byref(hdr), _ptr(ws), ws.numel(), _ptr(exp), _ptr(sm),
+           _ptr(chunk_bit), _ptr(lut), sh)
+    (stream or torch.cuda.current_stream()).synchronize()
+    return ChunkedStream(hdr, exp, sm, chunk_bit, lut,
+                         names=list(names) if names else [f"t{k}" for k in range(len(segs))],
+                         shapes=[tuple(t.shape) for t in segs])
+
+
+def chunked_from_arrays(code_len: np.ndarray, n_elems: int, total_bits: int, exp: np.ndarray, sm: np.ndarray,
+                        chunk_bit: np.ndarray, max_code_len: int = 32, seg_counts=None, shapes=None,
+                        device="cuda") -> ChunkedStream:
+    """Upload an independent-chunk stream made elsewhere."""
+    hdr = make_header(code_len, n_elems, total_bits, DEFAULT_THREADS_PER_BLOCK, max_code_len, seg_counts)
+    lut = build_lut(hdr)
+    up = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
+    cb = np.ascontiguousarray(chunk_bit, dtype=np.uint32).view(np.int32)
+    shapes = shapes or [(int(c),) for c in (seg_counts or [n_elems])]
+    return ChunkedStream(hdr, up(exp), up(sm), up(cb), up(lut), names=[f"t{k}" for k in range(len(shapes))],
+                         shapes=shapes)
+
+
+def decompress_chunked(cs: ChunkedStream, out: torch.Tensor | None = None, status: torch.Tensor | None = None,
+                       stream=None) -> torch.Tensor:
+    """One launch of the independent-chunk decoder; asynchronous."""
+    n = cs.n_elems
+    if out is None:
+        out = torch.empty(max(n, 8), dtype=torch.bfloat16, device=cs.exp.device)[:n]
+    if out.dtype != torch.bfloat16 or not out.is_contiguous() or out.numel() < n:
+        raise ValueError("out must be a contiguous bfloat16 tensor with n_elems elements")
+    B.call("df11_decompress_chunked", ctypes.byref(cs.header), _ptr(cs.exp), _ptr(cs.sm), _ptr(cs.chunk_bit),
+           _ptr(cs.lut), _ptr(out), _ptr(status) if status is not None else ctypes.c_void_p(0),
+           _stream_handle(stream))
+    return out

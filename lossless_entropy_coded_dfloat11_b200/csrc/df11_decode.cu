@@ -790,6 +790,156 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_warp_kernel(const Decode
 }
 
 // ---------------------------------------------------------------------------
+// Independent chunks, an ablation of the gap-and-scan design (the parallel
+// decoding of "EntroLLM: Compressao de Pesos Codificada por Entropia ...",
+// section "Metodologia", item 3, segments the coded weights so that segments
+// decode independently): the stream records the start bit of every
+// kIndChunk-element chunk instead of Gaps and block offsets, so a lane
+// decodes its chunk with no gap, count or prefix sum and writes exactly
+// kIndChunk symbols to a fixed slot.  A warp takes 32 consecutive chunks and
+// first stages their stream words in shared memory.
+// ---------------------------------------------------------------------------
+struct ChunkArgs {
+    const uint32_t* exp32;      // EncodedExponent as 32-bit words (stream byte order)
+    const uint2* sm8;           // PackedSignMantissa, 8 bytes per unit
+    const uint32_t* chunk_bit;  // start bit of each chunk, then total_bits
+    const uint4* lut;
+    uint16_t* out;
+    uint32_t* status;
+    uint32_t n_elems;
+    uint32_t n_chunks;
+    uint32_t exp_words;  // words of EncodedExponent that may be read
+};
+
+constexpr int kChunkWarps = 12;
+// 32 chunks of codes of at most 32 bits, plus the peek's lookahead word
+constexpr uint32_t kChunkStreamWords = 32 * kIndChunk + 4;
+// staged symbols per lane: the chunk plus up to 3 decoded past it, 8-byte aligned
+constexpr uint32_t kChunkSlot = kIndChunk + 8;
+constexpr uint32_t kChunkWarpBytes = 4 * kChunkStreamWords + 32 * kChunkSlot;
+static_assert(kChunkWarpBytes % 16 == 0 && kChunkSlot % 8 == 0, "aligned per-warp buffers");
+
+__global__ void __launch_bounds__(kChunkWarps * 32, 1) decode_chunk_kernel(const ChunkArgs a) {
+    extern __shared__ __align__(16) uint8_t smem[];
+    copy_compact_tables(smem, a.lut, kChunkWarps * 32);
+    __syncthreads();
+    Tables t;
+    t.ctab = nullptr;
+    t.mtab = reinterpret_cast<const uint16_t*>(smem + kCompactMask);
+    t.dtab = reinterpret_cast<const uint2*>(smem + kCompactDecode);
+    t.lj_end = reinterpret_cast<const unsigned long long*>(smem + kLutOffLjEnd);
+    t.delta = reinterpret_cast<const uint32_t*>(smem + kLutOffDelta);
+    t.syms = smem + kLutOffSyms;
+    const uint16_t* ltab = reinterpret_cast<const uint16_t*>(smem + kCompactLong);
+    const uint32_t long_base = reinterpret_cast<const LutHeader*>(smem)->long_base;
+    const uint32_t long_count = reinterpret_cast<const LutHeader*>(smem)->long_count;
+    const uint32_t lane = threadIdx.x & 31u;
+    const uint32_t warp = threadIdx.x >> 5;
+    uint32_t* s_stream = reinterpret_cast<uint32_t*>(smem + kCompactBytes + warp * kChunkWarpBytes);
+    uint8_t* s_slot = reinterpret_cast<uint8_t*>(s_stream + kChunkStreamWords);
+    uint32_t* my_slot = reinterpret_cast<uint32_t*>(s_slot + lane * kChunkSlot);
+    const uint32_t slot_s = uint32_t(__cvta_generic_to_shared(s_slot));
+    const uint32_t n_groups = (a.n_chunks + 31) / 32;
+    for (uint32_t g = warp * gridDim.x + blockIdx.x; g < n_groups; g += gridDim.x * kChunkWarps) {
+        const uint32_t k = 32 * g + lane;
+        const uint32_t kl = min(32 * g + 32, a.n_chunks);
+        const uint32_t b0 = __ldg(a.chunk_bit + 32 * g), b1 = __ldg(a.chunk_bit + kl);
+        const uint32_t my0 = k < a.n_chunks ? __ldg(a.chunk_bit + k) : b1;
+        const uint32_t my1 = k < a.n_chunks ? __ldg(a.chunk_bit + k + 1) : b1;
+        const uint32_t w0 = b0 >> 5;
+        // words [w0, w_end): every code of the group plus the peek's lookahead
+        const uint32_t w_end = min((b1 >> 5) + 2, a.exp_words);
+        // (every index into the staged words below stays inside them)
+        bool bad = b1 < b0 || my0 < b0 || my1 < my0 || my1 > b1 || w_end <= w0 || w_end - w0 > kChunkStreamWords ||
+                   (my0 >> 5) >= w_end;
+        if (__any_sync(0xFFFFFFFFu, bad)) {
+            if (lane == 0 && a.status) atomicOr(a.status, uint32_t(DF11_ERR_CORRUPT));
+            continue;
+        }
+        const uint32_t nwords = w_end - w0;
+        for (uint32_t j = lane; j < nwords; j += 32) s_stream[j] = bswap32(__ldg(a.exp32 + w0 + j));
+        __syncwarp();
+        // this lane's chunk: exactly cnt codes from bit my0
+        const uint32_t cnt = k < a.n_chunks ? min(kIndChunk, a.n_elems - k * kIndChunk) : 0u;
+        const uint32_t rel = my0 - 32 * w0;
+        uint32_t wi = rel >> 5, pos = rel & 31u;
+        uint32_t hi = s_stream[wi], lo = wi + 1 < nwords ? s_stream[wi + 1] : 0u;
+        uint32_t produced = 0, pend = 0;
+        for (uint32_t steps = 0; produced < cnt; steps++) {
+            if (steps >= kIndChunk) {  // every step decodes at least one code
+                bad = true;
+                break;
+            }
+            const uint32_t pk = __funnelshift_l(lo, hi, pos);
+            const uint2 e = t.dtab[pk >> (32 - kPeekBits)];
+            uint32_t x, nsym, used;
+            if ((e.y >> 16) >= kEscape) {  // a code longer than the table
+                const uint32_t li = (pk >> (32 - kLongBits)) - long_base;
+                const uint32_t le = li < long_count ? uint32_t(ltab[li]) : 0u;
+                if (le) {
+                    used = le >> 8;
+                    x = le & 0xFFu;
+                } else {
+                    used = uint32_t(code_length(t.lj_end, pk, kPeekBits + 1));
+                    if (!used) {
+                        bad = true;
+                        break;
+                    }
+                    x = code_symbol(t, pk, int(used));
+                }
+                nsym = 1;
+            } else {
+                x = e.x;
+                nsym = (e.y & 0xFFu) >> 3;
+                used = e.y >> 16;
+            }
+            // append nsym symbol bytes at byte `produced` of the slot
+            const uint32_t sh = 8 * (produced & 3u);
+            pend |= x << sh;
+            if ((produced & 3u) + nsym >= 4) {
+                my_slot[produced >> 2] = pend;
+                pend = sh ? x >> (32 - sh) : 0u;
+            }
+            produced += nsym;
+            pos += used;
+            while (pos >= 32) {
+                hi = lo;
+                wi++;
+                lo = wi + 1 < nwords ? s_stream[wi + 1] : 0u;
+                pos -= 32;
+            }
+            if (wi >= nwords) {
+                bad = true;
+                break;
+            }
+        }
+        if (produced & 3u) my_slot[produced >> 2] = pend;
+        // a chunk decoded without symbols past its end stops at the next start
+        if (produced == cnt && cnt && 32 * (w0 + wi) + pos != my1) bad = true;
+        if (__any_sync(0xFFFFFFFFu, bad)) {
+            if (lane == 0 && a.status) atomicOr(a.status, uint32_t(DF11_ERR_CORRUPT));
+            __syncwarp();
+            continue;
+        }
+        __syncwarp();
+        // merge the group's elements [e0, e1) in 8-element units
+        const uint32_t e0 = 32 * g * kIndChunk;
+        const uint32_t e1 = min(a.n_elems, e0 + 32 * kIndChunk);
+        const uint32_t nunits = (e1 - e0 + 7) / 8;
+        for (uint32_t q = lane; q < nunits; q += 32) {
+            const uint32_t off = (q / (kIndChunk / 8)) * kChunkSlot + 8 * (q % (kIndChunk / 8));
+            const uint32_t u = e0 / 8 + q;
+            const uint2 s8 = __ldcs(a.sm8 + u);
+            if (e0 + 8 * q + 8 <= e1)
+                merge_store8(slot_s + off, s8, reinterpret_cast<uint4*>(a.out) + u, 0x80808080u);
+            else
+                merge_unit(*reinterpret_cast<const uint2*>(s_slot + off), s8, u, e0, e1, a.out);
+        }
+        __syncwarp();
+    }
+}
+
+// ---------------------------------------------------------------------------
 // T >= 64: one CTA of T threads decodes one thread block per iteration, with
 // a block-wide scan.
 // ---------------------------------------------------------------------------
@@ -1044,4 +1194,51 @@ extern "C" df11_status df11_decompress_u8(const df11_header* hdr, const uint8_t*
                                           uint32_t* d_status, void* stream) {
     return decompress_on("df11_decompress_u8", true, hdr, d_exp, nullptr, d_gaps, d_block_off, d_lut, d_out,
                          d_status, UINT32_MAX, stream);
+}
+
+extern "C" df11_status df11_decompress_chunked(const df11_header* hdr, const uint8_t* d_exp, const uint8_t* d_sm,
+                                               const uint32_t* d_chunk_bit, const void* d_lut, uint16_t* d_out,
+                                               uint32_t* d_status, void* stream) {
+    df11_status st = check_header(hdr);
+    if (st != DF11_OK) return st;
+    if (hdr->n_elems == 0) return DF11_OK;
+    if (!d_exp || !d_sm || !d_chunk_bit || !d_lut || !d_out)
+        return fail(DF11_ERR_INVALID, "df11_decompress_chunked: null device pointer");
+    if (!aligned16(d_exp) || !aligned16(d_sm) || !aligned16(d_chunk_bit) || !aligned16(d_lut) || !aligned16(d_out))
+        return fail(DF11_ERR_INVALID, "df11_decompress_chunked: device pointers must be 16-byte aligned");
+    if (hdr->total_bits >= (uint64_t(1) << 32))
+        return fail(DF11_ERR_TOO_LARGE, "df11_decompress_chunked: chunk table positions are 32-bit");
+    ChunkArgs a;
+    a.exp32 = reinterpret_cast<const uint32_t*>(d_exp);
+    a.sm8 = reinterpret_cast<const uint2*>(d_sm);
+    a.chunk_bit = d_chunk_bit;
+    a.lut = reinterpret_cast<const uint4*>(d_lut);
+    a.out = d_out;
+    a.status = d_status;
+    a.n_elems = uint32_t(hdr->n_elems);
+    a.n_chunks = uint32_t((hdr->n_elems + kIndChunk - 1) / kIndChunk);
+    a.exp_words = uint32_t(hdr->bytes_exp / 4);
+    constexpr size_t smem = kCompactBytes + size_t(kChunkWarps) * kChunkWarpBytes;
+    static_assert(smem <= 227 * 1024, "shared memory per CTA");
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return fail(DF11_ERR_CUDA, "cudaGetDevice failed");
+    LaunchInfo& li = g_info[dev][9];
+    if (!li.ready.load(std::memory_order_acquire)) {
+        cudaError_t e = cudaFuncSetAttribute(decode_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             int(smem));
+        if (e != cudaSuccess) return fail(DF11_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+        int sms = 0;
+        e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return fail(DF11_ERR_CUDA, "SM count: %s", cudaGetErrorString(e));
+        li.per_sm = 1;
+        li.sms = sms;
+        li.ready.store(1, std::memory_order_release);
+    }
+    const uint64_t groups = (uint64_t(a.n_chunks) + 31) / 32;
+    const uint64_t want = (groups + kChunkWarps - 1) / kChunkWarps;
+    const unsigned grid = unsigned(want < uint64_t(li.sms) ? want : uint64_t(li.sms));
+    decode_chunk_kernel<<<grid, kChunkWarps * 32, smem, reinterpret_cast<cudaStream_t>(stream)>>>(a);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(DF11_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
+    return DF11_OK;
 }

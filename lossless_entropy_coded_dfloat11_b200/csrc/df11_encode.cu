@@ -366,7 +366,8 @@ __global__ void __launch_bounds__(kEncThreads) pack_kernel(const __grid_constant
                                                            const unsigned long long* __restrict__ chunk_start,
                                                            uint32_t* __restrict__ exp32, uint8_t* __restrict__ sm,
                                                            uint32_t* __restrict__ gaps32,
-                                                           uint32_t* __restrict__ block_off, uint64_t n_blocks) {
+                                                           uint32_t* __restrict__ block_off, uint64_t n_blocks,
+                                                           uint32_t* __restrict__ chunk_bit) {
     __shared__ SharedCodes sc;
     __shared__ __align__(16) uint32_t s_words[kPackWords];
     __shared__ uint32_t s_ev[kMaxEvents][kEncThreads];
@@ -447,16 +448,22 @@ __global__ void __launch_bounds__(kEncThreads) pack_kernel(const __grid_constant
                 u = nu;
             }
             if (fill) atomicOr(&s_words[w], cur_word);
-            for (uint32_t j = 0; j < ne; j++) {
-                const uint32_t e = s_ev[j][threadIdx.x];
-                window_event((e >> 10) - 63u, (e >> 4) & 63u, i0 + (e & 15u));
+            if (gaps32) {
+                for (uint32_t j = 0; j < ne; j++) {
+                    const uint32_t e = s_ev[j][threadIdx.x];
+                    window_event((e >> 10) - 63u, (e >> 4) & 63u, i0 + (e & 15u));
+                }
             }
         };
         if (valid == kEncPerThread)
             pack_codes(std::true_type{});
         else if (valid)
             pack_codes(std::false_type{});
-        if (valid && n - i0 <= kEncPerThread) block_off[n_blocks] = uint32_t(n);
+        if (block_off && valid && n - i0 <= kEncPerThread) block_off[n_blocks] = uint32_t(n);
+        if (chunk_bit && valid) {  // independent-chunk table: first bit of every kIndChunk elements
+            if (i0 % kIndChunk == 0) chunk_bit[i0 / kIndChunk] = uint32_t(S + my_off);
+            if (n - i0 <= kEncPerThread) chunk_bit[(n + kIndChunk - 1) / kIndChunk] = uint32_t(S + my_off + bits);
+        }
         if constexpr (ES == 2) if (valid) {
             // sign+mantissa bytes: sign (bit 15) to bit 7, mantissa bits 6..0
             uint32_t smw[kEncPerThread / 4];
@@ -601,10 +608,13 @@ df11_status compress_plan(const void* const* d_segs, const uint64_t* seg_counts,
 
 // Table upload, clears, then the chunk-bits, scan and bit-pack kernels.
 // d_sm is written for BF16 input (ES = 2) only.
+// With d_chunk_bit (the independent-chunk table instead of Gaps and block
+// offsets) d_gaps and d_block_off are not written and may be null.
 template <int ES>
 df11_status compress_encode(const char* fn, const void* const* d_segs, const df11_header* hdr,
                             uint32_t* chunk_bits, unsigned long long* chunk_start, uint8_t* d_exp, uint8_t* d_sm,
-                            uint8_t* d_gaps, uint32_t* d_block_off, void* d_lut, void* stream) {
+                            uint8_t* d_gaps, uint32_t* d_block_off, void* d_lut, void* stream,
+                            uint32_t* d_chunk_bit = nullptr) {
     df11_status st = check_header(hdr);
     if (st != DF11_OK) return st;
     uint64_t counts[DF11_MAX_SEGMENTS];
@@ -616,11 +626,14 @@ df11_status compress_encode(const char* fn, const void* const* d_segs, const df1
     st = build_segtable(d_segs, counts, hdr->n_segments, &sg, &n);
     if (st != DF11_OK) return st;
     if (n != hdr->n_elems) return fail(DF11_ERR_INVALID, "segments disagree with header n_elems");
-    if (!d_exp || (ES == 2 && !d_sm) || !d_gaps || !d_block_off || !d_lut)
+    const bool chunked = d_chunk_bit != nullptr;
+    if (!d_exp || (ES == 2 && !d_sm) || (!chunked && (!d_gaps || !d_block_off)) || !d_lut)
         return fail(DF11_ERR_INVALID, "%s: null output pointer", fn);
-    if (!aligned16(d_exp) || (ES == 2 && !aligned16(d_sm)) || !aligned16(d_gaps) || !aligned16(d_block_off) ||
-        !aligned16(d_lut))
+    if (!aligned16(d_exp) || (ES == 2 && !aligned16(d_sm)) || (!chunked && (!aligned16(d_gaps) ||
+        !aligned16(d_block_off))) || !aligned16(d_lut))
         return fail(DF11_ERR_INVALID, "%s: outputs must be 16-byte aligned", fn);
+    if (chunked && hdr->total_bits >= (uint64_t(1) << 32))
+        return fail(DF11_ERR_TOO_LARGE, "%s: chunk table positions are 32-bit", fn);
 
     CodeTable ct;
     std::memcpy(ct.len, hdr->code_len, 256);
@@ -635,8 +648,11 @@ df11_status compress_encode(const char* fn, const void* const* d_segs, const df1
     if ((e = cudaMemcpyAsync(d_lut, lut, kLutBytes, cudaMemcpyHostToDevice, s)) != cudaSuccess)
         return cuda_fail("table upload", e);
     if ((e = cudaMemsetAsync(d_exp, 0, hdr->bytes_exp, s)) != cudaSuccess) return cuda_fail("clear exp", e);
-    if ((e = cudaMemsetAsync(d_gaps, 0, hdr->bytes_gaps, s)) != cudaSuccess) return cuda_fail("clear gaps", e);
-    if ((e = cudaMemsetAsync(d_block_off, 0, hdr->bytes_off, s)) != cudaSuccess) return cuda_fail("clear off", e);
+    if (!chunked) {
+        if ((e = cudaMemsetAsync(d_gaps, 0, hdr->bytes_gaps, s)) != cudaSuccess) return cuda_fail("clear gaps", e);
+        if ((e = cudaMemsetAsync(d_block_off, 0, hdr->bytes_off, s)) != cudaSuccess)
+            return cuda_fail("clear off", e);
+    }
     if constexpr (ES == 2) {
         const uint64_t sm_tail = n & ~uint64_t(15);
         if (hdr->bytes_sm > sm_tail &&
@@ -654,7 +670,7 @@ df11_status compress_encode(const char* fn, const void* const* d_segs, const df1
     while ((1u << (log2_bb - 6)) < hdr->threads_per_block) log2_bb++;
     pack_kernel<ES><<<encode_grid(pack_kernel<ES>, chunks), kEncThreads, 0, s>>>(
         sg, ct, n, chunks, log2_bb, chunk_start, reinterpret_cast<uint32_t*>(d_exp), d_sm,
-        reinterpret_cast<uint32_t*>(d_gaps), d_block_off, hdr->n_blocks);
+        reinterpret_cast<uint32_t*>(d_gaps), d_block_off, hdr->n_blocks, d_chunk_bit);
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail("encode launch", e);
     return DF11_OK;
@@ -770,4 +786,17 @@ extern "C" df11_status df11_compress_encode_static(const void* const* d_segs, co
         reinterpret_cast<unsigned long long*>(static_cast<unsigned char*>(scratch) + kStaticBitsBytes);
     return compress_encode<2>("df11_compress_encode_static", d_segs, hdr, chunk_bits, chunk_start, d_exp, d_sm,
                               d_gaps, d_block_off, d_lut, stream);
+}
+
+extern "C" df11_status df11_compress_encode_chunked(const void* const* d_segs, const df11_header* hdr,
+                                                    void* d_workspace, uint64_t workspace_bytes, uint8_t* d_exp,
+                                                    uint8_t* d_sm, uint32_t* d_chunk_bit, void* d_lut,
+                                                    void* stream) {
+    if (!d_chunk_bit || (reinterpret_cast<uintptr_t>(d_chunk_bit) & 15u))
+        return fail(DF11_ERR_INVALID, "df11_compress_encode_chunked: chunk table null or not 16-byte aligned");
+    Workspace w{};
+    const df11_status st = carve(d_workspace, workspace_bytes, hdr ? hdr->n_elems : 0, &w);
+    if (st != DF11_OK) return st;
+    return compress_encode<2>("df11_compress_encode_chunked", d_segs, hdr, w.chunk_bits, w.chunk_start, d_exp,
+                              d_sm, nullptr, nullptr, d_lut, stream, d_chunk_bit);
 }

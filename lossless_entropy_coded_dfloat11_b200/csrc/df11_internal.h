@@ -92,5 +92,9 @@ df11_status fail(df11_status st, const char* fmt, ...);
 constexpr uint32_t kEncChunk = 4096;       // elements per bit-pack CTA
 constexpr uint32_t kEncThreads = 256;      // threads per bit-pack CTA
 constexpr uint32_t kEncPerThread = kEncChunk / kEncThreads;
+// Independent-chunk variant of the container: one 32-bit start bit per
+// kIndChunk elements replaces Gaps and block offsets.
+constexpr uint32_t kIndChunk = 64;
+static_assert(kIndChunk % kEncPerThread == 0, "chunk starts fall on encode-thread boundaries");
 
 }  // namespace df11

@@ -228,3 +228,19 @@ def decode_windowed(s: Stream, b0: int = 0, b1: int | None = None) -> np.ndarray
 def read_gap(gaps: np.ndarray, t: int) -> int:
     g = np.ascontiguousarray(gaps, dtype=np.uint8)
     return int(_load().oracle_read_gap(_ptr(g, ctypes.c_uint8), t))
+
+
+def chunk_starts(x: np.ndarray, code_len: np.ndarray, chunk: int) -> np.ndarray:
+    """Start bit of the code of element k*chunk, k = 0 .. ceil(n/chunk) - 1,
+    then total_bits: the table of the independent-chunk variant of the
+    container (segments that decode on their own, "EntroLLM: Compressao de
+    Pesos Codificada por Entropia ...", section "Metodologia", item 3).  By
+    definition the prefix sums of the code lengths of the elements' exponent
+    fields (summed per chunk first)."""
+    x = np.ascontiguousarray(x, dtype=np.uint16).reshape(-1)
+    n = x.size
+    ln = np.ascontiguousarray(code_len, dtype=np.uint8)[(x >> 7) & 0xFF]
+    if n == 0:
+        return np.zeros(1, dtype=np.uint64)
+    per_chunk = np.add.reduceat(ln.astype(np.uint64), np.arange(0, n, chunk))
+    return np.concatenate([[0], np.cumsum(per_chunk)]).astype(np.uint64)

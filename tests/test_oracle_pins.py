@@ -123,6 +123,29 @@ def test_golden_stream_A(golden_dir):
         np.testing.assert_array_equal(oracle.decode_windowed(s), x)
 
 
+def test_chunk_starts_golden_stream_A(golden_dir):
+    # every chunk start is where that element's hand-written code sits in the
+    # hand-derived bit string, and the table ends at total_bits
+    g = _golden(golden_dir)
+    ex, x = _golden_input(g)
+    bits = g["A.bits"]
+    want_codes = _kv(g["A.codes"], str)
+    lengths = np.zeros(256, np.uint8)
+    for sym, code in want_codes.items():
+        lengths[sym] = len(code)
+    starts = oracle.chunk_starts(x, lengths, 1)
+    assert starts.size == x.size + 1 and starts[-1] == int(g["A.total_bits"])
+    for i, e in enumerate(ex):
+        code = want_codes[int(e)]
+        assert bits[int(starts[i]): int(starts[i]) + len(code)] == code, i
+    # the leading 126 takes bits 0..1, then groups of 8 elements take 14 bits
+    assert list(oracle.chunk_starts(x, lengths, 8)) == [0, 13, 27, 41, 55, 69, 72]
+    for chunk in (2, 3, 5, 64):
+        np.testing.assert_array_equal(oracle.chunk_starts(x, lengths, chunk),
+                                      np.append(starts[:-1][::chunk], starts[-1]))
+    assert list(oracle.chunk_starts(x[:0], lengths, 4)) == [0]
+
+
 def test_golden_stream_B_empty_last_window(golden_dir):
     g = _golden(golden_dir)
     n = int(g["B.n_elems"])
