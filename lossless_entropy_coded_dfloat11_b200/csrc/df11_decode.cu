@@ -840,24 +840,76 @@ __global__ void __launch_bounds__(kChunkWarps * 32, 1) decode_chunk_kernel(const
     uint32_t* my_slot = reinterpret_cast<uint32_t*>(s_slot + lane * kChunkSlot);
     const uint32_t slot_s = uint32_t(__cvta_generic_to_shared(s_slot));
     const uint32_t n_groups = (a.n_chunks + 31) / 32;
-    for (uint32_t g = warp * gridDim.x + blockIdx.x; g < n_groups; g += gridDim.x * kChunkWarps) {
+    const uint32_t stride = gridDim.x * kChunkWarps;
+    // one group's start bits, and the first kPreWords of its stream words
+    constexpr uint32_t kPreWords = 8;  // per lane: 256 words cover a typical group
+    struct GroupBits {
+        uint32_t b0, b1, my0, my1;
+    };
+    auto load_bits = [&](uint32_t g) {
+        GroupBits r{0, 0, 0, 0};
+        if (g < n_groups) {
+            const uint32_t k = 32 * g + lane, kl = min(32 * g + 32, a.n_chunks);
+            r.b0 = __ldg(a.chunk_bit + 32 * g);
+            r.b1 = __ldg(a.chunk_bit + kl);
+            r.my0 = k < a.n_chunks ? __ldg(a.chunk_bit + k) : r.b1;
+            r.my1 = k < a.n_chunks ? __ldg(a.chunk_bit + k + 1) : r.b1;
+        }
+        return r;
+    };
+    auto word_range = [&](const GroupBits& gb, uint32_t& w0, uint32_t& w_end) {
+        w0 = gb.b0 >> 5;
+        w_end = min((gb.b1 >> 5) + 2, a.exp_words);
+    };
+    auto load_words = [&](const GroupBits& gb, uint32_t (&wv)[kPreWords]) {
+        uint32_t w0, w_end;
+        word_range(gb, w0, w_end);
+#pragma unroll
+        for (int r = 0; r < int(kPreWords); r++) {
+            const uint32_t j = lane + 32 * r;
+            wv[r] = w_end > w0 && j < w_end - w0 ? __ldg(a.exp32 + w0 + j) : 0u;
+        }
+    };
+    uint32_t g = warp * gridDim.x + blockIdx.x;
+    GroupBits nbits = load_bits(g);
+    uint32_t nwv[kPreWords];
+    load_words(nbits, nwv);
+    for (; g < n_groups; g += stride) {
+        const GroupBits gb = nbits;
+        uint32_t wv[kPreWords];
+#pragma unroll
+        for (int r = 0; r < int(kPreWords); r++) wv[r] = nwv[r];
+        nbits = load_bits(g + stride);  // in flight during this group's work
         const uint32_t k = 32 * g + lane;
-        const uint32_t kl = min(32 * g + 32, a.n_chunks);
-        const uint32_t b0 = __ldg(a.chunk_bit + 32 * g), b1 = __ldg(a.chunk_bit + kl);
-        const uint32_t my0 = k < a.n_chunks ? __ldg(a.chunk_bit + k) : b1;
-        const uint32_t my1 = k < a.n_chunks ? __ldg(a.chunk_bit + k + 1) : b1;
-        const uint32_t w0 = b0 >> 5;
-        // words [w0, w_end): every code of the group plus the peek's lookahead
-        const uint32_t w_end = min((b1 >> 5) + 2, a.exp_words);
+        const uint32_t b0 = gb.b0, b1 = gb.b1, my0 = gb.my0, my1 = gb.my1;
+        uint32_t w0, w_end;
+        word_range(gb, w0, w_end);
         // (every index into the staged words below stays inside them)
         bool bad = b1 < b0 || my0 < b0 || my1 < my0 || my1 > b1 || w_end <= w0 || w_end - w0 > kChunkStreamWords ||
                    (my0 >> 5) >= w_end;
         if (__any_sync(0xFFFFFFFFu, bad)) {
             if (lane == 0 && a.status) atomicOr(a.status, uint32_t(DF11_ERR_CORRUPT));
+            load_words(nbits, nwv);
             continue;
         }
         const uint32_t nwords = w_end - w0;
-        for (uint32_t j = lane; j < nwords; j += 32) s_stream[j] = bswap32(__ldg(a.exp32 + w0 + j));
+#pragma unroll
+        for (int r = 0; r < int(kPreWords); r++) {
+            const uint32_t j = lane + 32 * r;
+            if (j < nwords) s_stream[j] = bswap32(wv[r]);
+        }
+        for (uint32_t j = lane + 32 * kPreWords; j < nwords; j += 32) s_stream[j] = bswap32(__ldg(a.exp32 + w0 + j));
+        // this group's sign+mantissa units (32 kIndChunk / 8 over 32 lanes),
+        // requested before the decode
+        const uint32_t e0 = 32 * g * kIndChunk;
+        const uint32_t e1 = min(a.n_elems, e0 + 32 * kIndChunk);
+        const uint32_t nunits = (e1 - e0 + 7) / 8;
+        uint2 sv[kIndChunk / 8];
+#pragma unroll
+        for (int r = 0; r < int(kIndChunk / 8); r++) {
+            const uint32_t q = lane + 32 * r;
+            sv[r] = q < nunits ? __ldcs(a.sm8 + e0 / 8 + q) : make_uint2(0, 0);
+        }
         __syncwarp();
         // this lane's chunk: exactly cnt codes from bit my0
         const uint32_t cnt = k < a.n_chunks ? min(kIndChunk, a.n_elems - k * kIndChunk) : 0u;
@@ -916,6 +968,7 @@ __global__ void __launch_bounds__(kChunkWarps * 32, 1) decode_chunk_kernel(const
         if (produced & 3u) my_slot[produced >> 2] = pend;
         // a chunk decoded without symbols past its end stops at the next start
         if (produced == cnt && cnt && 32 * (w0 + wi) + pos != my1) bad = true;
+        load_words(nbits, nwv);  // the next group's words, in flight during the merge
         if (__any_sync(0xFFFFFFFFu, bad)) {
             if (lane == 0 && a.status) atomicOr(a.status, uint32_t(DF11_ERR_CORRUPT));
             __syncwarp();
@@ -923,17 +976,16 @@ __global__ void __launch_bounds__(kChunkWarps * 32, 1) decode_chunk_kernel(const
         }
         __syncwarp();
         // merge the group's elements [e0, e1) in 8-element units
-        const uint32_t e0 = 32 * g * kIndChunk;
-        const uint32_t e1 = min(a.n_elems, e0 + 32 * kIndChunk);
-        const uint32_t nunits = (e1 - e0 + 7) / 8;
-        for (uint32_t q = lane; q < nunits; q += 32) {
+#pragma unroll
+        for (int r = 0; r < int(kIndChunk / 8); r++) {
+            const uint32_t q = lane + 32 * r;
+            if (q >= nunits) break;
             const uint32_t off = (q / (kIndChunk / 8)) * kChunkSlot + 8 * (q % (kIndChunk / 8));
             const uint32_t u = e0 / 8 + q;
-            const uint2 s8 = __ldcs(a.sm8 + u);
             if (e0 + 8 * q + 8 <= e1)
-                merge_store8(slot_s + off, s8, reinterpret_cast<uint4*>(a.out) + u, 0x80808080u);
+                merge_store8(slot_s + off, sv[r], reinterpret_cast<uint4*>(a.out) + u, 0x80808080u);
             else
-                merge_unit(*reinterpret_cast<const uint2*>(s_slot + off), s8, u, e0, e1, a.out);
+                merge_unit(*reinterpret_cast<const uint2*>(s_slot + off), sv[r], u, e0, e1, a.out);
         }
         __syncwarp();
     }
