@@ -400,14 +400,16 @@ __device__ __forceinline__ void copy_compact_tables(uint8_t* s, const uint4* g, 
 }
 
 // One half of the window (bit positions below lim, peeking at hi:lo) through
-// the decode table, in hand-written PTX: 16 instructions per step, with no
+// the decode table, in hand-written PTX: 15 instructions per step, with no
 // branch but the loop's own.  `acc` is (bit position << 16 | 8 x bytes
 // produced so far); its low five bits place the next symbols in `pend`, and a
-// word is complete when bit 5 of acc flips.  The completed word is stored at
-// `wad` (a shared-window address, stepping 128 bytes in the transposed slot)
-// and `pend` becomes the spilled bytes through one clamped funnel shift.  The
-// loop is unrolled twice with acc alternating between two registers.  The
-// last entry's index and y word stay behind for the end-of-window correction.
+// word is complete when bit 5 of acc flips.  Every step stores the word under
+// construction at `wad` (a shared-window address, stepping 128 bytes in the
+// transposed slot), so a completed word is in place when wad moves on;
+// `pend` then becomes the spilled bytes through one clamped funnel shift.
+// The loop is unrolled twice with acc alternating between two registers.
+// The last entry's index and y word stay behind for the end-of-window
+// correction.
 __device__ __forceinline__ void decode_half(uint32_t& acc, uint32_t& pend, uint32_t& wad, uint32_t& idx,
                                             uint32_t& ylast, uint32_t hi, uint32_t lo, uint32_t lim,
                                             uint32_t dtab_s) {
@@ -422,13 +424,12 @@ __device__ __forceinline__ void decode_half(uint32_t& acc, uint32_t& pend, uint3
     "shf.l.wrap.b32 spill, x, zero, " A ";\n\t"           \
     "add.u32 " B ", " A ", %4;\n\t"                       \
     "lop3.b32 t1, " B ", " A ", c32, 0x28;\n\t"           \
-    "setp.ne.u32 q, t1, 0;\n\t"                           \
-    "@q st.shared.u32 [%2], %1;\n\t"                      \
+    "st.shared.u32 [%2], %1;\n\t"                         \
     "mad.lo.u32 %2, t1, 4, %2;\n\t"                       \
     "shf.r.clamp.b32 %1, %1, spill, t1;\n\t"
     asm volatile(
         "{\n\t"
-        ".reg .pred p, q;\n\t"
+        ".reg .pred p;\n\t"
         ".reg .u32 sh, pk, ad, x, t1, spill, zero, c32, b;\n\t"
         "mov.u32 zero, 0;\n\t"
         "mov.u32 c32, 32;\n\t"
@@ -615,25 +616,8 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_warp_kernel(const Decode
     // elements per merge unit, 16 output bytes either way
     constexpr uint32_t kUnit = U8 ? 16u : 8u;
     extern __shared__ __align__(16) uint8_t smem[];
-    copy_compact_tables(smem, a.lut, WARPS * 32);
-    __syncthreads();
-    Tables t;
-    t.ctab = nullptr;
-    t.mtab = reinterpret_cast<const uint16_t*>(smem + kCompactMask);
-    t.dtab = reinterpret_cast<const uint2*>(smem + kCompactDecode);
-    t.lj_end = reinterpret_cast<const unsigned long long*>(smem + kLutOffLjEnd);
-    t.delta = reinterpret_cast<const uint32_t*>(smem + kLutOffDelta);
-    t.syms = smem + kLutOffSyms;
-    const uint32_t dtab_s = uint32_t(__cvta_generic_to_shared(t.dtab));
-    const uint16_t* ltab = reinterpret_cast<const uint16_t*>(smem + kCompactLong);
-    const uint32_t long_base = reinterpret_cast<const LutHeader*>(smem)->long_base;
-    const uint32_t long_count = reinterpret_cast<const LutHeader*>(smem)->long_count;
     const uint32_t lane = threadIdx.x & 31u;
     const uint32_t warp = threadIdx.x >> 5;
-    uint8_t* wbase = smem + kCompactBytes + warp * L::kBytes;
-    uint32_t* slot = reinterpret_cast<uint32_t*>(wbase) + lane;
-    const uint32_t slot_s = uint32_t(__cvta_generic_to_shared(slot));
-    uint8_t* stage = wbase + L::kSlots;
     // the gap field of the lane's first window, WPL (32b + lane), lies in the
     // block's 5 WPL gap words
     const uint32_t lane_gword = (5 * WPL * lane) >> 5;
@@ -648,6 +632,8 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_warp_kernel(const Decode
     uint32_t b = g * per + (g < extra ? g : extra);
     const uint32_t b_end = b + per + (g < extra ? 1u : 0u);
 
+    copy_compact_tables(smem, a.lut, WARPS * 32);
+    __syncthreads();
     RawLane<WPL> nraw{};
     uint32_t noff0 = 0, noff1 = 0;
     if (b < b_end) {
@@ -655,6 +641,21 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_warp_kernel(const Decode
         noff0 = __ldg(a.off + b);
         noff1 = __ldg(a.off + b + 1);
     }
+    Tables t;
+    t.ctab = nullptr;
+    t.mtab = reinterpret_cast<const uint16_t*>(smem + kCompactMask);
+    t.dtab = reinterpret_cast<const uint2*>(smem + kCompactDecode);
+    t.lj_end = reinterpret_cast<const unsigned long long*>(smem + kLutOffLjEnd);
+    t.delta = reinterpret_cast<const uint32_t*>(smem + kLutOffDelta);
+    t.syms = smem + kLutOffSyms;
+    const uint32_t dtab_s = uint32_t(__cvta_generic_to_shared(t.dtab));
+    const uint16_t* ltab = reinterpret_cast<const uint16_t*>(smem + kCompactLong);
+    const uint32_t long_base = reinterpret_cast<const LutHeader*>(smem)->long_base;
+    const uint32_t long_count = reinterpret_cast<const LutHeader*>(smem)->long_count;
+    uint8_t* wbase = smem + kCompactBytes + warp * L::kBytes;
+    uint32_t* slot = reinterpret_cast<uint32_t*>(wbase) + lane;
+    const uint32_t slot_s = uint32_t(__cvta_generic_to_shared(slot));
+    uint8_t* stage = wbase + L::kSlots;
     const uint2* sm8 = reinterpret_cast<const uint2*>(a.sm);
     uint4 carry = make_uint4(0, 0, 0, 0);  // staging bytes of the unit left by the previous block
     bool have_carry = false;
@@ -678,6 +679,12 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_warp_kernel(const Decode
         const uint32_t uw = keep_tail && u1 > u0 ? u1 - 1 : u1;
         const bool use_carry = have_carry && head != 0;
         const uint32_t lo = use_carry ? (off0 & ~(kUnit - 1)) : off0;
+        // lane q of a merge round r takes unit ub + q + 32 r, with ub = u0
+        // rounded down to 16 units (8 for 8-bit symbols), so that every warp
+        // access covers whole 128-byte lines (256 sign+mantissa bytes, 512
+        // output bytes); lanes whose unit lies before u0 idle in the first round
+        const uint32_t a_sh = u0 & (U8 ? 7u : 15u);
+        const uint32_t ub = u0 - a_sh;
         // sign+mantissa units requested before the decode: 4 rounds of 32
         // (a 32-window block has ~100 units), 7 for two windows per lane
         constexpr int kPre = WPL == 1 ? 4 : 7;
@@ -685,7 +692,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_warp_kernel(const Decode
         if constexpr (!U8) {
 #pragma unroll
             for (int r = 0; r < kPre; r++)
-                sv[r] = u0 + lane + 32 * r < uw ? __ldcs(sm8 + u0 + lane + 32 * r) : make_uint2(0, 0);
+                sv[r] = ub + lane + 32 * r < uw ? __ldcs(sm8 + ub + lane + 32 * r) : make_uint2(0, 0);
         }
 
         const LaneWindow<WPL> w = finish_lane<WPL>(a, raw, WPL * (32 * b + lane), lane_gshift, lane);
@@ -724,26 +731,27 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_warp_kernel(const Decode
                 const uint2* ev = reinterpret_cast<const uint2*>(stage);
                 const uint32_t stage_s = uint32_t(__cvta_generic_to_shared(stage));
                 const uint32_t nu = uw - u0;  // units this block stores
+                const uint32_t qe = nu + a_sh;  // lanes [a_sh, qe) of the rounds hold them
                 const uint32_t m = 0x80808080u;
                 if (lo == 8 * u0 && (keep_tail || (off1 & 7u) == 0)) {
                     // every unit is whole (all but the first and last block of a run)
-                    const uint32_t ev_s = stage_s + 8 * lane;
-                    uint4* dst = reinterpret_cast<uint4*>(a.out) + u0 + lane;
-                    if (lane < nu) merge_store8<0, 0>(ev_s, sv[0], dst, m);
-                    if (lane + 32 < nu) merge_store8<256, 512>(ev_s, sv[1], dst, m);
-                    if (lane + 64 < nu) merge_store8<512, 1024>(ev_s, sv[2], dst, m);
-                    if (lane + 96 < nu) merge_store8<768, 1536>(ev_s, sv[3], dst, m);
+                    const uint32_t ev_s = stage_s + 8 * lane - 8 * a_sh;
+                    uint4* dst = reinterpret_cast<uint4*>(a.out) + ub + lane;
+                    if (lane >= a_sh && lane < qe) merge_store8<0, 0>(ev_s, sv[0], dst, m);
+                    if (lane + 32 < qe) merge_store8<256, 512>(ev_s, sv[1], dst, m);
+                    if (lane + 64 < qe) merge_store8<512, 1024>(ev_s, sv[2], dst, m);
+                    if (lane + 96 < qe) merge_store8<768, 1536>(ev_s, sv[3], dst, m);
                     if constexpr (kPre == 7) {
-                        if (lane + 128 < nu) merge_store8<1024, 2048>(ev_s, sv[4], dst, m);
-                        if (lane + 160 < nu) merge_store8<1280, 2560>(ev_s, sv[5], dst, m);
-                        if (lane + 192 < nu) merge_store8<1536, 3072>(ev_s, sv[6], dst, m);
+                        if (lane + 128 < qe) merge_store8<1024, 2048>(ev_s, sv[4], dst, m);
+                        if (lane + 160 < qe) merge_store8<1280, 2560>(ev_s, sv[5], dst, m);
+                        if (lane + 192 < qe) merge_store8<1536, 3072>(ev_s, sv[6], dst, m);
                     }
-                    for (uint32_t k = 32 * kPre; lane + k < nu; k += 32)
-                        merge_store8(ev_s + 8 * k, __ldcs(sm8 + u0 + lane + k), dst + k, m);
+                    for (uint32_t k = 32 * kPre; lane + k < qe; k += 32)
+                        merge_store8(ev_s + 8 * k, __ldcs(sm8 + ub + lane + k), dst + k, m);
                 } else {
                     const uint32_t uf = (lo + 7) >> 3, ul = off1 >> 3;  // whole units: [uf, ul)
-                    auto unit = [&](uint32_t k, const uint2 s8) {
-                        const uint32_t u = u0 + k;
+                    auto unit = [&](uint32_t q, const uint2 s8) {  // unit u0 + q - a_sh
+                        const uint32_t k = q - a_sh, u = u0 + k;
                         if (u >= uf && u < ul)
                             merge_store8(stage_s + 8 * k, s8, reinterpret_cast<uint4*>(a.out) + u, m);
                         else
@@ -751,8 +759,8 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_warp_kernel(const Decode
                     };
     #pragma unroll
                     for (int r = 0; r < kPre; r++)
-                        if (lane + 32 * r < nu) unit(lane + 32 * r, sv[r]);
-                    for (uint32_t k = lane + 32 * kPre; k < nu; k += 32) unit(k, __ldcs(sm8 + u0 + k));
+                        if (lane + 32 * r >= a_sh && lane + 32 * r < qe) unit(lane + 32 * r, sv[r]);
+                    for (uint32_t q = lane + 32 * kPre; q < qe; q += 32) unit(q, __ldcs(sm8 + ub + q));
                 }
                 if (keep_tail) {
                     const uint2 c = ev[u1 - 1 - u0];
@@ -762,12 +770,15 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_warp_kernel(const Decode
                 // 8-bit symbols: the staged bytes themselves, rotated back
                 const uint4* ev16 = reinterpret_cast<const uint4*>(stage);
                 const uint32_t nu = uw - u0;  // units this block stores
+                const uint32_t qe = nu + a_sh;
                 uint4* out16 = reinterpret_cast<uint4*>(a.out8);
                 if (lo == kUnit * u0 && (keep_tail || (off1 & (kUnit - 1)) == 0)) {
-                    for (uint32_t k = lane; k < nu; k += 32) __stcs(out16 + u0 + k, unrotate16(ev16[k]));
+                    for (uint32_t q = lane; q < qe; q += 32)
+                        if (q >= a_sh) __stcs(out16 + ub + q, unrotate16(ev16[q - a_sh]));
                 } else {
-                    for (uint32_t k = lane; k < nu; k += 32) {
-                        const uint32_t u = u0 + k;
+                    for (uint32_t q = lane; q < qe; q += 32) {
+                        if (q < a_sh) continue;
+                        const uint32_t k = q - a_sh, u = u0 + k;
                         const uint4 v = unrotate16(ev16[k]);
                         const uint32_t i0 = kUnit * u;
                         if (i0 >= lo && i0 + kUnit <= off1) {
@@ -775,8 +786,8 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_warp_kernel(const Decode
                         } else {
                             const uint32_t words[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-                            for (int q = 0; q < 16; q++)
-                                if (i0 + q >= lo && i0 + q < off1) a.out8[i0 + q] = uint8_t(words[q >> 2] >> (8 * (q & 3)));
+                            for (int e = 0; e < 16; e++)
+                                if (i0 + e >= lo && i0 + e < off1) a.out8[i0 + e] = uint8_t(words[e >> 2] >> (8 * (e & 3)));
                         }
                     }
                 }
