@@ -233,6 +233,34 @@ df11_status df11_decompress_u8(const df11_header* hdr, const uint8_t* d_exp, con
                                const uint32_t* d_block_off, const void* d_lut, uint8_t* d_out,
                                uint32_t* d_status, void* stream);
 
+/* Decompress thread blocks [block_begin, block_end) of a stream only.  The
+ * per-block output positions of "Kernel de GPU em 2 etapas e metadados
+ * auxiliares" make every thread block decodable on its own, so a stream can
+ * be decoded piece by piece, e.g. while the next piece is still being copied
+ * to the device and the previous one copied back (our extension; the pages
+ * decode a whole block of matrices at once).  Pointers as for
+ * df11_decompress / df11_decompress_u8: the whole stream's arrays, of which
+ * the call reads, for b0 = block_begin, b1 = block_end:
+ *   d_exp        bytes [8 T b0, 8 T b1 + 16), within bytes_exp
+ *   d_gaps       bytes [5 T b0 / 8, 5 T b1 / 8 + 8), within bytes_gaps
+ *   d_block_off  entries b0 .. b1
+ *   d_sm         bytes [off[b0] rounded down to 128, off[b1] rounded up to 16),
+ *                within bytes_sm; only bytes [off[b0], off[b1]) affect d_out
+ *   d_lut        all of it
+ * and writes exactly output elements [off[b0], off[b1]) of d_out (the whole
+ * stream's output buffer); other elements are left as they are, so calls on
+ * disjoint ranges may run concurrently into one buffer.  block_begin ==
+ * block_end is a no-op; block_begin > block_end or block_end > n_blocks is
+ * DF11_ERR_INVALID.  Asynchronous, no allocation. */
+df11_status df11_decompress_blocks(const df11_header* hdr, const uint8_t* d_exp, const uint8_t* d_sm,
+                                   const uint8_t* d_gaps, const uint32_t* d_block_off, const void* d_lut,
+                                   uint16_t* d_out, uint64_t block_begin, uint64_t block_end,
+                                   uint32_t* d_status, void* stream);
+df11_status df11_decompress_u8_blocks(const df11_header* hdr, const uint8_t* d_exp, const uint8_t* d_gaps,
+                                      const uint32_t* d_block_off, const void* d_lut, uint8_t* d_out,
+                                      uint64_t block_begin, uint64_t block_end, uint32_t* d_status,
+                                      void* stream);
+
 /* Independent chunks: a variant of the container for comparison with the
  * Gaps-and-block-offsets design ("EntroLLM: Compressao de Pesos Codificada
  * por Entropia ...", section "Metodologia", item 3, decodes independently

@@ -20,7 +20,7 @@ EXPORTED = ["df11_version", "df11_last_error", "df11_code_lengths", "df11_header
             "df11_compress_workspace_size", "df11_compress_plan", "df11_compress_encode", "df11_decompress",
             "df11_compress_encode_static", "df11_decompress_sms", "df11_compress_plan_u8",
             "df11_compress_encode_u8", "df11_decompress_u8", "df11_compress_encode_chunked",
-            "df11_decompress_chunked"]
+            "df11_decompress_chunked", "df11_decompress_blocks", "df11_decompress_u8_blocks"]
 
 
 class Header(ctypes.Structure):
@@ -95,6 +95,8 @@ def load(build_if_missing: bool = True):
     lib.df11_decompress_u8.argtypes = [hp, vp, vp, vp, vp, vp, vp, vp]
     lib.df11_compress_encode_chunked.argtypes = [vp, hp, vp, u64, vp, vp, vp, vp, vp]
     lib.df11_decompress_chunked.argtypes = [hp, vp, vp, vp, vp, vp, vp, vp]
+    lib.df11_decompress_blocks.argtypes = [hp, vp, vp, vp, vp, vp, vp, u64, u64, vp, vp]
+    lib.df11_decompress_u8_blocks.argtypes = [hp, vp, vp, vp, vp, vp, u64, u64, vp, vp]
     for name in EXPORTED[2:]:
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib

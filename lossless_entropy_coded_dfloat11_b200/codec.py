@@ -228,10 +228,61 @@ def decompress(cs: CompressedStream, out: torch.Tensor | None = None, status: to
     return out
 
 
+def decompress_blocks(cs: CompressedStream, block_begin: int, block_end: int, out: torch.Tensor,
+                      status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Decode thread blocks [block_begin, block_end) of the stream only
+    (df11_decompress_blocks, or df11_decompress_u8_blocks for 8-bit symbols):
+    writes output elements [off[block_begin], off[block_end]) of `out`, the
+    whole stream's output buffer, and leaves the rest as it is.  Reads only
+    the bytes `piece_ranges` lists.  Asynchronous."""
+    u8 = cs.symbols == "u8"
+    dtype = torch.uint8 if u8 else torch.bfloat16
+    if out.dtype != dtype or not out.is_contiguous() or out.numel() < cs.n_elems:
+        raise ValueError(f"out must be a contiguous {dtype} tensor with n_elems elements")
+    st = _ptr(status) if status is not None else ctypes.c_void_p(0)
+    b0, b1 = ctypes.c_uint64(block_begin), ctypes.c_uint64(block_end)
+    if u8:
+        B.call("df11_decompress_u8_blocks", ctypes.byref(cs.header), _ptr(cs.exp), _ptr(cs.gaps),
+               _ptr(cs.block_off), _ptr(cs.lut), _ptr(out), b0, b1, st, _stream_handle(stream))
+    else:
+        B.call("df11_decompress_blocks", ctypes.byref(cs.header), _ptr(cs.exp), _ptr(cs.sm), _ptr(cs.gaps),
+               _ptr(cs.block_off), _ptr(cs.lut), _ptr(out), b0, b1, st, _stream_handle(stream))
+    return out
+
+
+def piece_ranges(header, block_off, b0: int, b1: int, u8: bool = False) -> dict[str, tuple[int, int]]:
+    """Byte ranges [lo, hi) of each stream array that decoding thread blocks
+    [b0, b1) reads (the contract of df11_decompress_blocks): EncodedExponent
+    from the piece's first window to 16 bytes past its last, the gap fields
+    of its windows plus one 8-byte lookahead, block offsets b0..b1, and the
+    sign+mantissa bytes of its elements widened to 128 bytes below and 16
+    above; each clipped to the array's size.  `block_off` is the host copy of
+    the offsets (any integer sequence)."""
+    T = int(header.threads_per_block)
+    lo_e, hi_e = int(block_off[b0]), int(block_off[b1])
+    r = {
+        "exp": (8 * T * b0, min(8 * T * b1 + 16, int(header.bytes_exp))),
+        "gaps": ((5 * T * b0) // 8, min((5 * T * b1 + 7) // 8 + 8, int(header.bytes_gaps))),
+        "block_off": (4 * b0, 4 * (b1 + 1)),
+    }
+    if not u8:
+        r["sm"] = (lo_e & ~127, min((hi_e + 15) & ~15, int(header.bytes_sm)))
+    return r
+
+
 class HostStream:
     """A stream kept in pinned host memory, decompressed end to end: copy the
     compressed arrays to the device, decode, copy the result (BF16, or bytes
-    for a stream of 8-bit symbols) back."""
+    for a stream of 8-bit symbols) back.
+
+    `run` splits the stream into pieces of whole thread blocks and pipelines
+    them over three CUDA streams: the copy of piece i+1 to the device, the
+    decode of piece i (on the caller's stream) and the copy of piece i-1
+    back run at the same time, so the two directions of the host link
+    overlap each other and the decode."""
+
+    PIECE_OUT_BYTES = 12 << 20  # output bytes per piece when `pieces` is not given
+    MAX_PIECES = 64
 
     def __init__(self, cs: CompressedStream):
         self.header = cs.header
@@ -247,20 +298,67 @@ class HostStream:
         n = cs.n_elems
         self.out_dev = torch.empty(max(n, 16), dtype=dtype, device=dev)[:n]
         self.out_host = torch.empty(max(n, 16), dtype=dtype).pin_memory()[:n]
+        self.off = self.host["block_off"].numpy().view(np.uint32)
+        self._side = None
+        self.last_h2d_bytes = 0
 
     def h2d_bytes(self) -> int:
-        return sum(v.numel() * v.element_size() for v in self.host.values())
+        """Bytes the last `run` copied to the device (every array once, plus
+        the few bytes pieces share); before any run, the arrays' sizes."""
+        return self.last_h2d_bytes or sum(v.numel() * v.element_size() for v in self.host.values())
 
     def d2h_bytes(self) -> int:
         return self.out_host.element_size() * int(self.header.n_elems)
 
-    def run(self, stream=None) -> torch.Tensor:
+    def default_pieces(self) -> int:
+        return max(1, min(self.MAX_PIECES, self.d2h_bytes() // self.PIECE_OUT_BYTES))
+
+    def run(self, stream=None, pieces: int | None = None) -> torch.Tensor:
         s = stream or torch.cuda.current_stream()
-        with torch.cuda.stream(s):
-            for k, v in self.host.items():
-                self.dev[k].copy_(v, non_blocking=True)
-            (decompress_u8 if self.u8 else decompress)(self.dev_stream, self.out_dev, stream=s)
-            self.out_host.copy_(self.out_dev, non_blocking=True)
+        nb = int(self.header.n_blocks)
+        n_pieces = max(1, min(self.default_pieces() if pieces is None else int(pieces), nb))
+        decode = decompress_u8 if self.u8 else decompress
+        if n_pieces == 1:
+            with torch.cuda.stream(s):
+                for k, v in self.host.items():
+                    self.dev[k].copy_(v, non_blocking=True)
+                decode(self.dev_stream, self.out_dev, stream=s)
+                self.out_host.copy_(self.out_dev, non_blocking=True)
+            self.last_h2d_bytes = sum(v.numel() * v.element_size() for v in self.host.values())
+            return self.out_host
+        if self._side is None:
+            dev = self.out_dev.device
+            self._side = (torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev))
+        s_in, s_out = self._side
+        # the buffers may still be in use by work already queued on the caller's stream
+        s_in.wait_stream(s)
+        s_out.wait_stream(s)
+        h2d = 0
+        with torch.cuda.stream(s_in):
+            self.dev["lut"].copy_(self.host["lut"], non_blocking=True)
+            h2d += self.host["lut"].numel()
+        bounds = [nb * i // n_pieces for i in range(n_pieces + 1)]
+        for i in range(n_pieces):
+            b0, b1 = bounds[i], bounds[i + 1]
+            with torch.cuda.stream(s_in):
+                for k, (lo, hi) in piece_ranges(self.header, self.off, b0, b1, self.u8).items():
+                    src, dst = self.host[k], self.dev[k]
+                    if k == "block_off":  # int32 entries
+                        lo, hi = lo // 4, hi // 4
+                    dst[lo:hi].copy_(src[lo:hi], non_blocking=True)
+                    h2d += (hi - lo) * src.element_size()
+            ready = torch.cuda.Event()
+            ready.record(s_in)
+            s.wait_event(ready)
+            decompress_blocks(self.dev_stream, b0, b1, self.out_dev, stream=s)
+            done = torch.cuda.Event()
+            done.record(s)
+            s_out.wait_event(done)
+            e0, e1 = int(self.off[b0]), int(self.off[b1])
+            with torch.cuda.stream(s_out):
+                self.out_host[e0:e1].copy_(self.out_dev[e0:e1], non_blocking=True)
+        s.wait_stream(s_out)
+        self.last_h2d_bytes = h2d
         return self.out_host
 
 

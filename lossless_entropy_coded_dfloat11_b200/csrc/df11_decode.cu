@@ -61,7 +61,8 @@ struct DecodeArgs {
     uint32_t* status;
     uint32_t n_elems;
     uint32_t n_threads;
-    uint32_t n_blocks;
+    uint32_t block0;     // first thread block to decode
+    uint32_t n_blocks;   // thread blocks to decode, from block0
     uint32_t last_wend;  // bits of the last window inside the stream, 1..64
 };
 
@@ -629,7 +630,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_warp_kernel(const Decode
     const uint32_t nw = gridDim.x * WARPS;
     const uint32_t g = warp * gridDim.x + blockIdx.x;
     const uint32_t per = a.n_blocks / nw, extra = a.n_blocks % nw;
-    uint32_t b = g * per + (g < extra ? g : extra);
+    uint32_t b = a.block0 + g * per + (g < extra ? g : extra);
     const uint32_t b_end = b + per + (g < extra ? 1u : 0u);
 
     copy_compact_tables(smem, a.lut, WARPS * 32);
@@ -1025,19 +1026,20 @@ __global__ void __launch_bounds__(T) decode_block_kernel(const DecodeArgs a) {
     const uint32_t my_gshift = (5 * threadIdx.x) & 31u;
     constexpr uint32_t kGwordsPerBlock = 5 * T / 32;
 
-    uint32_t b = blockIdx.x;
+    const uint32_t b_end = a.block0 + a.n_blocks;
+    uint32_t b = a.block0 + blockIdx.x;
     RawWindow nraw{};
     uint32_t noff0 = 0, noff1 = 0;
-    if (b < a.n_blocks) {
+    if (b < b_end) {
         nraw = load_window(a, T * b + threadIdx.x, kGwordsPerBlock * b + my_gword);
         noff0 = __ldg(a.off + b);
         noff1 = __ldg(a.off + b + 1);
     }
-    while (b < a.n_blocks) {
+    while (b < b_end) {
         const RawWindow raw = nraw;
         const uint32_t off0 = noff0, off1 = noff1;
         const uint32_t bn = b + gridDim.x;
-        if (bn < a.n_blocks) {
+        if (bn < b_end) {
             nraw = load_window(a, T * bn + threadIdx.x, kGwordsPerBlock * bn + my_gword);
             noff0 = __ldg(a.off + bn);
             noff1 = __ldg(a.off + bn + 1);
@@ -1186,10 +1188,16 @@ namespace {
 // of 8-bit symbols (u8 = true): no d_sm, d_out holds n_elems bytes.
 df11_status decompress_on(const char* fn, bool u8, const df11_header* hdr, const uint8_t* d_exp,
                           const uint8_t* d_sm, const uint8_t* d_gaps, const uint32_t* d_block_off,
-                          const void* d_lut, void* d_out, uint32_t* d_status, uint32_t max_sms, void* stream) {
+                          const void* d_lut, void* d_out, uint32_t* d_status, uint32_t max_sms, void* stream,
+                          uint64_t block_begin = 0, uint64_t block_end = UINT64_MAX) {
     df11_status st = check_header(hdr);
     if (st != DF11_OK) return st;
-    if (hdr->n_elems == 0) return DF11_OK;
+    if (block_end == UINT64_MAX) block_end = hdr->n_blocks;
+    if (block_begin > block_end || block_end > hdr->n_blocks)
+        return fail(DF11_ERR_INVALID, "%s: block range [%llu, %llu) outside [0, %llu)", fn,
+                    (unsigned long long)block_begin, (unsigned long long)block_end,
+                    (unsigned long long)hdr->n_blocks);
+    if (hdr->n_elems == 0 || block_begin == block_end) return DF11_OK;
     if (!d_exp || (!u8 && !d_sm) || !d_gaps || !d_block_off || !d_lut || !d_out)
         return fail(DF11_ERR_INVALID, "%s: null device pointer", fn);
     if (!aligned16(d_exp) || (!u8 && !aligned16(d_sm)) || !aligned16(d_gaps) || !aligned16(d_block_off) ||
@@ -1206,7 +1214,8 @@ df11_status decompress_on(const char* fn, bool u8, const df11_header* hdr, const
     a.status = d_status;
     a.n_elems = uint32_t(hdr->n_elems);
     a.n_threads = uint32_t(hdr->n_threads);
-    a.n_blocks = uint32_t(hdr->n_blocks);
+    a.block0 = uint32_t(block_begin);
+    a.n_blocks = uint32_t(block_end - block_begin);
     a.last_wend = uint32_t(hdr->total_bits - 64 * (hdr->n_threads - 1));
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     uint32_t min_len = 32;
@@ -1257,6 +1266,22 @@ extern "C" df11_status df11_decompress_u8(const df11_header* hdr, const uint8_t*
                                           uint32_t* d_status, void* stream) {
     return decompress_on("df11_decompress_u8", true, hdr, d_exp, nullptr, d_gaps, d_block_off, d_lut, d_out,
                          d_status, UINT32_MAX, stream);
+}
+
+extern "C" df11_status df11_decompress_blocks(const df11_header* hdr, const uint8_t* d_exp, const uint8_t* d_sm,
+                                              const uint8_t* d_gaps, const uint32_t* d_block_off,
+                                              const void* d_lut, uint16_t* d_out, uint64_t block_begin,
+                                              uint64_t block_end, uint32_t* d_status, void* stream) {
+    return decompress_on("df11_decompress_blocks", false, hdr, d_exp, d_sm, d_gaps, d_block_off, d_lut, d_out,
+                         d_status, UINT32_MAX, stream, block_begin, block_end);
+}
+
+extern "C" df11_status df11_decompress_u8_blocks(const df11_header* hdr, const uint8_t* d_exp, const uint8_t* d_gaps,
+                                                 const uint32_t* d_block_off, const void* d_lut, uint8_t* d_out,
+                                                 uint64_t block_begin, uint64_t block_end, uint32_t* d_status,
+                                                 void* stream) {
+    return decompress_on("df11_decompress_u8_blocks", true, hdr, d_exp, nullptr, d_gaps, d_block_off, d_lut,
+                         d_out, d_status, UINT32_MAX, stream, block_begin, block_end);
 }
 
 extern "C" df11_status df11_decompress_chunked(const df11_header* hdr, const uint8_t* d_exp, const uint8_t* d_sm,
