@@ -40,7 +40,9 @@ UNIT = "GB/s"
 FALLBACK_HBM_GBS = 6650.0
 L2_BYTES = 126 * 2**20  # B200 L2 capacity
 KERNEL_SOURCE = os.path.join(ROOT, "lossless_entropy_coded_dfloat11_b200", "csrc", "df11_decode.cu")
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_kernel_llama8b_block.txt")
+# committed ncu summaries giving the decode kernel's DRAM bytes per launch, by workload
+TRAFFIC_FILES = {"c3": os.path.join(ROOT, "profiles", "decode_kernel_llama8b_block.txt"),
+                 "c5": os.path.join(ROOT, "profiles", "decode_kernel_u8_llama8b_block.txt")}
 
 CONFIGS = {
     "c1": "matrix_1k: one 1024x1024 BF16 matrix, N(0, 0.02)",
@@ -104,12 +106,12 @@ def measured_peak_gbs() -> tuple[float, str]:
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def recorded_traffic() -> float | None:
-    """DRAM bytes per launch from the committed ncu summary, only while the
-    kernel source still matches the one that was profiled."""
+def recorded_traffic(config: str = "c3") -> float | None:
+    """DRAM bytes per launch from the committed ncu summary of this workload,
+    only while the kernel source still matches the one that was profiled."""
     try:
-        text = open(TRAFFIC_FILE).read()
-    except OSError:
+        text = open(TRAFFIC_FILES[config]).read()
+    except (KeyError, OSError):
         return None
     m_sha = re.search(r"kernel_source_sha256:\s*([0-9a-f]{64})", text)
     m_tr = re.search(r"traffic_bytes_per_launch_full_size:\s*([0-9.eE+]+)", text)
@@ -478,7 +480,7 @@ def run_native(args, rank: int, world: int, local_rank: int) -> None:
     peak, peak_kind = measured_peak_gbs()
     launch_ms = elapsed / (args.steps * launches_per_step)
     achieved = (alg_bytes / launches_per_step) / (launch_ms * 1e-3) / 1e9
-    traffic = recorded_traffic() if args.config == "c3" and not chunks else None
+    traffic = recorded_traffic(args.config) if not chunks else None
     cs0 = streams[0]
     line = {
         "metric": METRIC_U8 if u8 else METRIC, "value": agg["gbs"], "unit": UNIT, "n_gpus": world,
