@@ -26,7 +26,6 @@ import json
 import os
 import platform
 import re
-import subprocess
 import sys
 import threading
 import time

@@ -8,7 +8,6 @@ torch and pass raw pointers through the C ABI of include/df11.h.
 from __future__ import annotations
 
 import ctypes
-import math
 from dataclasses import dataclass, field
 
 import numpy as np

@@ -8,7 +8,6 @@ self-consistency of the auxiliary arrays under a windowed re-decode.
 """
 import heapq
 import itertools
-import math
 import os
 
 import numpy as np
