@@ -3,9 +3,12 @@
 Each case plants one mistake in a copy of oracle/df11_oracle.c (a dropped
 term, a wrong shift, sign or index, a transposed field), builds it, and runs
 the pin suite (tests/test_oracle_pins.py) against that build: the suite must
-fail.  Nothing here touches the real oracle or the CUDA library.
+fail.  The Python part of the oracle (the chunk start table) gets the same
+treatment through a mutated copy of the package, imported ahead of the real
+one.  Nothing here touches the real oracle or the CUDA library.
 """
 import os
+import shutil
 import subprocess
 import sys
 
@@ -57,3 +60,35 @@ def test_pins_catch_planted_mistake(name, old, new, tmp_path):
                           os.path.join(ROOT, "tests", "test_oracle_pins.py")],
                          capture_output=True, text=True, env=env, cwd=ROOT, timeout=600)
     assert res.returncode != 0, f"pins did not catch: {name}\n{res.stdout[-1500:]}"
+
+
+PY_SRC = os.path.join(ROOT, "oracle", "__init__.py")
+
+PY_MUTATIONS = [
+    ("chunk table without its leading zero", "return np.concatenate([[0], np.cumsum(per_chunk)]).astype(np.uint64)",
+     "return np.concatenate([np.cumsum(per_chunk), [per_chunk.sum()]]).astype(np.uint64)"),
+    ("chunk lengths from the wrong field", "ln = np.ascontiguousarray(code_len, dtype=np.uint8)[(x >> 7) & 0xFF]",
+     "ln = np.ascontiguousarray(code_len, dtype=np.uint8)[(x >> 8) & 0xFF]"),
+    ("chunks start one element late", "per_chunk = np.add.reduceat(ln.astype(np.uint64), np.arange(0, n, chunk))",
+     "per_chunk = np.add.reduceat(ln.astype(np.uint64), np.minimum(np.arange(0, n, chunk) + 1, n - 1))"),
+]
+
+
+@pytest.mark.parametrize("name,old,new", PY_MUTATIONS, ids=[m[0] for m in PY_MUTATIONS])
+def test_pins_catch_planted_mistake_in_python_oracle(name, old, new, tmp_path):
+    src = open(PY_SRC).read()
+    assert src.count(old) == 1, f"mutation site not found: {name}"
+    pkg = tmp_path / "oracle"
+    pkg.mkdir()
+    (pkg / "__init__.py").write_text(src.replace(old, new))
+    shutil.copy(os.path.join(ROOT, "oracle", "df11_oracle.c"), pkg / "df11_oracle.c")
+    import oracle
+    env = dict(os.environ, DF11_ORACLE_LIB=oracle.build())  # the real C part
+    pins = os.path.join(ROOT, "tests", "test_oracle_pins.py")
+    code = (f"import sys; sys.path.insert(0, {str(tmp_path)!r}); import oracle; "
+            f"assert oracle.__file__.startswith({str(tmp_path)!r}); import pytest; "
+            f"sys.exit(pytest.main(['-x', '-q', '-p', 'no:cacheprovider', {pins!r}]))")
+    res = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, env=env, cwd=ROOT,
+                         timeout=600)
+    assert res.returncode != 0, f"pins did not catch: {name}\n{res.stdout[-1500:]}"
+    assert "failed" in res.stdout, res.stdout[-800:] + res.stderr[-800:]
