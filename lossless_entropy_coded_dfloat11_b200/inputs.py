@@ -199,6 +199,23 @@ def quantize_u8(t: torch.Tensor) -> torch.Tensor:
     return torch.round((x - lo) / scale).clamp_(0, 255).to(torch.uint8)
 
 
+def quantize_u4(t: torch.Tensor) -> torch.Tensor:
+    """Per-tensor asymmetric 4-bit quantisation onto 0..15 (round to nearest),
+    one value per byte: the 16-symbol alphabet of uint4 weights, coded whole
+    by the same 8-bit-symbol streams."""
+    x = t.float()
+    lo, hi = x.min(), x.max()
+    scale = (hi - lo).clamp_min(1e-30) / 15.0
+    return torch.round((x - lo) / scale).clamp_(0, 15).to(torch.uint8)
+
+
+def llama_block_u4(cfg: dict = LLAMA_8B, seed_base: int = 3, device: str = "cpu") -> Workload:
+    """The matrices of `llama_block` quantized per tensor to 4 bits, one value
+    per byte."""
+    w = llama_block(cfg, seed_base, device)
+    return Workload(w.name + "-u4", list(w.names), [quantize_u4(t) for t in w.tensors])
+
+
 def llama_block_u8(cfg: dict = LLAMA_8B, seed_base: int = 3, device: str = "cpu") -> Workload:
     """The matrices of `llama_block` quantized per tensor to uint8."""
     w = llama_block(cfg, seed_base, device)

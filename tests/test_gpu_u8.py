@@ -74,6 +74,21 @@ def test_quantized_matrix(T):
     assert 0.88 < cs.compressed_bytes() / cs.n_elems < 0.95
 
 
+@pytest.mark.parametrize("T", [32, 64])
+def test_uint4_values_one_per_byte(T):
+    """uint4 weights (the other alphabet the EntroLLM page codes), one value
+    per byte: a 16-symbol alphabet on the same streams and kernels."""
+    w = inputs.Workload("q4", ["w"], [inputs.quantize_u4(inputs.gaussian((1024, 1024), 0.02, 1))])
+    cs = both_directions(w, T)
+    # ~2.69 code bits per value (entropy 2.65) plus a 5-bit gap per 64-bit
+    # window: ~0.365 bytes per value
+    assert 0.34 < cs.compressed_bytes() / cs.n_elems < 0.40
+
+
+def test_uint4_block():
+    both_directions(inputs.llama_block_u4(dict(hidden=512, intermediate=1408, kv=128), seed_base=150))
+
+
 @pytest.mark.parametrize("dist", inputs.EDGE_DISTS)
 @pytest.mark.parametrize("n", [1, 2, 31, 33, 255, 4097, 65537, (1 << 20) + 7])
 def test_edge_cases(n, dist):
