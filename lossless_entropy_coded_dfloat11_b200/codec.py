@@ -74,8 +74,9 @@ class CompressedStream:
                 + 4 * (h.n_blocks + 1) + 256)
 
     def read_bytes(self) -> int:
-        """Bytes one decompress reads from HBM (the format's arrays as the
-        kernel fetches them, plus the decode tables once per CTA from L2)."""
+        """Bytes of the format's arrays one decompress reads (exponent
+        stream, sign+mantissa bytes, gaps, block offsets); the decode tables,
+        fetched once per CTA and served from L2, are not counted."""
         h = self.header
         side = h.n_elems if self.symbols == "bf16" else 0
         return (h.total_bits + 7) // 8 + side + (5 * h.n_threads + 7) // 8 + 4 * (h.n_blocks + 1)
