@@ -38,6 +38,7 @@ METRIC_U8 = "decompressed 8-bit symbols GB/s on 1 B200 (bit-exact), % of HBM roo
 UNIT = "GB/s"
 FALLBACK_HBM_GBS = 6650.0
 L2_BYTES = 126 * 2**20  # B200 L2 capacity
+LEAD_CYCLES = 200_000    # ~0.1 ms device-side wait before a timed region
 KERNEL_SOURCE = os.path.join(ROOT, "lossless_entropy_coded_dfloat11_b200", "csrc", "df11_decode.cu")
 # committed ncu summaries giving the decode kernel's DRAM bytes per launch, by workload
 TRAFFIC_FILES = {"c3": os.path.join(ROOT, "profiles", "decode_kernel_llama8b_block.txt"),
@@ -52,6 +53,12 @@ CONFIGS = {
           "per block, each block one launch into one reused buffer",
     "c5": "llama3.1-8b-block quantized per tensor to uint8 (asymmetric, round to nearest); 218,112,000 "
           "8-bit symbols coded whole with one table, no side array, one launch",
+    "edge_one_value": "edge sweep, n = 2^26+13: 99.9% of exponents one value (1-bit code), sign+mantissa "
+                      "a uniform byte",
+    "edge_uniform": "edge sweep, n = 2^26+13: exponents uniform over 0..254 (the stream expands), "
+                    "sign+mantissa a uniform byte",
+    "edge_zipf": "edge sweep, n = 2^26+13: exponents Zipf(s=1.2) over 255 ranks mapped by a seeded "
+                 "permutation, sign+mantissa a uniform byte",
 }
 U8_CONFIGS = {"c5"}
 
@@ -199,9 +206,16 @@ def cpu_model() -> str:
 # --------------------------------------------------------------------------- #
 # workloads                                                                   #
 # --------------------------------------------------------------------------- #
+EDGE_N = 2 ** 26 + 13  # the edge sweep's largest size
+
+
 def make_workloads(config: str, rank: int, device: str):
     from lossless_entropy_coded_dfloat11_b200 import inputs as I
     off = rank_seed_offset(rank)
+    if config.startswith("edge_"):
+        dist = config[len("edge_"):]
+        w = I.edge_case(EDGE_N, dist, 500 + len(I.EDGE_SIZES) - 1 + off)
+        return [I.Workload(w.name, w.names, [t.to(device) for t in w.tensors])]
     if config == "c1":
         return [I.Workload("matrix_1k", ["w"], [I.gaussian((1024, 1024), 0.02, 1 + off, device=device)])]
     if config == "c2":
@@ -260,12 +274,12 @@ def time_oracle_decode(x, steps: int, warmup: int):
     return dt, s
 
 
-def time_oracle_decode_parallel(s, x, threads: int) -> float:
+def time_oracle_decode_parallel(s, x, threads: int):
     """The oracle's windowed decoder on `threads` host threads, one range of
     thread blocks per task: ranges decode independently through their Gaps and
     block offsets, the format's own parallel structure (the C oracle runs
-    without the interpreter lock).  Returns seconds for one full decode,
-    checked against x."""
+    without the interpreter lock).  Returns (seconds for one full decode, the
+    decoded elements), checked against x."""
     import numpy as np
     import oracle
     from concurrent.futures import ThreadPoolExecutor
@@ -280,8 +294,9 @@ def time_oracle_decode_parallel(s, x, threads: int) -> float:
         t0 = time.perf_counter()
         outs = run(pool)
         dt = time.perf_counter() - t0
-    assert np.array_equal(np.concatenate(outs), x), "parallel oracle decode failed"
-    return dt
+    y = np.concatenate(outs)
+    assert np.array_equal(y, x), "parallel oracle decode failed"
+    return dt, y
 
 
 # --------------------------------------------------------------------------- #
@@ -298,7 +313,7 @@ def run_reference(args, rank: int, world: int) -> None:
     line = {
         "impl": "reference", "metric": METRIC_U8 if esize == 1 else METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u8",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u8" if esize == 1 else "bf16",
         "data": "synthetic",
         "config": {"workload": CONFIGS[args.config], "reference_sample_elements": int(x.size)},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
@@ -335,6 +350,152 @@ def time_compress(df11, w, repeats: int, u8: bool = False, chunks: bool = False)
                     "table build, bit-pack kernels; median wall clock, synchronised"}
 
 
+def step_stats(per_step_ms: list[float]) -> dict:
+    """Median, min and max of per-step device times (CUDA events)."""
+    v = sorted(per_step_ms)
+    return {"median": v[len(v) // 2], "min": v[0], "max": v[-1], "n": len(v)}
+
+
+def time_steps(step, steps: int, warmup: int, stream, flush=None) -> tuple[float, list[float]]:
+    """Run `warmup` untimed steps, then time `steps` steps with one CUDA event
+    between consecutive steps on the launching stream.  Without `flush` the
+    steps run back to back and the total is the first-to-last event span; with
+    it, a write of the flush buffer (larger than L2) precedes every step and
+    only the steps are summed."""
+    import torch
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    if flush is None:
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+        # a short device-side wait ahead of the first event lets the host queue
+        # the first launches before the GPU reaches it, so the first step does
+        # not include the host's launch latency (the GPU would otherwise idle
+        # between the event and the kernel)
+        torch.cuda._sleep(LEAD_CYCLES)
+        ev[0].record(stream)
+        for i in range(steps):
+            step()
+            ev[i + 1].record(stream)
+        torch.cuda.synchronize()
+        per = [ev[i].elapsed_time(ev[i + 1]) for i in range(steps)]
+        return ev[0].elapsed_time(ev[-1]), per
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for i, (e0, e1) in enumerate(evs):
+        flush.fill_(i & 0xFF)
+        e0.record(stream)
+        step()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    per = [e0.elapsed_time(e1) for e0, e1 in evs]
+    return sum(per), per
+
+
+class Prepared:
+    """One workload compressed on this GPU, with its decode step and a
+    whole-output bit-exactness check to run after the timed region."""
+
+    def __init__(self, df11, config: str, rank: int, dev, chunks: bool = False, compress_repeats: int = 0,
+                 options=None):
+        import torch
+        self.config = config
+        self.options = options
+        self.u8 = config in U8_CONFIGS
+        self.chunks = chunks
+        self.esize = 1 if self.u8 else 2
+        self.compress = None
+        compress = df11.compress_u8 if self.u8 else df11.compress_chunked if chunks else df11.compress
+        self.decode = df11.decompress_u8 if self.u8 else df11.decompress_chunked if chunks else df11.decompress
+        self.streams, self.originals, self.seeds = [], [], []
+        bits = (lambda t: t) if self.u8 else (lambda t: t.view(torch.int16))
+        self.bits = bits
+        for w in make_workloads(config, rank, "cuda"):
+            if self.compress is None and compress_repeats:
+                self.compress = time_compress(df11, w, compress_repeats, self.u8, chunks)
+            self.streams.append(compress(w.tensors, names=w.names))
+            if config == "c4":  # 6.9B weights: regenerate each block for the check instead of keeping it
+                self.originals.append(None)
+            else:
+                self.originals.append(bits(torch.cat([t.reshape(-1) for t in w.tensors])))
+            del w
+        torch.cuda.synchronize()
+        self.n_max = max(cs.n_elems for cs in self.streams)
+        self.out = torch.empty(max(self.n_max, 16), dtype=torch.uint8 if self.u8 else torch.bfloat16, device=dev)
+        self.out_bytes = sum(self.esize * cs.n_elems for cs in self.streams)
+        self.alg_bytes = sum(cs.read_bytes() + self.esize * cs.n_elems for cs in self.streams)
+        self.elements = sum(cs.n_elems for cs in self.streams)
+
+    def step(self, stream):
+        if self.options is None:
+            for cs in self.streams:
+                self.decode(cs, out=self.out[: cs.n_elems], stream=stream)
+        else:
+            for cs in self.streams:
+                self.decode(cs, out=self.out[: cs.n_elems], stream=stream, options=self.options)
+
+    def check(self, rank: int, stream) -> tuple[bool, str]:
+        """Decode every stream once more and compare every element with the
+        original weights (C4: the block regenerated on the device from its
+        seeds, since the eight blocks are not kept)."""
+        import torch
+        from lossless_entropy_coded_dfloat11_b200 import inputs as I
+        ok = True
+        for b, (cs, orig) in enumerate(zip(self.streams, self.originals)):
+            if self.options is None:
+                got = self.decode(cs, out=self.out[: cs.n_elems], stream=stream)
+            else:
+                got = self.decode(cs, out=self.out[: cs.n_elems], stream=stream, options=self.options)
+            if orig is None:
+                w = I.llama_block(I.LLAMA_70B, seed_base=100 + 16 * b + rank_seed_offset(rank), device="cuda")
+                orig = self.bits(torch.cat([t.reshape(-1) for t in w.tensors]))
+                del w
+            ok &= bool(torch.equal(self.bits(got), orig))
+        torch.cuda.synchronize()
+        scope = (f"every element of every block ({len(self.streams)} blocks, each decoded again after the timed "
+                 "region and compared with the block regenerated on the device)" if self.config == "c4" else
+                 "every element of the output, decoded again after the timed region")
+        return ok, scope
+
+
+def measure(pw: Prepared, steps: int, warmup: int, stream, dev, world: int) -> dict:
+    """Time one prepared workload and check it; the record every workload
+    line carries."""
+    import torch
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev) if pw.alg_bytes < 2 * L2_BYTES else None
+    elapsed, per = time_steps(lambda: pw.step(stream), steps, warmup, stream, flush)
+    del flush
+    elapsed = max_over_ranks(elapsed, dev)
+    exact, scope = pw.check(0, stream)
+    exact = min_over_ranks(exact, dev)
+    agg = aggregate([elapsed] * world, pw.out_bytes, steps)
+    peak, peak_kind = measured_peak_gbs()
+    launches = len(pw.streams)
+    launch_ms = elapsed / (steps * launches)
+    achieved = (pw.alg_bytes / launches) / (launch_ms * 1e-3) / 1e9
+    cs0 = pw.streams[0]
+    return {
+        "workload": CONFIGS[pw.config], "metric": METRIC_U8 if pw.u8 else METRIC, "value": agg["gbs"],
+        "unit": UNIT, "ms_per_step": agg["ms_per_step"], "per_step_ms": step_stats(per),
+        "elements_per_step": pw.elements, "elements_per_s": agg["gbs"] * 1e9 / pw.esize,
+        "launches_per_step": launches, "bit_exact": exact, "bit_exact_scope": scope,
+        "compression_ratio": sum(c.compressed_bytes() for c in pw.streams) / pw.out_bytes,
+        "threads_per_block": None if pw.chunks else cs0.threads_per_block,
+        "decode_kernel": None if pw.chunks else cs0.kernel_info(pw.u8),
+        "l2": ("no flush: compressed input + output per step exceed the 126 MB L2" if pw.alg_bytes >= 2 * L2_BYTES
+               else f"flushed: a {2 * L2_BYTES >> 20} MiB buffer is written before each step; per-step CUDA "
+                    "events time the decode alone"),
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "peak_kind": f"{peak_kind} (copy bandwidth)",
+                     "algorithmic_bytes_per_launch": pw.alg_bytes / launches,
+                     "frac_of_8000_nominal": achieved / 8000.0},
+        "_elapsed_ms": elapsed,
+    }
+
+
+# the workloads measured besides the headline one in a default run
+EXTRA_CONFIGS = ["c4", "c2", "c1", "c5", "edge_one_value", "edge_uniform", "edge_zipf"]
+
+
 def run_native(args, rank: int, world: int, local_rank: int) -> None:
     import numpy as np
     import torch
@@ -344,44 +505,16 @@ def run_native(args, rank: int, world: int, local_rank: int) -> None:
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     df11.load_library()
-
-    # ---- build the compressed workload on this GPU ------------------------
-    workloads = make_workloads(args.config, rank, "cuda")
-    u8 = args.config in U8_CONFIGS  # 8-bit symbols: uint8 out, no side array
     chunks = args.layout == "chunks"  # independent-chunk variant of the container
-    if chunks and u8:
+    if chunks and args.config in U8_CONFIGS:
         raise SystemExit("--layout chunks takes BF16 configurations")
-    esize = 1 if u8 else 2          # output bytes per element
-    bits16 = (lambda t: t) if u8 else (lambda t: t.view(torch.int16))
-    streams, originals = [], []
-    compress = None
-    for w in workloads:
-        if compress is None and not args.no_compress:
-            compress = time_compress(df11, w, args.compress_repeats, u8, chunks)
-        cs = (df11.compress_u8 if u8 else df11.compress_chunked if chunks else df11.compress)(
-            w.tensors, names=w.names)
-        streams.append(cs)
-        originals.append(bits16(torch.cat([t.reshape(-1) for t in w.tensors]))
-                         if len(workloads) == 1 else None)
-        if len(workloads) > 1:
-            # keep a fingerprint per block instead of all 6.9B weights
-            originals[-1] = [t.reshape(-1).view(torch.int16)[:: 4093].clone() for t in w.tensors]
-        del w
-    torch.cuda.synchronize()
-    n_max = max(cs.n_elems for cs in streams)
-    out = torch.empty(max(n_max, 16), dtype=torch.uint8 if u8 else torch.bfloat16, device=dev)
     stream = torch.cuda.current_stream()
-    out_bytes = sum(esize * cs.n_elems for cs in streams)
-    alg_bytes = sum(cs.read_bytes() + esize * cs.n_elems for cs in streams)
-    launches_per_step = len(streams)
-    decode = df11.decompress_u8 if u8 else df11.decompress_chunked if chunks else df11.decompress
 
-    def step():
-        for cs in streams:
-            decode(cs, out=out[: cs.n_elems], stream=stream)
-
+    # ---- the headline workload, built and compressed on this GPU ----------
+    opts = df11.decode_options(peek_bits=args.peek_bits) if args.peek_bits else None
+    pw = Prepared(df11, args.config, rank, dev, chunks, 0 if args.no_compress else args.compress_repeats, opts)
     for _ in range(args.warmup):
-        step()
+        pw.step(stream)
     torch.cuda.synchronize()
 
     # ---- timed region -------------------------------------------------------
@@ -389,50 +522,21 @@ def run_native(args, rank: int, world: int, local_rank: int) -> None:
         dist.barrier()
     torch.cuda.synchronize()
     sampler = ClockSampler(local_rank)
-    # a step whose bytes could stay in L2 is preceded by a write of a buffer
-    # twice the L2 size and timed on its own
-    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev) if alg_bytes < 2 * L2_BYTES else None
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev) if pw.alg_bytes < 2 * L2_BYTES else None
     with sampler:
-        if flush is None:
-            ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            ev0.record(stream)
-            for _ in range(args.steps):
-                step()
-            ev1.record(stream)
-            torch.cuda.synchronize()
-            elapsed = ev0.elapsed_time(ev1)
-        else:
-            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                   for _ in range(args.steps)]
-            for i, (e0, e1) in enumerate(evs):
-                flush.fill_(i & 0xFF)
-                e0.record(stream)
-                step()
-                e1.record(stream)
-            torch.cuda.synchronize()
-            elapsed = sum(e0.elapsed_time(e1) for e0, e1 in evs)
+        elapsed, per_step = time_steps(lambda: pw.step(stream), args.steps, 0, stream, flush)
     if world > 1:
         dist.barrier()
-
-    # ---- bit-exact check of the last step's output --------------------------
-    exact = True
-    if len(streams) == 1:
-        exact = bool(torch.equal(bits16(out[: streams[0].n_elems]), originals[0]))
-    else:
-        for cs, fp in zip(streams, originals):
-            step_out = decode(cs, out=out[: cs.n_elems], stream=stream)
-            for v, f in zip(cs.views(step_out), fp):
-                exact &= bool(torch.equal(v.reshape(-1).view(torch.int16)[:: 4093], f))
-    torch.cuda.synchronize()
-
+    del flush
+    exact, exact_scope = pw.check(rank, stream)
     per_rank = [max_over_ranks(elapsed, dev)] * world
     exact = min_over_ranks(exact, dev)
-    agg = aggregate(per_rank, out_bytes, args.steps)
+    agg = aggregate(per_rank, pw.out_bytes, args.steps)
 
     # ---- end to end: host buffers through the public API --------------------
     e2e = None
-    if not args.no_e2e and len(streams) == 1 and not chunks:
-        hs = df11.HostStream(streams[0])
+    if not args.no_e2e and len(pw.streams) == 1 and not chunks:
+        hs = df11.HostStream(pw.streams[0])
         for _ in range(2):
             hs.run(stream)
         torch.cuda.synchronize()
@@ -447,8 +551,8 @@ def run_native(args, rank: int, world: int, local_rank: int) -> None:
         e1.record(stream)
         torch.cuda.synchronize()
         ems = max_over_ranks(e0.elapsed_time(e1), dev)
-        e2e_exact = bool(torch.equal(bits16(res), originals[0].cpu()))
-        e2e = {"value": esize * streams[0].n_elems * k * world / (ems * 1e-3) / 1e9, "unit": UNIT,
+        e2e_exact = bool(torch.equal(pw.bits(res), pw.originals[0].cpu()))
+        e2e = {"value": pw.esize * pw.streams[0].n_elems * k * world / (ems * 1e-3) / 1e9, "unit": UNIT,
                "h2d_bytes_per_step": hs.h2d_bytes(), "d2h_bytes_per_step": hs.d2h_bytes(),
                "steps": k, "bit_exact": e2e_exact}
         del hs
@@ -456,63 +560,83 @@ def run_native(args, rank: int, world: int, local_rank: int) -> None:
     # ---- CPU baseline (oracle, rank 0, one GPU) ----------------------------
     cpu = cpu_parallel = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not chunks:
-        n_sample = min(args.cpu_sample, streams[0].n_elems)
-        if len(streams) == 1:
-            x = originals[0][:n_sample].cpu().numpy()
+        n_sample = min(args.cpu_sample, pw.streams[0].n_elems)
+        if pw.originals[0] is not None:
+            x = pw.originals[0][:n_sample].cpu().numpy()
             # the oracle codes byte v as the exponent field of the BF16 pattern v << 7
-            x = x.astype(np.uint16) << 7 if u8 else x.view(np.uint16)
+            x = x.astype(np.uint16) << 7 if pw.u8 else x.view(np.uint16)
         else:
             x = reference_sample(args.config, n_sample)
         dt, sx = time_oracle_decode(x, 1, 0)
-        cpu = {"value": esize * x.size / dt / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
+        cpu = {"value": pw.esize * x.size / dt / 1e9, "unit": UNIT, "cores": 1, "kind": "oracle",
                "sample": f"first {x.size} elements of the workload, oracle bit-serial decode, one "
                          f"thread on {cpu_model()} ({os.cpu_count()} host cores present)",
                "seconds": dt}
         threads = os.cpu_count() or 1
-        dtp = time_oracle_decode_parallel(sx, x, threads)
-        cpu_parallel = {"value": esize * x.size / dtp / 1e9, "unit": UNIT, "cores": threads,
+        dtp, _ = time_oracle_decode_parallel(sx, x, threads)
+        cpu_parallel = {"value": pw.esize * x.size / dtp / 1e9, "unit": UNIT, "cores": threads,
                         "kind": "oracle windowed decode, ranges of thread blocks on host threads",
                         "sample": cpu["sample"].split(", oracle")[0], "seconds": dtp}
 
-    if rank != 0:
-        return
+    # ---- headline record ----------------------------------------------------
     peak, peak_kind = measured_peak_gbs()
-    launch_ms = elapsed / (args.steps * launches_per_step)
-    achieved = (alg_bytes / launches_per_step) / (launch_ms * 1e-3) / 1e9
+    launches = len(pw.streams)
+    launch_ms = per_rank[0] / (args.steps * launches)
+    achieved = (pw.alg_bytes / launches) / (launch_ms * 1e-3) / 1e9
     traffic = recorded_traffic(args.config) if not chunks else None
-    cs0 = streams[0]
+    cs0 = pw.streams[0]
     line = {
-        "metric": METRIC_U8 if u8 else METRIC, "value": agg["gbs"], "unit": UNIT, "n_gpus": world,
+        "metric": METRIC_U8 if pw.u8 else METRIC, "value": agg["gbs"], "unit": UNIT, "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": agg["ms_per_step"], "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "u8", "data": "synthetic",
-        "config": {"workload": CONFIGS[args.config], "elements_per_step": sum(c.n_elems for c in streams),
+        "scaling": "weak", "vs_baseline": None, "dtype": "u8" if pw.u8 else "bf16", "data": "synthetic",
+        "config": {"workload": CONFIGS[args.config], "elements_per_step": pw.elements,
                    "threads_per_block": None if chunks else cs0.threads_per_block,
                    "layout": (f"independent chunks of {df11.IND_CHUNK} elements (start-bit table), no gaps or scan"
                               if chunks else "gaps + thread-block offsets"),
-                   "launches_per_step": launches_per_step,
+                   "launches_per_step": launches,
+                   "decode_kernel": None if chunks else cs0.kernel_info(pw.u8, opts),
                    "l2": ("no flush: compressed input + output per step exceed the 126 MB L2"
-                          if flush is None else
+                          if pw.alg_bytes >= 2 * L2_BYTES else
                           f"flushed: a {2 * L2_BYTES >> 20} MiB buffer is written before each step; "
                           "per-step CUDA events time the decode alone"),
                    "parallelism": f"replicas x{world} (independent streams per rank)"},
-        "bit_exact": exact,
-        "elements_per_s": agg["gbs"] * 1e9 / esize,
-        "compression_ratio": sum(c.compressed_bytes() for c in streams) / out_bytes,
+        "per_step_ms": step_stats(per_step),
+        "bit_exact": exact, "bit_exact_scope": exact_scope,
+        "elements_per_s": agg["gbs"] * 1e9 / pw.esize,
+        "compression_ratio": sum(c.compressed_bytes() for c in pw.streams) / pw.out_bytes,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic,
                      "peak_kind": f"{peak_kind} (copy bandwidth)",
-                     "algorithmic_bytes_per_launch": alg_bytes / launches_per_step,
+                     "algorithmic_bytes_per_launch": pw.alg_bytes / launches,
                      "frac_of_8000_nominal": achieved / 8000.0},
         "cpu_baseline": cpu,
         "cpu_parallel": cpu_parallel,
         "e2e": e2e,
-        "gpu_launches": args.steps * launches_per_step,
-        "compress": compress,
+        "gpu_launches": args.steps * launches,
+        "compress": pw.compress,
         "clocks": sampler.record(),
-        "when": datetime.datetime.now(datetime.timezone.utc).isoformat(timespec="seconds"),
     }
-    print(json.dumps(line), flush=True)
+    del pw
+    torch.cuda.empty_cache()
+
+    # ---- every other workload, each timed the same way ----------------------
+    if world == 1 and not args.headline_only and not chunks and not args.peek_bits:
+        extra = {}
+        for c in EXTRA_CONFIGS:
+            if c == args.config:
+                continue
+            other = Prepared(df11, c, rank, dev)
+            rec = measure(other, args.steps, args.warmup, stream, dev, world)
+            line["gpu_launches"] += (args.steps + args.warmup + 1) * rec["launches_per_step"]
+            rec.pop("_elapsed_ms")
+            extra[c] = rec
+            del other
+            torch.cuda.empty_cache()
+        line["workloads"] = extra
+    line["when"] = datetime.datetime.now(datetime.timezone.utc).isoformat(timespec="seconds")
+    if rank == 0:
+        print(json.dumps(line), flush=True)
 
 
 def run_pipeline(args, local_rank: int) -> None:
@@ -566,6 +690,36 @@ def run_pipeline(args, local_rank: int) -> None:
         pf = df11.BlockPrefetcher(streams, max_sms=cap)
         res["prefetch_all_sms" if cap is None else f"prefetch_{cap}_sms"] = timed(
             lambda: [consume(views) for _, views in pf])
+    # many small CTAs that queue behind the consumer's kernels and take the
+    # SMs those leave idle (cuBLAS's B200 GEMMs run 128 CTAs of up to 226 KB
+    # of shared memory: one per SM on 128 of the 148 SMs)
+    for ctas, warps in args.pipeline_shapes:
+        pf = df11.BlockPrefetcher(streams, options=df11.decode_options(ctas=ctas, max_warps_per_cta=warps))
+        res[f"prefetch_{ctas}x{warps}w"] = timed(lambda: [consume(views) for _, views in pf])
+    # the consumer on a high-priority stream and the decode on the lowest: when
+    # an SM frees up, the block scheduler hands it to the consumer's CTAs
+    # first, so the decode's CTAs take what the consumer leaves idle
+    hi = torch.cuda.Stream(priority=-100)
+    lo = torch.cuda.Stream(priority=0)
+
+    def timed_on(st, fn, reps=3):
+        with torch.cuda.stream(st):
+            fn()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(st)
+            for _ in range(reps):
+                fn()
+            e1.record(st)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / (reps * len(streams))
+
+    for ctas, warps in [(0, 0)] + list(args.pipeline_shapes):
+        opts = df11.decode_options(ctas=ctas, max_warps_per_cta=warps) if ctas else None
+        pf = df11.BlockPrefetcher(streams, options=opts, decode_stream=lo)
+        key = "prefetch_prio_all_sms" if not ctas else f"prefetch_prio_{ctas}x{warps}w"
+        res[key] = timed_on(hi, lambda: [consume(views) for _, views in pf])
+    res["serial_hi_stream"] = timed_on(hi, serial)
     best = min(v for k, v in res.items() if k.startswith("prefetch"))
     hidden = (res["serial"] - best) / min(res["decode_only"], res["consumer_only"])
     flops = 2 * args.tokens * sum(cs.n_elems for cs in streams) / len(streams)
@@ -596,6 +750,11 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-compress", action="store_true", help="skip timing the compress call")
+    ap.add_argument("--peek-bits", type=int, default=0,
+                    help="first-level table width of the timed decode: 12 (default), or 8, 9, 10 for a "
+                         "narrow table in 16 shared-memory copies (BF16 configurations)")
+    ap.add_argument("--headline-only", action="store_true",
+                    help="time the --config workload only, not the other workloads")
     ap.add_argument("--layout", choices=["gaps", "chunks"], default="gaps",
                     help="chunks: the independent-chunk variant of the container (an ablation)")
     ap.add_argument("--compress-repeats", type=int, default=5)
@@ -604,6 +763,9 @@ def main(argv=None):
     ap.add_argument("--pipeline-blocks", type=int, default=4)
     ap.add_argument("--tokens", type=int, default=1024, help="consumer activation rows (--pipeline)")
     ap.add_argument("--pipeline-sms", type=int, nargs="*", default=[16, 32, 64])
+    ap.add_argument("--pipeline-shapes", type=lambda v: tuple(int(x) for x in v.split("x")), nargs="*",
+                    default=[(1184, 4), (4736, 4), (9472, 2)],
+                    help="CTAsxWARPS launch shapes of the prefetched decode (many small CTAs)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("at least 3 warm-up steps")

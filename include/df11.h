@@ -165,14 +165,20 @@ df11_status df11_compress_encode(const void* const* d_segs, const df11_header* h
  * instance) where allocating would recurse.  It calls no cudaMalloc/cudaFree.
  *   - At most DF11_STATIC_MAX_ELEMS (2^28) elements per call; larger streams
  *     get DF11_ERR_TOO_LARGE (use df11_compress_encode with a workspace).
- *   - The scratch is 786,432 bytes of device memory that every GPU loading
- *     the library holds until exit.
- *   - The first call on a device looks up the scratch's device address (with
- *     that device current); make that first call before any stream capture.
- *   - All calls share the one scratch array and every call overwrites all of
- *     it that it reads, so no clearing is needed; calls whose work overlaps
- *     on the GPU (other streams, other host threads) race on it and must be
- *     serialised by the caller.
+ *   - The scratch is 524,304 bytes of device memory that every GPU using the
+ *     library's device code holds until exit.
+ *   - That device code, and the scratch with it, is put on a GPU when the
+ *     library first uses the GPU (CUDA loads modules lazily by default), and
+ *     that first use may itself need device memory.  So make one call of this
+ *     entry point (or any compress or decompress) on each device at start-up,
+ *     before handing HBM to other pools and before any stream capture.
+ *   - Every call looks up the scratch's address for the current device and
+ *     context on the host; once the device code is loaded this allocates
+ *     nothing.
+ *   - All calls share the one scratch array, which keeps the last call's
+ *     contents; every call clears, on its stream, the part it uses before
+ *     its kernel.  Calls whose work overlaps on the GPU (other streams, other
+ *     host threads) race on it and must be serialised by the caller.
  * Arguments as for df11_compress_encode, minus the workspace. */
 df11_status df11_compress_encode_static(const void* const* d_segs, const df11_header* hdr,
                                         uint8_t* d_exp, uint8_t* d_sm, uint8_t* d_gaps,
@@ -280,6 +286,61 @@ df11_status df11_compress_encode_chunked(const void* const* d_segs, const df11_h
 df11_status df11_decompress_chunked(const df11_header* hdr, const uint8_t* d_exp, const uint8_t* d_sm,
                                     const uint32_t* d_chunk_bit, const void* d_lut, uint16_t* d_out,
                                     uint32_t* d_status, void* stream);
+
+/* Options of df11_decompress_opts (all zero = exactly df11_decompress /
+ * df11_decompress_u8).  The pages' first-level tables have 256 entries
+ * ("Decodificacao com LUT hierarquica"); the library's default is a 12-bit,
+ * multi-symbol table in one shared-memory copy, which measured fastest on
+ * LLM weights.  peek_bits selects the alternatives for comparison. */
+typedef struct {
+    uint32_t peek_bits;          /* 0 or 12: default table; 8, 9 or 10: a 2^K-entry
+                                    first-level table held in 16 copies, one per
+                                    8-byte bank pair (BF16 streams, T = 64, codes of
+                                    >= 2 bits; DF11_ERR_INVALID otherwise)       */
+    uint32_t max_sms;            /* 0 = every SM; else size the grid for this many */
+    uint32_t max_warps_per_cta;  /* 0 = the kernel's maximum                      */
+    uint32_t ctas;               /* 0 = one persistent CTA per SM (fewer for small
+                                    streams); else this many CTAs at most, each
+                                    decoding a contiguous run of thread blocks --
+                                    more CTAs than fit at once simply queue, so
+                                    many small CTAs interleave with other kernels */
+    uint32_t reserved[2];        /* must be zero                                  */
+} df11_decode_options;
+
+/* df11_decompress (symbols_u8 = 0, d_out: n_elems uint16) or
+ * df11_decompress_u8 (symbols_u8 = 1, d_out: n_elems bytes, d_sm unused) with
+ * the options above; same arguments otherwise, same result (every option gives
+ * bit-identical output), asynchronous, no allocation. */
+df11_status df11_decompress_opts(const df11_header* hdr, const uint8_t* d_exp, const uint8_t* d_sm,
+                                 const uint8_t* d_gaps, const uint32_t* d_block_off, const void* d_lut,
+                                 void* d_out, uint32_t symbols_u8, const df11_decode_options* opt,
+                                 uint32_t* d_status, void* stream);
+
+/* Which decode kernel a stream gets on the current device, and its launch
+ * shape: a host-side query with no launch and no allocation (the first query
+ * for a kernel on a device sets its shared-memory limit and reads its
+ * occupancy, as the first decode does).  The pages have no counterpart; it
+ * reports the on-chip choices of "Decodificacao com LUT hierarquica" (the
+ * width of the first-level table and how many copies of it shared memory
+ * holds) and of "Kernel de GPU em 2 etapas e metadados auxiliares" (threads
+ * per CTA, CTAs) for a whole-stream df11_decompress / df11_decompress_u8.
+ *   hdr         in: the stream's header (checked as df11_decompress checks it)
+ *   symbols_u8  in: 0 for BF16 streams, 1 for streams of 8-bit symbols
+ *   opt         in, may be NULL: options as for df11_decompress_opts
+ *   info        out: see the fields
+ * Returns DF11_ERR_INVALID for a header no kernel decodes. */
+typedef struct {
+    char kernel[64];          /* kernel name with its template arguments        */
+    uint32_t grid;            /* CTAs                                            */
+    uint32_t block;           /* threads per CTA                                 */
+    uint32_t smem_bytes;      /* dynamic shared memory per CTA                   */
+    uint32_t peek_bits;       /* first-level table index width K (2^K entries)   */
+    uint32_t table_copies;    /* copies of the first-level decode table per CTA  */
+    uint32_t reserved;
+    uint64_t thread_blocks;   /* format thread blocks (n_blocks)                 */
+} df11_kernel_info;
+df11_status df11_decode_kernel_info(const df11_header* hdr, uint32_t symbols_u8, const df11_decode_options* opt,
+                                    df11_kernel_info* info);
 
 #ifdef __cplusplus
 }

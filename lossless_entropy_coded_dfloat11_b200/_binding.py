@@ -20,7 +20,8 @@ EXPORTED = ["df11_version", "df11_last_error", "df11_code_lengths", "df11_header
             "df11_compress_workspace_size", "df11_compress_plan", "df11_compress_encode", "df11_decompress",
             "df11_compress_encode_static", "df11_decompress_sms", "df11_compress_plan_u8",
             "df11_compress_encode_u8", "df11_decompress_u8", "df11_compress_encode_chunked",
-            "df11_decompress_chunked", "df11_decompress_blocks", "df11_decompress_u8_blocks"]
+            "df11_decompress_chunked", "df11_decompress_blocks", "df11_decompress_u8_blocks",
+            "df11_decode_kernel_info", "df11_decompress_opts"]
 
 
 class Header(ctypes.Structure):
@@ -43,6 +44,31 @@ class Header(ctypes.Structure):
         ("bytes_gaps", ctypes.c_uint64),
         ("bytes_off", ctypes.c_uint64),
         ("bytes_lut", ctypes.c_uint64),
+    ]
+
+
+class DecodeOptions(ctypes.Structure):
+    """Mirror of df11_decode_options."""
+    _fields_ = [
+        ("peek_bits", ctypes.c_uint32),
+        ("max_sms", ctypes.c_uint32),
+        ("max_warps_per_cta", ctypes.c_uint32),
+        ("ctas", ctypes.c_uint32),
+        ("reserved", ctypes.c_uint32 * 2),
+    ]
+
+
+class KernelInfo(ctypes.Structure):
+    """Mirror of df11_kernel_info."""
+    _fields_ = [
+        ("kernel", ctypes.c_char * 64),
+        ("grid", ctypes.c_uint32),
+        ("block", ctypes.c_uint32),
+        ("smem_bytes", ctypes.c_uint32),
+        ("peek_bits", ctypes.c_uint32),
+        ("table_copies", ctypes.c_uint32),
+        ("reserved", ctypes.c_uint32),
+        ("thread_blocks", ctypes.c_uint64),
     ]
 
 
@@ -97,6 +123,8 @@ def load(build_if_missing: bool = True):
     lib.df11_decompress_chunked.argtypes = [hp, vp, vp, vp, vp, vp, vp, vp]
     lib.df11_decompress_blocks.argtypes = [hp, vp, vp, vp, vp, vp, vp, u64, u64, vp, vp]
     lib.df11_decompress_u8_blocks.argtypes = [hp, vp, vp, vp, vp, vp, u64, u64, vp, vp]
+    lib.df11_decode_kernel_info.argtypes = [hp, u32, ctypes.POINTER(DecodeOptions), ctypes.POINTER(KernelInfo)]
+    lib.df11_decompress_opts.argtypes = [hp, vp, vp, vp, vp, vp, vp, u32, ctypes.POINTER(DecodeOptions), vp, vp]
     for name in EXPORTED[2:]:
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib

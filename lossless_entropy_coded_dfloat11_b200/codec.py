@@ -81,6 +81,18 @@ class CompressedStream:
         side = h.n_elems if self.symbols == "bf16" else 0
         return (h.total_bits + 7) // 8 + side + (5 * h.n_threads + 7) // 8 + 4 * (h.n_blocks + 1)
 
+    def kernel_info(self, u8: bool | None = None, options=None) -> dict:
+        """The decode kernel a whole-stream decompress of this stream launches
+        on the current device, with its grid, CTA size, shared memory, table
+        width and table copies (df11_decode_kernel_info)."""
+        info = B.KernelInfo()
+        u8 = self.symbols == "u8" if u8 is None else u8
+        B.call("df11_decode_kernel_info", ctypes.byref(self.header), 1 if u8 else 0,
+               ctypes.byref(options) if options is not None else None, ctypes.byref(info))
+        return {"kernel": info.kernel.decode(), "grid": int(info.grid), "block": int(info.block),
+                "smem_bytes": int(info.smem_bytes), "peek_bits": int(info.peek_bits),
+                "table_copies": int(info.table_copies), "thread_blocks": int(info.thread_blocks)}
+
     def views(self, flat: torch.Tensor) -> list[torch.Tensor]:
         """Per-matrix views of a decompressed flat buffer."""
         out = []
@@ -206,25 +218,34 @@ def to_host(cs: CompressedStream) -> dict:
                 block_off=cs.block_off.cpu().numpy().view(np.uint32)[: int(h.n_blocks) + 1])
 
 
+def decode_options(peek_bits: int = 0, max_sms: int = 0, max_warps_per_cta: int = 0, ctas: int = 0):
+    """df11_decode_options (all zero: the library's defaults)."""
+    return B.DecodeOptions(peek_bits, max_sms, max_warps_per_cta, ctas)
+
+
 def decompress(cs: CompressedStream, out: torch.Tensor | None = None, status: torch.Tensor | None = None,
-               stream=None, max_sms: int | None = None) -> torch.Tensor:
+               stream=None, max_sms: int | None = None, options=None) -> torch.Tensor:
     """One kernel launch rebuilding all n_elems BF16 values of the stream.
     Asynchronous; `out` (bfloat16, n_elems, contiguous) may be reused across
     calls.  `status` (int32 device word, zeroed by the caller) receives
     DF11_ERR_CORRUPT if the stream disagrees with its metadata.  `max_sms`
     caps the SMs the decode occupies (df11_decompress_sms), leaving the rest
-    to kernels on other streams."""
+    to kernels on other streams; `options` (decode_options) selects the
+    table width and launch shape (df11_decompress_opts)."""
     n = cs.n_elems
     if out is None:
         out = torch.empty(max(n, 1), dtype=torch.bfloat16, device=cs.exp.device)[:n]
     if out.dtype != torch.bfloat16 or not out.is_contiguous() or out.numel() < n:
         raise ValueError("out must be a contiguous bfloat16 tensor with n_elems elements")
+    st = _ptr(status) if status is not None else ctypes.c_void_p(0)
     args = (ctypes.byref(cs.header), _ptr(cs.exp), _ptr(cs.sm), _ptr(cs.gaps), _ptr(cs.block_off),
-            _ptr(cs.lut), _ptr(out), _ptr(status) if status is not None else ctypes.c_void_p(0))
-    if max_sms is None:
-        B.call("df11_decompress", *args, _stream_handle(stream))
+            _ptr(cs.lut), _ptr(out))
+    if options is not None:
+        B.call("df11_decompress_opts", *args, 0, ctypes.byref(options), st, _stream_handle(stream))
+    elif max_sms is None:
+        B.call("df11_decompress", *args, st, _stream_handle(stream))
     else:
-        B.call("df11_decompress_sms", *args, ctypes.c_uint32(max_sms), _stream_handle(stream))
+        B.call("df11_decompress_sms", *args, st, ctypes.c_uint32(max_sms), _stream_handle(stream))
     return out
 
 
@@ -370,8 +391,8 @@ def compress_u8(tensors, names=None, threads_per_block: int = DEFAULT_THREADS_PE
                 stream=None) -> CompressedStream:
     """Compress one uint8 tensor (e.g. per-tensor quantized weights), or a
     list, coding each byte whole with one shared table; no side array.  T = 64
-    falls back to T = 32 when the code has a 1-bit symbol (the two-window
-    decoder needs codes of 2 bits or more)."""
+    or 128 falls back to T = 32 when the code has a 1-bit symbol (the decoders
+    with two or four windows per lane need codes of 2 bits or more)."""
     segs = _as_segments(tensors, torch.uint8)
     device = segs[0].device
     n = sum(t.numel() for t in segs)
@@ -383,7 +404,7 @@ def compress_u8(tensors, names=None, threads_per_block: int = DEFAULT_THREADS_PE
     B.call("df11_compress_plan_u8", ptrs, counts, len(segs), threads_per_block, max_code_len, _ptr(ws),
            ws.numel(), ctypes.byref(hdr), sh)
     ln = np.frombuffer(bytes(hdr.code_len), dtype=np.uint8)
-    if threads_per_block == 64 and n and ln[ln > 0].min() == 1:
+    if threads_per_block in (64, 128) and n and ln[ln > 0].min() == 1:
         hdr = make_header(ln, int(hdr.n_elems), int(hdr.total_bits), 32, max_code_len,
                           [t.numel() for t in segs])
     exp = torch.empty(int(hdr.bytes_exp), dtype=torch.uint8, device=device)
@@ -399,10 +420,10 @@ def compress_u8(tensors, names=None, threads_per_block: int = DEFAULT_THREADS_PE
 
 
 def decompress_u8(cs: CompressedStream, out: torch.Tensor | None = None, status: torch.Tensor | None = None,
-                  stream=None) -> torch.Tensor:
+                  stream=None, options=None) -> torch.Tensor:
     """One kernel launch rebuilding all n_elems bytes of a stream of 8-bit
     symbols.  Asynchronous; `out` (uint8, n_elems, contiguous, 16-byte
-    aligned) may be reused."""
+    aligned) may be reused; `options` as for decompress."""
     if cs.symbols != "u8":
         raise ValueError("decompress_u8 takes streams of 8-bit symbols (compress_u8)")
     n = cs.n_elems
@@ -410,9 +431,13 @@ def decompress_u8(cs: CompressedStream, out: torch.Tensor | None = None, status:
         out = torch.empty(max(n, 16), dtype=torch.uint8, device=cs.exp.device)[:n]
     if out.dtype != torch.uint8 or not out.is_contiguous() or out.numel() < n:
         raise ValueError("out must be a contiguous uint8 tensor with n_elems elements")
-    B.call("df11_decompress_u8", ctypes.byref(cs.header), _ptr(cs.exp), _ptr(cs.gaps), _ptr(cs.block_off),
-           _ptr(cs.lut), _ptr(out), _ptr(status) if status is not None else ctypes.c_void_p(0),
-           _stream_handle(stream))
+    st = _ptr(status) if status is not None else ctypes.c_void_p(0)
+    if options is not None:
+        B.call("df11_decompress_opts", ctypes.byref(cs.header), _ptr(cs.exp), ctypes.c_void_p(0), _ptr(cs.gaps),
+               _ptr(cs.block_off), _ptr(cs.lut), _ptr(out), 1, ctypes.byref(options), st, _stream_handle(stream))
+    else:
+        B.call("df11_decompress_u8", ctypes.byref(cs.header), _ptr(cs.exp), _ptr(cs.gaps), _ptr(cs.block_off),
+               _ptr(cs.lut), _ptr(out), st, _stream_handle(stream))
     return out
 
 

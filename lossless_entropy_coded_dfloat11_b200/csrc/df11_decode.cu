@@ -44,6 +44,7 @@
 
 #include <atomic>
 #include <cstdio>
+#include <cstring>
 
 #include "df11_internal.h"
 
@@ -340,13 +341,73 @@ __device__ __forceinline__ uint4 unrotate16(const uint4 r) {
     return make_uint4(rol1(r.x), rol1(r.y), rol1(r.z), rol1(r.w));
 }
 
-__device__ __forceinline__ void copy_tables(uint8_t* s_lut, const uint4* g_lut, int nthreads) {
-    for (int i = threadIdx.x; i < int(kLutBytes / 16); i += nthreads)
-        reinterpret_cast<uint4*>(s_lut)[i] = __ldg(g_lut + i);
-}
+// the K = 12 tables: everything before the narrow sections
+constexpr uint64_t kLutWideBytes = kLutOffNarrow;
+
 
 __device__ __forceinline__ bool block_consistent(uint32_t off0, uint32_t off1, uint32_t total, uint32_t n) {
     return off0 <= off1 && off1 <= n && total == off1 - off0;
+}
+
+// ---------------------------------------------------------------------------
+// Table staging through the bulk-copy engine: one thread initialises an
+// mbarrier, announces the bytes and issues one cp.async.bulk per piece; the
+// copies then run without any thread's registers, whatever the CTA size (a
+// CTA of a few warps would otherwise need many dependent load rounds).  The
+// issuing thread waits on the mbarrier -- a bounded wait -- and a CTA barrier
+// passes the tables on.  A wait that runs out (never expected) waits once
+// more for the copies in flight, then the CTA reports the stream corrupt and
+// stops.
+// ---------------------------------------------------------------------------
+constexpr uint32_t kBulkWaitLimit = 1u << 20;
+
+__device__ __forceinline__ void bulk_begin(uint32_t bar, uint32_t tx_bytes) {
+    asm volatile(
+        "mbarrier.init.shared::cta.b64 [%0], 1;\n\t"
+        "fence.mbarrier_init.release.cluster;\n\t"
+        "fence.proxy.async.shared::cta;\n\t"
+        "mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;"
+        ::"r"(bar), "r"(tx_bytes) : "memory");
+}
+
+// bytes: a multiple of 16; both addresses 16-byte aligned
+__device__ __forceinline__ void bulk_copy(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(dst), "l"(src), "r"(bytes), "r"(bar) : "memory");
+}
+
+__device__ __forceinline__ bool bulk_wait(uint32_t bar) {
+    for (uint32_t i = 0; i < kBulkWaitLimit; i++) {
+        uint32_t done;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], 0;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(done) : "r"(bar) : "memory");
+        if (done) return true;
+    }
+    return false;
+}
+
+// Thread 0: wait for the staged tables; false (after a second bounded wait
+// for the copies still in flight) if they never arrived.
+__device__ __forceinline__ bool bulk_end(uint32_t bar) {
+    if (bulk_wait(bar)) return true;
+    bulk_wait(bar);
+    return false;
+}
+
+// Kernels launched with programmatic stream serialisation start while the
+// previous kernel on the stream drains; nothing is read before this.
+__device__ __forceinline__ void wait_for_prior_grids() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// After the table copy and a CTA barrier: false (and the stream reported
+// corrupt) when the staged tables do not carry the library's magic word -- a
+// table buffer never filled, or the tables of a stream whose encode gave up.
+__device__ __forceinline__ bool tables_valid(const uint8_t* s_lut, uint32_t* status) {
+    if (reinterpret_cast<const LutHeader*>(s_lut)->magic == kLutMagic) return true;
+    if (threadIdx.x == 0 && status) atomicOr(status, uint32_t(DF11_ERR_CORRUPT));
+    return false;
 }
 
 // ---------------------------------------------------------------------------
@@ -390,14 +451,68 @@ constexpr uint32_t kCompactSmall = uint32_t(kLutOffCount);
 constexpr uint32_t kCompactMask = kCompactSmall;
 constexpr uint32_t kCompactDecode = kCompactMask + uint32_t(kLutOffDecode - kLutOffMask);
 constexpr uint32_t kCompactLong = kCompactDecode + uint32_t(kLutOffLong - kLutOffDecode);
-constexpr uint32_t kCompactBytes = kCompactDecode + uint32_t(kLutBytes - kLutOffDecode);
+constexpr uint32_t kCompactBytes = kCompactDecode + uint32_t(kLutWideBytes - kLutOffDecode);
 
-__device__ __forceinline__ void copy_compact_tables(uint8_t* s, const uint4* g, int nthreads) {
-    for (int i = threadIdx.x; i < int(kCompactSmall / 16); i += nthreads)
-        reinterpret_cast<uint4*>(s)[i] = __ldg(g + i);
-    const uint4* g2 = g + kLutOffMask / 16;
-    uint4* s2 = reinterpret_cast<uint4*>(s + kCompactMask);
-    for (int i = threadIdx.x; i < int((kLutBytes - kLutOffMask) / 16); i += nthreads) s2[i] = __ldg(g2 + i);
+
+// Shared-memory layout of the tables a warp kernel decodes with.  K = 12: the
+// compact copy above, decode table in one copy (8-byte entries at random
+// 12-bit indices: ~5 wavefronts per warp lookup).  K < 12: a narrow section,
+// its decode table stored once per 8-byte bank pair -- entry i of copy c at
+// 8-byte slot 16 i + c, lane L reading copy L % 16 -- so every lookup takes
+// one wavefront per half-warp.
+template <int K>
+struct TableLayout {
+    static constexpr bool kNarrow = K != kPeekBits;
+    static constexpr uint32_t kRep = kNarrow ? 16u : 1u;  // copies of the decode table
+    static constexpr uint32_t kStride = 8 * kRep;          // bytes between entries
+    static constexpr uint32_t kMask = kNarrow ? kCompactSmall : kCompactMask;
+    static constexpr uint32_t kLong = kNarrow ? kMask + (2u << K) : kCompactLong;
+    static constexpr uint32_t kLongEnd = kNarrow ? kLong + 2 * narrow_long_entries(K) : kCompactBytes;
+    static constexpr uint32_t kDecode = kNarrow ? (kLongEnd + 127) & ~127u : kCompactDecode;
+    static constexpr uint32_t kBytes = kNarrow ? kDecode + (kRep * 8u << K) : kCompactBytes;
+};
+
+
+// Thread 0: the warp kernel's tables by bulk copies (the small part, then
+// the mask and long tables, and for K = 12 the decode table); the narrow
+// decode table's 16 copies are written by every thread (copy_narrow_decode).
+template <int K>
+__device__ __forceinline__ void bulk_warp_tables(uint8_t* s, const uint8_t* g, uint32_t bar) {
+    using TL = TableLayout<K>;
+    const uint32_t s0 = uint32_t(__cvta_generic_to_shared(s));
+    if constexpr (!TL::kNarrow) {
+        constexpr uint32_t rest = uint32_t(kLutWideBytes - kLutOffMask);
+        bulk_begin(bar, kCompactSmall + rest);
+        bulk_copy(s0, g, kCompactSmall, bar);
+        bulk_copy(s0 + kCompactMask, g + kLutOffMask, rest, bar);
+    } else {
+        constexpr uint32_t rest = TL::kLongEnd - TL::kMask;
+        bulk_begin(bar, kCompactSmall + rest);
+        bulk_copy(s0, g, kCompactSmall, bar);
+        bulk_copy(s0 + TL::kMask, g + narrow_off(K), rest, bar);
+    }
+}
+
+template <int K>
+__device__ __forceinline__ void copy_narrow_decode(uint8_t* s, const uint4* g, int nthreads) {
+    if constexpr (TableLayout<K>::kNarrow) {
+        using TL = TableLayout<K>;
+        const uint2* gd = reinterpret_cast<const uint2*>(g) + (narrow_off(K) + narrow_decode_off(K)) / 8;
+        uint2* sd = reinterpret_cast<uint2*>(s + TL::kDecode);
+        for (int j = threadIdx.x; j < int(TL::kRep << K); j += nthreads) sd[j] = __ldg(gd + (j >> 4));
+    }
+}
+
+template <int K>
+__device__ __forceinline__ void long_table_of(const uint8_t* s, uint32_t& base, uint32_t& count) {
+    const LutHeader* h = reinterpret_cast<const LutHeader*>(s);
+    if constexpr (TableLayout<K>::kNarrow) {
+        base = h->narrow_long[narrow_index(K)][0];
+        count = h->narrow_long[narrow_index(K)][1];
+    } else {
+        base = h->long_base;
+        count = h->long_count;
+    }
 }
 
 // One half of the window (bit positions below lim, peeking at hi:lo) through
@@ -411,14 +526,15 @@ __device__ __forceinline__ void copy_compact_tables(uint8_t* s, const uint4* g, 
 // The loop is unrolled twice with acc alternating between two registers.
 // The last entry's index and y word stay behind for the end-of-window
 // correction.
+template <int K, uint32_t STRIDE>
 __device__ __forceinline__ void decode_half(uint32_t& acc, uint32_t& pend, uint32_t& wad, uint32_t& idx,
                                             uint32_t& ylast, uint32_t hi, uint32_t lo, uint32_t lim,
                                             uint32_t dtab_s) {
 #define DF11_STEP(A, B)                                  \
     "shr.u32 sh, " A ", 16;\n\t"                          \
     "shf.l.wrap.b32 pk, %6, %5, sh;\n\t"                  \
-    "shr.u32 %3, pk, 20;\n\t"                             \
-    "mad.lo.u32 ad, %3, 8, %8;\n\t"                       \
+    "shr.u32 %3, pk, %9;\n\t"                             \
+    "mad.lo.u32 ad, %3, %10, %8;\n\t"                     \
     "ld.shared.v2.u32 {x, %4}, [ad];\n\t"                 \
     "shf.l.wrap.b32 t1, zero, x, " A ";\n\t"              \
     "or.b32 %1, %1, t1;\n\t"                              \
@@ -449,7 +565,7 @@ __device__ __forceinline__ void decode_half(uint32_t& acc, uint32_t& pend, uint3
         "DONE:\n\t"
         "}"
         : "+r"(acc), "+r"(pend), "+r"(wad), "+r"(idx), "+r"(ylast)
-        : "r"(hi), "r"(lo), "r"(lim), "r"(dtab_s)
+        : "r"(hi), "r"(lo), "r"(lim), "r"(dtab_s), "n"(32 - K), "n"(STRIDE)
         : "memory");
 #undef DF11_STEP
 }
@@ -479,10 +595,13 @@ __device__ __forceinline__ RawLane<WPL> load_lane(const DecodeArgs& a, uint32_t 
     RawLane<WPL> r;
     if (tg0 < a.n_threads) {
         const uint8_t* base = a.exp + 8 * size_t(tg0);
-        if constexpr (WPL == 2) {
-            const uint4 q = __ldg(reinterpret_cast<const uint4*>(base));
-            r.v[0] = q.x; r.v[1] = q.y; r.v[2] = q.z; r.v[3] = q.w;
-            r.look = lane == 31 ? __ldg(reinterpret_cast<const uint32_t*>(base + 16)) : 0u;
+        if constexpr (WPL >= 2) {
+#pragma unroll
+            for (int h = 0; h < WPL / 2; h++) {
+                const uint4 q = __ldg(reinterpret_cast<const uint4*>(base) + h);
+                r.v[4 * h] = q.x; r.v[4 * h + 1] = q.y; r.v[4 * h + 2] = q.z; r.v[4 * h + 3] = q.w;
+            }
+            r.look = lane == 31 ? __ldg(reinterpret_cast<const uint32_t*>(base + 8 * WPL)) : 0u;
         } else {
             const uint2 q = __ldg(reinterpret_cast<const uint2*>(base));
             r.v[0] = q.x; r.v[1] = q.y;
@@ -505,7 +624,7 @@ __device__ __forceinline__ LaneWindow<WPL> finish_lane(const DecodeArgs& a, cons
     LaneWindow<WPL> w;
 #pragma unroll
     for (int k = 0; k < 2 * WPL; k++) w.w[k] = bswap32(r.v[k]);
-    if constexpr (WPL == 2) {
+    if constexpr (WPL >= 2) {
         const uint32_t next = __shfl_down_sync(0xFFFFFFFFu, r.v[0], 1);  // the next lane's first word
         w.w[2 * WPL] = bswap32(lane == 31 ? r.look : next);
     } else {
@@ -522,7 +641,7 @@ __device__ __forceinline__ LaneWindow<WPL> finish_lane(const DecodeArgs& a, cons
 
 // Decode the lane's run into its (transposed) slot at shared address slot_s;
 // returns the number of codes that start in the run.
-template <int WPL>
+template <int WPL, int K>
 __device__ __forceinline__ uint32_t decode_lane_once(const LaneWindow<WPL>& w, const Tables& t, uint32_t dtab_s,
                                                      uint32_t slot_s, const uint16_t* ltab, uint32_t long_base,
                                                      uint32_t long_count, bool& bad) {
@@ -532,22 +651,22 @@ __device__ __forceinline__ uint32_t decode_lane_once(const LaneWindow<WPL>& w, c
     for (;;) {
 #pragma unroll
         for (int k = 0; k < 2 * WPL; k++)  // one loop per 32 bits, each peeking at one word pair
-            decode_half(acc, pend, wad, idx, ylast, w.w[k], w.w[k + 1], min(w.wend, 32u * (k + 1)) << 16,
-                        dtab_s);
+            decode_half<K, TableLayout<K>::kStride>(acc, pend, wad, idx, ylast, w.w[k], w.w[k + 1],
+                                                    min(w.wend, 32u * (k + 1)) << 16, dtab_s);
         if (acc < (kEscape << 16)) break;
         // a code longer than the table: undo the escape, take it from level 2
         acc -= kEscape << 16;
         const uint32_t pos = acc >> 16;
         // the word pair holding bit pos, by selects (an indexed pick would
         // put the window in local memory)
-        const bool odd = (pos >> 5) & 1u;
-        uint32_t hi = odd ? w.w[1] : w.w[0], lo = odd ? w.w[2] : w.w[1];
-        if constexpr (WPL == 2) {
-            if ((pos >> 5) & 2u) {
-                hi = odd ? w.w[3] : w.w[2];
-                lo = odd ? w.w[4] : w.w[3];
+        const uint32_t kw = pos >> 5;
+        uint32_t hi = w.w[0], lo = w.w[1];
+#pragma unroll
+        for (int k = 1; k < 2 * WPL; k++)
+            if (kw == uint32_t(k)) {
+                hi = w.w[k];
+                lo = w.w[k + 1];
             }
-        }
         const uint32_t pk = __funnelshift_l(lo, hi, pos);
         const uint32_t li = (pk >> (32 - kLongBits)) - long_base;
         const uint32_t le = li < long_count ? uint32_t(ltab[li]) : 0u;
@@ -557,7 +676,7 @@ __device__ __forceinline__ uint32_t decode_lane_once(const LaneWindow<WPL>& w, c
             l = int(le >> 8);
             sym = le & 0xFFu;
         } else {
-            l = code_length(t.lj_end, pk, kPeekBits + 1);
+            l = code_length(t.lj_end, pk, K + 1);
             if (!l) {
                 bad = true;
                 return 0;
@@ -578,7 +697,7 @@ __device__ __forceinline__ uint32_t decode_lane_once(const LaneWindow<WPL>& w, c
     uint32_t cnt = (acc & 0xFFFFu) >> 3;
     if (ylast) {  // codes of the last table step that start at or past wend
         const uint32_t s = w.wend - ((acc >> 16) - (ylast >> 16));
-        if (s < uint32_t(kPeekBits)) {
+        if (s < uint32_t(K)) {
             const uint32_t n = (ylast & 0xFFu) >> 3;
             const uint32_t before = __popc(uint32_t(t.mtab[idx]) & ((1u << s) - 1u));
             cnt -= n - min(n, before);
@@ -611,9 +730,22 @@ __device__ __forceinline__ uint32_t copy_slot(const uint32_t* slot, uint32_t* st
     return first;
 }
 
-template <int WARPS, int MIN_LEN, int WPL, bool U8>
+// Rounds R .. N-1 of a block's whole-unit merge: round r merges unit
+// lane + 32 r from staging bytes 256 r on and stores to dst + 32 r, with the
+// offsets as immediates.
+template <int R, int N>
+__device__ __forceinline__ void merge_rounds(uint32_t ev_s, const uint2 (&sv)[N], uint4* dst, uint32_t m,
+                                             uint32_t lane, uint32_t qe) {
+    if constexpr (R < N) {
+        if (lane + 32 * R < qe) merge_store8<256 * R, 512 * R>(ev_s, sv[R], dst, m);
+        merge_rounds<R + 1, N>(ev_s, sv, dst, m, lane, qe);
+    }
+}
+
+template <int WARPS, int MIN_LEN, int WPL, bool U8, int K>
 __global__ void __launch_bounds__(WARPS * 32, 1) decode_warp_kernel(const DecodeArgs a) {
     using L = WarpLayout<MIN_LEN, WPL>;
+    using TL = TableLayout<K>;
     // elements per merge unit, 16 output bytes either way
     constexpr uint32_t kUnit = U8 ? 16u : 8u;
     extern __shared__ __align__(16) uint8_t smem[];
@@ -627,14 +759,21 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_warp_kernel(const Decode
     // this warp's run of thread blocks [b, b_end); warps are numbered across
     // the CTAs first, so the runs one block longer than the rest (the first
     // n_blocks mod nw) fall at most one per SM instead of filling a few SMs
-    const uint32_t nw = gridDim.x * WARPS;
+    // (a stream of few thread blocks runs with fewer warps per CTA, so that
+    // its warps spread over all SMs)
+    const uint32_t nw = gridDim.x * (blockDim.x >> 5);
     const uint32_t g = warp * gridDim.x + blockIdx.x;
     const uint32_t per = a.n_blocks / nw, extra = a.n_blocks % nw;
     uint32_t b = a.block0 + g * per + (g < extra ? g : extra);
     const uint32_t b_end = b + per + (g < extra ? 1u : 0u);
 
-    copy_compact_tables(smem, a.lut, WARPS * 32);
-    __syncthreads();
+    __shared__ __align__(8) unsigned long long s_bar;
+    __shared__ uint32_t s_abort;
+    const uint32_t bar = uint32_t(__cvta_generic_to_shared(&s_bar));
+    wait_for_prior_grids();
+    if (threadIdx.x == 0) bulk_warp_tables<K>(smem, reinterpret_cast<const uint8_t*>(a.lut), bar);
+    copy_narrow_decode<K>(smem, a.lut, int(blockDim.x));
+    // the first block's loads overlap the table copy
     RawLane<WPL> nraw{};
     uint32_t noff0 = 0, noff1 = 0;
     if (b < b_end) {
@@ -642,18 +781,26 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_warp_kernel(const Decode
         noff0 = __ldg(a.off + b);
         noff1 = __ldg(a.off + b + 1);
     }
+    if (threadIdx.x == 0) s_abort = bulk_end(bar) ? 0u : 1u;
+    __syncthreads();
+    if (s_abort) {
+        if (threadIdx.x == 0 && a.status) atomicOr(a.status, uint32_t(DF11_ERR_CORRUPT));
+        return;
+    }
+    if (!tables_valid(smem, a.status)) return;
     Tables t;
     t.ctab = nullptr;
-    t.mtab = reinterpret_cast<const uint16_t*>(smem + kCompactMask);
-    t.dtab = reinterpret_cast<const uint2*>(smem + kCompactDecode);
+    t.mtab = reinterpret_cast<const uint16_t*>(smem + TL::kMask);
+    t.dtab = reinterpret_cast<const uint2*>(smem + TL::kDecode);
     t.lj_end = reinterpret_cast<const unsigned long long*>(smem + kLutOffLjEnd);
     t.delta = reinterpret_cast<const uint32_t*>(smem + kLutOffDelta);
     t.syms = smem + kLutOffSyms;
-    const uint32_t dtab_s = uint32_t(__cvta_generic_to_shared(t.dtab));
-    const uint16_t* ltab = reinterpret_cast<const uint16_t*>(smem + kCompactLong);
-    const uint32_t long_base = reinterpret_cast<const LutHeader*>(smem)->long_base;
-    const uint32_t long_count = reinterpret_cast<const LutHeader*>(smem)->long_count;
-    uint8_t* wbase = smem + kCompactBytes + warp * L::kBytes;
+    // a replicated table is read through the lane's own copy
+    const uint32_t dtab_s = uint32_t(__cvta_generic_to_shared(t.dtab)) + (TL::kNarrow ? 8 * (lane & 15) : 0);
+    const uint16_t* ltab = reinterpret_cast<const uint16_t*>(smem + TL::kLong);
+    uint32_t long_base, long_count;
+    long_table_of<K>(smem, long_base, long_count);
+    uint8_t* wbase = smem + TL::kBytes + warp * L::kBytes;
     uint32_t* slot = reinterpret_cast<uint32_t*>(wbase) + lane;
     const uint32_t slot_s = uint32_t(__cvta_generic_to_shared(slot));
     uint8_t* stage = wbase + L::kSlots;
@@ -687,8 +834,9 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_warp_kernel(const Decode
         const uint32_t a_sh = u0 & (U8 ? 7u : 15u);
         const uint32_t ub = u0 - a_sh;
         // sign+mantissa units requested before the decode: 4 rounds of 32
-        // (a 32-window block has ~100 units), 7 for two windows per lane
-        constexpr int kPre = WPL == 1 ? 4 : 7;
+        // (a 32-window block of LLM weights has ~100 units), 7 for two
+        // windows per lane, 13 for four
+        constexpr int kPre = WPL == 1 ? 4 : WPL == 2 ? 7 : 13;
         uint2 sv[kPre];
         if constexpr (!U8) {
 #pragma unroll
@@ -698,7 +846,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_warp_kernel(const Decode
 
         const LaneWindow<WPL> w = finish_lane<WPL>(a, raw, WPL * (32 * b + lane), lane_gshift, lane);
         bool bad = false;
-        const uint32_t cnt = decode_lane_once<WPL>(w, t, dtab_s, slot_s, ltab, long_base, long_count, bad);
+        const uint32_t cnt = decode_lane_once<WPL, K>(w, t, dtab_s, slot_s, ltab, long_base, long_count, bad);
         uint32_t incl = cnt;
 #pragma unroll
         for (int d = 1; d < 32; d <<= 1) {
@@ -739,14 +887,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_warp_kernel(const Decode
                     const uint32_t ev_s = stage_s + 8 * lane - 8 * a_sh;
                     uint4* dst = reinterpret_cast<uint4*>(a.out) + ub + lane;
                     if (lane >= a_sh && lane < qe) merge_store8<0, 0>(ev_s, sv[0], dst, m);
-                    if (lane + 32 < qe) merge_store8<256, 512>(ev_s, sv[1], dst, m);
-                    if (lane + 64 < qe) merge_store8<512, 1024>(ev_s, sv[2], dst, m);
-                    if (lane + 96 < qe) merge_store8<768, 1536>(ev_s, sv[3], dst, m);
-                    if constexpr (kPre == 7) {
-                        if (lane + 128 < qe) merge_store8<1024, 2048>(ev_s, sv[4], dst, m);
-                        if (lane + 160 < qe) merge_store8<1280, 2560>(ev_s, sv[5], dst, m);
-                        if (lane + 192 < qe) merge_store8<1536, 3072>(ev_s, sv[6], dst, m);
-                    }
+                    merge_rounds<1, kPre>(ev_s, sv, dst, m, lane, qe);
                     for (uint32_t k = 32 * kPre; lane + k < qe; k += 32)
                         merge_store8(ev_s + 8 * k, __ldcs(sm8 + ub + lane + k), dst + k, m);
                 } else {
@@ -833,8 +974,20 @@ static_assert(kChunkWarpBytes % 16 == 0 && kChunkSlot % 8 == 0, "aligned per-war
 
 __global__ void __launch_bounds__(kChunkWarps * 32, 1) decode_chunk_kernel(const ChunkArgs a) {
     extern __shared__ __align__(16) uint8_t smem[];
-    copy_compact_tables(smem, a.lut, kChunkWarps * 32);
+    __shared__ __align__(8) unsigned long long s_bar;
+    __shared__ uint32_t s_abort;
+    const uint32_t bar = uint32_t(__cvta_generic_to_shared(&s_bar));
+    wait_for_prior_grids();
+    if (threadIdx.x == 0) {
+        bulk_warp_tables<kPeekBits>(smem, reinterpret_cast<const uint8_t*>(a.lut), bar);
+        s_abort = bulk_end(bar) ? 0u : 1u;
+    }
     __syncthreads();
+    if (s_abort) {
+        if (threadIdx.x == 0 && a.status) atomicOr(a.status, uint32_t(DF11_ERR_CORRUPT));
+        return;
+    }
+    if (!tables_valid(smem, a.status)) return;
     Tables t;
     t.ctab = nullptr;
     t.mtab = reinterpret_cast<const uint16_t*>(smem + kCompactMask);
@@ -1015,10 +1168,23 @@ constexpr size_t block_stage_bytes() {
 template <int T>
 __global__ void __launch_bounds__(T) decode_block_kernel(const DecodeArgs a) {
     extern __shared__ __align__(16) uint8_t smem[];
-    copy_tables(smem, a.lut, T);
-    uint8_t* stage = smem + kLutBytes;
+    __shared__ __align__(8) unsigned long long s_bar;
+    __shared__ uint32_t s_abort;
+    const uint32_t bar = uint32_t(__cvta_generic_to_shared(&s_bar));
+    wait_for_prior_grids();
+    if (threadIdx.x == 0) {
+        bulk_begin(bar, uint32_t(kLutWideBytes));
+        bulk_copy(uint32_t(__cvta_generic_to_shared(smem)), a.lut, uint32_t(kLutWideBytes), bar);
+        s_abort = bulk_end(bar) ? 0u : 1u;
+    }
+    uint8_t* stage = smem + kLutWideBytes;
     uint32_t* s_warp = reinterpret_cast<uint32_t*>(stage + block_stage_bytes<T>());
     __syncthreads();
+    if (s_abort) {
+        if (threadIdx.x == 0 && a.status) atomicOr(a.status, uint32_t(DF11_ERR_CORRUPT));
+        return;
+    }
+    if (!tables_valid(smem, a.status)) return;
     const Tables t = tables_at(smem);
     const uint32_t lane = threadIdx.x & 31u;
     const uint32_t warp = threadIdx.x >> 5;
@@ -1092,7 +1258,7 @@ struct LaunchInfo {
     int sms = 0;
 };
 constexpr int kMaxDev = 64;
-LaunchInfo g_info[kMaxDev][16];  // [device][variant]: BF16 0..7, 8-bit symbols 8..15
+LaunchInfo g_info[kMaxDev][32];  // [device][variant]: BF16 0..15, 8-bit symbols 16..31
 
 // One CTA per SM: all warps share one copy of the tables.  With one window
 // per lane, 32 warps at 64 registers measured faster than two CTAs of 20
@@ -1102,19 +1268,77 @@ constexpr int kWarpsShort = 32;  // every code has 2 bits or more
 // two windows per lane: 28 warps leave 72 registers per thread (the merge's
 // seven prefetched rounds fit) and measured faster than 24, 26, 30 or 32
 constexpr int kWarpsTwoWindows = 28;
+// four windows per lane with 2-bit codes: 8,384 bytes of slots and staging
+// per warp, so 20 warps fit beside the tables
+constexpr int kWarpsFourWindows = 20;
 
-template <typename Kernel>
-df11_status launch_persistent(Kernel kernel, int slot, int threads, size_t smem, uint64_t work_units,
-                              uint32_t max_sms, const DecodeArgs& a, cudaStream_t stream) {
+// How one stream is decoded: which kernel, its CTA shape and its shared
+// memory.  Warp kernels take up to `warps` warps per CTA, one CTA per SM; a
+// stream with fewer thread blocks than warps x SMs gets ceil(blocks / SMs)
+// warps per CTA so that it still spreads over every SM.  Block kernels take T
+// threads per CTA.
+struct Plan {
+    const void* kernel;
+    int slot;            // LaunchInfo slot
+    uint32_t warps;      // warp kernels: warps per CTA at most; 0 for block kernels
+    uint32_t threads;    // block kernels: T
+    size_t smem_fixed;   // tables (+ block kernels' staging)
+    size_t smem_per_warp;
+    uint32_t peek_bits, copies;
+    char name[64];
+};
+
+template <int WARPS, int MIN_LEN, int WPL, bool U8, int K = kPeekBits>
+Plan warp_plan(int slot) {
+    using TL = TableLayout<K>;
+    static_assert(TL::kBytes + size_t(WARPS) * WarpLayout<MIN_LEN, WPL>::kBytes <= 227 * 1024,
+                  "shared memory per CTA");
+    Plan p{};
+    p.kernel = reinterpret_cast<const void*>(&decode_warp_kernel<WARPS, MIN_LEN, WPL, U8, K>);
+    p.slot = slot + (U8 ? 16 : 0);
+    p.warps = WARPS;
+    p.smem_fixed = TL::kBytes;
+    p.smem_per_warp = WarpLayout<MIN_LEN, WPL>::kBytes;
+    p.peek_bits = K;
+    p.copies = TL::kRep;
+    std::snprintf(p.name, sizeof(p.name), "decode_warp_kernel<%d,%d,%d,%d,%d>", WARPS, MIN_LEN, WPL, int(U8), K);
+    return p;
+}
+
+template <int T>
+Plan block_plan(int slot) {
+    Plan p{};
+    p.kernel = reinterpret_cast<const void*>(&decode_block_kernel<T>);
+    p.slot = slot;
+    p.threads = T;
+    p.smem_fixed = kLutWideBytes + block_stage_bytes<T>() + 4 * (T / 32);
+    p.peek_bits = kPeekBits;
+    p.copies = 1;
+    std::snprintf(p.name, sizeof(p.name), "decode_block_kernel<%d>", T);
+    return p;
+}
+
+struct Shape {
+    unsigned grid, block;
+    size_t smem;
+};
+
+// Grid and CTA shape of a plan for n_blocks thread blocks on at most max_sms
+// SMs of the current device (first use per device and kernel: sets the
+// kernel's shared-memory limit and queries its occupancy).
+df11_status shape_of(const Plan& p, uint64_t n_blocks, const df11_decode_options& o, Shape* out) {
+    const uint32_t max_sms = o.max_sms ? o.max_sms : UINT32_MAX;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev)
         return fail(DF11_ERR_CUDA, "cudaGetDevice failed");
-    LaunchInfo& li = g_info[dev][slot];
+    const size_t smem_max = p.smem_fixed + (p.warps ? p.warps * p.smem_per_warp : 0);
+    const int threads_max = p.warps ? int(32 * p.warps) : int(p.threads);
+    LaunchInfo& li = g_info[dev][p.slot];
     if (!li.ready.load(std::memory_order_acquire)) {
-        cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+        cudaError_t e = cudaFuncSetAttribute(p.kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem_max));
         if (e != cudaSuccess) return fail(DF11_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
         int per_sm = 0, sms = 0;
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, smem);
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, p.kernel, threads_max, smem_max);
         if (e != cudaSuccess) return fail(DF11_ERR_CUDA, "occupancy query: %s", cudaGetErrorString(e));
         e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
         if (e != cudaSuccess) return fail(DF11_ERR_CUDA, "SM count: %s", cudaGetErrorString(e));
@@ -1123,34 +1347,50 @@ df11_status launch_persistent(Kernel kernel, int slot, int threads, size_t smem,
         li.ready.store(1, std::memory_order_release);
     }
     const uint64_t sms = max_sms < uint32_t(li.sms) ? max_sms : uint32_t(li.sms);
-    const uint64_t want = uint64_t(li.per_sm) * sms;
-    const unsigned grid = unsigned(work_units < want ? work_units : want);
-    kernel<<<grid, threads, smem, stream>>>(a);
-    const cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return fail(DF11_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
+    if (!p.warps) {
+        const uint64_t want = o.ctas ? uint64_t(o.ctas) : uint64_t(li.per_sm) * sms;
+        *out = Shape{unsigned(n_blocks < want ? n_blocks : want), p.threads, p.smem_fixed};
+        return DF11_OK;
+    }
+    // The slowest warp decodes ceil(n_blocks / all warps) thread blocks; the
+    // fewest warps per CTA that keep that count let each of them run faster
+    // (a stream of 38 K blocks: 26 warps per SM doing 10 blocks each instead
+    // of 28 doing 9 or 10).  Few blocks: fewer warps per CTA, every SM.
+    const uint64_t cap = o.max_warps_per_cta && o.max_warps_per_cta < p.warps ? o.max_warps_per_cta : p.warps;
+    uint64_t warps = cap;
+    const uint64_t per = (n_blocks + warps * sms - 1) / (warps * sms);
+    if (per > 0) warps = ((n_blocks + per - 1) / per + sms - 1) / sms;
+    if (warps > cap) warps = cap;
+    if (warps < 1) warps = 1;
+    const uint64_t ctas = (n_blocks + warps - 1) / warps;
+    const uint64_t want = o.ctas ? uint64_t(o.ctas) : uint64_t(li.per_sm) * sms;
+    *out = Shape{unsigned(ctas < want ? ctas : want), unsigned(32 * warps), p.smem_fixed + warps * p.smem_per_warp};
     return DF11_OK;
 }
 
-template <int T>
-df11_status launch_block(const DecodeArgs& a, cudaStream_t s, int slot, uint32_t max_sms) {
-    const size_t smem = kLutBytes + block_stage_bytes<T>() + 4 * (T / 32);
-    return launch_persistent(decode_block_kernel<T>, slot, T, smem, a.n_blocks, max_sms, a, s);
-}
-
-template <int WARPS, int MIN_LEN, int WPL, bool U8>
-df11_status launch_warp_variant(const DecodeArgs& a, cudaStream_t s, int slot, uint32_t max_sms) {
-    constexpr size_t smem = kCompactBytes + size_t(WARPS) * WarpLayout<MIN_LEN, WPL>::kBytes;
-    static_assert(smem <= 227 * 1024, "shared memory per CTA");
-    const uint64_t ctas = (uint64_t(a.n_blocks) + WARPS - 1) / WARPS;
-    return launch_persistent(decode_warp_kernel<WARPS, MIN_LEN, WPL, U8>, slot + (U8 ? 8 : 0), WARPS * 32, smem,
-                             ctas, max_sms, a, s);
-}
-
-// T = 32: one window per lane (T = 64 streams: two, see decompress_on).
-template <bool U8>
-df11_status launch_warp(const DecodeArgs& a, cudaStream_t s, uint32_t min_len, uint32_t max_sms) {
-    if (min_len >= 2) return launch_warp_variant<kWarpsShort, 2, 1, U8>(a, s, 6, max_sms);
-    return launch_warp_variant<kWarpsLong, 1, 1, U8>(a, s, 0, max_sms);
+df11_status launch_plan(const Plan& p, const DecodeArgs& a, const df11_decode_options& o, cudaStream_t stream) {
+    Shape sh;
+    df11_status st = shape_of(p, a.n_blocks, o, &sh);
+    if (st != DF11_OK) return st;
+    DecodeArgs args = a;
+    void* params[] = {&args};
+    // programmatic stream serialisation: the CTAs may be placed while the
+    // previous kernel on the stream drains; each waits for it (and its
+    // memory) before reading anything
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(sh.grid);
+    cfg.blockDim = dim3(sh.block);
+    cfg.dynamicSmemBytes = sh.smem;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelExC(&cfg, p.kernel, params);
+    if (e == cudaSuccess) e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(DF11_ERR_CUDA, "decode launch (%s): %s", p.name, cudaGetErrorString(e));
+    return DF11_OK;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -1184,12 +1424,72 @@ using namespace df11;
 namespace df11 {
 namespace {
 
+// The decode kernel for a stream.  T = 64 (the library default) and codes of
+// at least 2 bits: the warp kernel with two windows per lane.  T = 32: one
+// window per lane.  T = 64 with a 1-bit code (a lane could then hold 128
+// codes, too many for its slot) and T >= 128: the block kernel, whose two
+// decode passes need no slot.
+df11_status plan_for(const char* fn, const df11_header* hdr, bool u8, uint32_t peek_bits, Plan* out) {
+    if (peek_bits != 0 && peek_bits != uint32_t(kPeekBits) &&
+        (u8 || hdr->threads_per_block != 64 || peek_bits < 8 || peek_bits > 10))
+        return fail(DF11_ERR_INVALID, "%s: peek_bits %u (8, 9 or 10 only for BF16 streams with T = 64)", fn,
+                    peek_bits);
+    uint32_t min_len = 32;
+    for (int v = 0; v < 256; v++)
+        if (hdr->code_len[v] && hdr->code_len[v] < min_len) min_len = hdr->code_len[v];
+    const uint32_t T = hdr->threads_per_block;
+    if (u8) {  // the warp kernel only
+        if (T == 32) {
+            *out = min_len >= 2 ? warp_plan<kWarpsShort, 2, 1, true>(6) : warp_plan<kWarpsLong, 1, 1, true>(0);
+            return DF11_OK;
+        }
+        if (T == 64 && min_len >= 2) {
+            *out = warp_plan<kWarpsTwoWindows, 2, 2, true>(7);
+            return DF11_OK;
+        }
+        if (T == 128 && min_len >= 2) {  // four windows per lane
+            *out = min_len >= 4 ? warp_plan<kWarpsTwoWindows, 4, 4, true>(14)
+                                : warp_plan<kWarpsFourWindows, 2, 4, true>(15);
+            return DF11_OK;
+        }
+        return fail(DF11_ERR_INVALID,
+                    "%s: streams of 8-bit symbols decode with T = 32, or T = 64 or 128 when no code is 1 bit long",
+                    fn);
+    }
+    switch (T) {
+        case 32:
+            *out = min_len >= 2 ? warp_plan<kWarpsShort, 2, 1, false>(6) : warp_plan<kWarpsLong, 1, 1, false>(0);
+            return DF11_OK;
+        case 64:
+            if (min_len >= 2) {
+                // the narrow first-level tables, 16 copies each (an ablation:
+                // slower on LLM weights, see df11_decode_options)
+                if (peek_bits == 10) *out = warp_plan<20, 2, 2, false, 10>(10);
+                else if (peek_bits == 9) *out = warp_plan<kWarpsTwoWindows, 2, 2, false, 9>(11);
+                else if (peek_bits == 8) *out = warp_plan<kWarpsTwoWindows, 2, 2, false, 8>(12);
+                else *out = warp_plan<kWarpsTwoWindows, 2, 2, false>(7);
+                return DF11_OK;
+            }
+            if (peek_bits && peek_bits != uint32_t(kPeekBits))
+                return fail(DF11_ERR_INVALID, "%s: narrow tables need codes of 2 bits or more", fn);
+            *out = block_plan<64>(1);
+            return DF11_OK;
+        case 128:  // four windows per lane when every code has 2 bits or more
+            *out = min_len >= 2 ? warp_plan<kWarpsFourWindows, 2, 4, false>(14) : block_plan<128>(2);
+            return DF11_OK;
+        case 256: *out = block_plan<256>(3); return DF11_OK;
+        case 512: *out = block_plan<512>(4); return DF11_OK;
+        case 1024: *out = block_plan<1024>(5); return DF11_OK;
+        default: return fail(DF11_ERR_INVALID, "threads_per_block %u", T);
+    }
+}
+
 // BF16 streams (u8 = false): d_sm read, d_out holds n_elems uint16; streams
 // of 8-bit symbols (u8 = true): no d_sm, d_out holds n_elems bytes.
 df11_status decompress_on(const char* fn, bool u8, const df11_header* hdr, const uint8_t* d_exp,
                           const uint8_t* d_sm, const uint8_t* d_gaps, const uint32_t* d_block_off,
-                          const void* d_lut, void* d_out, uint32_t* d_status, uint32_t max_sms, void* stream,
-                          uint64_t block_begin = 0, uint64_t block_end = UINT64_MAX) {
+                          const void* d_lut, void* d_out, uint32_t* d_status, const df11_decode_options& opt,
+                          void* stream, uint64_t block_begin = 0, uint64_t block_end = UINT64_MAX) {
     df11_status st = check_header(hdr);
     if (st != DF11_OK) return st;
     if (block_end == UINT64_MAX) block_end = hdr->n_blocks;
@@ -1217,29 +1517,13 @@ df11_status decompress_on(const char* fn, bool u8, const df11_header* hdr, const
     a.block0 = uint32_t(block_begin);
     a.n_blocks = uint32_t(block_end - block_begin);
     a.last_wend = uint32_t(hdr->total_bits - 64 * (hdr->n_threads - 1));
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    uint32_t min_len = 32;
-    for (int v = 0; v < 256; v++)
-        if (hdr->code_len[v] && hdr->code_len[v] < min_len) min_len = hdr->code_len[v];
-    if (u8) {  // the warp kernel only
-        if (hdr->threads_per_block == 32) return launch_warp<true>(a, s, min_len, max_sms);
-        if (hdr->threads_per_block == 64 && min_len >= 2)
-            return launch_warp_variant<kWarpsTwoWindows, 2, 2, true>(a, s, 7, max_sms);
-        return fail(DF11_ERR_INVALID,
-                    "%s: streams of 8-bit symbols decode with T = 32, or T = 64 when no code is 1 bit long", fn);
-    }
-    switch (hdr->threads_per_block) {
-        case 32: return launch_warp<false>(a, s, min_len, max_sms);
-        case 64:  // two windows per lane when every code has 2 bits or more (the slots then fit)
-            if (min_len >= 2) return launch_warp_variant<kWarpsTwoWindows, 2, 2, false>(a, s, 7, max_sms);
-            return launch_block<64>(a, s, 1, max_sms);
-        case 128: return launch_block<128>(a, s, 2, max_sms);
-        case 256: return launch_block<256>(a, s, 3, max_sms);
-        case 512: return launch_block<512>(a, s, 4, max_sms);
-        case 1024: return launch_block<1024>(a, s, 5, max_sms);
-        default: return fail(DF11_ERR_INVALID, "threads_per_block %u", hdr->threads_per_block);
-    }
+    Plan p;
+    st = plan_for(fn, hdr, u8, opt.peek_bits, &p);
+    if (st != DF11_OK) return st;
+    return launch_plan(p, a, opt, reinterpret_cast<cudaStream_t>(stream));
 }
+
+constexpr df11_decode_options kDefaultOptions{0, 0, 0, 0, 0, 0};
 
 }  // namespace
 }  // namespace df11
@@ -1249,7 +1533,7 @@ extern "C" df11_status df11_decompress(const df11_header* hdr, const uint8_t* d_
                                        const void* d_lut, uint16_t* d_out, uint32_t* d_status,
                                        void* stream) {
     return decompress_on("df11_decompress", false, hdr, d_exp, d_sm, d_gaps, d_block_off, d_lut, d_out, d_status,
-                         UINT32_MAX, stream);
+                         kDefaultOptions, stream);
 }
 
 extern "C" df11_status df11_decompress_sms(const df11_header* hdr, const uint8_t* d_exp, const uint8_t* d_sm,
@@ -1257,15 +1541,28 @@ extern "C" df11_status df11_decompress_sms(const df11_header* hdr, const uint8_t
                                            const void* d_lut, uint16_t* d_out, uint32_t* d_status,
                                            uint32_t max_sms, void* stream) {
     if (max_sms == 0) return fail(DF11_ERR_INVALID, "df11_decompress_sms: max_sms must be at least 1");
+    df11_decode_options o = kDefaultOptions;
+    o.max_sms = max_sms;
     return decompress_on("df11_decompress_sms", false, hdr, d_exp, d_sm, d_gaps, d_block_off, d_lut, d_out,
-                         d_status, max_sms, stream);
+                         d_status, o, stream);
+}
+
+extern "C" df11_status df11_decompress_opts(const df11_header* hdr, const uint8_t* d_exp, const uint8_t* d_sm,
+                                            const uint8_t* d_gaps, const uint32_t* d_block_off,
+                                            const void* d_lut, void* d_out, uint32_t symbols_u8,
+                                            const df11_decode_options* opt, uint32_t* d_status, void* stream) {
+    if (!opt) return fail(DF11_ERR_INVALID, "df11_decompress_opts: null options");
+    for (uint32_t r : opt->reserved)
+        if (r) return fail(DF11_ERR_INVALID, "df11_decompress_opts: reserved fields must be zero");
+    return decompress_on("df11_decompress_opts", symbols_u8 != 0, hdr, d_exp, d_sm, d_gaps, d_block_off, d_lut,
+                         d_out, d_status, *opt, stream);
 }
 
 extern "C" df11_status df11_decompress_u8(const df11_header* hdr, const uint8_t* d_exp, const uint8_t* d_gaps,
                                           const uint32_t* d_block_off, const void* d_lut, uint8_t* d_out,
                                           uint32_t* d_status, void* stream) {
     return decompress_on("df11_decompress_u8", true, hdr, d_exp, nullptr, d_gaps, d_block_off, d_lut, d_out,
-                         d_status, UINT32_MAX, stream);
+                         d_status, kDefaultOptions, stream);
 }
 
 extern "C" df11_status df11_decompress_blocks(const df11_header* hdr, const uint8_t* d_exp, const uint8_t* d_sm,
@@ -1273,7 +1570,7 @@ extern "C" df11_status df11_decompress_blocks(const df11_header* hdr, const uint
                                               const void* d_lut, uint16_t* d_out, uint64_t block_begin,
                                               uint64_t block_end, uint32_t* d_status, void* stream) {
     return decompress_on("df11_decompress_blocks", false, hdr, d_exp, d_sm, d_gaps, d_block_off, d_lut, d_out,
-                         d_status, UINT32_MAX, stream, block_begin, block_end);
+                         d_status, kDefaultOptions, stream, block_begin, block_end);
 }
 
 extern "C" df11_status df11_decompress_u8_blocks(const df11_header* hdr, const uint8_t* d_exp, const uint8_t* d_gaps,
@@ -1281,7 +1578,7 @@ extern "C" df11_status df11_decompress_u8_blocks(const df11_header* hdr, const u
                                                  uint64_t block_begin, uint64_t block_end, uint32_t* d_status,
                                                  void* stream) {
     return decompress_on("df11_decompress_u8_blocks", true, hdr, d_exp, nullptr, d_gaps, d_block_off, d_lut,
-                         d_out, d_status, UINT32_MAX, stream, block_begin, block_end);
+                         d_out, d_status, kDefaultOptions, stream, block_begin, block_end);
 }
 
 extern "C" df11_status df11_decompress_chunked(const df11_header* hdr, const uint8_t* d_exp, const uint8_t* d_sm,
@@ -1328,5 +1625,27 @@ extern "C" df11_status df11_decompress_chunked(const df11_header* hdr, const uin
     decode_chunk_kernel<<<grid, kChunkWarps * 32, smem, reinterpret_cast<cudaStream_t>(stream)>>>(a);
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return fail(DF11_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
+    return DF11_OK;
+}
+
+extern "C" df11_status df11_decode_kernel_info(const df11_header* hdr, uint32_t symbols_u8,
+                                               const df11_decode_options* opt, df11_kernel_info* info) {
+    if (!info) return fail(DF11_ERR_INVALID, "df11_decode_kernel_info: null info");
+    df11_status st = check_header(hdr);
+    if (st != DF11_OK) return st;
+    Plan p;
+    st = plan_for("df11_decode_kernel_info", hdr, symbols_u8 != 0, opt ? opt->peek_bits : 0, &p);
+    if (st != DF11_OK) return st;
+    Shape sh;
+    st = shape_of(p, hdr->n_blocks, opt ? *opt : kDefaultOptions, &sh);
+    if (st != DF11_OK) return st;
+    std::memset(info, 0, sizeof(*info));
+    std::snprintf(info->kernel, sizeof(info->kernel), "%s", p.name);
+    info->grid = sh.grid;
+    info->block = sh.block;
+    info->smem_bytes = uint32_t(sh.smem);
+    info->peek_bits = p.peek_bits;
+    info->table_copies = p.copies;
+    info->thread_blocks = hdr->n_blocks;
     return DF11_OK;
 }

@@ -10,9 +10,7 @@
 // position per thread block).
 #include <cuda_runtime.h>
 
-#include <atomic>
 #include <cstring>
-#include <mutex>
 #include <type_traits>
 #include <vector>
 
@@ -38,57 +36,54 @@ struct CodeTable {
 };
 
 // ---------------------------------------------------------------------------
-// Histogram of the symbols of one segment (the exponent field of BF16
-// elements, or 8-bit symbols); per-warp shared-memory histograms, flushed
-// into 64-bit global counters.
+// Histogram of the symbols of every segment in one launch (the exponent field
+// of BF16 elements, or 8-bit symbols); per-warp shared-memory histograms,
+// flushed into 64-bit global counters.  The CTAs stride over each segment's
+// 16-byte vectors in turn, two vectors in flight per thread.
 // ---------------------------------------------------------------------------
 constexpr int kHistThreads = 256;
 
-__global__ void __launch_bounds__(kHistThreads) histogram_u8_kernel(const uint8_t* __restrict__ x, uint64_t n,
-                                                                    unsigned long long* __restrict__ hist) {
-    __shared__ uint32_t sh[kHistThreads / 32][256];
-    uint32_t* mine = sh[threadIdx.x >> 5];
-    for (int i = threadIdx.x; i < (kHistThreads / 32) * 256; i += kHistThreads) (&sh[0][0])[i] = 0;
-    __syncthreads();
-    const uint64_t nvec = n / 16;
-    const uint4* xv = reinterpret_cast<const uint4*>(x);
-    const uint64_t stride = uint64_t(gridDim.x) * kHistThreads;
-    for (uint64_t v = uint64_t(blockIdx.x) * kHistThreads + threadIdx.x; v < nvec; v += stride) {
-        const uint4 q = __ldcs(xv + v);
-        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+template <int ES>
+__device__ __forceinline__ void count16(uint32_t* mine, const uint4 q) {
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
-        for (int k = 0; k < 16; k++) atomicAdd(&mine[(w[k >> 2] >> (8 * (k & 3))) & 0xFFu], 1u);
-    }
-    for (uint64_t i = nvec * 16 + uint64_t(blockIdx.x) * kHistThreads + threadIdx.x; i < n; i += stride)
-        atomicAdd(&mine[x[i]], 1u);
-    __syncthreads();
-    for (int s = threadIdx.x; s < 256; s += kHistThreads) {
-        uint64_t t = 0;
-        for (int w = 0; w < kHistThreads / 32; w++) t += sh[w][s];
-        if (t) atomicAdd(hist + s, (unsigned long long)t);
+    for (int k = 0; k < 4; k++) {
+        if constexpr (ES == 2) {
+            atomicAdd(&mine[(w[k] >> 7) & 0xFFu], 1u);
+            atomicAdd(&mine[(w[k] >> 23) & 0xFFu], 1u);
+        } else {
+#pragma unroll
+            for (int b = 0; b < 4; b++) atomicAdd(&mine[(w[k] >> (8 * b)) & 0xFFu], 1u);
+        }
     }
 }
 
-__global__ void __launch_bounds__(kHistThreads) histogram_kernel(const uint16_t* __restrict__ x, uint64_t n,
+template <int ES>
+__global__ void __launch_bounds__(kHistThreads) histogram_kernel(const __grid_constant__ SegTable sg,
                                                                  unsigned long long* __restrict__ hist) {
     __shared__ uint32_t sh[kHistThreads / 32][256];
     uint32_t* mine = sh[threadIdx.x >> 5];
     for (int i = threadIdx.x; i < (kHistThreads / 32) * 256; i += kHistThreads) (&sh[0][0])[i] = 0;
     __syncthreads();
-    const uint64_t nvec = n / 8;
-    const uint4* xv = reinterpret_cast<const uint4*>(x);
     const uint64_t stride = uint64_t(gridDim.x) * kHistThreads;
-    for (uint64_t v = uint64_t(blockIdx.x) * kHistThreads + threadIdx.x; v < nvec; v += stride) {
-        const uint4 q = __ldcs(xv + v);
-        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-        for (int k = 0; k < 4; k++) {
-            atomicAdd(&mine[(w[k] >> 7) & 0xFFu], 1u);
-            atomicAdd(&mine[(w[k] >> 23) & 0xFFu], 1u);
+    const uint64_t tid = uint64_t(blockIdx.x) * kHistThreads + threadIdx.x;
+    for (uint32_t seg = 0; seg < sg.n; seg++) {
+        const uint64_t cnt = sg.start[seg + 1] - sg.start[seg];
+        const uint8_t* p = sg.ptr[seg];
+        const uint64_t nvec = cnt * ES / 16;
+        const uint4* xv = reinterpret_cast<const uint4*>(p);
+        uint64_t v = tid;
+        for (; v + stride < nvec; v += 2 * stride) {
+            const uint4 a = __ldcs(xv + v), b = __ldcs(xv + v + stride);
+            count16<ES>(mine, a);
+            count16<ES>(mine, b);
+        }
+        if (v < nvec) count16<ES>(mine, __ldcs(xv + v));
+        for (uint64_t i = nvec * 16 / ES + tid; i < cnt; i += stride) {
+            const uint32_t x = ES == 2 ? uint32_t(reinterpret_cast<const uint16_t*>(p)[i] >> 7) : uint32_t(p[i]);
+            atomicAdd(&mine[x & 0xFFu], 1u);
         }
     }
-    for (uint64_t i = nvec * 8 + uint64_t(blockIdx.x) * kHistThreads + threadIdx.x; i < n; i += stride)
-        atomicAdd(&mine[(x[i] >> 7) & 0xFFu], 1u);
     __syncthreads();
     for (int s = threadIdx.x; s < 256; s += kHistThreads) {
         uint64_t t = 0;
@@ -246,170 +241,205 @@ __device__ __forceinline__ uint32_t thread_bits(const SharedCodes& sc, const uin
     return bits;
 }
 
-// Bits of code per chunk.
-template <int ES>
-__global__ void __launch_bounds__(kEncThreads) chunk_bits_kernel(const __grid_constant__ SegTable sg,
-                                                                 const __grid_constant__ CodeTable ct,
-                                                                 uint64_t n, uint64_t n_chunks,
-                                                                 uint32_t* __restrict__ chunk_bits) {
-    __shared__ SharedCodes sc;
-    __shared__ uint32_t s_warp[kEncThreads / 32];
-    stage_codes(sc, ct);
-    __syncthreads();
-    const uint64_t tofs = uint64_t(threadIdx.x) * kEncPerThread;
-    uint64_t c = blockIdx.x;
-    RawElems next = load_raw<ES>(sg, c * kEncChunk, c * kEncChunk + tofs, n);
-    for (; c < n_chunks; c += gridDim.x) {
-        const RawElems cur = next;
-        const uint64_t i0 = c * kEncChunk + tofs;
-        if (c + gridDim.x < n_chunks)
-            next = load_raw<ES>(sg, (c + gridDim.x) * kEncChunk, (c + gridDim.x) * kEncChunk + tofs, n);
-        uint32_t bits = 0;
-        if (i0 < n) {
-            uint32_t w[kWords<ES>];
-            raw_words<ES>(sg, cur, i0, n, w);
-            const uint64_t left = n - i0;
-            bits = thread_bits<ES>(sc, w, left < kEncPerThread ? uint32_t(left) : kEncPerThread);
-        }
-        uint32_t total;
-        block_exclusive_scan<kEncThreads>(bits, s_warp, total);
-        if (threadIdx.x == 0) chunk_bits[c] = total;
-        __syncthreads();  // s_warp is reused by the next chunk
-    }
-}
-
-// Exclusive prefix sum of the chunk totals in one CTA, 4096 chunks per tile
-// (four per thread, 16-byte loads), the next tile's loads issued before the
-// current tile is scanned.
-constexpr int kScanThreads = 1024;
-__global__ void __launch_bounds__(kScanThreads) chunk_scan_kernel(const uint32_t* __restrict__ chunk_bits,
-                                                                  uint64_t n_chunks,
-                                                                  unsigned long long* __restrict__ chunk_start) {
-    __shared__ unsigned long long s_warp[kScanThreads / 32];
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    constexpr uint64_t kTile = 4 * kScanThreads;
-    auto load4 = [&](uint64_t base) {
-        const uint64_t c = base + 4 * uint64_t(threadIdx.x);
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (c + 4 <= n_chunks) {
-            v = __ldg(reinterpret_cast<const uint4*>(chunk_bits + c));
-        } else {
-            if (c < n_chunks) v.x = chunk_bits[c];
-            if (c + 1 < n_chunks) v.y = chunk_bits[c + 1];
-            if (c + 2 < n_chunks) v.z = chunk_bits[c + 2];
-            if (c + 3 < n_chunks) v.w = chunk_bits[c + 3];
-        }
-        return v;
-    };
-    unsigned long long carry = 0;
-    uint4 v = load4(0);
-    for (uint64_t base = 0; base < n_chunks; base += kTile) {
-        const uint4 cur = v;
-        if (base + kTile < n_chunks) v = load4(base + kTile);
-        const unsigned long long own = (unsigned long long)cur.x + cur.y + cur.z + cur.w;
-        unsigned long long incl = own;
-#pragma unroll
-        for (int d = 1; d < 32; d <<= 1) {
-            const unsigned long long y = __shfl_up_sync(0xFFFFFFFFu, incl, d);
-            if (lane >= d) incl += y;
-        }
-        if (lane == 31) s_warp[warp] = incl;
-        __syncthreads();
-        unsigned long long before = 0, total = 0;
-        for (int w = 0; w < kScanThreads / 32; w++) {
-            const unsigned long long t = s_warp[w];
-            total += t;
-            before += w < warp ? t : 0ull;
-        }
-        __syncthreads();  // s_warp is rewritten by the next tile
-        unsigned long long run = carry + before + incl - own;
-        const uint64_t c = base + 4 * uint64_t(threadIdx.x);
-        const uint32_t e[4] = {cur.x, cur.y, cur.z, cur.w};
-#pragma unroll
-        for (int k = 0; k < 4; k++) {
-            if (c + k < n_chunks) chunk_start[c + k] = run;
-            run += e[k];
-        }
-        carry += total;
-    }
-}
-
 // ---------------------------------------------------------------------------
-// Bit-pack.  Each thread appends its codes to a register word with funnel
-// shifts; its first word (which it may share with the previous thread) and
-// its last, partial word (shared with the next) are OR-ed into a
-// shared-memory image of the chunk, the words in between are stored.  The
-// image's interior words are then stored to EncodedExponent and its two
-// boundary words, shared with the neighbouring chunks, are OR-ed into global
-// memory.  The same pass writes the sign+mantissa bytes, each window's gap
-// and each thread block's output position from the element's own start bit
-// s and length l:
+// Single-pass encode.  Chunks of kEncChunk elements are handed out in order by
+// an atomic ticket.  A chunk's CTA looks up every element's code, sums the
+// bits per thread and per chunk, and learns the chunk's first bit by a
+// decoupled look-back over per-chunk descriptors (64 bits: a 2-bit state,
+// then a bit count): it publishes its own total as an "aggregate", walks back
+// over its predecessors adding aggregates until it meets an "inclusive" prefix,
+// and publishes its own inclusive prefix.  A predecessor holds an earlier
+// ticket, so it is already running and publishes its aggregate without waiting
+// on anything; every wait here is therefore short, and each is bounded anyway
+// (after kSpinLimit polls the chunk gives up, zeroes the decode tables' magic
+// word -- the decoders then report the stream as corrupt -- and goes on).
+//
+// Packing, for a chunk starting at stream bit S.  Each thread appends its
+// codes to a register word with funnel shifts; its first word (which it may
+// share with the previous thread) and its last, partial word (shared with the
+// next) are OR-ed into a shared-memory image of the chunk, the words in
+// between are stored.  The image's interior words are then stored to
+// EncodedExponent and its two boundary words, shared with the neighbouring
+// chunks, are OR-ed into global memory.  The same pass writes the
+// sign+mantissa bytes, the gaps and the thread blocks' output positions from
+// each code's start bit s and length l:
 //   * a code that starts inside window w-1 and runs into window w sets
 //     gap[w] = s + l - 64w (gaps of windows that begin exactly at a code start
-//     stay 0);
+//     stay 0); the chunk's gap fields are assembled in shared memory and
+//     stored as whole words, the two boundary words OR-ed in;
 //   * a code that starts exactly at bit 64*T*b sets off[b] = i, one that runs
 //     over that bit sets off[b] = i + 1.
-// Positions are kept 32-bit relative to the chunk's first bit rounded down to
-// a thread-block boundary; a code covers a window boundary exactly when
-// (u >> 6) changes across it, u = relative start + 63, which is one test per
-// element.
+// Positions are kept 32-bit relative to S rounded down to a thread-block
+// boundary; a code covers a window boundary exactly when (u >> 6) changes
+// across it, u = relative start + 63, which is one test per element.
 // ---------------------------------------------------------------------------
 constexpr int kPackWords = kEncChunk + 4;  // 32 bits per element at most, plus the misalignment
 // windows a thread's codes can reach into: 16 codes of at most 32 bits
 constexpr int kMaxEvents = (int(kEncPerThread) * 32) / 64 + 1;
+// gap words a chunk can touch: 32 kEncChunk bits -> 512 kEncChunk / 64 + 2 windows of 5 bits
+constexpr int kGapWords = (5 * (int(kEncChunk) * 32 / 64 + 2)) / 32 + 2;
 static_assert(kPackWords % 4 == 0, "image cleared in 16-byte stores");
+constexpr unsigned long long kDescAggregate = 1ull << 62, kDescInclusive = 2ull << 62;
+constexpr unsigned long long kDescValue = (1ull << 62) - 1;
+constexpr uint32_t kSpinLimit = 1u << 20;
+
+// A descriptor is read only for its own value (no other memory is ordered by
+// it), so relaxed GPU-scope accesses suffice: no fence, which would make every
+// poll wait for the lane's outstanding pack stores.  Aligned 64-bit accesses
+// are single-copy atomic.
+__device__ __forceinline__ void publish(unsigned long long* p, unsigned long long v) {
+    asm volatile("st.relaxed.gpu.global.b64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+__device__ __forceinline__ unsigned long long observe(const unsigned long long* p) {
+    unsigned long long v;
+    asm volatile("ld.relaxed.gpu.global.b64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Warp 0: the exclusive prefix (first bit) of chunk c, whose own bits are
+// `total`; publishes c's aggregate first and its inclusive prefix last.  The
+// warp reads its predecessors kLookBack at a time (lane l, round r: the
+// (l + 32 r)-th nearest), every load of a window in flight at once: with a
+// few hundred chunks in flight, most look-backs end within one or two windows.
+constexpr int kLookRounds = 4;
+constexpr int kLookBack = 32 * kLookRounds;
+
+__device__ __forceinline__ unsigned long long look_back(unsigned long long* desc, uint32_t c, uint32_t total,
+                                                        uint32_t* lut_magic) {
+    const uint32_t lane = threadIdx.x & 31u;
+    if (c == 0) {
+        if (lane == 0) publish(desc, kDescInclusive | total);
+        return 0;
+    }
+    if (lane == 0) publish(desc + c, kDescAggregate | total);
+    unsigned long long prefix = 0;
+    int64_t base = int64_t(c) - 1;  // the nearest predecessor not yet added
+    uint32_t spins = 0;
+    for (;;) {
+        unsigned long long d[kLookRounds];
+#pragma unroll
+        for (int r = 0; r < kLookRounds; r++) {
+            const int64_t j = base - int64_t(lane) - 32 * r;
+            d[r] = j >= 0 ? observe(desc + j) : kDescInclusive;
+        }
+        // walk the window nearest first; stop at the first inclusive prefix
+        bool stall = false, found = false;
+        unsigned long long v = 0;
+#pragma unroll
+        for (int r = 0; r < kLookRounds; r++) {
+            const uint32_t state = uint32_t(d[r] >> 62);
+            const uint32_t incl = __ballot_sync(0xFFFFFFFFu, state == 2u);
+            const uint32_t empty = __ballot_sync(0xFFFFFFFFu, state == 0u);
+            // lanes up to the nearest inclusive prefix (all 32 if none) must be ready
+            const uint32_t upto = incl ? (incl & (0u - incl)) * 2u - 1u : 0xFFFFFFFFu;
+            if (empty & upto) {
+                stall = true;
+                break;
+            }
+            v += ((upto >> lane) & 1u) ? (d[r] & kDescValue) : 0ull;
+            if (incl) {
+                found = true;
+                break;
+            }
+        }
+        if (stall) {
+            ++spins;
+            // never expected: give up, mark the stream bad; once one chunk
+            // has given up, the others stop waiting too
+            const bool abort = spins >= kSpinLimit ||
+                               ((spins & 63u) == 0 && *reinterpret_cast<volatile uint32_t*>(lut_magic) == 0u);
+            if (abort) {
+                if (lane == 0) atomicExch(lut_magic, 0u);
+                return prefix;
+            }
+            __nanosleep(32);
+            continue;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+        prefix += v;
+        if (found) break;
+        base -= kLookBack;
+    }
+    if (lane == 0) publish(desc + c, kDescInclusive | (prefix + total));
+    return prefix;
+}
 
 template <int ES>
-__global__ void __launch_bounds__(kEncThreads) pack_kernel(const __grid_constant__ SegTable sg,
-                                                           const __grid_constant__ CodeTable ct, uint64_t n,
-                                                           uint64_t n_chunks, uint32_t log2_block_bits,
-                                                           const unsigned long long* __restrict__ chunk_start,
-                                                           uint32_t* __restrict__ exp32, uint8_t* __restrict__ sm,
-                                                           uint32_t* __restrict__ gaps32,
-                                                           uint32_t* __restrict__ block_off, uint64_t n_blocks,
-                                                           uint32_t* __restrict__ chunk_bit) {
+__global__ void __launch_bounds__(kEncThreads) encode_kernel(const __grid_constant__ SegTable sg,
+                                                             const __grid_constant__ CodeTable ct, uint64_t n,
+                                                             uint64_t n_chunks, uint32_t log2_block_bits,
+                                                             unsigned long long* __restrict__ desc,
+                                                             uint32_t* __restrict__ ticket, uint32_t* lut_magic,
+                                                             uint32_t* __restrict__ exp32, uint8_t* __restrict__ sm,
+                                                             uint32_t* __restrict__ gaps32,
+                                                             uint32_t* __restrict__ block_off, uint64_t n_blocks,
+                                                             uint32_t* __restrict__ chunk_bit) {
     __shared__ SharedCodes sc;
     __shared__ __align__(16) uint32_t s_words[kPackWords];
+    __shared__ uint32_t s_gap[kGapWords];
     __shared__ uint32_t s_ev[kMaxEvents][kEncThreads];
     __shared__ uint32_t s_warp[kEncThreads / 32];
+    __shared__ uint32_t s_ticket;
+    __shared__ unsigned long long s_prefix;
     stage_codes(sc, ct);
+    if (threadIdx.x == 0) s_ticket = atomicAdd(ticket, 1u);
     __syncthreads();
     const uint64_t block_mask = (uint64_t(1) << log2_block_bits) - 1;
     const uint64_t tofs = uint64_t(threadIdx.x) * kEncPerThread;
-    uint64_t c = blockIdx.x;
+    uint64_t c = s_ticket;
     RawElems next = load_raw<ES>(sg, c * kEncChunk, c * kEncChunk + tofs, n);
-    for (; c < n_chunks; c += gridDim.x) {
+    while (c < n_chunks) {
         const RawElems cur = next;
         const uint64_t i0 = c * kEncChunk + tofs;
-        if (c + gridDim.x < n_chunks)
-            next = load_raw<ES>(sg, (c + gridDim.x) * kEncChunk, (c + gridDim.x) * kEncChunk + tofs, n);
+        __syncthreads();  // everyone has read s_ticket; s_* of the last chunk are free
         uint32_t w8[kWords<ES>];
+        uint2 ce[kEncPerThread];  // code (left-aligned) and length of each element
         uint32_t valid = 0, bits = 0;
         if (i0 < n) {
             raw_words<ES>(sg, cur, i0, n, w8);
             const uint64_t left = n - i0;
             valid = left < kEncPerThread ? uint32_t(left) : kEncPerThread;
-            bits = thread_bits<ES>(sc, w8, valid);
+#pragma unroll
+            for (int k = 0; k < int(kEncPerThread); k++) {
+                ce[k] = uint32_t(k) < valid ? sc.e[symbol<ES>(w8, k)] : make_uint2(0, 0);
+                bits += ce[k].y;
+            }
         }
         for (int j = threadIdx.x; j < kPackWords / 4; j += kEncThreads)
             reinterpret_cast<uint4*>(s_words)[j] = make_uint4(0, 0, 0, 0);
+        for (int j = threadIdx.x; j < kGapWords; j += kEncThreads) s_gap[j] = 0;
         uint32_t chunk_total;
         const uint32_t my_off = block_exclusive_scan<kEncThreads>(bits, s_warp, chunk_total);
-        const uint64_t S = chunk_start[c];
+        if (threadIdx.x < 32) {
+            const unsigned long long pre = look_back(desc, uint32_t(c), chunk_total, lut_magic);
+            // the next ticket only now: a chunk's aggregate must follow its
+            // ticket quickly (a ticket held across this chunk's work would
+            // make the next chunk's look-back wait for all of it)
+            if (threadIdx.x == 0) {
+                s_prefix = pre;
+                s_ticket = atomicAdd(ticket, 1u);
+            }
+        }
+        __syncthreads();
+        const uint64_t nc = s_ticket;
+        next = load_raw<ES>(sg, nc * kEncChunk, nc * kEncChunk + tofs, n);  // in flight during the pack
+        const uint64_t S = s_prefix;
         const uint32_t lead = uint32_t(S & 31u);
         const uint64_t Sb = S & ~block_mask;  // a thread-block (and window) boundary
-        // gap and output position for a code at relative start r (bits from
-        // Sb) of length l, element i, that covers a window boundary
-        const uint64_t gap_base = 5 * (Sb >> 6);
+        // gap fields of this chunk: windows (S >> 6, (S + total - 1) >> 6], at
+        // gap array bits 5w .. 5w + 4; s_gap word 0 = gap array word g0
+        const uint64_t g0 = (5 * ((S >> 6) + 1)) >> 5;
         const uint64_t blk_base = Sb >> log2_block_bits;
         auto window_event = [&](uint32_t r, uint32_t l, uint64_t i) {
             if (r & 63u) {
-                const uint32_t wr = (r >> 6) + 1;
-                const uint32_t g = r + l - 64 * wr;
-                const uint64_t gb = gap_base + 5 * uint64_t(wr);
+                const uint64_t w = ((Sb + r) >> 6) + 1;  // the window the code runs into
+                const uint32_t g = uint32_t((Sb + r + l) - 64 * w);
+                const uint64_t gb = 5 * w;
                 const uint32_t sh = uint32_t(gb & 31);
-                atomicOr(gaps32 + (gb >> 5), g << sh);
-                if (sh > 27) atomicOr(gaps32 + (gb >> 5) + 1, g >> (32 - sh));
+                const uint32_t k = uint32_t((gb >> 5) - g0);
+                atomicOr(&s_gap[k], g << sh);
+                if (sh > 27) atomicOr(&s_gap[k + 1], g >> (32 - sh));
             }
             const uint32_t br = r >> log2_block_bits;
             if ((r & uint32_t(block_mask)) == 0) {
@@ -423,22 +453,22 @@ __global__ void __launch_bounds__(kEncThreads) pack_kernel(const __grid_constant
         // cover a window boundary (at most 9 for 16 codes of <= 32 bits) are
         // only noted in the thread's column of s_ev and handled after the
         // loop, so the warp does not run that handler on every element.
-        auto pack_codes = [&](auto full_tag) {
-            constexpr bool kFull = decltype(full_tag)::value;  // all kEncPerThread elements valid
+        if (valid) {
             const uint32_t q = lead + my_off;  // bit position in the chunk image
             uint32_t w = q >> 5, fill = q & 31u, cur_word = 0;
             uint32_t u = uint32_t(S - Sb) + my_off + 63u;  // relative start + 63
             uint32_t ne = 0;
+            bool first = true;
 #pragma unroll
             for (int k = 0; k < int(kEncPerThread); k++) {
-                if (!kFull && uint32_t(k) >= valid) break;
-                const uint2 ce = sc.e[symbol<ES>(w8, k)];
-                const uint32_t t = ce.x, l = ce.y;
+                const uint32_t t = ce[k].x, l = ce[k].y;  // l = 0 past the valid elements
                 cur_word |= t >> fill;
                 const uint32_t spill = __funnelshift_r(0u, t, fill);  // bits that did not fit
                 fill += l;
                 if (fill >= 32u) {
-                    atomicOr(&s_words[w], cur_word);
+                    if (first) atomicOr(&s_words[w], cur_word);
+                    else s_words[w] = cur_word;
+                    first = false;
                     w++;
                     cur_word = spill;
                     fill -= 32u;
@@ -454,11 +484,7 @@ __global__ void __launch_bounds__(kEncThreads) pack_kernel(const __grid_constant
                     window_event((e >> 10) - 63u, (e >> 4) & 63u, i0 + (e & 15u));
                 }
             }
-        };
-        if (valid == kEncPerThread)
-            pack_codes(std::true_type{});
-        else if (valid)
-            pack_codes(std::false_type{});
+        }
         if (block_off && valid && n - i0 <= kEncPerThread) block_off[n_blocks] = uint32_t(n);
         if (chunk_bit && valid) {  // independent-chunk table: first bit of every kIndChunk elements
             if (i0 % kIndChunk == 0) chunk_bit[i0 / kIndChunk] = uint32_t(S + my_off);
@@ -493,7 +519,23 @@ __global__ void __launch_bounds__(kEncThreads) pack_kernel(const __grid_constant
                 exp32[W0 + j] = v;
             }
         }
-        __syncthreads();  // s_words and s_warp are reused by the next chunk
+        if (gaps32) {
+            // gap words g0 .. g1; the first and last may hold other chunks' fields
+            const uint64_t w_last = (S + chunk_total - 1) >> 6;
+            const uint64_t g1 = (5 * w_last + 4) >> 5;
+            if (w_last > (S >> 6)) {
+                const uint32_t ng = uint32_t(g1 - g0 + 1);
+                for (uint32_t j = threadIdx.x; j < ng; j += kEncThreads) {
+                    const uint32_t v = s_gap[j];
+                    if (j == 0 || j == ng - 1) {
+                        if (v) atomicOr(gaps32 + g0 + j, v);
+                    } else {
+                        gaps32[g0 + j] = v;
+                    }
+                }
+            }
+        }
+        c = nc;
     }
 }
 
@@ -512,10 +554,13 @@ unsigned encode_grid(Kernel kernel, uint64_t chunks) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Encode scratch: one look-back descriptor per chunk, then the chunk ticket
+// (zeroed by every encode call before its kernel).
+constexpr uint64_t encode_scratch_bytes(uint64_t chunks) { return 8 * (chunks + 2); }
+
 struct Workspace {
     unsigned long long* hist;
-    uint32_t* chunk_bits;
-    unsigned long long* chunk_start;
+    unsigned long long* desc;
 };
 
 df11_status carve(void* ws, uint64_t ws_bytes, uint64_t n_elems, Workspace* w) {
@@ -529,8 +574,8 @@ df11_status carve(void* ws, uint64_t ws_bytes, uint64_t n_elems, Workspace* w) {
     const uint64_t chunks = (n_elems + kEncChunk - 1) / kEncChunk;
     uint8_t* p = static_cast<uint8_t*>(ws);
     w->hist = reinterpret_cast<unsigned long long*>(p);
-    w->chunk_bits = reinterpret_cast<uint32_t*>(p + 2048);
-    w->chunk_start = reinterpret_cast<unsigned long long*>(p + 2048 + align16(4 * chunks));
+    (void)chunks;
+    w->desc = reinterpret_cast<unsigned long long*>(p + 2048);
     return DF11_OK;
 }
 
@@ -579,17 +624,11 @@ df11_status compress_plan(const void* const* d_segs, const uint64_t* seg_counts,
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    for (uint32_t k = 0; k < n_segs; k++) {
-        const uint64_t cnt = seg_counts[k];
-        if (!cnt) continue;
-        const uint64_t vec_blocks = (cnt / (16 / ES) + kHistThreads - 1) / kHistThreads;
+    if (n) {
+        const uint64_t vec_blocks = (n * ES / 16 + kHistThreads - 1) / kHistThreads;
         uint64_t grid = vec_blocks < uint64_t(4 * sms) ? vec_blocks : uint64_t(4 * sms);
         if (grid == 0) grid = 1;
-        if constexpr (ES == 2)
-            histogram_kernel<<<unsigned(grid), kHistThreads, 0, s>>>(
-                reinterpret_cast<const uint16_t*>(sg.ptr[k]), cnt, w.hist);
-        else
-            histogram_u8_kernel<<<unsigned(grid), kHistThreads, 0, s>>>(sg.ptr[k], cnt, w.hist);
+        histogram_kernel<ES><<<unsigned(grid), kHistThreads, 0, s>>>(sg, w.hist);
     }
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail("histogram launch", e);
@@ -612,7 +651,7 @@ df11_status compress_plan(const void* const* d_segs, const uint64_t* seg_counts,
 // offsets) d_gaps and d_block_off are not written and may be null.
 template <int ES>
 df11_status compress_encode(const char* fn, const void* const* d_segs, const df11_header* hdr,
-                            uint32_t* chunk_bits, unsigned long long* chunk_start, uint8_t* d_exp, uint8_t* d_sm,
+                            unsigned long long* desc, uint8_t* d_exp, uint8_t* d_sm,
                             uint8_t* d_gaps, uint32_t* d_block_off, void* d_lut, void* stream,
                             uint32_t* d_chunk_bit = nullptr) {
     df11_status st = check_header(hdr);
@@ -663,13 +702,13 @@ df11_status compress_encode(const char* fn, const void* const* d_segs, const df1
 
     const uint64_t chunks = (n + kEncChunk - 1) / kEncChunk;
     if (chunks >= (uint64_t(1) << 31)) return fail(DF11_ERR_TOO_LARGE, "too many chunks");
-    chunk_bits_kernel<ES><<<encode_grid(chunk_bits_kernel<ES>, chunks), kEncThreads, 0, s>>>(sg, ct, n, chunks,
-                                                                                          chunk_bits);
-    chunk_scan_kernel<<<1, kScanThreads, 0, s>>>(chunk_bits, chunks, chunk_start);
+    if ((e = cudaMemsetAsync(desc, 0, encode_scratch_bytes(chunks), s)) != cudaSuccess)
+        return cuda_fail("clear encode scratch", e);
     uint32_t log2_bb = 6;
     while ((1u << (log2_bb - 6)) < hdr->threads_per_block) log2_bb++;
-    pack_kernel<ES><<<encode_grid(pack_kernel<ES>, chunks), kEncThreads, 0, s>>>(
-        sg, ct, n, chunks, log2_bb, chunk_start, reinterpret_cast<uint32_t*>(d_exp), d_sm,
+    encode_kernel<ES><<<encode_grid(encode_kernel<ES>, chunks), kEncThreads, 0, s>>>(
+        sg, ct, n, chunks, log2_bb, desc, reinterpret_cast<uint32_t*>(desc + chunks),
+        static_cast<uint32_t*>(d_lut), reinterpret_cast<uint32_t*>(d_exp), d_sm,
         reinterpret_cast<uint32_t*>(d_gaps), d_block_off, hdr->n_blocks, d_chunk_bit);
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail("encode launch", e);
@@ -695,7 +734,7 @@ extern "C" df11_status df11_compress_encode(const void* const* d_segs, const df1
     Workspace w{};
     const df11_status st = carve(d_workspace, workspace_bytes, hdr ? hdr->n_elems : 0, &w);
     if (st != DF11_OK) return st;
-    return compress_encode<2>("df11_compress_encode", d_segs, hdr, w.chunk_bits, w.chunk_start, d_exp, d_sm, d_gaps,
+    return compress_encode<2>("df11_compress_encode", d_segs, hdr, w.desc, d_exp, d_sm, d_gaps,
                               d_block_off, d_lut, stream);
 }
 
@@ -714,7 +753,7 @@ extern "C" df11_status df11_compress_encode_u8(const void* const* d_segs, const 
     Workspace w{};
     const df11_status st = carve(d_workspace, workspace_bytes, hdr ? hdr->n_elems : 0, &w);
     if (st != DF11_OK) return st;
-    return compress_encode<1>("df11_compress_encode_u8", d_segs, hdr, w.chunk_bits, w.chunk_start, d_exp,
+    return compress_encode<1>("df11_compress_encode_u8", d_segs, hdr, w.desc, d_exp,
                               nullptr, d_gaps, d_block_off, d_lut, stream);
 }
 
@@ -731,36 +770,24 @@ namespace df11 {
 namespace {
 
 constexpr uint64_t kStaticChunks = DF11_STATIC_MAX_ELEMS / kEncChunk;
-constexpr uint64_t kStaticBitsBytes = 4 * kStaticChunks;
-constexpr uint64_t kStaticScratchBytes = kStaticBitsBytes + 8 * kStaticChunks;
+constexpr uint64_t kStaticScratchBytes = encode_scratch_bytes(kStaticChunks);
 static_assert(DF11_STATIC_MAX_ELEMS % kEncChunk == 0, "whole chunks");
 
-// Loaded with the library on every GPU that uses it and held until exit.
-// Every call overwrites all of the scratch it reads, so nothing has to be
-// cleared between calls; two calls that overlap on the GPU share it and race.
+// Loaded with the library's device code on every GPU that uses it and held
+// until exit.  Every call clears the part it uses (the look-back descriptors
+// and the chunk ticket must start at zero) before its kernel; two calls that
+// overlap on the GPU share it and race.
 static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
 
-// Device address of the scratch, looked up once per device with that device
-// current (host code cannot use the symbol itself as a device pointer).
-constexpr int kMaxDevices = 64;
-std::atomic<void*> g_static_scratch_addr[kMaxDevices];
-std::mutex g_static_scratch_mu;
-
+// Device address of the scratch for the current device and context.  Host
+// code cannot use the symbol itself as a device pointer, and the address can
+// change when the module is loaded again (after cudaDeviceReset, or in another
+// context on the same device), so it is looked up on every call; once the
+// library's device code is loaded, the lookup allocates nothing.
 df11_status static_scratch_address(void** out) {
-    int dev = -1;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return cuda_fail("cudaGetDevice", e);
-    if (dev < 0 || dev >= kMaxDevices) return fail(DF11_ERR_INVALID, "device ordinal %d above %d", dev, kMaxDevices);
-    void* p = g_static_scratch_addr[dev].load(std::memory_order_acquire);
-    if (!p) {
-        std::lock_guard<std::mutex> lock(g_static_scratch_mu);
-        p = g_static_scratch_addr[dev].load(std::memory_order_relaxed);
-        if (!p) {
-            e = cudaGetSymbolAddress(&p, g_static_scratch);
-            if (e != cudaSuccess) return cuda_fail("cudaGetSymbolAddress(static scratch)", e);
-            g_static_scratch_addr[dev].store(p, std::memory_order_release);
-        }
-    }
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_static_scratch);
+    if (e != cudaSuccess) return cuda_fail("cudaGetSymbolAddress(static scratch)", e);
     *out = p;
     return DF11_OK;
 }
@@ -781,10 +808,8 @@ extern "C" df11_status df11_compress_encode_static(const void* const* d_segs, co
     void* scratch = nullptr;
     st = static_scratch_address(&scratch);
     if (st != DF11_OK) return st;
-    uint32_t* chunk_bits = static_cast<uint32_t*>(scratch);
-    unsigned long long* chunk_start =
-        reinterpret_cast<unsigned long long*>(static_cast<unsigned char*>(scratch) + kStaticBitsBytes);
-    return compress_encode<2>("df11_compress_encode_static", d_segs, hdr, chunk_bits, chunk_start, d_exp, d_sm,
+    return compress_encode<2>("df11_compress_encode_static", d_segs, hdr, static_cast<unsigned long long*>(scratch),
+                              d_exp, d_sm,
                               d_gaps, d_block_off, d_lut, stream);
 }
 
@@ -797,6 +822,6 @@ extern "C" df11_status df11_compress_encode_chunked(const void* const* d_segs, c
     Workspace w{};
     const df11_status st = carve(d_workspace, workspace_bytes, hdr ? hdr->n_elems : 0, &w);
     if (st != DF11_OK) return st;
-    return compress_encode<2>("df11_compress_encode_chunked", d_segs, hdr, w.chunk_bits, w.chunk_start, d_exp,
+    return compress_encode<2>("df11_compress_encode_chunked", d_segs, hdr, w.desc, d_exp,
                               d_sm, nullptr, nullptr, d_lut, stream, d_chunk_bit);
 }

@@ -254,52 +254,76 @@ df11_status df11_build_lut(const df11_header* hdr, void* h_lut, uint64_t cap) {
         delta[l] = base[l] - uint32_t(first[l]);  // wraps; used modulo 2^32
     }
 
-    // length of the code at the top of a 32-bit left-justified peek, 0 if none
-    auto code_length = [&](uint64_t peek32) -> int {
-        for (int l = 1; l <= 32; l++)
-            if (peek32 < lj_end[l]) return l;
-        return 0;
-    };
-
-    // level 1: walk the complete codes at the front of every 12-bit peek
-    uint32_t* ctab = reinterpret_cast<uint32_t*>(blob + kLutOffCount);
-    uint16_t* mtab = reinterpret_cast<uint16_t*>(blob + kLutOffMask);
-    uint32_t* dtab = reinterpret_cast<uint32_t*>(blob + kLutOffDecode);  // pairs (x, y)
-    for (uint32_t v = 0; v < kLutEntries; v++) {
-        uint32_t mask = 0, count = 0, syms4 = 0, n4 = 0, used4 = 0;
-        int pos = 0;
-        while (pos < kPeekBits) {
-            const uint64_t peek = (uint64_t(v) << (32 - kPeekBits + pos)) & 0xFFFFFFFFull;
-            const int l = code_length(peek);
-            if (l == 0 || pos + l > kPeekBits) break;
-            mask |= 1u << pos;
-            count++;
-            if (n4 < kDecodeSyms) {
-                const uint32_t value = uint32_t(peek >> (32 - l));
-                syms4 |= uint32_t(syms[(value + delta[l]) & 0xFFu]) << (8 * n4);
-                n4++;
-                used4 = uint32_t(pos + l);
+    // the code at the front of every 12-bit value, when it has at most 12
+    // bits: front[v] = length << 8 | rotated symbol, 0 if longer (canonical
+    // codes are ranges of consecutive values, so each fills its range)
+    static_assert(kPeekBits == 12, "front table covers the widest level-1 table");
+    uint16_t front[1u << kPeekBits] = {0};
+    {
+        int idx = 0;
+        for (int l = 1; l <= kPeekBits; l++) {
+            for (uint64_t j = 0; j < count[l]; j++, idx++) {
+                const uint32_t lo = uint32_t((first[l] + j) << (kPeekBits - l));
+                const uint32_t hi = lo + (1u << (kPeekBits - l));
+                for (uint32_t v = lo; v < hi; v++) front[v] = uint16_t((l << 8) | syms[idx]);
             }
-            pos += l;
         }
-        ctab[v] = count ? ((uint32_t(pos) << 16) | count) : (kEscape << 16);
-        mtab[v] = uint16_t(mask);
-        dtab[2 * v] = n4 ? syms4 : 0u;
-        dtab[2 * v + 1] = n4 ? ((used4 << 16) | (8 * n4)) : (kEscape << 16);
     }
-    // level 2: long codes of up to kLongBits bits by their 20-bit prefix
-    uint16_t* ltab = reinterpret_cast<uint16_t*>(blob + kLutOffLong);
-    const uint64_t region = (uint64_t(1) << 32) - lj_end[kPeekBits];  // code space of long codes
-    const uint64_t n_long = (region + (uint64_t(1) << (32 - kLongBits)) - 1) >> (32 - kLongBits);
-    lh.long_base = uint32_t(lj_end[kPeekBits] >> (32 - kLongBits));
-    lh.long_count = (lj_end[kPeekBits] < (uint64_t(1) << 32) && n_long <= kLongEntries) ? uint32_t(n_long) : 0u;
-    for (uint32_t i = 0; i < lh.long_count; i++) {
-        const uint64_t peek = uint64_t(lh.long_base + i) << (32 - kLongBits);
-        const int l = code_length(peek);
-        if (l > kPeekBits && l <= int(kLongBits)) {
-            const uint32_t value = uint32_t(peek >> (32 - l));
-            ltab[i] = uint16_t(syms[(value + delta[l]) & 0xFFu] | (uint32_t(l) << 8));
+
+    // level 1 for a K-bit peek: walk the complete codes at the front of every
+    // K-bit value; the count table only exists for K = 12
+    auto level1 = [&](int K, uint32_t* ctab, uint16_t* mtab, uint32_t* dtab) {
+        for (uint32_t v = 0; v < (1u << K); v++) {
+            uint32_t mask = 0, count = 0, syms4 = 0, n4 = 0, used4 = 0;
+            int pos = 0;
+            while (pos < K) {
+                // the bits of v from pos on, at the front of 12 bits (zeros after)
+                const uint32_t f = front[(v << (kPeekBits - K + pos)) & ((1u << kPeekBits) - 1)];
+                const int l = int(f >> 8);
+                if (l == 0 || pos + l > K) break;
+                mask |= 1u << pos;
+                count++;
+                if (n4 < kDecodeSyms) {
+                    syms4 |= uint32_t(f & 0xFFu) << (8 * n4);
+                    n4++;
+                    used4 = uint32_t(pos + l);
+                }
+                pos += l;
+            }
+            if (ctab) ctab[v] = count ? ((uint32_t(pos) << 16) | count) : (kEscape << 16);
+            mtab[v] = uint16_t(mask);
+            dtab[2 * v] = n4 ? syms4 : 0u;
+            dtab[2 * v + 1] = n4 ? ((used4 << 16) | (8 * n4)) : (kEscape << 16);
         }
+    };
+    // level 2 for codes longer than K: up to kLongBits bits by their 20-bit
+    // prefix, from the first code longer than K on; none (count 0) when the
+    // long codes need more than `cap` prefixes.  A code of l bits covers
+    // 2^(20 - l) consecutive prefixes.
+    auto level2 = [&](int K, uint16_t* ltab, uint32_t cap, uint32_t* long_base, uint32_t* long_count) {
+        const uint64_t region = (uint64_t(1) << 32) - lj_end[K];  // code space of long codes
+        const uint64_t n_long = (region + (uint64_t(1) << (32 - kLongBits)) - 1) >> (32 - kLongBits);
+        *long_base = uint32_t(lj_end[K] >> (32 - kLongBits));
+        *long_count = (lj_end[K] < (uint64_t(1) << 32) && n_long <= cap) ? uint32_t(n_long) : 0u;
+        if (!*long_count) return;
+        for (int l = K + 1; l <= int(kLongBits); l++) {
+            for (uint64_t j = 0; j < count[l]; j++) {
+                const uint64_t lo = (first[l] + j) << (kLongBits - l);
+                const uint64_t hi = lo + (uint64_t(1) << (kLongBits - l));
+                const uint16_t e = uint16_t(syms[base[l] + j] | (uint32_t(l) << 8));
+                for (uint64_t v = lo; v < hi; v++) ltab[v - *long_base] = e;
+            }
+        }
+    };
+    level1(kPeekBits, reinterpret_cast<uint32_t*>(blob + kLutOffCount), reinterpret_cast<uint16_t*>(blob + kLutOffMask),
+           reinterpret_cast<uint32_t*>(blob + kLutOffDecode));
+    level2(kPeekBits, reinterpret_cast<uint16_t*>(blob + kLutOffLong), kLongEntries, &lh.long_base, &lh.long_count);
+    for (int K = 10; K >= 8; K--) {
+        uint8_t* sec = blob + narrow_off(K);
+        level1(K, nullptr, reinterpret_cast<uint16_t*>(sec + narrow_mask_off(K)),
+               reinterpret_cast<uint32_t*>(sec + narrow_decode_off(K)));
+        level2(K, reinterpret_cast<uint16_t*>(sec + narrow_long_off(K)), narrow_long_entries(K),
+               &lh.narrow_long[narrow_index(K)][0], &lh.narrow_long[narrow_index(K)][1]);
     }
     std::memcpy(blob, &lh, sizeof(lh));
     return DF11_OK;
@@ -308,8 +332,9 @@ df11_status df11_build_lut(const df11_header* hdr, void* h_lut, uint64_t cap) {
 df11_status df11_compress_workspace_size(uint64_t n_elems, uint64_t* bytes) {
     if (!bytes) return fail(DF11_ERR_INVALID, "df11_compress_workspace_size: null pointer");
     const uint64_t chunks = (n_elems + kEncChunk - 1) / kEncChunk;
-    // histogram (256 x u64) + per-chunk bit counts (u32) + chunk starts (u64)
-    *bytes = 2048 + align16(4 * chunks) + align16(8 * chunks) + 64;
+    // histogram (256 x u64), then one look-back descriptor (u64) per chunk and
+    // the chunk ticket
+    *bytes = 2048 + align16(8 * (chunks + 2)) + 64;
     return DF11_OK;
 }
 

@@ -48,7 +48,7 @@ namespace df11 {
 // ---------------------------------------------------------------------------
 constexpr uint32_t kLutMagic = 0x31314644u;  // "DF11"
 constexpr int kPeekBits = 12;
-constexpr uint32_t kEscape = 256;            // > any bit position a thread decodes (<= 128) + K
+constexpr uint32_t kEscape = 512;            // > any bit position a thread decodes (<= 256) + K
 constexpr uint32_t kDecodeSyms = 4;          // symbols per decode-table entry
 
 struct LutHeader {
@@ -60,7 +60,8 @@ struct LutHeader {
     uint32_t max_len;
     uint32_t long_base;   // (lj_end[K] >> 12): 20-bit prefix of the first long code
     uint32_t long_count;  // entries of the long table, 0 = ladder only
-    uint32_t pad[8];
+    uint32_t narrow_long[3][2];  // long_base, long_count of the narrow sections (K = 10, 9, 8)
+    uint32_t pad[2];
 };
 static_assert(sizeof(LutHeader) == 64, "LutHeader is 64 bytes");
 
@@ -75,7 +76,26 @@ constexpr uint64_t kLutOffDecode = align16(kLutOffMask + 2 * kLutEntries);  // u
 constexpr uint32_t kLongEntries = 4096;
 constexpr uint32_t kLongBits = 20;                                          // long-table resolution
 constexpr uint64_t kLutOffLong = align16(kLutOffDecode + 8 * kLutEntries);  // uint16[kLongEntries]
-constexpr uint64_t kLutBytes = align16(kLutOffLong + 2 * kLongEntries);
+
+// Narrow level-1 sections: the same mask and decode tables for a K-bit peek,
+// K = 10, 9 or 8 (the pages' 256-entry first level), each with its own long
+// table for the codes longer than K.  A table of 2^K entries is small enough
+// to be staged in shared memory once per 8-byte bank pair (16 copies, copy c
+// in bank pair c), so the 16 lanes of a half-warp always read distinct bank
+// pairs: one wavefront per half-warp, whatever the indices.
+//   section(K) = mask u16[2^K] | long u16[narrow_long_entries(K)] | decode uint2[2^K]
+constexpr uint32_t narrow_long_entries(int K) { return K == 8 ? 8192u : 4096u; }
+constexpr uint64_t narrow_mask_off(int) { return 0; }
+constexpr uint64_t narrow_long_off(int K) { return uint64_t(2) << K; }
+constexpr uint64_t narrow_decode_off(int K) { return narrow_long_off(K) + 2 * uint64_t(narrow_long_entries(K)); }
+constexpr uint64_t narrow_bytes(int K) { return align16(narrow_decode_off(K) + (uint64_t(8) << K)); }
+constexpr int narrow_index(int K) { return 10 - K; }  // LutHeader::narrow_long row
+constexpr uint64_t kLutOffNarrow = align16(kLutOffLong + 2 * kLongEntries);
+constexpr uint64_t narrow_off(int K) {
+    return K == 10 ? kLutOffNarrow : K == 9 ? kLutOffNarrow + narrow_bytes(10)
+                                            : kLutOffNarrow + narrow_bytes(10) + narrow_bytes(9);
+}
+constexpr uint64_t kLutBytes = narrow_off(8) + narrow_bytes(8);
 
 // Canonical code per value (DEFLATE-style construction); false if the
 // lengths overflow the code space.

@@ -28,18 +28,23 @@ class BlockPrefetcher:
     n_buffers   BF16 buffers cycled through (2 = double buffering)
     max_sms     cap on the SMs each decode occupies (None = all), so that the
                 caller's kernels can run beside it
+    options     decode options (decode_options), e.g. many small CTAs that
+                queue behind the caller's kernels and fill the SMs they leave
+                idle; overrides max_sms
     status      optional int32 device word, OR-ed with DF11_ERR_CORRUPT by a
                 decode that finds its stream inconsistent
     """
 
     def __init__(self, streams: list[CompressedStream], n_buffers: int = 2, max_sms: int | None = None,
-                 status: torch.Tensor | None = None, decode_stream: torch.cuda.Stream | None = None):
+                 status: torch.Tensor | None = None, decode_stream: torch.cuda.Stream | None = None,
+                 options=None):
         if n_buffers < 2:
             raise ValueError("n_buffers must be at least 2")
         if not streams:
             raise ValueError("no blocks")
         self.streams = list(streams)
         self.max_sms = max_sms
+        self.options = options
         self.status = status
         dev = self.streams[0].exp.device
         n_max = max(max(cs.n_elems for cs in self.streams), 1)
@@ -55,7 +60,7 @@ class BlockPrefetcher:
             self.decode_stream.wait_event(free[slot])
         cs = self.streams[i]
         decompress(cs, out=self.buffers[slot][: cs.n_elems], status=self.status, stream=self.decode_stream,
-                   max_sms=self.max_sms)
+                   max_sms=self.max_sms, options=self.options)
         ready = torch.cuda.Event()
         ready.record(self.decode_stream)
         return ready

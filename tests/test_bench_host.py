@@ -59,3 +59,25 @@ def test_every_config_has_a_workload_description():
     assert set(bench.CONFIGS) >= {"c1", "c2", "c3", "c4", "c5"}
     assert bench.U8_CONFIGS <= set(bench.CONFIGS)
     assert all(isinstance(v, str) and v for v in bench.CONFIGS.values())
+
+
+def test_step_stats_median_min_max():
+    st = bench.step_stats([0.3, 0.1, 0.2, 0.5, 0.4])
+    assert st == {"median": 0.3, "min": 0.1, "max": 0.5, "n": 5}
+    assert bench.step_stats([1.0])["median"] == 1.0
+
+
+def test_extra_workloads_are_described_and_distinct():
+    assert len(set(bench.EXTRA_CONFIGS)) == len(bench.EXTRA_CONFIGS)
+    assert set(bench.EXTRA_CONFIGS) <= set(bench.CONFIGS)
+    # every synthetic workload of the edge sweep has a full-size line
+    assert {"edge_uniform", "edge_one_value", "edge_zipf"} <= set(bench.EXTRA_CONFIGS)
+    assert bench.EDGE_N == 2 ** 26 + 13
+
+
+def test_edge_workload_uses_the_parity_sweep_seed():
+    from lossless_entropy_coded_dfloat11_b200 import inputs as I
+    w = bench.make_workloads("edge_zipf", 0, "cpu")[0]
+    ref = I.edge_case(bench.EDGE_N, "zipf", 500 + len(I.EDGE_SIZES) - 1)
+    assert w.n_elems == bench.EDGE_N
+    assert (w.flat_u16()[:4096] == ref.flat_u16()[:4096]).all()

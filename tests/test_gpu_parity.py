@@ -91,6 +91,22 @@ def test_edge_sweep(idx, dist):
 
 
 @pytest.mark.parametrize("dist", inputs.EDGE_DISTS)
+@pytest.mark.parametrize("n", [1, 33, 127, 4097, 65537, (1 << 20) + 7, (1 << 24) + 3])
+def test_edge_cases_four_windows_per_lane(n, dist):
+    both_directions(inputs.edge_case(n, dist, 950 + n % 97), T=128)
+
+
+def test_llama8b_block_four_windows_per_lane():
+    w = inputs.llama_block(inputs.LLAMA_8B, seed_base=3)
+    x = w.flat_u16()
+    cs = df11.compress(to_device(w), threads_per_block=128)
+    assert cs.kernel_info()["kernel"].startswith("decode_warp_kernel")
+    np.testing.assert_array_equal(decode_on_gpu(cs), x)
+    s = oracle.encode(x, threads_per_block=128)
+    assert_same_stream(cs, s)
+
+
+@pytest.mark.parametrize("dist", inputs.EDGE_DISTS)
 @pytest.mark.parametrize("n", [1, 33, 127, 4097, 65537, (1 << 20) + 7])
 def test_edge_cases_one_window_per_lane(n, dist):
     # the sweep above runs the default T = 64 (two windows per lane when every
@@ -195,9 +211,9 @@ def test_empty_and_single_element():
     both_directions(w)
 
 
-def test_corrupt_block_offsets_are_reported_not_trapped():
+@pytest.mark.parametrize("T", [64, 128])
+def test_corrupt_block_offsets_are_reported_not_trapped(T):
     x = inputs.matrix_1k().flat_u16()
-    T = df11.DEFAULT_THREADS_PER_BLOCK
     s = oracle.encode(x, threads_per_block=T)
     guard = 4096
     for b, delta in ((5, 1), (100, -3), (s.n_blocks, 1000)):
@@ -212,9 +228,9 @@ def test_corrupt_block_offsets_are_reported_not_trapped():
         assert bool((buf[s.n_elems:] == 7.0).all())       # nothing written past the output
 
 
-def test_corrupt_gaps_and_bits_terminate():
+@pytest.mark.parametrize("T", [64, 128])
+def test_corrupt_gaps_and_bits_terminate(T):
     x = inputs.matrix_outliers(512, 512, seed=5).flat_u16()
-    T = df11.DEFAULT_THREADS_PER_BLOCK
     s = oracle.encode(x, threads_per_block=T)
     gaps = s.gaps.copy()
     gaps[40] ^= 0x1F
@@ -234,6 +250,23 @@ def test_corrupt_gaps_and_bits_terminate():
         torch.cuda.synchronize()
         assert int(status.item()) in (0, B.DF11_ERR_CORRUPT)
         assert out.numel() == s.n_elems
+
+
+@pytest.mark.parametrize("T", [32, 64, 256])
+def test_tables_without_the_magic_word_are_reported(T):
+    """Decode tables whose magic word is not the library's (a table buffer
+    never filled, or the tables of an encode that gave up waiting): every
+    decode kernel reports the stream corrupt and writes nothing."""
+    x = inputs.matrix_1k().flat_u16()
+    s = oracle.encode(x, threads_per_block=T)
+    cs = lib_stream_from_oracle(s)
+    cs.lut[:4] = 0
+    buf = torch.full((s.n_elems,), 7.0, dtype=torch.bfloat16, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    df11.decompress(cs, out=buf, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == B.DF11_ERR_CORRUPT
+    assert bool((buf == 7.0).all())
 
 
 def test_host_side_argument_checks():

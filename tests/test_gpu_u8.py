@@ -40,7 +40,7 @@ def decode_u8(cs) -> np.ndarray:
 def both_directions(w: inputs.Workload, T: int = df11.DEFAULT_THREADS_PER_BLOCK):
     v = flat_u8(w)
     counts = [t.numel() for t in w.tensors]
-    # library encoder (T = 64 falls back to 32 when a code is 1 bit long)
+    # library encoder (T = 64 or 128 falls back to 32 when a code is 1 bit long)
     cs = df11.compress_u8([t.cuda() for t in w.tensors], threads_per_block=T)
     s = oracle_stream(v, cs.threads_per_block)
     # oracle stream -> library u8 kernel
@@ -65,7 +65,7 @@ def both_directions(w: inputs.Workload, T: int = df11.DEFAULT_THREADS_PER_BLOCK)
     return cs
 
 
-@pytest.mark.parametrize("T", [32, 64])
+@pytest.mark.parametrize("T", [32, 64, 128])
 def test_quantized_matrix(T):
     w = inputs.Workload("q", ["w"], [inputs.quantize_u8(inputs.gaussian((1024, 1024), 0.02, 1))])
     cs = both_directions(w, T)
@@ -74,7 +74,7 @@ def test_quantized_matrix(T):
     assert 0.88 < cs.compressed_bytes() / cs.n_elems < 0.95
 
 
-@pytest.mark.parametrize("T", [32, 64])
+@pytest.mark.parametrize("T", [32, 64, 128])
 def test_uint4_values_one_per_byte(T):
     """uint4 weights (the other alphabet the EntroLLM page codes), one value
     per byte: a 16-symbol alphabet on the same streams and kernels."""
@@ -93,6 +93,20 @@ def test_uint4_block():
 @pytest.mark.parametrize("n", [1, 2, 31, 33, 255, 4097, 65537, (1 << 20) + 7])
 def test_edge_cases(n, dist):
     both_directions(inputs.edge_case_u8(n, dist, 600 + n % 89))
+
+
+@pytest.mark.parametrize("dist", inputs.EDGE_DISTS)
+@pytest.mark.parametrize("n", [1, 33, 4097, 65537, (1 << 20) + 7])
+def test_edge_cases_four_windows_per_lane(n, dist):
+    both_directions(inputs.edge_case_u8(n, dist, 700 + n % 89), T=128)
+
+
+def test_llama8b_block_quantized_four_windows_per_lane():
+    w = inputs.llama_block_u8(inputs.LLAMA_8B, seed_base=3)
+    v = flat_u8(w)
+    cs = df11.compress_u8([t.cuda() for t in w.tensors], names=w.names, threads_per_block=128)
+    assert cs.threads_per_block == 128
+    np.testing.assert_array_equal(decode_u8(cs), v)
 
 
 def test_ragged_segments():

@@ -142,14 +142,31 @@ def test_header_validation():
 
 
 PEEK_BITS = 12
-ESCAPE = 256
+ESCAPE = 512
 # table offsets: 64-byte header, lj_end u64[33], delta u32[33], syms u8[256],
 # then count u32[4096], mask u16[4096], decode (u32, u32)[4096]
 OFF_COUNT = 736
 OFF_MASK = OFF_COUNT + 4 * 4096
 OFF_DECODE = OFF_MASK + 2 * 4096
 OFF_LONG = OFF_DECODE + 8 * 4096
-LUT_BYTES = OFF_LONG + 2 * 4096
+# then the narrow sections for K = 10, 9, 8: mask u16[2^K], long u16[4096
+# (8192 for K = 8)], decode (u32, u32)[2^K], each rounded up to 16 bytes
+OFF_NARROW = OFF_LONG + 2 * 4096
+
+
+def narrow_long_entries(k):
+    return 8192 if k == 8 else 4096
+
+
+def narrow_bytes(k):
+    return -(-(2 * 2 ** k + 2 * narrow_long_entries(k) + 8 * 2 ** k) // 16) * 16
+
+
+def narrow_off(k):
+    return OFF_NARROW + sum(narrow_bytes(j) for j in range(10, k, -1))
+
+
+LUT_BYTES = narrow_off(8) + narrow_bytes(8)
 
 
 def _oracle_prefix_decoder(code_len):
@@ -212,6 +229,64 @@ def test_decode_tables_agree_with_oracle_codes(source):
             assert (x >> (8 * k)) & 0xFF == ((sym >> 1) | (sym << 7)) & 0xFF
 
 
+@pytest.mark.parametrize("k", [10, 9, 8])
+@pytest.mark.parametrize("source", ["matrix_1k", "zipf", "fibonacci"])
+def test_narrow_tables_agree_with_oracle_codes(source, k):
+    """The narrow first levels (a K-bit peek, K = 10, 9 and the pages' 8-bit
+    256-entry table): every mask and decode entry describes exactly the
+    complete oracle codes at the front of its K-bit index, and entry i of the
+    section's long table the code at the top of the 20-bit prefix
+    long_base + i when that code is longer than K and at most 20 bits."""
+    if source == "matrix_1k":
+        x = inputs.matrix_1k().flat_u16()
+    elif source == "fibonacci":
+        x = inputs.fibonacci().flat_u16()
+    else:
+        x = inputs.edge_case(65537, source, 515).flat_u16()
+    s = oracle.encode(x)
+    hdr = df11.make_header(s.code_len, s.n_elems, s.total_bits, 64)
+    lut = df11.build_lut(hdr)
+    assert lut.size == LUT_BYTES == int(hdr.bytes_lut)
+    sec = lut[narrow_off(k):narrow_off(k) + narrow_bytes(k)]
+    mtab = sec[: 2 * 2 ** k].view(np.uint16)
+    nl = narrow_long_entries(k)
+    ltab = sec[2 * 2 ** k: 2 * 2 ** k + 2 * nl].view(np.uint16)
+    dtab = sec[2 * 2 ** k + 2 * nl: 2 * 2 ** k + 2 * nl + 8 * 2 ** k].view(np.uint32).reshape(-1, 2)
+    table = _oracle_prefix_decoder(s.code_len)
+    for v in range(2 ** k):
+        bits = format(v, "0%db" % k)
+        codes, _ = _decode_bits(table, bits, None)
+        assert int(mtab[v]) == sum(1 << p for _, p in codes), (v, bits)
+        codes4, used4 = _decode_bits(table, bits, 4)
+        x_, y = int(dtab[v, 0]), int(dtab[v, 1])
+        if not codes4:
+            assert (x_, y) == (0, ESCAPE << 16)
+            continue
+        assert y == (used4 << 16) | (8 * len(codes4))
+        assert len(codes4) == 4 or x_ >> (8 * len(codes4)) == 0
+        for j, (sym, _) in enumerate(codes4):
+            assert (x_ >> (8 * j)) & 0xFF == ((sym >> 1) | (sym << 7)) & 0xFF
+    row = 10 - k   # LutHeader: 8 words, then (long_base, long_count) per narrow K
+    long_base, long_count = (int(v) for v in lut[32 + 8 * row: 40 + 8 * row].view(np.uint32))
+    short_space = sum(1 << (32 - int(l)) for l in s.code_len if 0 < l <= k)
+    assert long_base == short_space >> 12
+    need = -(-((1 << 32) - short_space) // 4096)
+    assert long_count == (need if short_space < (1 << 32) and need <= nl else 0)
+    rng = np.random.default_rng(k)
+    picks = range(long_count) if long_count <= 600 else rng.integers(0, long_count, size=600)
+    for i in picks:
+        bits = format(long_base + int(i), "020b")
+        codes, _ = _decode_bits(table, bits, 1)
+        e = int(ltab[i])
+        if not codes:
+            assert e == 0
+            continue
+        sym, _ = codes[0]
+        length = next(len(c) for c, v in table.items() if v == sym)
+        assert length > k
+        assert e == (((sym >> 1) | (sym << 7)) & 0xFF) | (length << 8)
+
+
 @pytest.mark.parametrize("source", ["outliers", "fibonacci", "matrix_1k"])
 def test_long_code_table_agrees_with_oracle_codes(source):
     """Level 2: entry i of the long table describes the code at the top of the
@@ -227,7 +302,7 @@ def test_long_code_table_agrees_with_oracle_codes(source):
     lut = df11.build_lut(hdr)
     long_base, long_count = (int(v) for v in lut[24:32].view(np.uint32))
     assert 0 < long_count <= 4096
-    ltab = lut[OFF_LONG:LUT_BYTES].view(np.uint16)
+    ltab = lut[OFF_LONG:OFF_NARROW].view(np.uint16)
     table = _oracle_prefix_decoder(s.code_len)
     # the first long prefix is where the codes of more than 12 bits begin
     short_space = sum(1 << (32 - int(l)) for l in s.code_len if 0 < l <= 12)
