@@ -667,16 +667,24 @@ def run_pipeline(args, local_rank: int) -> None:
             if v.dim() == 2:
                 torch.matmul(act[:, : v.shape[1]], v.t())
 
-    def timed(fn, reps=3):
-        fn()
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(reps):
+    def timed_on(st, fn, reps=None):
+        """Median over `reps` passes (each over every block) of the ms per
+        block, events on stream `st` around each pass."""
+        reps = reps or args.pipeline_reps
+        with torch.cuda.stream(st):
             fn()
-        e1.record(stream)
+            torch.cuda.synchronize()
+            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+            for e0, e1 in evs:
+                e0.record(st)
+                fn()
+                e1.record(st)
         torch.cuda.synchronize()
-        return e0.elapsed_time(e1) / (reps * len(streams))
+        per = sorted(e0.elapsed_time(e1) / len(streams) for e0, e1 in evs)
+        return per[len(per) // 2]
+
+    def timed(fn, reps=None):
+        return timed_on(stream, fn, reps)
 
     first = streams[0].views(df11.decompress(streams[0], out=buf[: streams[0].n_elems]))
     res = {"consumer_only": timed(lambda: [consume(first) for _ in streams]),
@@ -701,27 +709,21 @@ def run_pipeline(args, local_rank: int) -> None:
     # first, so the decode's CTAs take what the consumer leaves idle
     hi = torch.cuda.Stream(priority=-100)
     lo = torch.cuda.Stream(priority=0)
-
-    def timed_on(st, fn, reps=3):
-        with torch.cuda.stream(st):
-            fn()
-            torch.cuda.synchronize()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(st)
-            for _ in range(reps):
-                fn()
-            e1.record(st)
-        torch.cuda.synchronize()
-        return e0.elapsed_time(e1) / (reps * len(streams))
-
     for ctas, warps in [(0, 0)] + list(args.pipeline_shapes):
         opts = df11.decode_options(ctas=ctas, max_warps_per_cta=warps) if ctas else None
         pf = df11.BlockPrefetcher(streams, options=opts, decode_stream=lo)
         key = "prefetch_prio_all_sms" if not ctas else f"prefetch_prio_{ctas}x{warps}w"
         res[key] = timed_on(hi, lambda: [consume(views) for _, views in pf])
+    # split: part of the next block on the SMs the consumer leaves idle, the
+    # rest after the consumer (consumer on the high-priority stream)
+    for frac in args.pipeline_split:
+        pf = df11.BlockPrefetcher(streams, decode_stream=lo, split=frac, side_sms=args.side_sms)
+        res[f"prefetch_split_{frac:g}_on_{args.side_sms}_sms"] = timed_on(hi, lambda: [consume(views) for _, views in pf])
     res["serial_hi_stream"] = timed_on(hi, serial)
+    res["serial_again"] = timed(serial)  # drift check: serial timed first and last
     best = min(v for k, v in res.items() if k.startswith("prefetch"))
-    hidden = (res["serial"] - best) / min(res["decode_only"], res["consumer_only"])
+    serial_ms = min(res["serial"], res["serial_again"])
+    hidden = (serial_ms - best) / min(res["decode_only"], res["consumer_only"])
     flops = 2 * args.tokens * sum(cs.n_elems for cs in streams) / len(streams)
     line = {"metric": "decompress-into-consumer, ms per transformer block", "unit": "ms",
             "higher_is_better": False, "n_gpus": 1, "data": "synthetic",
@@ -761,6 +763,11 @@ def main(argv=None):
     ap.add_argument("--pipeline", action="store_true",
                     help="time decompress-into-consumer (BlockPrefetcher) instead of the decode alone")
     ap.add_argument("--pipeline-blocks", type=int, default=4)
+    ap.add_argument("--pipeline-split", type=float, nargs="*", default=[0.2, 0.3, 0.4],
+                    help="fractions of the next block decoded beside the consumer (split prefetch)")
+    ap.add_argument("--side-sms", type=int, default=20, help="SMs of the overlapped decode (split prefetch)")
+    ap.add_argument("--pipeline-reps", type=int, default=9,
+                    help="passes per pipeline variant; the median pass is reported")
     ap.add_argument("--tokens", type=int, default=1024, help="consumer activation rows (--pipeline)")
     ap.add_argument("--pipeline-sms", type=int, nargs="*", default=[16, 32, 64])
     ap.add_argument("--pipeline-shapes", type=lambda v: tuple(int(x) for x in v.split("x")), nargs="*",

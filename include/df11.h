@@ -304,6 +304,11 @@ typedef struct {
                                     decoding a contiguous run of thread blocks --
                                     more CTAs than fit at once simply queue, so
                                     many small CTAs interleave with other kernels */
+    uint32_t block_begin;        /* block_begin = block_end = 0: every thread    */
+    uint32_t block_end;          /* block; else thread blocks [block_begin,
+                                    block_end) only, exactly as
+                                    df11_decompress_blocks (same reads, writes
+                                    only those blocks' output elements)          */
     uint32_t reserved[2];        /* must be zero                                  */
 } df11_decode_options;
 

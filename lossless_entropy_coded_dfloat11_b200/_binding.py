@@ -54,6 +54,8 @@ class DecodeOptions(ctypes.Structure):
         ("max_sms", ctypes.c_uint32),
         ("max_warps_per_cta", ctypes.c_uint32),
         ("ctas", ctypes.c_uint32),
+        ("block_begin", ctypes.c_uint32),
+        ("block_end", ctypes.c_uint32),
         ("reserved", ctypes.c_uint32 * 2),
     ]
 

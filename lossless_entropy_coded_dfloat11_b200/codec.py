@@ -218,9 +218,11 @@ def to_host(cs: CompressedStream) -> dict:
                 block_off=cs.block_off.cpu().numpy().view(np.uint32)[: int(h.n_blocks) + 1])
 
 
-def decode_options(peek_bits: int = 0, max_sms: int = 0, max_warps_per_cta: int = 0, ctas: int = 0):
-    """df11_decode_options (all zero: the library's defaults)."""
-    return B.DecodeOptions(peek_bits, max_sms, max_warps_per_cta, ctas)
+def decode_options(peek_bits: int = 0, max_sms: int = 0, max_warps_per_cta: int = 0, ctas: int = 0,
+                   block_begin: int = 0, block_end: int = 0):
+    """df11_decode_options (all zero: the library's defaults; a block range
+    decodes only those thread blocks, as decompress_blocks)."""
+    return B.DecodeOptions(peek_bits, max_sms, max_warps_per_cta, ctas, block_begin, block_end)
 
 
 def decompress(cs: CompressedStream, out: torch.Tensor | None = None, status: torch.Tensor | None = None,

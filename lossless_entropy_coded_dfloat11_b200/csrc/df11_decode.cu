@@ -1523,7 +1523,7 @@ df11_status decompress_on(const char* fn, bool u8, const df11_header* hdr, const
     return launch_plan(p, a, opt, reinterpret_cast<cudaStream_t>(stream));
 }
 
-constexpr df11_decode_options kDefaultOptions{0, 0, 0, 0, 0, 0};
+constexpr df11_decode_options kDefaultOptions{0, 0, 0, 0, 0, 0, {0, 0}};
 
 }  // namespace
 }  // namespace df11
@@ -1554,6 +1554,9 @@ extern "C" df11_status df11_decompress_opts(const df11_header* hdr, const uint8_
     if (!opt) return fail(DF11_ERR_INVALID, "df11_decompress_opts: null options");
     for (uint32_t r : opt->reserved)
         if (r) return fail(DF11_ERR_INVALID, "df11_decompress_opts: reserved fields must be zero");
+    if (opt->block_begin || opt->block_end)
+        return decompress_on("df11_decompress_opts", symbols_u8 != 0, hdr, d_exp, d_sm, d_gaps, d_block_off, d_lut,
+                             d_out, d_status, *opt, stream, opt->block_begin, opt->block_end);
     return decompress_on("df11_decompress_opts", symbols_u8 != 0, hdr, d_exp, d_sm, d_gaps, d_block_off, d_lut,
                          d_out, d_status, *opt, stream);
 }

@@ -180,11 +180,14 @@ struct RawElems {
 // for every thread), a thread whose elements lie in a later segment looks
 // up its own.
 template <int ES>
-__device__ __forceinline__ RawElems load_raw(const SegTable& sg, uint64_t c0, uint64_t i0, uint64_t n) {
+__device__ __forceinline__ RawElems load_raw(const SegTable& sg, uint64_t c0, uint64_t i0, uint64_t n,
+                                             uint32_t seg_hint = 0xFFFFFFFFu) {
     RawElems r;
     r.direct = false;
     if (i0 < n) {
-        uint32_t seg = find_seg(sg, c0);
+        // the chunk's segment (given, or looked up); threads past its end
+        // look up their own
+        uint32_t seg = seg_hint != 0xFFFFFFFFu ? seg_hint : find_seg(sg, c0);
         if (i0 >= sg.start[seg + 1]) seg = find_seg(sg, i0);
         const uint8_t* p = sg.ptr[seg] + ES * (i0 - sg.start[seg]);
         if (i0 + kEncPerThread <= sg.start[seg + 1] && (reinterpret_cast<uintptr_t>(p) & 15u) == 0) {
@@ -366,9 +369,10 @@ __device__ __forceinline__ unsigned long long look_back(unsigned long long* desc
 }
 
 template <int ES>
-__global__ void __launch_bounds__(kEncThreads) encode_kernel(const __grid_constant__ SegTable sg,
+__global__ void __launch_bounds__(kEncThreads, 3) encode_kernel(const __grid_constant__ SegTable sg,
                                                              const __grid_constant__ CodeTable ct, uint64_t n,
-                                                             uint64_t n_chunks, uint32_t log2_block_bits,
+                                                             uint64_t n_chunks, uint64_t chunks_per_range,
+                                                             uint32_t log2_block_bits,
                                                              unsigned long long* __restrict__ desc,
                                                              uint32_t* __restrict__ ticket, uint32_t* lut_magic,
                                                              uint32_t* __restrict__ exp32, uint8_t* __restrict__ sm,
@@ -387,44 +391,72 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(const __grid_consta
     __syncthreads();
     const uint64_t block_mask = (uint64_t(1) << log2_block_bits) - 1;
     const uint64_t tofs = uint64_t(threadIdx.x) * kEncPerThread;
-    uint64_t c = s_ticket;
-    RawElems next = load_raw<ES>(sg, c * kEncChunk, c * kEncChunk + tofs, n);
-    while (c < n_chunks) {
+    const uint32_t range = s_ticket;
+    const uint64_t c_begin = uint64_t(range) * chunks_per_range;
+    const uint64_t c_end = c_begin + chunks_per_range < n_chunks ? c_begin + chunks_per_range : n_chunks;
+    if (c_begin >= c_end) return;  // (the grid has exactly one range per CTA)
+
+    // the segment holding a chunk's first element, advanced chunk by chunk
+    auto seg_of = [&](uint32_t seg, uint64_t c) {
+        while (seg + 1 < sg.n && c * kEncChunk >= sg.start[seg + 1]) seg++;
+        return seg;
+    };
+    const uint32_t seg0 = find_seg(sg, c_begin * kEncChunk);
+
+    // pass 1: the code bits of this range, read once for the sum
+    uint32_t mine = 0;
+    uint32_t seg = seg0;
+    RawElems next = load_raw<ES>(sg, c_begin * kEncChunk, c_begin * kEncChunk + tofs, n, seg);
+    for (uint64_t c = c_begin; c < c_end; c++) {
         const RawElems cur = next;
+        if (c + 1 < c_end) {
+            seg = seg_of(seg, c + 1);
+            next = load_raw<ES>(sg, (c + 1) * kEncChunk, (c + 1) * kEncChunk + tofs, n, seg);
+        }
         const uint64_t i0 = c * kEncChunk + tofs;
-        __syncthreads();  // everyone has read s_ticket; s_* of the last chunk are free
+        if (i0 < n) {
+            uint32_t w8[kWords<ES>];
+            raw_words<ES>(sg, cur, i0, n, w8);
+            const uint64_t left = n - i0;
+            mine += thread_bits<ES>(sc, w8, left < kEncPerThread ? uint32_t(left) : kEncPerThread);
+        }
+    }
+    uint32_t range_total;
+    block_exclusive_scan<kEncThreads>(mine, s_warp, range_total);
+    // the range's first bit: one look-back per range; every earlier range's
+    // CTA is already running (it holds an earlier ticket) and publishes its
+    // aggregate as soon as its own pass 1 ends
+    if (threadIdx.x < 32) {
+        const unsigned long long pre = look_back(desc, range, range_total, lut_magic);
+        if (threadIdx.x == 0) s_prefix = pre;
+    }
+    __syncthreads();
+    uint64_t S = s_prefix;
+
+    // pass 2: each chunk packed at the running prefix
+    seg = seg0;
+    next = load_raw<ES>(sg, c_begin * kEncChunk, c_begin * kEncChunk + tofs, n, seg);
+    for (uint64_t c = c_begin; c < c_end; c++) {
+        const RawElems cur = next;
+        if (c + 1 < c_end) {
+            seg = seg_of(seg, c + 1);
+            next = load_raw<ES>(sg, (c + 1) * kEncChunk, (c + 1) * kEncChunk + tofs, n, seg);
+        }
+        const uint64_t i0 = c * kEncChunk + tofs;
+        __syncthreads();  // s_words, s_gap, s_warp and s_ev of the last chunk are free
         uint32_t w8[kWords<ES>];
-        uint2 ce[kEncPerThread];  // code (left-aligned) and length of each element
         uint32_t valid = 0, bits = 0;
         if (i0 < n) {
             raw_words<ES>(sg, cur, i0, n, w8);
             const uint64_t left = n - i0;
             valid = left < kEncPerThread ? uint32_t(left) : kEncPerThread;
-#pragma unroll
-            for (int k = 0; k < int(kEncPerThread); k++) {
-                ce[k] = uint32_t(k) < valid ? sc.e[symbol<ES>(w8, k)] : make_uint2(0, 0);
-                bits += ce[k].y;
-            }
+            bits = thread_bits<ES>(sc, w8, valid);
         }
         for (int j = threadIdx.x; j < kPackWords / 4; j += kEncThreads)
             reinterpret_cast<uint4*>(s_words)[j] = make_uint4(0, 0, 0, 0);
         for (int j = threadIdx.x; j < kGapWords; j += kEncThreads) s_gap[j] = 0;
         uint32_t chunk_total;
         const uint32_t my_off = block_exclusive_scan<kEncThreads>(bits, s_warp, chunk_total);
-        if (threadIdx.x < 32) {
-            const unsigned long long pre = look_back(desc, uint32_t(c), chunk_total, lut_magic);
-            // the next ticket only now: a chunk's aggregate must follow its
-            // ticket quickly (a ticket held across this chunk's work would
-            // make the next chunk's look-back wait for all of it)
-            if (threadIdx.x == 0) {
-                s_prefix = pre;
-                s_ticket = atomicAdd(ticket, 1u);
-            }
-        }
-        __syncthreads();
-        const uint64_t nc = s_ticket;
-        next = load_raw<ES>(sg, nc * kEncChunk, nc * kEncChunk + tofs, n);  // in flight during the pack
-        const uint64_t S = s_prefix;
         const uint32_t lead = uint32_t(S & 31u);
         const uint64_t Sb = S & ~block_mask;  // a thread-block (and window) boundary
         // gap fields of this chunk: windows (S >> 6, (S + total - 1) >> 6], at
@@ -448,36 +480,38 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(const __grid_consta
                 block_off[blk_base + br + 1] = uint32_t(i + 1);
             }
         };
-        // Append this thread's codes to the image.  A completed word is OR-ed
-        // in (the first may be shared with the previous thread).  Codes that
-        // cover a window boundary (at most 9 for 16 codes of <= 32 bits) are
-        // only noted in the thread's column of s_ev and handled after the
-        // loop, so the warp does not run that handler on every element.
+        // OR each of this thread's codes into the image at its own bit
+        // position: one shared-memory atomic, a second when the code runs into
+        // the next word -- no per-thread word bookkeeping for the warp to
+        // diverge on (neighbouring threads share boundary words, hence the
+        // atomics).  Codes that cover a window boundary (at most 9 for 16
+        // codes of <= 32 bits) are only noted in the thread's column of s_ev
+        // and handled after the loop.
         if (valid) {
-            const uint32_t q = lead + my_off;  // bit position in the chunk image
-            uint32_t w = q >> 5, fill = q & 31u, cur_word = 0;
+            uint32_t pos = lead + my_off;  // bit position in the chunk image
             uint32_t u = uint32_t(S - Sb) + my_off + 63u;  // relative start + 63
             uint32_t ne = 0;
-            bool first = true;
+            auto pack = [&](auto full_tag) {
+                constexpr bool kFull = decltype(full_tag)::value;  // all kEncPerThread elements valid
 #pragma unroll
-            for (int k = 0; k < int(kEncPerThread); k++) {
-                const uint32_t t = ce[k].x, l = ce[k].y;  // l = 0 past the valid elements
-                cur_word |= t >> fill;
-                const uint32_t spill = __funnelshift_r(0u, t, fill);  // bits that did not fit
-                fill += l;
-                if (fill >= 32u) {
-                    if (first) atomicOr(&s_words[w], cur_word);
-                    else s_words[w] = cur_word;
-                    first = false;
-                    w++;
-                    cur_word = spill;
-                    fill -= 32u;
+                for (int k = 0; k < int(kEncPerThread); k++) {
+                    // code (left-aligned) and length; l = 0, t = 0 past the valid elements
+                    const uint2 e = (kFull || uint32_t(k) < valid) ? sc.e[symbol<ES>(w8, k)] : make_uint2(0, 0);
+                    const uint32_t t = e.x, l = e.y;
+                    const uint32_t wi = pos >> 5, sh = pos & 31u;
+                    atomicOr(&s_words[wi], t >> sh);
+                    const uint32_t spill = __funnelshift_r(0u, t, sh);  // bits that did not fit
+                    if (spill) atomicOr(&s_words[wi + 1], spill);
+                    const uint32_t nu = u + l;
+                    if ((u ^ nu) >= 64u) s_ev[ne++][threadIdx.x] = (u << 10) | (l << 4) | uint32_t(k);
+                    u = nu;
+                    pos += l;
                 }
-                const uint32_t nu = u + l;
-                if ((u ^ nu) >= 64u) s_ev[ne++][threadIdx.x] = (u << 10) | (l << 4) | uint32_t(k);
-                u = nu;
-            }
-            if (fill) atomicOr(&s_words[w], cur_word);
+            };
+            if (valid == kEncPerThread)
+                pack(std::true_type{});
+            else
+                pack(std::false_type{});
             if (gaps32) {
                 for (uint32_t j = 0; j < ne; j++) {
                     const uint32_t e = s_ev[j][threadIdx.x];
@@ -535,7 +569,7 @@ __global__ void __launch_bounds__(kEncThreads) encode_kernel(const __grid_consta
                 }
             }
         }
-        c = nc;
+        S += chunk_total;
     }
 }
 
@@ -706,8 +740,12 @@ df11_status compress_encode(const char* fn, const void* const* d_segs, const df1
         return cuda_fail("clear encode scratch", e);
     uint32_t log2_bb = 6;
     while ((1u << (log2_bb - 6)) < hdr->threads_per_block) log2_bb++;
-    encode_kernel<ES><<<encode_grid(encode_kernel<ES>, chunks), kEncThreads, 0, s>>>(
-        sg, ct, n, chunks, log2_bb, desc, reinterpret_cast<uint32_t*>(desc + chunks),
+    // one contiguous range of chunks per CTA of a full persistent grid
+    const uint64_t slots = encode_grid(encode_kernel<ES>, chunks);
+    const uint64_t per_range = (chunks + slots - 1) / slots;
+    const unsigned grid = unsigned((chunks + per_range - 1) / per_range);
+    encode_kernel<ES><<<grid, kEncThreads, 0, s>>>(
+        sg, ct, n, chunks, per_range, log2_bb, desc, reinterpret_cast<uint32_t*>(desc + chunks),
         static_cast<uint32_t*>(d_lut), reinterpret_cast<uint32_t*>(d_exp), d_sm,
         reinterpret_cast<uint32_t*>(d_gaps), d_block_off, hdr->n_blocks, d_chunk_bit);
     e = cudaGetLastError();

@@ -13,7 +13,7 @@ from __future__ import annotations
 
 import torch
 
-from .codec import CompressedStream, decompress
+from .codec import CompressedStream, decode_options, decompress
 
 
 class BlockPrefetcher:
@@ -33,18 +33,28 @@ class BlockPrefetcher:
                 idle; overrides max_sms
     status      optional int32 device word, OR-ed with DF11_ERR_CORRUPT by a
                 decode that finds its stream inconsistent
+    split       None, or the fraction of block i+1's thread blocks decoded on
+                at most side_sms SMs while the caller works on block i; the
+                rest is decoded on every SM once the caller's work on block i
+                is done.  For consumers that leave SMs idle: cuBLAS's BF16
+                GEMMs on B200 run 128 CTAs, one per SM, on 128 of 148 SMs.
+    side_sms    SMs for the overlapped part (split mode)
     """
 
     def __init__(self, streams: list[CompressedStream], n_buffers: int = 2, max_sms: int | None = None,
                  status: torch.Tensor | None = None, decode_stream: torch.cuda.Stream | None = None,
-                 options=None):
+                 options=None, split: float | None = None, side_sms: int = 20):
         if n_buffers < 2:
             raise ValueError("n_buffers must be at least 2")
         if not streams:
             raise ValueError("no blocks")
         self.streams = list(streams)
+        if split is not None and not 0.0 <= split <= 1.0:
+            raise ValueError("split must lie in [0, 1]")
         self.max_sms = max_sms
         self.options = options
+        self.split = split
+        self.side_sms = side_sms
         self.status = status
         dev = self.streams[0].exp.device
         n_max = max(max(cs.n_elems for cs in self.streams), 1)
@@ -54,13 +64,36 @@ class BlockPrefetcher:
     def __len__(self) -> int:
         return len(self.streams)
 
-    def _launch(self, i: int, free: list) -> torch.cuda.Event:
+    def _decode(self, i: int, options=None) -> None:
+        cs = self.streams[i]
+        slot = i % len(self.buffers)
+        decompress(cs, out=self.buffers[slot][: cs.n_elems], status=self.status, stream=self.decode_stream,
+                   max_sms=None if options is not None else self.max_sms,
+                   options=options if options is not None else self.options)
+
+    def _launch(self, i: int, free: list) -> torch.cuda.Event | None:
+        """Block i's decode (split mode: its first part only); returns the
+        event that marks it ready, or None when a second part follows."""
         slot = i % len(self.buffers)
         if free[slot] is not None:
             self.decode_stream.wait_event(free[slot])
-        cs = self.streams[i]
-        decompress(cs, out=self.buffers[slot][: cs.n_elems], status=self.status, stream=self.decode_stream,
-                   max_sms=self.max_sms, options=self.options)
+        if self.split is None:
+            self._decode(i)
+        else:
+            cut = int(self.streams[i].header.n_blocks * self.split)
+            if cut > 0:
+                self._decode(i, decode_options(max_sms=self.side_sms, block_begin=0, block_end=cut))
+            return None
+        ready = torch.cuda.Event()
+        ready.record(self.decode_stream)
+        return ready
+
+    def _finish(self, i: int) -> torch.cuda.Event:
+        """Split mode: the rest of block i on every SM."""
+        nb = int(self.streams[i].header.n_blocks)
+        cut = int(nb * self.split)
+        if cut < nb:
+            self._decode(i, decode_options(block_begin=cut, block_end=nb))
         ready = torch.cuda.Event()
         ready.record(self.decode_stream)
         return ready
@@ -71,12 +104,18 @@ class BlockPrefetcher:
         self.decode_stream.wait_stream(compute)
         free = [None] * len(self.buffers)
         ready = self._launch(0, free)
+        if ready is None:
+            ready = self._finish(0)
         for i, cs in enumerate(self.streams):
             compute.wait_event(ready)
-            if i + 1 < len(self.streams):
+            nxt = i + 1 < len(self.streams)
+            if nxt:
                 ready = self._launch(i + 1, free)
             slot = i % len(self.buffers)
             yield i, cs.views(self.buffers[slot][: cs.n_elems])
             done = torch.cuda.Event()
             done.record(compute)
             free[slot] = done
+            if nxt and ready is None:  # split: the rest after the caller's work on block i
+                self.decode_stream.wait_event(done)
+                ready = self._finish(i + 1)

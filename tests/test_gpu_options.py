@@ -96,6 +96,30 @@ def test_many_small_ctas_on_a_full_size_block():
     assert cs.kernel_info(options=opts)["grid"] == 4 * 148 * 4
 
 
+@pytest.mark.parametrize("T", [32, 64, 256])
+def test_block_ranges_write_only_their_elements(T):
+    """A block range in the options decodes exactly as df11_decompress_blocks:
+    output elements [off[b0], off[b1]) and nothing else; ranges that tile the
+    stream rebuild it, on any launch shape."""
+    x, cs = oracle_stream_on_gpu(inputs.llama_block(SMALL_BLOCK, seed_base=97), T=T)
+    nb = int(cs.header.n_blocks)
+    off = cs.block_off.cpu().numpy().view(np.uint32)
+    cuts = [0, 1, nb // 3, nb // 3 + 1, nb - 1, nb]
+    out = torch.full((cs.n_elems,), 3.0, dtype=torch.bfloat16, device="cuda")
+    for b0, b1 in zip(cuts[:-1], cuts[1:]):
+        before = u16(out)
+        opts = df11.decode_options(block_begin=b0, block_end=b1, max_sms=7 if b0 % 2 else 0)
+        df11.decompress(cs, out=out, options=opts)
+        torch.cuda.synchronize()
+        after = u16(out)
+        e0, e1 = int(off[b0]), int(off[b1])
+        np.testing.assert_array_equal(after[e0:e1], x[e0:e1])
+        np.testing.assert_array_equal(np.delete(after, np.s_[e0:e1]), np.delete(before, np.s_[e0:e1]))
+    np.testing.assert_array_equal(u16(out), x)
+    with pytest.raises(df11.DF11Error):
+        df11.decompress(cs, out=out, options=df11.decode_options(block_begin=2, block_end=1))
+
+
 def test_u8_streams_take_launch_shapes():
     w = inputs.Workload("q", ["w"], [inputs.quantize_u8(inputs.gaussian((1024, 1024), 0.02, 95))])
     cs = df11.compress_u8([t.cuda() for t in w.tensors])

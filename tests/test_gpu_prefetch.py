@@ -47,8 +47,9 @@ def test_zero_sm_cap_is_rejected():
     assert e.value.code == B.DF11_ERR_INVALID
 
 
-@pytest.mark.parametrize("n_buffers,max_sms", [(2, None), (2, 8), (3, 31)])
-def test_block_prefetcher_overlaps_and_is_exact(n_buffers, max_sms):
+@pytest.mark.parametrize("n_buffers,max_sms,split", [(2, None, None), (2, 8, None), (3, 31, None),
+                                                    (2, None, 0.0), (2, None, 0.35), (3, None, 1.0)])
+def test_block_prefetcher_overlaps_and_is_exact(n_buffers, max_sms, split):
     blocks = [inputs.llama_block(SMALL_BLOCK, seed_base=200 + 16 * b) for b in range(5)]
     streams = [df11.compress([t.cuda() for t in w.tensors], names=w.names) for w in blocks]
     # the oracle agrees with every input (the reference the GPU results are held to)
@@ -58,7 +59,8 @@ def test_block_prefetcher_overlaps_and_is_exact(n_buffers, max_sms):
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     act = torch.randn(64, SMALL_BLOCK["intermediate"], device="cuda").to(torch.bfloat16)
     copies, sums = [], []
-    pf = df11.BlockPrefetcher(streams, n_buffers=n_buffers, max_sms=max_sms, status=status)
+    pf = df11.BlockPrefetcher(streams, n_buffers=n_buffers, max_sms=max_sms, status=status, split=split,
+                              side_sms=5)
     for i, views in pf:
         acc = torch.zeros((), dtype=torch.float32, device="cuda")
         for v in views:
