@@ -480,7 +480,7 @@ def measure(pw: Prepared, steps: int, warmup: int, stream, dev, world: int) -> d
         "launches_per_step": launches, "bit_exact": exact, "bit_exact_scope": scope,
         "compression_ratio": sum(c.compressed_bytes() for c in pw.streams) / pw.out_bytes,
         "threads_per_block": None if pw.chunks else cs0.threads_per_block,
-        "decode_kernel": None if pw.chunks else cs0.kernel_info(pw.u8),
+        "decode_kernel": None if pw.chunks else cs0.kernel_info(pw.u8, pw.options),
         "l2": ("no flush: compressed input + output per step exceed the 126 MB L2" if pw.alg_bytes >= 2 * L2_BYTES
                else f"flushed: a {2 * L2_BYTES >> 20} MiB buffer is written before each step; per-step CUDA "
                     "events time the decode alone"),
@@ -492,8 +492,12 @@ def measure(pw: Prepared, steps: int, warmup: int, stream, dev, world: int) -> d
     }
 
 
-# the workloads measured besides the headline one in a default run
-EXTRA_CONFIGS = ["c4", "c2", "c1", "c5", "edge_one_value", "edge_uniform", "edge_zipf"]
+# the workloads measured besides the headline one in a default run; the
+# last two are the C3 block again, through the independent-chunk container
+# (an ablation of the gap layout) and through the pages' 8-bit first-level
+# table (an ablation of the 12-bit one)
+EXTRA_CONFIGS = ["c4", "c2", "c1", "c5", "edge_one_value", "edge_uniform", "edge_zipf", "c3_chunks", "c3_peek8"]
+EXTRA_VARIANTS = {"c3_chunks": ("c3", dict(chunks=True)), "c3_peek8": ("c3", dict(peek_bits=8))}
 
 
 def run_native(args, rank: int, world: int, local_rank: int) -> None:
@@ -626,9 +630,15 @@ def run_native(args, rank: int, world: int, local_rank: int) -> None:
         for c in EXTRA_CONFIGS:
             if c == args.config:
                 continue
-            other = Prepared(df11, c, rank, dev)
+            base, var = EXTRA_VARIANTS.get(c, (c, {}))
+            opts = df11.decode_options(peek_bits=var["peek_bits"]) if "peek_bits" in var else None
+            other = Prepared(df11, base, rank, dev, chunks=var.get("chunks", False), options=opts)
             rec = measure(other, args.steps, args.warmup, stream, dev, world)
-            line["gpu_launches"] += (args.steps + args.warmup + 1) * rec["launches_per_step"]
+            if var:
+                rec["variant"] = ("independent chunks of 64 elements (start-bit table), no gaps or scan"
+                                  if var.get("chunks") else
+                                  f"first-level table of {var['peek_bits']} bits held in 16 shared-memory copies")
+            rec["gpu_launches"] = args.steps * rec["launches_per_step"]  # in its own timed region
             rec.pop("_elapsed_ms")
             extra[c] = rec
             del other

@@ -1368,7 +1368,17 @@ df11_status shape_of(const Plan& p, uint64_t n_blocks, const df11_decode_options
     return DF11_OK;
 }
 
-df11_status launch_plan(const Plan& p, const DecodeArgs& a, const df11_decode_options& o, cudaStream_t stream) {
+// Forget a kernel's set-up on the current device: the next launch sets its
+// shared-memory limit again.  A device reset, or another context on the same
+// device, loads the module again with the attribute back at its default.
+void forget_setup(const Plan& p) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < kMaxDev)
+        g_info[dev][p.slot].ready.store(0, std::memory_order_release);
+}
+
+df11_status launch_plan(const Plan& p, const DecodeArgs& a, const df11_decode_options& o, cudaStream_t stream,
+                        bool retried = false) {
     Shape sh;
     df11_status st = shape_of(p, a.n_blocks, o, &sh);
     if (st != DF11_OK) return st;
@@ -1389,6 +1399,10 @@ df11_status launch_plan(const Plan& p, const DecodeArgs& a, const df11_decode_op
     cfg.numAttrs = 1;
     cudaError_t e = cudaLaunchKernelExC(&cfg, p.kernel, params);
     if (e == cudaSuccess) e = cudaGetLastError();
+    if (e != cudaSuccess && !retried) {  // a stale set-up: redo it once
+        forget_setup(p);
+        return launch_plan(p, a, o, stream, true);
+    }
     if (e != cudaSuccess) return fail(DF11_ERR_CUDA, "decode launch (%s): %s", p.name, cudaGetErrorString(e));
     return DF11_OK;
 }
@@ -1611,23 +1625,30 @@ extern "C" df11_status df11_decompress_chunked(const df11_header* hdr, const uin
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return fail(DF11_ERR_CUDA, "cudaGetDevice failed");
     LaunchInfo& li = g_info[dev][9];
-    if (!li.ready.load(std::memory_order_acquire)) {
-        cudaError_t e = cudaFuncSetAttribute(decode_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             int(smem));
-        if (e != cudaSuccess) return fail(DF11_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
-        int sms = 0;
-        e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        if (e != cudaSuccess) return fail(DF11_ERR_CUDA, "SM count: %s", cudaGetErrorString(e));
-        li.per_sm = 1;
-        li.sms = sms;
-        li.ready.store(1, std::memory_order_release);
+    for (int attempt = 0;; attempt++) {
+        if (!li.ready.load(std::memory_order_acquire)) {
+            cudaError_t e = cudaFuncSetAttribute(decode_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 int(smem));
+            if (e != cudaSuccess) return fail(DF11_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+            int sms = 0;
+            e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+            if (e != cudaSuccess) return fail(DF11_ERR_CUDA, "SM count: %s", cudaGetErrorString(e));
+            li.per_sm = 1;
+            li.sms = sms;
+            li.ready.store(1, std::memory_order_release);
+        }
+        const uint64_t groups = (uint64_t(a.n_chunks) + 31) / 32;
+        const uint64_t want = (groups + kChunkWarps - 1) / kChunkWarps;
+        const unsigned grid = unsigned(want < uint64_t(li.sms) ? want : uint64_t(li.sms));
+        decode_chunk_kernel<<<grid, kChunkWarps * 32, smem, reinterpret_cast<cudaStream_t>(stream)>>>(a);
+        const cudaError_t e = cudaGetLastError();
+        if (e == cudaSuccess) break;
+        if (attempt == 0) {  // a stale set-up (device reset, another context): redo it once
+            li.ready.store(0, std::memory_order_release);
+            continue;
+        }
+        return fail(DF11_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
     }
-    const uint64_t groups = (uint64_t(a.n_chunks) + 31) / 32;
-    const uint64_t want = (groups + kChunkWarps - 1) / kChunkWarps;
-    const unsigned grid = unsigned(want < uint64_t(li.sms) ? want : uint64_t(li.sms));
-    decode_chunk_kernel<<<grid, kChunkWarps * 32, smem, reinterpret_cast<cudaStream_t>(stream)>>>(a);
-    const cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return fail(DF11_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
     return DF11_OK;
 }
 
