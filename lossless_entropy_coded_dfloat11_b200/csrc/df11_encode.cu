@@ -274,11 +274,11 @@ __device__ __forceinline__ uint32_t thread_bits(const SharedCodes& sc, const uin
 //     over that bit sets off[b] = i + 1.
 // Positions are kept 32-bit relative to S rounded down to a thread-block
 // boundary; a code covers a window boundary exactly when (u >> 6) changes
-// across it, u = relative start + 63, which is one test per element.
+// across it, u = relative start + 63: one test per element marks the code in
+// a bit mask, and the marked codes' gap and offset writes follow the packing
+// loop, their positions read back from shared memory.
 // ---------------------------------------------------------------------------
 constexpr int kPackWords = kEncChunk + 4;  // 32 bits per element at most, plus the misalignment
-// windows a thread's codes can reach into: 16 codes of at most 32 bits
-constexpr int kMaxEvents = (int(kEncPerThread) * 32) / 64 + 1;
 // gap words a chunk can touch: 32 kEncChunk bits -> 512 kEncChunk / 64 + 2 windows of 5 bits
 constexpr int kGapWords = (5 * (int(kEncChunk) * 32 / 64 + 2)) / 32 + 2;
 static_assert(kPackWords % 4 == 0, "image cleared in 16-byte stores");
@@ -369,7 +369,7 @@ __device__ __forceinline__ unsigned long long look_back(unsigned long long* desc
 }
 
 template <int ES>
-__global__ void __launch_bounds__(kEncThreads, 3) encode_kernel(const __grid_constant__ SegTable sg,
+__global__ void __launch_bounds__(kEncThreads, 4) encode_kernel(const __grid_constant__ SegTable sg,
                                                              const __grid_constant__ CodeTable ct, uint64_t n,
                                                              uint64_t n_chunks, uint64_t chunks_per_range,
                                                              uint32_t log2_block_bits,
@@ -382,7 +382,7 @@ __global__ void __launch_bounds__(kEncThreads, 3) encode_kernel(const __grid_con
     __shared__ SharedCodes sc;
     __shared__ __align__(16) uint32_t s_words[kPackWords];
     __shared__ uint32_t s_gap[kGapWords];
-    __shared__ uint32_t s_ev[kMaxEvents][kEncThreads];
+    __shared__ uint32_t s_pos[kEncPerThread][kEncThreads];  // (relative start + 63) << 6 | length
     __shared__ uint32_t s_warp[kEncThreads / 32];
     __shared__ uint32_t s_ticket;
     __shared__ unsigned long long s_prefix;
@@ -443,7 +443,7 @@ __global__ void __launch_bounds__(kEncThreads, 3) encode_kernel(const __grid_con
             next = load_raw<ES>(sg, (c + 1) * kEncChunk, (c + 1) * kEncChunk + tofs, n, seg);
         }
         const uint64_t i0 = c * kEncChunk + tofs;
-        __syncthreads();  // s_words, s_gap, s_warp and s_ev of the last chunk are free
+        __syncthreads();  // s_words, s_gap, s_warp and s_pos of the last chunk are free
         uint32_t w8[kWords<ES>];
         uint32_t valid = 0, bits = 0;
         if (i0 < n) {
@@ -463,13 +463,17 @@ __global__ void __launch_bounds__(kEncThreads, 3) encode_kernel(const __grid_con
         // gap array bits 5w .. 5w + 4; s_gap word 0 = gap array word g0
         const uint64_t g0 = (5 * ((S >> 6) + 1)) >> 5;
         const uint64_t blk_base = Sb >> log2_block_bits;
-        auto window_event = [&](uint32_t r, uint32_t l, uint64_t i) {
+        // gap array bit 5w of window w = Sb / 64 + j, counted from s_gap's
+        // first bit: gap_bit0 + 5 j (small: Sb is at most one thread block,
+        // 64 T bits, before the chunk's first window)
+        const int32_t gap_bit0 = int32_t(int64_t(5 * (Sb >> 6)) - int64_t(32 * g0));
+        auto window_event = [&](uint32_t r, uint32_t l, uint32_t i) {
             if (r & 63u) {
-                const uint64_t w = ((Sb + r) >> 6) + 1;  // the window the code runs into
-                const uint32_t g = uint32_t((Sb + r + l) - 64 * w);
-                const uint64_t gb = 5 * w;
-                const uint32_t sh = uint32_t(gb & 31);
-                const uint32_t k = uint32_t((gb >> 5) - g0);
+                const uint32_t j = (r >> 6) + 1;          // the window the code runs into, from Sb
+                const uint32_t g = r + l - 64 * j;         // its gap
+                const uint32_t gb = uint32_t(gap_bit0 + int32_t(5 * j));
+                const uint32_t sh = gb & 31u;
+                const uint32_t k = gb >> 5;
                 atomicOr(&s_gap[k], g << sh);
                 if (sh > 27) atomicOr(&s_gap[k + 1], g >> (32 - sh));
             }
@@ -484,13 +488,13 @@ __global__ void __launch_bounds__(kEncThreads, 3) encode_kernel(const __grid_con
         // position: one shared-memory atomic, a second when the code runs into
         // the next word -- no per-thread word bookkeeping for the warp to
         // diverge on (neighbouring threads share boundary words, hence the
-        // atomics).  Codes that cover a window boundary (at most 9 for 16
-        // codes of <= 32 bits) are only noted in the thread's column of s_ev
-        // and handled after the loop.
+        // atomics).  Every code's relative start and length go to the
+        // thread's column of s_pos and a bit of `cross` marks the codes that
+        // cover a window boundary; those few are handled after the loop.
         if (valid) {
             uint32_t pos = lead + my_off;  // bit position in the chunk image
             uint32_t u = uint32_t(S - Sb) + my_off + 63u;  // relative start + 63
-            uint32_t ne = 0;
+            uint32_t cross = 0;
             auto pack = [&](auto full_tag) {
                 constexpr bool kFull = decltype(full_tag)::value;  // all kEncPerThread elements valid
 #pragma unroll
@@ -503,7 +507,8 @@ __global__ void __launch_bounds__(kEncThreads, 3) encode_kernel(const __grid_con
                     const uint32_t spill = __funnelshift_r(0u, t, sh);  // bits that did not fit
                     if (spill) atomicOr(&s_words[wi + 1], spill);
                     const uint32_t nu = u + l;
-                    if ((u ^ nu) >= 64u) s_ev[ne++][threadIdx.x] = (u << 10) | (l << 4) | uint32_t(k);
+                    s_pos[k][threadIdx.x] = (u << 6) | l;
+                    cross |= uint32_t((u ^ nu) >= 64u) << k;
                     u = nu;
                     pos += l;
                 }
@@ -513,9 +518,10 @@ __global__ void __launch_bounds__(kEncThreads, 3) encode_kernel(const __grid_con
             else
                 pack(std::false_type{});
             if (gaps32) {
-                for (uint32_t j = 0; j < ne; j++) {
-                    const uint32_t e = s_ev[j][threadIdx.x];
-                    window_event((e >> 10) - 63u, (e >> 4) & 63u, i0 + (e & 15u));
+                for (; cross; cross &= cross - 1) {
+                    const int k = __ffs(cross) - 1;
+                    const uint32_t e = s_pos[k][threadIdx.x];
+                    window_event((e >> 6) - 63u, e & 63u, uint32_t(i0) + uint32_t(k));
                 }
             }
         }
