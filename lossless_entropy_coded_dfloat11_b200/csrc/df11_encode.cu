@@ -245,27 +245,31 @@ __device__ __forceinline__ uint32_t thread_bits(const SharedCodes& sc, const uin
 }
 
 // ---------------------------------------------------------------------------
-// Single-pass encode.  Chunks of kEncChunk elements are handed out in order by
-// an atomic ticket.  A chunk's CTA looks up every element's code, sums the
-// bits per thread and per chunk, and learns the chunk's first bit by a
-// decoupled look-back over per-chunk descriptors (64 bits: a 2-bit state,
-// then a bit count): it publishes its own total as an "aggregate", walks back
-// over its predecessors adding aggregates until it meets an "inclusive" prefix,
-// and publishes its own inclusive prefix.  A predecessor holds an earlier
-// ticket, so it is already running and publishes its aggregate without waiting
-// on anything; every wait here is therefore short, and each is bounded anyway
-// (after kSpinLimit polls the chunk gives up, zeroes the decode tables' magic
-// word -- the decoders then report the stream as corrupt -- and goes on).
+// Encode: one persistent grid; CTA r (by an atomic ticket, so that every
+// lower ticket's CTA is already running) takes a contiguous range of chunks
+// of kEncChunk elements, 16 per thread.
+//   pass 1: every element's code length, summed over the range (one read of
+//     the input);
+//   look-back: the range's first stream bit by a decoupled look-back over
+//     per-range descriptors (64 bits: a 2-bit state, then a bit count): the
+//     CTA publishes its total as an "aggregate", walks back over its
+//     predecessors adding aggregates until it meets an "inclusive" prefix, and
+//     publishes its own inclusive prefix.  A predecessor holds an earlier
+//     ticket, so it is running and publishes its aggregate without waiting on
+//     anything; every wait is bounded anyway (after kSpinLimit polls the
+//     range gives up and raises an abort flag, which marks the stream's
+//     decode tables invalid once they are uploaded -- the decoders then
+//     report the stream as corrupt);
+//   pass 2: chunk by chunk, the input read again, each thread's bit offset
+//     by a CTA scan, and the chunk packed at the running prefix.
 //
-// Packing, for a chunk starting at stream bit S.  Each thread appends its
-// codes to a register word with funnel shifts; its first word (which it may
-// share with the previous thread) and its last, partial word (shared with the
-// next) are OR-ed into a shared-memory image of the chunk, the words in
-// between are stored.  The image's interior words are then stored to
-// EncodedExponent and its two boundary words, shared with the neighbouring
-// chunks, are OR-ed into global memory.  The same pass writes the
-// sign+mantissa bytes, the gaps and the thread blocks' output positions from
-// each code's start bit s and length l:
+// Packing a chunk that starts at stream bit S: every code is OR-ed into a
+// shared-memory image of the chunk at its bit position (shared-memory
+// atomics; a code may run into the next word).  The image's interior words
+// are then stored to EncodedExponent and its two boundary words, shared with
+// the neighbouring chunks, are OR-ed into global memory.  The same pass
+// writes the sign+mantissa bytes, the gaps and the thread blocks' output
+// positions from each code's start bit s and length l:
 //   * a code that starts inside window w-1 and runs into window w sets
 //     gap[w] = s + l - 64w (gaps of windows that begin exactly at a code start
 //     stay 0); the chunk's gap fields are assembled in shared memory and
@@ -308,7 +312,7 @@ constexpr int kLookRounds = 4;
 constexpr int kLookBack = 32 * kLookRounds;
 
 __device__ __forceinline__ unsigned long long look_back(unsigned long long* desc, uint32_t c, uint32_t total,
-                                                        uint32_t* lut_magic) {
+                                                        uint32_t* abort_flag) {
     const uint32_t lane = threadIdx.x & 31u;
     if (c == 0) {
         if (lane == 0) publish(desc, kDescInclusive | total);
@@ -347,12 +351,13 @@ __device__ __forceinline__ unsigned long long look_back(unsigned long long* desc
         }
         if (stall) {
             ++spins;
-            // never expected: give up, mark the stream bad; once one chunk
-            // has given up, the others stop waiting too
+            // never expected: give up and raise the abort flag (the stream
+            // is then marked bad, mark_if_aborted); once one range has
+            // given up, the others stop waiting too
             const bool abort = spins >= kSpinLimit ||
-                               ((spins & 63u) == 0 && *reinterpret_cast<volatile uint32_t*>(lut_magic) == 0u);
+                               ((spins & 63u) == 0 && *reinterpret_cast<volatile uint32_t*>(abort_flag) != 0u);
             if (abort) {
-                if (lane == 0) atomicExch(lut_magic, 0u);
+                if (lane == 0) atomicExch(abort_flag, 1u);
                 return prefix;
             }
             __nanosleep(32);
@@ -374,7 +379,7 @@ __global__ void __launch_bounds__(kEncThreads, 4) encode_kernel(const __grid_con
                                                              uint64_t n_chunks, uint64_t chunks_per_range,
                                                              uint32_t log2_block_bits,
                                                              unsigned long long* __restrict__ desc,
-                                                             uint32_t* __restrict__ ticket, uint32_t* lut_magic,
+                                                             uint32_t* __restrict__ ticket, uint32_t* abort_flag,
                                                              uint32_t* __restrict__ exp32, uint8_t* __restrict__ sm,
                                                              uint32_t* __restrict__ gaps32,
                                                              uint32_t* __restrict__ block_off, uint64_t n_blocks,
@@ -382,7 +387,9 @@ __global__ void __launch_bounds__(kEncThreads, 4) encode_kernel(const __grid_con
     __shared__ SharedCodes sc;
     __shared__ __align__(16) uint32_t s_words[kPackWords];
     __shared__ uint32_t s_gap[kGapWords];
-    __shared__ uint32_t s_pos[kEncPerThread][kEncThreads];  // (relative start + 63) << 6 | length
+    // per element: BF16, the code's start relative to its thread's first bit;
+    // 8-bit symbols, (start relative to Sb + 63) << 6 | length
+    __shared__ uint32_t s_pos[kEncPerThread][kEncThreads];
     __shared__ uint32_t s_warp[kEncThreads / 32];
     __shared__ uint32_t s_ticket;
     __shared__ unsigned long long s_prefix;
@@ -427,7 +434,7 @@ __global__ void __launch_bounds__(kEncThreads, 4) encode_kernel(const __grid_con
     // CTA is already running (it holds an earlier ticket) and publishes its
     // aggregate as soon as its own pass 1 ends
     if (threadIdx.x < 32) {
-        const unsigned long long pre = look_back(desc, range, range_total, lut_magic);
+        const unsigned long long pre = look_back(desc, range, range_total, abort_flag);
         if (threadIdx.x == 0) s_prefix = pre;
     }
     __syncthreads();
@@ -446,11 +453,34 @@ __global__ void __launch_bounds__(kEncThreads, 4) encode_kernel(const __grid_con
         __syncthreads();  // s_words, s_gap, s_warp and s_pos of the last chunk are free
         uint32_t w8[kWords<ES>];
         uint32_t valid = 0, bits = 0;
+        uint32_t xhi = 0, xlo = 0;  // BF16: the thread's codes in a row, right-aligned (the last 64 bits)
         if (i0 < n) {
             raw_words<ES>(sg, cur, i0, n, w8);
             const uint64_t left = n - i0;
             valid = left < kEncPerThread ? uint32_t(left) : kEncPerThread;
-            bits = thread_bits<ES>(sc, w8, valid);
+            if constexpr (ES == 2) {
+                // one lookup per code: its start relative to the thread's
+                // first bit to s_pos, the code appended to xhi:xlo
+                auto gather = [&](auto full_tag) {
+                    constexpr bool kFull = decltype(full_tag)::value;
+#pragma unroll
+                    for (int k = 0; k < int(kEncPerThread); k++) {
+                        // code (left-aligned) and length; 0, 0 past the valid elements
+                        const uint2 e = (kFull || uint32_t(k) < valid) ? sc.e[symbol<ES>(w8, k)] : make_uint2(0, 0);
+                        s_pos[k][threadIdx.x] = bits;
+                        const uint32_t r = __funnelshift_r(e.x, 0u, 32u - e.y);  // right-aligned (l = 32: e.x)
+                        xhi = __funnelshift_lc(xlo, xhi, e.y);
+                        xlo = __funnelshift_lc(0u, xlo, e.y) | r;
+                        bits += e.y;
+                    }
+                };
+                if (valid == kEncPerThread)
+                    gather(std::true_type{});
+                else
+                    gather(std::false_type{});
+            } else {
+                bits = thread_bits<ES>(sc, w8, valid);
+            }
         }
         for (int j = threadIdx.x; j < kPackWords / 4; j += kEncThreads)
             reinterpret_cast<uint4*>(s_words)[j] = make_uint4(0, 0, 0, 0);
@@ -484,39 +514,84 @@ __global__ void __launch_bounds__(kEncThreads, 4) encode_kernel(const __grid_con
                 block_off[blk_base + br + 1] = uint32_t(i + 1);
             }
         };
-        // OR each of this thread's codes into the image at its own bit
+        // Per-code packing: OR each code into the image at its own bit
         // position: one shared-memory atomic, a second when the code runs into
-        // the next word -- no per-thread word bookkeeping for the warp to
-        // diverge on (neighbouring threads share boundary words, hence the
-        // atomics).  Every code's relative start and length go to the
-        // thread's column of s_pos and a bit of `cross` marks the codes that
-        // cover a window boundary; those few are handled after the loop.
-        if (valid) {
-            uint32_t pos = lead + my_off;  // bit position in the chunk image
+        // the next word (neighbouring threads share boundary words, hence the
+        // atomics).
+        auto pack_codes = [&](uint32_t pos, auto full_tag, auto note) {
+            constexpr bool kFull = decltype(full_tag)::value;  // all kEncPerThread elements valid
+#pragma unroll
+            for (int k = 0; k < int(kEncPerThread); k++) {
+                // code (left-aligned) and length; l = 0, t = 0 past the valid elements
+                const uint2 e = (kFull || uint32_t(k) < valid) ? sc.e[symbol<ES>(w8, k)] : make_uint2(0, 0);
+                const uint32_t t = e.x, l = e.y;
+                const uint32_t wi = pos >> 5, sh = pos & 31u;
+                atomicOr(&s_words[wi], t >> sh);
+                const uint32_t spill = __funnelshift_r(0u, t, sh);  // bits that did not fit
+                if (spill) atomicOr(&s_words[wi + 1], spill);
+                note(k, l);
+                pos += l;
+            }
+        };
+        if constexpr (ES == 2) {
+            if (valid) {
+                const uint32_t pos = lead + my_off;  // bit position in the chunk image
+                if (bits <= 64) {
+                    // the whole row of codes at once: at most three words
+                    if (bits) {
+                        const unsigned long long y = ((static_cast<unsigned long long>(xhi) << 32) | xlo)
+                                                     << (64 - bits);
+                        const uint32_t yh = uint32_t(y >> 32), yl = uint32_t(y);
+                        const uint32_t wi = pos >> 5, sh = pos & 31u;
+                        atomicOr(&s_words[wi], yh >> sh);
+                        const uint32_t w1 = __funnelshift_r(yl, yh, sh);
+                        if (w1) atomicOr(&s_words[wi + 1], w1);
+                        const uint32_t w2 = __funnelshift_r(0u, yl, sh);
+                        if (w2) atomicOr(&s_words[wi + 2], w2);
+                    }
+                } else {  // rare: more than 64 code bits in 16 elements
+                    auto none = [](int, uint32_t) {};
+                    if (valid == kEncPerThread)
+                        pack_codes(pos, std::true_type{}, none);
+                    else
+                        pack_codes(pos, std::false_type{}, none);
+                }
+                if (gaps32) {
+                    // every window boundary 64 m (relative to Sb) in the
+                    // thread's bits [A, A + bits) is covered by one code: the
+                    // last one starting at or before it (binary search over
+                    // the thread's starts; starts past the valid elements
+                    // equal bits)
+                    const uint32_t A = uint32_t(S - Sb) + my_off;
+                    for (uint32_t m = (A + 63) >> 6; 64 * m < A + bits; m++) {
+                        const uint32_t q = 64 * m - A;
+                        uint32_t k = 0;
+                        if (s_pos[k + 8][threadIdx.x] <= q) k += 8;
+                        if (s_pos[k + 4][threadIdx.x] <= q) k += 4;
+                        if (s_pos[k + 2][threadIdx.x] <= q) k += 2;
+                        if (s_pos[k + 1][threadIdx.x] <= q) k += 1;
+                        const uint32_t a = s_pos[k][threadIdx.x];
+                        const uint32_t b = k + 1 < kEncPerThread ? s_pos[k + 1][threadIdx.x] : bits;
+                        window_event(A + a, b - a, uint32_t(i0) + k);
+                    }
+                }
+            }
+        } else if (valid) {
+            // Every code's relative start and length go to the thread's
+            // column of s_pos and a bit of `cross` marks the codes that cover
+            // a window boundary; those few are handled after the loop.
             uint32_t u = uint32_t(S - Sb) + my_off + 63u;  // relative start + 63
             uint32_t cross = 0;
-            auto pack = [&](auto full_tag) {
-                constexpr bool kFull = decltype(full_tag)::value;  // all kEncPerThread elements valid
-#pragma unroll
-                for (int k = 0; k < int(kEncPerThread); k++) {
-                    // code (left-aligned) and length; l = 0, t = 0 past the valid elements
-                    const uint2 e = (kFull || uint32_t(k) < valid) ? sc.e[symbol<ES>(w8, k)] : make_uint2(0, 0);
-                    const uint32_t t = e.x, l = e.y;
-                    const uint32_t wi = pos >> 5, sh = pos & 31u;
-                    atomicOr(&s_words[wi], t >> sh);
-                    const uint32_t spill = __funnelshift_r(0u, t, sh);  // bits that did not fit
-                    if (spill) atomicOr(&s_words[wi + 1], spill);
-                    const uint32_t nu = u + l;
-                    s_pos[k][threadIdx.x] = (u << 6) | l;
-                    cross |= uint32_t((u ^ nu) >= 64u) << k;
-                    u = nu;
-                    pos += l;
-                }
+            auto note = [&](int k, uint32_t l) {
+                const uint32_t nu = u + l;
+                s_pos[k][threadIdx.x] = (u << 6) | l;
+                cross |= uint32_t((u ^ nu) >= 64u) << k;
+                u = nu;
             };
             if (valid == kEncPerThread)
-                pack(std::true_type{});
+                pack_codes(lead + my_off, std::true_type{}, note);
             else
-                pack(std::false_type{});
+                pack_codes(lead + my_off, std::false_type{}, note);
             if (gaps32) {
                 for (; cross; cross &= cross - 1) {
                     const int k = __ffs(cross) - 1;
@@ -579,6 +654,12 @@ __global__ void __launch_bounds__(kEncThreads, 4) encode_kernel(const __grid_con
     }
 }
 
+// After the decode tables' upload: a stream whose encode gave up (see
+// look_back) gets a zero table magic, so that every decode of it fails.
+__global__ void mark_if_aborted(const uint32_t* abort_flag, uint32_t* lut_magic) {
+    if (*abort_flag) *lut_magic = 0u;
+}
+
 // Persistent grid for an encode kernel: as many CTAs as can be resident on
 // every SM at once.
 template <typename Kernel>
@@ -595,7 +676,8 @@ unsigned encode_grid(Kernel kernel, uint64_t chunks) {
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // Encode scratch: one look-back descriptor per chunk, then the chunk ticket
-// (zeroed by every encode call before its kernel).
+// and the abort flag, 8 bytes each (zeroed by every encode call before its
+// kernel).
 constexpr uint64_t encode_scratch_bytes(uint64_t chunks) { return 8 * (chunks + 2); }
 
 struct Workspace {
@@ -685,7 +767,8 @@ df11_status compress_plan(const void* const* d_segs, const uint64_t* seg_counts,
     return df11_header_init(hdr, len, n, bits, threads_per_block, max_code_len, seg_counts, n_segs);
 }
 
-// Table upload, clears, then the chunk-bits, scan and bit-pack kernels.
+// Clears and the encode kernel, then the decode tables: built on the host
+// while the kernel runs, uploaded after it.
 // d_sm is written for BF16 input (ES = 2) only.
 // With d_chunk_bit (the independent-chunk table instead of Gaps and block
 // offsets) d_gaps and d_block_off are not written and may be null.
@@ -717,15 +800,9 @@ df11_status compress_encode(const char* fn, const void* const* d_segs, const df1
     CodeTable ct;
     std::memcpy(ct.len, hdr->code_len, 256);
     if (!canonical_codes(hdr->code_len, ct.code)) return fail(DF11_ERR_INVALID, "code lengths overflow");
-    // decode tables are built in this thread's own host buffer (no heap)
-    static thread_local unsigned char lut[kLutBytes];
-    st = df11_build_lut(hdr, lut, sizeof(lut));
-    if (st != DF11_OK) return st;
 
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     cudaError_t e;
-    if ((e = cudaMemcpyAsync(d_lut, lut, kLutBytes, cudaMemcpyHostToDevice, s)) != cudaSuccess)
-        return cuda_fail("table upload", e);
     if ((e = cudaMemsetAsync(d_exp, 0, hdr->bytes_exp, s)) != cudaSuccess) return cuda_fail("clear exp", e);
     if (!chunked) {
         if ((e = cudaMemsetAsync(d_gaps, 0, hdr->bytes_gaps, s)) != cudaSuccess) return cuda_fail("clear gaps", e);
@@ -738,24 +815,38 @@ df11_status compress_encode(const char* fn, const void* const* d_segs, const df1
             (e = cudaMemsetAsync(d_sm + sm_tail, 0, hdr->bytes_sm - sm_tail, s)) != cudaSuccess)
             return cuda_fail("clear sm tail", e);
     }
-    if (n == 0) return DF11_OK;
-
     const uint64_t chunks = (n + kEncChunk - 1) / kEncChunk;
     if (chunks >= (uint64_t(1) << 31)) return fail(DF11_ERR_TOO_LARGE, "too many chunks");
-    if ((e = cudaMemsetAsync(desc, 0, encode_scratch_bytes(chunks), s)) != cudaSuccess)
-        return cuda_fail("clear encode scratch", e);
-    uint32_t log2_bb = 6;
-    while ((1u << (log2_bb - 6)) < hdr->threads_per_block) log2_bb++;
-    // one contiguous range of chunks per CTA of a full persistent grid
-    const uint64_t slots = encode_grid(encode_kernel<ES>, chunks);
-    const uint64_t per_range = (chunks + slots - 1) / slots;
-    const unsigned grid = unsigned((chunks + per_range - 1) / per_range);
-    encode_kernel<ES><<<grid, kEncThreads, 0, s>>>(
-        sg, ct, n, chunks, per_range, log2_bb, desc, reinterpret_cast<uint32_t*>(desc + chunks),
-        static_cast<uint32_t*>(d_lut), reinterpret_cast<uint32_t*>(d_exp), d_sm,
-        reinterpret_cast<uint32_t*>(d_gaps), d_block_off, hdr->n_blocks, d_chunk_bit);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_fail("encode launch", e);
+    uint32_t* abort_flag = reinterpret_cast<uint32_t*>(desc + chunks + 1);
+    if (n) {
+        if ((e = cudaMemsetAsync(desc, 0, encode_scratch_bytes(chunks), s)) != cudaSuccess)
+            return cuda_fail("clear encode scratch", e);
+        uint32_t log2_bb = 6;
+        while ((1u << (log2_bb - 6)) < hdr->threads_per_block) log2_bb++;
+        // one contiguous range of chunks per CTA of a full persistent grid
+        const uint64_t slots = encode_grid(encode_kernel<ES>, chunks);
+        const uint64_t per_range = (chunks + slots - 1) / slots;
+        const unsigned grid = unsigned((chunks + per_range - 1) / per_range);
+        encode_kernel<ES><<<grid, kEncThreads, 0, s>>>(
+            sg, ct, n, chunks, per_range, log2_bb, desc, reinterpret_cast<uint32_t*>(desc + chunks), abort_flag,
+            reinterpret_cast<uint32_t*>(d_exp), d_sm, reinterpret_cast<uint32_t*>(d_gaps), d_block_off,
+            hdr->n_blocks, d_chunk_bit);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail("encode launch", e);
+    }
+    // The decode tables are built while the encode kernel runs, in this
+    // thread's own host buffer (no heap; an asynchronous copy from pageable
+    // memory has taken the bytes when it returns), and uploaded after it.
+    static thread_local unsigned char lut[kLutBytes];
+    st = df11_build_lut(hdr, lut, sizeof(lut));
+    if (st != DF11_OK) return st;
+    if ((e = cudaMemcpyAsync(d_lut, lut, kLutBytes, cudaMemcpyHostToDevice, s)) != cudaSuccess)
+        return cuda_fail("table upload", e);
+    if (n) {
+        mark_if_aborted<<<1, 1, 0, s>>>(abort_flag, static_cast<uint32_t*>(d_lut));
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail("abort mark launch", e);
+    }
     return DF11_OK;
 }
 
