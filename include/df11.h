@@ -84,7 +84,11 @@ typedef struct {
     uint64_t n_blocks;           /* ceil(n_threads / T)                        */
     uint8_t code_len[256];       /* code length per exponent value, 0 = absent */
     uint32_t n_segments;         /* matrices in the stream, 1..64              */
-    uint32_t reserved;
+    uint32_t plan_token;         /* set by df11_compress_plan (0 otherwise):
+                                    names the per-range histograms it left in
+                                    its workspace; df11_compress_encode with
+                                    that workspace uses them instead of
+                                    counting code bits in a pass of its own    */
     uint64_t seg_elem_off[DF11_MAX_SEGMENTS + 1]; /* segment k = elements
                                     [seg_elem_off[k], seg_elem_off[k+1])       */
     uint64_t bytes_exp;          /* EncodedExponent buffer size                */
@@ -149,7 +153,11 @@ df11_status df11_compress_plan(const void* const* d_segs, const uint64_t* seg_co
 /* Compress, step 2 of 2: bit-pack kernel.  Writes EncodedExponent,
  * PackedSignMantissa, Gaps and block offsets into caller buffers of at least
  * the header's sizes, and the decode tables into d_lut (hdr->bytes_lut).
- * Asynchronous on `stream`; d_segs must hold the data the plan saw. */
+ * Asynchronous on `stream`; d_segs must hold the data the plan saw.  With
+ * the workspace the plan filled (and its header) the kernel takes each
+ * range's code bits from the plan's per-range histograms; any other
+ * workspace of the needed size gives the same output, reading the input
+ * once more to count them. */
 df11_status df11_compress_encode(const void* const* d_segs, const df11_header* hdr,
                                  void* d_workspace, uint64_t workspace_bytes, uint8_t* d_exp,
                                  uint8_t* d_sm, uint8_t* d_gaps, uint32_t* d_block_off,
@@ -157,7 +165,7 @@ df11_status df11_compress_encode(const void* const* d_segs, const df11_header* h
 
 /* Compress, step 2 of 2, without allocating: the pages have no counterpart
  * to this entry point.  It writes exactly what df11_compress_encode writes,
- * but keeps its scratch (per-chunk bit totals and start bits) in a fixed
+ * but keeps its scratch (look-back descriptors, chunk ticket, abort flag) in a fixed
  * array inside the library instead of a caller workspace.  It is for callers
  * that cannot allocate device memory at compress time: serving engines that
  * hand all of HBM to their own pools at start-up and forbid later cudaMalloc

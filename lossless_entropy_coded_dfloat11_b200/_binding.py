@@ -37,7 +37,7 @@ class Header(ctypes.Structure):
         ("n_blocks", ctypes.c_uint64),
         ("code_len", ctypes.c_uint8 * 256),
         ("n_segments", ctypes.c_uint32),
-        ("reserved", ctypes.c_uint32),
+        ("plan_token", ctypes.c_uint32),
         ("seg_elem_off", ctypes.c_uint64 * (DF11_MAX_SEGMENTS + 1)),
         ("bytes_exp", ctypes.c_uint64),
         ("bytes_sm", ctypes.c_uint64),

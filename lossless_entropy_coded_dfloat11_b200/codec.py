@@ -407,8 +407,10 @@ def compress_u8(tensors, names=None, threads_per_block: int = DEFAULT_THREADS_PE
            ws.numel(), ctypes.byref(hdr), sh)
     ln = np.frombuffer(bytes(hdr.code_len), dtype=np.uint8)
     if threads_per_block in (64, 128) and n and ln[ln > 0].min() == 1:
+        token = hdr.plan_token  # the plan's per-range histograms do not depend on T
         hdr = make_header(ln, int(hdr.n_elems), int(hdr.total_bits), 32, max_code_len,
                           [t.numel() for t in segs])
+        hdr.plan_token = token
     exp = torch.empty(int(hdr.bytes_exp), dtype=torch.uint8, device=device)
     gaps = torch.empty(int(hdr.bytes_gaps), dtype=torch.uint8, device=device)
     off = torch.empty(int(hdr.n_blocks) + 1, dtype=torch.int32, device=device)

@@ -10,6 +10,8 @@
 // position per thread block).
 #include <cuda_runtime.h>
 
+#include <atomic>
+#include <chrono>
 #include <cstring>
 #include <type_traits>
 #include <vector>
@@ -37,11 +39,24 @@ struct CodeTable {
 
 // ---------------------------------------------------------------------------
 // Histogram of the symbols of every segment in one launch (the exponent field
-// of BF16 elements, or 8-bit symbols); per-warp shared-memory histograms,
-// flushed into 64-bit global counters.  The CTAs stride over each segment's
-// 16-byte vectors in turn, two vectors in flight per thread.
+// of BF16 elements, or 8-bit symbols); per-warp shared-memory histograms.
+// CTA r counts elements [r E, (r + 1) E) of the concatenated segments -- the
+// elements of the encode kernel's range r -- and stores that range's
+// histogram (32-bit counts) besides adding it to the 64-bit global counters;
+// the encode kernel then needs no pass over its range to learn the range's
+// code bits.  Within each segment's part of the range the threads read
+// 16-byte vectors, two in flight per thread, and the unaligned ends element
+// by element.
 // ---------------------------------------------------------------------------
 constexpr int kHistThreads = 256;
+
+// Which plan left the per-range histograms in a workspace, and for which
+// partition (written by the histogram kernel, checked by the encode kernel).
+struct RangeTag {
+    uint32_t token;     // the plan's token (never 0), also in df11_header.plan_token
+    uint32_t n_ranges;
+    uint64_t range_chunks;
+};
 
 template <int ES>
 __device__ __forceinline__ void count16(uint32_t* mine, const uint4 q) {
@@ -59,37 +74,54 @@ __device__ __forceinline__ void count16(uint32_t* mine, const uint4 q) {
 }
 
 template <int ES>
+__device__ __forceinline__ uint32_t symbol_at(const uint8_t* p, uint64_t i) {
+    if constexpr (ES == 2) return uint32_t(reinterpret_cast<const uint16_t*>(p)[i] >> 7) & 0xFFu;
+    else return uint32_t(p[i]);
+}
+
+template <int ES>
 __global__ void __launch_bounds__(kHistThreads) histogram_kernel(const __grid_constant__ SegTable sg,
-                                                                 unsigned long long* __restrict__ hist) {
+                                                                 uint64_t range_elems,
+                                                                 unsigned long long* __restrict__ hist,
+                                                                 uint32_t* __restrict__ range_hist,
+                                                                 RangeTag* __restrict__ tag, const RangeTag tag_value) {
     __shared__ uint32_t sh[kHistThreads / 32][256];
     uint32_t* mine = sh[threadIdx.x >> 5];
     for (int i = threadIdx.x; i < (kHistThreads / 32) * 256; i += kHistThreads) (&sh[0][0])[i] = 0;
     __syncthreads();
-    const uint64_t stride = uint64_t(gridDim.x) * kHistThreads;
-    const uint64_t tid = uint64_t(blockIdx.x) * kHistThreads + threadIdx.x;
+    const uint64_t n = sg.start[sg.n];
+    const uint64_t e0 = uint64_t(blockIdx.x) * range_elems;
+    const uint64_t e1 = e0 + range_elems < n ? e0 + range_elems : n;
+    constexpr uint64_t kPerVec = 16 / ES;
     for (uint32_t seg = 0; seg < sg.n; seg++) {
-        const uint64_t cnt = sg.start[seg + 1] - sg.start[seg];
-        const uint8_t* p = sg.ptr[seg];
-        const uint64_t nvec = cnt * ES / 16;
+        const uint64_t s0 = sg.start[seg], s1 = sg.start[seg + 1];
+        if (s1 <= e0 || s0 >= e1) continue;
+        // this range's part of the segment, local element indices [a, b)
+        const uint64_t a = (e0 > s0 ? e0 : s0) - s0, b = (e1 < s1 ? e1 : s1) - s0;
+        const uint8_t* p = sg.ptr[seg];  // 16-byte aligned
+        uint64_t va = (a + kPerVec - 1) / kPerVec, vb = b / kPerVec;
+        if (va > vb) va = vb = 0;  // no whole vector: every element below goes one by one
+        const uint64_t h1 = va < vb ? va * kPerVec : b;  // scalar head [a, h1), tail [t0, b)
+        const uint64_t t0 = va < vb ? vb * kPerVec : b;
+        for (uint64_t i = a + threadIdx.x; i < h1; i += kHistThreads) atomicAdd(&mine[symbol_at<ES>(p, i)], 1u);
+        for (uint64_t i = t0 + threadIdx.x; i < b; i += kHistThreads) atomicAdd(&mine[symbol_at<ES>(p, i)], 1u);
         const uint4* xv = reinterpret_cast<const uint4*>(p);
-        uint64_t v = tid;
-        for (; v + stride < nvec; v += 2 * stride) {
-            const uint4 a = __ldcs(xv + v), b = __ldcs(xv + v + stride);
-            count16<ES>(mine, a);
-            count16<ES>(mine, b);
+        uint64_t v = va + threadIdx.x;
+        for (; v + kHistThreads < vb; v += 2 * kHistThreads) {
+            const uint4 x = __ldcs(xv + v), y = __ldcs(xv + v + kHistThreads);
+            count16<ES>(mine, x);
+            count16<ES>(mine, y);
         }
-        if (v < nvec) count16<ES>(mine, __ldcs(xv + v));
-        for (uint64_t i = nvec * 16 / ES + tid; i < cnt; i += stride) {
-            const uint32_t x = ES == 2 ? uint32_t(reinterpret_cast<const uint16_t*>(p)[i] >> 7) : uint32_t(p[i]);
-            atomicAdd(&mine[x & 0xFFu], 1u);
-        }
+        if (v < vb) count16<ES>(mine, __ldcs(xv + v));
     }
     __syncthreads();
     for (int s = threadIdx.x; s < 256; s += kHistThreads) {
-        uint64_t t = 0;
+        uint32_t t = 0;
         for (int w = 0; w < kHistThreads / 32; w++) t += sh[w][s];
+        range_hist[uint64_t(blockIdx.x) * 256 + s] = t;
         if (t) atomicAdd(hist + s, (unsigned long long)t);
     }
+    if (blockIdx.x == 0 && threadIdx.x == 0) *tag = tag_value;
 }
 
 // Element i of the concatenated segments.
@@ -383,7 +415,9 @@ __global__ void __launch_bounds__(kEncThreads, 4) encode_kernel(const __grid_con
                                                              uint32_t* __restrict__ exp32, uint8_t* __restrict__ sm,
                                                              uint32_t* __restrict__ gaps32,
                                                              uint32_t* __restrict__ block_off, uint64_t n_blocks,
-                                                             uint32_t* __restrict__ chunk_bit) {
+                                                             uint32_t* __restrict__ chunk_bit,
+                                                             const uint32_t* __restrict__ range_hist,
+                                                             const RangeTag* __restrict__ tag, const RangeTag expect) {
     __shared__ SharedCodes sc;
     __shared__ __align__(16) uint32_t s_words[kPackWords];
     __shared__ uint32_t s_gap[kGapWords];
@@ -410,29 +444,45 @@ __global__ void __launch_bounds__(kEncThreads, 4) encode_kernel(const __grid_con
     };
     const uint32_t seg0 = find_seg(sg, c_begin * kEncChunk);
 
-    // pass 1: the code bits of this range, read once for the sum
+    // the code bits of this range: from the plan's histogram of the range
+    // when the workspace holds this partition's (thread s: symbol s), else
+    // pass 1 reads the range once for the sum
     uint32_t mine = 0;
-    uint32_t seg = seg0;
-    RawElems next = load_raw<ES>(sg, c_begin * kEncChunk, c_begin * kEncChunk + tofs, n, seg);
-    for (uint64_t c = c_begin; c < c_end; c++) {
-        const RawElems cur = next;
-        if (c + 1 < c_end) {
-            seg = seg_of(seg, c + 1);
-            next = load_raw<ES>(sg, (c + 1) * kEncChunk, (c + 1) * kEncChunk + tofs, n, seg);
-        }
-        const uint64_t i0 = c * kEncChunk + tofs;
-        if (i0 < n) {
-            uint32_t w8[kWords<ES>];
-            raw_words<ES>(sg, cur, i0, n, w8);
-            const uint64_t left = n - i0;
-            mine += thread_bits<ES>(sc, w8, left < kEncPerThread ? uint32_t(left) : kEncPerThread);
+    bool from_hist = false;
+    if (expect.token != 0) {
+        const RangeTag have = *tag;
+        from_hist = have.token == expect.token && have.n_ranges == expect.n_ranges &&
+                    have.range_chunks == expect.range_chunks;
+    }
+    if (from_hist) {
+        static_assert(kEncThreads == 256, "one thread per symbol");
+        mine = range_hist[uint64_t(range) * 256 + threadIdx.x] * sc.e[threadIdx.x].y;
+    } else {
+        uint32_t seg = seg0;
+        RawElems next = load_raw<ES>(sg, c_begin * kEncChunk, c_begin * kEncChunk + tofs, n, seg);
+        for (uint64_t c = c_begin; c < c_end; c++) {
+            const RawElems cur = next;
+            if (c + 1 < c_end) {
+                seg = seg_of(seg, c + 1);
+                next = load_raw<ES>(sg, (c + 1) * kEncChunk, (c + 1) * kEncChunk + tofs, n, seg);
+            }
+            const uint64_t i0 = c * kEncChunk + tofs;
+            if (i0 < n) {
+                uint32_t w8[kWords<ES>];
+                raw_words<ES>(sg, cur, i0, n, w8);
+                const uint64_t left = n - i0;
+                mine += thread_bits<ES>(sc, w8, left < kEncPerThread ? uint32_t(left) : kEncPerThread);
+            }
         }
     }
+    // pass 2's first loads go out before the look-back
+    uint32_t seg = seg0;
+    RawElems next = load_raw<ES>(sg, c_begin * kEncChunk, c_begin * kEncChunk + tofs, n, seg);
     uint32_t range_total;
     block_exclusive_scan<kEncThreads>(mine, s_warp, range_total);
     // the range's first bit: one look-back per range; every earlier range's
     // CTA is already running (it holds an earlier ticket) and publishes its
-    // aggregate as soon as its own pass 1 ends
+    // aggregate as soon as it has its range's bits
     if (threadIdx.x < 32) {
         const unsigned long long pre = look_back(desc, range, range_total, abort_flag);
         if (threadIdx.x == 0) s_prefix = pre;
@@ -441,8 +491,6 @@ __global__ void __launch_bounds__(kEncThreads, 4) encode_kernel(const __grid_con
     uint64_t S = s_prefix;
 
     // pass 2: each chunk packed at the running prefix
-    seg = seg0;
-    next = load_raw<ES>(sg, c_begin * kEncChunk, c_begin * kEncChunk + tofs, n, seg);
     for (uint64_t c = c_begin; c < c_end; c++) {
         const RawElems cur = next;
         if (c + 1 < c_end) {
@@ -669,8 +717,31 @@ unsigned encode_grid(Kernel kernel, uint64_t chunks) {
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kEncThreads, 0) != cudaSuccess || per_sm < 1)
         per_sm = 1;
-    const uint64_t want = uint64_t(sms) * uint64_t(per_sm);
+    uint64_t want = uint64_t(sms) * uint64_t(per_sm);
+    if (want > kMaxEncRanges) want = kMaxEncRanges;
     return unsigned(chunks < want ? chunks : want);
+}
+
+// The encode kernel's partition of `chunks` chunks: one contiguous range of
+// range_chunks chunks per CTA of a full persistent grid (the last range may
+// be shorter).  The plan's histogram kernel counts by the same ranges.
+template <int ES>
+RangeTag encode_partition(uint64_t chunks) {
+    RangeTag t{0u, 0u, 0u};
+    if (!chunks) return t;
+    const uint64_t slots = encode_grid(encode_kernel<ES>, chunks);
+    t.range_chunks = (chunks + slots - 1) / slots;
+    t.n_ranges = uint32_t((chunks + t.range_chunks - 1) / t.range_chunks);
+    return t;
+}
+
+// A fresh nonzero token per plan (an odd stride visits every 32-bit value).
+uint32_t next_plan_token() {
+    static std::atomic<uint32_t> counter{
+        uint32_t(std::chrono::steady_clock::now().time_since_epoch().count()) | 1u};
+    uint32_t t;
+    do t = counter.fetch_add(0x9E3779B9u); while (t == 0);
+    return t;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -682,7 +753,9 @@ constexpr uint64_t encode_scratch_bytes(uint64_t chunks) { return 8 * (chunks + 
 
 struct Workspace {
     unsigned long long* hist;
+    RangeTag* tag;
     unsigned long long* desc;
+    uint32_t* range_hist;
 };
 
 df11_status carve(void* ws, uint64_t ws_bytes, uint64_t n_elems, Workspace* w) {
@@ -696,8 +769,9 @@ df11_status carve(void* ws, uint64_t ws_bytes, uint64_t n_elems, Workspace* w) {
     const uint64_t chunks = (n_elems + kEncChunk - 1) / kEncChunk;
     uint8_t* p = static_cast<uint8_t*>(ws);
     w->hist = reinterpret_cast<unsigned long long*>(p);
-    (void)chunks;
-    w->desc = reinterpret_cast<unsigned long long*>(p + 2048);
+    w->tag = reinterpret_cast<RangeTag*>(p + kWsTagOff);
+    w->desc = reinterpret_cast<unsigned long long*>(p + kWsDescOff);
+    w->range_hist = reinterpret_cast<uint32_t*>(p + ws_range_hist_off(chunks));
     return DF11_OK;
 }
 
@@ -727,7 +801,8 @@ df11_status build_segtable(const void* const* d_segs, const uint64_t* counts, ui
     return DF11_OK;
 }
 
-// Histogram kernels (one launch per segment), host code builder, header.
+// Histogram kernel (one launch; a histogram per encode range too), host code
+// builder, header.
 template <int ES>
 df11_status compress_plan(const void* const* d_segs, const uint64_t* seg_counts, uint32_t n_segs,
                           uint32_t threads_per_block, uint32_t max_code_len, void* d_workspace,
@@ -743,14 +818,12 @@ df11_status compress_plan(const void* const* d_segs, const uint64_t* seg_counts,
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     cudaError_t e = cudaMemsetAsync(w.hist, 0, 2048, s);
     if (e != cudaSuccess) return cuda_fail("histogram clear", e);
-    int dev = 0, sms = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    uint32_t token = 0;
     if (n) {
-        const uint64_t vec_blocks = (n * ES / 16 + kHistThreads - 1) / kHistThreads;
-        uint64_t grid = vec_blocks < uint64_t(4 * sms) ? vec_blocks : uint64_t(4 * sms);
-        if (grid == 0) grid = 1;
-        histogram_kernel<ES><<<unsigned(grid), kHistThreads, 0, s>>>(sg, w.hist);
+        RangeTag tag = encode_partition<ES>((n + kEncChunk - 1) / kEncChunk);
+        tag.token = token = next_plan_token();
+        histogram_kernel<ES><<<tag.n_ranges, kHistThreads, 0, s>>>(sg, tag.range_chunks * kEncChunk, w.hist,
+                                                                   w.range_hist, w.tag, tag);
     }
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail("histogram launch", e);
@@ -764,7 +837,9 @@ df11_status compress_plan(const void* const* d_segs, const uint64_t* seg_counts,
     if (st != DF11_OK) return st;
     uint64_t bits = 0;
     for (int v = 0; v < 256; v++) bits += hist[v] * len[v];
-    return df11_header_init(hdr, len, n, bits, threads_per_block, max_code_len, seg_counts, n_segs);
+    st = df11_header_init(hdr, len, n, bits, threads_per_block, max_code_len, seg_counts, n_segs);
+    if (st == DF11_OK) hdr->plan_token = token;
+    return st;
 }
 
 // Clears and the encode kernel, then the decode tables: built on the host
@@ -774,7 +849,8 @@ df11_status compress_plan(const void* const* d_segs, const uint64_t* seg_counts,
 // offsets) d_gaps and d_block_off are not written and may be null.
 template <int ES>
 df11_status compress_encode(const char* fn, const void* const* d_segs, const df11_header* hdr,
-                            unsigned long long* desc, uint8_t* d_exp, uint8_t* d_sm,
+                            unsigned long long* desc, const uint32_t* range_hist, const RangeTag* tag,
+                            uint8_t* d_exp, uint8_t* d_sm,
                             uint8_t* d_gaps, uint32_t* d_block_off, void* d_lut, void* stream,
                             uint32_t* d_chunk_bit = nullptr) {
     df11_status st = check_header(hdr);
@@ -823,14 +899,15 @@ df11_status compress_encode(const char* fn, const void* const* d_segs, const df1
             return cuda_fail("clear encode scratch", e);
         uint32_t log2_bb = 6;
         while ((1u << (log2_bb - 6)) < hdr->threads_per_block) log2_bb++;
-        // one contiguous range of chunks per CTA of a full persistent grid
-        const uint64_t slots = encode_grid(encode_kernel<ES>, chunks);
-        const uint64_t per_range = (chunks + slots - 1) / slots;
-        const unsigned grid = unsigned((chunks + per_range - 1) / per_range);
-        encode_kernel<ES><<<grid, kEncThreads, 0, s>>>(
-            sg, ct, n, chunks, per_range, log2_bb, desc, reinterpret_cast<uint32_t*>(desc + chunks), abort_flag,
-            reinterpret_cast<uint32_t*>(d_exp), d_sm, reinterpret_cast<uint32_t*>(d_gaps), d_block_off,
-            hdr->n_blocks, d_chunk_bit);
+        // one contiguous range of chunks per CTA of a full persistent grid;
+        // the plan's per-range histograms are used when the workspace holds
+        // this header's plan for this partition (the kernel compares tags)
+        RangeTag expect = encode_partition<ES>(chunks);
+        expect.token = range_hist && tag ? hdr->plan_token : 0u;
+        encode_kernel<ES><<<expect.n_ranges, kEncThreads, 0, s>>>(
+            sg, ct, n, chunks, expect.range_chunks, log2_bb, desc, reinterpret_cast<uint32_t*>(desc + chunks),
+            abort_flag, reinterpret_cast<uint32_t*>(d_exp), d_sm, reinterpret_cast<uint32_t*>(d_gaps),
+            d_block_off, hdr->n_blocks, d_chunk_bit, range_hist, tag, expect);
         e = cudaGetLastError();
         if (e != cudaSuccess) return cuda_fail("encode launch", e);
     }
@@ -869,8 +946,8 @@ extern "C" df11_status df11_compress_encode(const void* const* d_segs, const df1
     Workspace w{};
     const df11_status st = carve(d_workspace, workspace_bytes, hdr ? hdr->n_elems : 0, &w);
     if (st != DF11_OK) return st;
-    return compress_encode<2>("df11_compress_encode", d_segs, hdr, w.desc, d_exp, d_sm, d_gaps,
-                              d_block_off, d_lut, stream);
+    return compress_encode<2>("df11_compress_encode", d_segs, hdr, w.desc, w.range_hist, w.tag, d_exp, d_sm,
+                              d_gaps, d_block_off, d_lut, stream);
 }
 
 extern "C" df11_status df11_compress_plan_u8(const void* const* d_segs, const uint64_t* seg_counts,
@@ -888,13 +965,13 @@ extern "C" df11_status df11_compress_encode_u8(const void* const* d_segs, const 
     Workspace w{};
     const df11_status st = carve(d_workspace, workspace_bytes, hdr ? hdr->n_elems : 0, &w);
     if (st != DF11_OK) return st;
-    return compress_encode<1>("df11_compress_encode_u8", d_segs, hdr, w.desc, d_exp,
+    return compress_encode<1>("df11_compress_encode_u8", d_segs, hdr, w.desc, w.range_hist, w.tag, d_exp,
                               nullptr, d_gaps, d_block_off, d_lut, stream);
 }
 
 // ---------------------------------------------------------------------------
 // Encode without any allocation: the same kernels as df11_compress_encode,
-// with their scratch (per-chunk bit totals and chunk start bits) in a
+// with their scratch (look-back descriptors, chunk ticket, abort flag) in a
 // fixed-size array that lives in the library's own device memory.  For
 // callers that cannot allocate device memory when they compress: serving
 // engines that hand all of HBM to their own pools at start-up and forbid
@@ -944,7 +1021,7 @@ extern "C" df11_status df11_compress_encode_static(const void* const* d_segs, co
     st = static_scratch_address(&scratch);
     if (st != DF11_OK) return st;
     return compress_encode<2>("df11_compress_encode_static", d_segs, hdr, static_cast<unsigned long long*>(scratch),
-                              d_exp, d_sm,
+                              nullptr, nullptr, d_exp, d_sm,
                               d_gaps, d_block_off, d_lut, stream);
 }
 
@@ -957,6 +1034,6 @@ extern "C" df11_status df11_compress_encode_chunked(const void* const* d_segs, c
     Workspace w{};
     const df11_status st = carve(d_workspace, workspace_bytes, hdr ? hdr->n_elems : 0, &w);
     if (st != DF11_OK) return st;
-    return compress_encode<2>("df11_compress_encode_chunked", d_segs, hdr, w.desc, d_exp,
+    return compress_encode<2>("df11_compress_encode_chunked", d_segs, hdr, w.desc, w.range_hist, w.tag, d_exp,
                               d_sm, nullptr, nullptr, d_lut, stream, d_chunk_bit);
 }

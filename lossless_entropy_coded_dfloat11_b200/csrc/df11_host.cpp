@@ -332,9 +332,7 @@ df11_status df11_build_lut(const df11_header* hdr, void* h_lut, uint64_t cap) {
 df11_status df11_compress_workspace_size(uint64_t n_elems, uint64_t* bytes) {
     if (!bytes) return fail(DF11_ERR_INVALID, "df11_compress_workspace_size: null pointer");
     const uint64_t chunks = (n_elems + kEncChunk - 1) / kEncChunk;
-    // histogram (256 x u64), then one look-back descriptor (u64) per chunk and
-    // the chunk ticket
-    *bytes = 2048 + align16(8 * (chunks + 2)) + 64;
+    *bytes = ws_bytes(chunks);
     return DF11_OK;
 }
 

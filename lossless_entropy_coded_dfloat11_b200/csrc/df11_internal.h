@@ -112,6 +112,20 @@ df11_status fail(df11_status st, const char* fmt, ...);
 constexpr uint32_t kEncChunk = 4096;       // elements per bit-pack CTA
 constexpr uint32_t kEncThreads = 256;      // threads per bit-pack CTA
 constexpr uint32_t kEncPerThread = kEncChunk / kEncThreads;
+// At most this many CTAs (chunk ranges) in an encode grid; the workspace holds
+// one 256-entry histogram per range.
+constexpr uint32_t kMaxEncRanges = 2048;
+// Workspace layout of the compress entry points, in bytes: the global
+// histogram (256 x u64), the range tag, the look-back descriptors, chunk
+// ticket and abort flag (8 (chunks + 2)), then the per-range histograms
+// (256 x u32 each).
+constexpr uint64_t kWsTagOff = 2048;
+constexpr uint64_t kWsDescOff = kWsTagOff + 64;
+inline uint64_t ws_range_hist_off(uint64_t chunks) { return kWsDescOff + ((8 * (chunks + 2) + 15) & ~uint64_t(15)); }
+inline uint64_t ws_bytes(uint64_t chunks) {
+    const uint64_t ranges = chunks < kMaxEncRanges ? chunks : kMaxEncRanges;
+    return ws_range_hist_off(chunks) + 1024 * ranges + 64;
+}
 // Independent-chunk variant of the container: one 32-bit start bit per
 // kIndChunk elements replaces Gaps and block offsets.
 constexpr uint32_t kIndChunk = 64;
