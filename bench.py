@@ -327,9 +327,10 @@ def run_reference(args, rank: int, world: int) -> None:
 
 def time_compress(df11, w, repeats: int, u8: bool = False, chunks: bool = False) -> dict:
     """Wall-clock time of the public compress call on device-resident BF16
-    tensors (histogram kernel, host code build, table upload, bit-pack
-    kernels), synchronised on both sides; the median of `repeats` calls after
-    one untimed call."""
+    tensors (histogram kernel with per-range counts, host code build, encode
+    kernel with the decode tables built on the host meanwhile and uploaded
+    after it), synchronised on both sides; the median of `repeats` calls
+    after one untimed call."""
     import torch
     times = []
     for r in range(repeats + 1):
@@ -346,8 +347,9 @@ def time_compress(df11, w, repeats: int, u8: bool = False, chunks: bool = False)
             "ms": t * 1e3,
             "repeats": repeats, "elements": sum(x.numel() for x in w.tensors),
             "what": f"df11.{'compress_u8' if u8 else 'compress'} on device-resident "
-                    f"{'uint8' if u8 else 'BF16'} tensors: histogram kernel, host package-merge and "
-                    "table build, bit-pack kernels; median wall clock, synchronised"}
+                    f"{'uint8' if u8 else 'BF16'} tensors: histogram kernel (per-range counts), host "
+                    "package-merge, encode kernel (decode tables built on the host meanwhile, uploaded "
+                    "after it); median wall clock, synchronised"}
 
 
 def step_stats(per_step_ms: list[float]) -> dict:
