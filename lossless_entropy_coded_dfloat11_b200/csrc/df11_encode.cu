@@ -45,7 +45,7 @@ struct CodeTable {
 // histogram (32-bit counts) besides adding it to the 64-bit global counters;
 // the encode kernel then needs no pass over its range to learn the range's
 // code bits.  Within each segment's part of the range the threads read
-// 16-byte vectors, two in flight per thread, and the unaligned ends element
+// 16-byte vectors, four in flight per thread, and the unaligned ends element
 // by element.
 // ---------------------------------------------------------------------------
 constexpr int kHistThreads = 256;
@@ -107,12 +107,14 @@ __global__ void __launch_bounds__(kHistThreads) histogram_kernel(const __grid_co
         for (uint64_t i = t0 + threadIdx.x; i < b; i += kHistThreads) atomicAdd(&mine[symbol_at<ES>(p, i)], 1u);
         const uint4* xv = reinterpret_cast<const uint4*>(p);
         uint64_t v = va + threadIdx.x;
-        for (; v + kHistThreads < vb; v += 2 * kHistThreads) {
-            const uint4 x = __ldcs(xv + v), y = __ldcs(xv + v + kHistThreads);
-            count16<ES>(mine, x);
-            count16<ES>(mine, y);
+        for (; v + 3 * kHistThreads < vb; v += 4 * kHistThreads) {
+            uint4 x[4];
+#pragma unroll
+            for (int k = 0; k < 4; k++) x[k] = __ldcs(xv + v + k * kHistThreads);
+#pragma unroll
+            for (int k = 0; k < 4; k++) count16<ES>(mine, x[k]);
         }
-        if (v < vb) count16<ES>(mine, __ldcs(xv + v));
+        for (; v < vb; v += kHistThreads) count16<ES>(mine, __ldcs(xv + v));
     }
     __syncthreads();
     for (int s = threadIdx.x; s < 256; s += kHistThreads) {
@@ -186,13 +188,17 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* s
 // exponent in every lane would serialise in the constant cache.)
 // ---------------------------------------------------------------------------
 struct SharedCodes {
-    uint2 e[256];  // x = code left-aligned in 32 bits, y = its length (0 = absent)
+    // x = the code, right-aligned for BF16 input (appended to a register
+    // row), left-aligned in 32 bits for 8-bit symbols (OR-ed in place);
+    // y = its length (0 = absent)
+    uint2 e[256];
 };
 
+template <int ES>
 __device__ __forceinline__ void stage_codes(SharedCodes& sc, const CodeTable& ct) {
     for (int v = threadIdx.x; v < 256; v += blockDim.x) {
         const uint32_t l = ct.len[v];
-        sc.e[v] = make_uint2(l ? ct.code[v] << (32u - l) : 0u, l);
+        sc.e[v] = make_uint2(ES == 2 ? ct.code[v] : (l ? ct.code[v] << (32u - l) : 0u), l);
     }
 }
 
@@ -427,7 +433,7 @@ __global__ void __launch_bounds__(kEncThreads, 4) encode_kernel(const __grid_con
     __shared__ uint32_t s_warp[kEncThreads / 32];
     __shared__ uint32_t s_ticket;
     __shared__ unsigned long long s_prefix;
-    stage_codes(sc, ct);
+    stage_codes<ES>(sc, ct);
     if (threadIdx.x == 0) s_ticket = atomicAdd(ticket, 1u);
     __syncthreads();
     const uint64_t block_mask = (uint64_t(1) << log2_block_bits) - 1;
@@ -513,12 +519,11 @@ __global__ void __launch_bounds__(kEncThreads, 4) encode_kernel(const __grid_con
                     constexpr bool kFull = decltype(full_tag)::value;
 #pragma unroll
                     for (int k = 0; k < int(kEncPerThread); k++) {
-                        // code (left-aligned) and length; 0, 0 past the valid elements
+                        // code and length; 0, 0 past the valid elements
                         const uint2 e = (kFull || uint32_t(k) < valid) ? sc.e[symbol<ES>(w8, k)] : make_uint2(0, 0);
                         s_pos[k][threadIdx.x] = bits;
-                        const uint32_t r = __funnelshift_r(e.x, 0u, 32u - e.y);  // right-aligned (l = 32: e.x)
                         xhi = __funnelshift_lc(xlo, xhi, e.y);
-                        xlo = __funnelshift_lc(0u, xlo, e.y) | r;
+                        xlo = __funnelshift_lc(0u, xlo, e.y) | e.x;  // e.x right-aligned
                         bits += e.y;
                     }
                 };
@@ -570,9 +575,10 @@ __global__ void __launch_bounds__(kEncThreads, 4) encode_kernel(const __grid_con
             constexpr bool kFull = decltype(full_tag)::value;  // all kEncPerThread elements valid
 #pragma unroll
             for (int k = 0; k < int(kEncPerThread); k++) {
-                // code (left-aligned) and length; l = 0, t = 0 past the valid elements
+                // code, left-aligned, and length; l = 0, t = 0 past the valid elements
                 const uint2 e = (kFull || uint32_t(k) < valid) ? sc.e[symbol<ES>(w8, k)] : make_uint2(0, 0);
-                const uint32_t t = e.x, l = e.y;
+                const uint32_t l = e.y;
+                const uint32_t t = ES == 2 ? __funnelshift_l(0u, e.x, 32u - l) : e.x;  // l = 32: shift 0
                 const uint32_t wi = pos >> 5, sh = pos & 31u;
                 atomicOr(&s_words[wi], t >> sh);
                 const uint32_t spill = __funnelshift_r(0u, t, sh);  // bits that did not fit
@@ -674,12 +680,28 @@ __global__ void __launch_bounds__(kEncThreads, 4) encode_kernel(const __grid_con
         __syncthreads();
         const uint32_t nwords = (lead + chunk_total + 31) >> 5;
         const uint64_t W0 = S >> 5;
-        for (uint32_t j = threadIdx.x; j < nwords; j += kEncThreads) {
-            const uint32_t v = __byte_perm(s_words[j], 0, 0x0123);  // MSB-first bytes
-            if (j == 0 || j == nwords - 1) {
-                if (v) atomicOr(exp32 + W0 + j, v);
-            } else {
-                exp32[W0 + j] = v;
+        auto word = [&](uint32_t j) { return __byte_perm(s_words[j], 0, 0x0123); };  // MSB-first bytes
+        // the first and last words are shared with the neighbouring chunks
+        if (threadIdx.x == 0 || (threadIdx.x == 32 && nwords > 1)) {
+            const uint32_t j = threadIdx.x == 0 ? 0u : nwords - 1;
+            const uint32_t v = word(j);
+            if (v) atomicOr(exp32 + W0 + j, v);
+        }
+        // the words between: 16-byte stores from the first one at a 16-byte
+        // boundary of EncodedExponent, single words before and after
+        if (nwords > 2) {
+            const uint32_t jb = nwords - 1;                                // interior [1, jb)
+            const uint32_t ja = 1u + ((4u - uint32_t((W0 + 1) & 3u)) & 3u);  // W0 + ja is 4-word aligned
+            const uint32_t groups = ja < jb ? (jb - ja) / 4 : 0u;
+            const uint32_t jv = ja + 4 * groups;
+            if (threadIdx.x >= 64 && threadIdx.x < 70) {  // at most 3 words before, 3 after
+                const uint32_t k = threadIdx.x - 64;
+                const uint32_t j = k < 3 ? 1 + k : jv + (k - 3);
+                if (k < 3 ? j < min(ja, jb) : j < jb) exp32[W0 + j] = word(j);
+            }
+            for (uint32_t g = threadIdx.x; g < groups; g += kEncThreads) {
+                const uint32_t j = ja + 4 * g;
+                *reinterpret_cast<uint4*>(exp32 + W0 + j) = make_uint4(word(j), word(j + 1), word(j + 2), word(j + 3));
             }
         }
         if (gaps32) {
