@@ -152,7 +152,9 @@ def compress(tensors, names=None, threads_per_block: int = DEFAULT_THREADS_PER_B
              stream=None) -> CompressedStream:
     """Compress one BF16 tensor, or a list (a transformer block) into one
     stream with a shared code table: histogram kernel, host code builder,
-    bit-pack kernel.  Synchronises the stream once (histogram readback)."""
+    encode kernel (the decode tables are built on the host while it runs).
+    Synchronises the stream once for the histogram readback, and again at
+    the end, before the workspace is released."""
     segs = _as_segments(tensors)
     device = segs[0].device
     n = sum(t.numel() for t in segs)

@@ -1,7 +1,7 @@
-// DF11 compression on the GPU: exponent histogram, then (after the host has
-// built the code) per-chunk code-bit totals, their prefix sum, and the
-// bit-pack kernel that writes EncodedExponent, PackedSignMantissa, Gaps and
-// the per-thread-block output positions.
+// DF11 compression on the GPU: the exponent histogram (also per range of the
+// encode grid), then, after the host has built the code, one encode kernel
+// that finds each range's first stream bit and writes EncodedExponent,
+// PackedSignMantissa, Gaps and the per-thread-block output positions.
 //
 // Format: "DFloat11: compressao sem perda para inferencia em GPU que reduz
 // LLMs para 70% do tamanho", sections "O formato DFloat11" (Huffman-coded
@@ -286,8 +286,9 @@ __device__ __forceinline__ uint32_t thread_bits(const SharedCodes& sc, const uin
 // Encode: one persistent grid; CTA r (by an atomic ticket, so that every
 // lower ticket's CTA is already running) takes a contiguous range of chunks
 // of kEncChunk elements, 16 per thread.
-//   pass 1: every element's code length, summed over the range (one read of
-//     the input);
+//   the range's code bits: the dot product of the range's histogram (left
+//     by the plan's histogram kernel) with the code lengths, or, without
+//     that histogram, a first pass summing every element's code length;
 //   look-back: the range's first stream bit by a decoupled look-back over
 //     per-range descriptors (64 bits: a 2-bit state, then a bit count): the
 //     CTA publishes its total as an "aggregate", walks back over its
@@ -298,8 +299,8 @@ __device__ __forceinline__ uint32_t thread_bits(const SharedCodes& sc, const uin
 //     range gives up and raises an abort flag, which marks the stream's
 //     decode tables invalid once they are uploaded -- the decoders then
 //     report the stream as corrupt);
-//   pass 2: chunk by chunk, the input read again, each thread's bit offset
-//     by a CTA scan, and the chunk packed at the running prefix.
+//   pack: chunk by chunk, each thread's bit offset by a CTA scan, and the
+//     chunk packed at the running prefix.
 //
 // Packing a chunk that starts at stream bit S: every code is OR-ed into a
 // shared-memory image of the chunk at its bit position (shared-memory
@@ -452,7 +453,7 @@ __global__ void __launch_bounds__(kEncThreads, 4) encode_kernel(const __grid_con
 
     // the code bits of this range: from the plan's histogram of the range
     // when the workspace holds this partition's (thread s: symbol s), else
-    // pass 1 reads the range once for the sum
+    // a first pass reads the range once for the sum
     uint32_t mine = 0;
     bool from_hist = false;
     if (expect.token != 0) {
@@ -481,7 +482,7 @@ __global__ void __launch_bounds__(kEncThreads, 4) encode_kernel(const __grid_con
             }
         }
     }
-    // pass 2's first loads go out before the look-back
+    // the pack's first loads go out before the look-back
     uint32_t seg = seg0;
     RawElems next = load_raw<ES>(sg, c_begin * kEncChunk, c_begin * kEncChunk + tofs, n, seg);
     uint32_t range_total;
@@ -496,7 +497,7 @@ __global__ void __launch_bounds__(kEncThreads, 4) encode_kernel(const __grid_con
     __syncthreads();
     uint64_t S = s_prefix;
 
-    // pass 2: each chunk packed at the running prefix
+    // pack: each chunk at the running prefix
     for (uint64_t c = c_begin; c < c_end; c++) {
         const RawElems cur = next;
         if (c + 1 < c_end) {
