@@ -426,12 +426,14 @@ __global__ void __launch_bounds__(kEncThreads, 4) encode_kernel(const __grid_con
                                                              const uint32_t* __restrict__ range_hist,
                                                              const RangeTag* __restrict__ tag, const RangeTag expect) {
     __shared__ SharedCodes sc;
-    __shared__ __align__(16) uint32_t s_words[kPackWords];
-    __shared__ uint32_t s_gap[kGapWords];
+    // 8-bit symbols: the chunk's image and gap fields are assembled here
+    // (BF16 rows go to global memory directly)
+    __shared__ __align__(16) uint32_t s_words[ES == 1 ? kPackWords : 4];
+    __shared__ uint32_t s_gap[ES == 1 ? kGapWords : 1];
     // per element: BF16, the code's start relative to its thread's first bit;
     // 8-bit symbols, (start relative to Sb + 63) << 6 | length
     __shared__ uint32_t s_pos[kEncPerThread][kEncThreads];
-    __shared__ uint32_t s_warp[kEncThreads / 32];
+    __shared__ uint32_t s_warp[2][kEncThreads / 32];  // scan partials, two chunks apart
     __shared__ uint32_t s_ticket;
     __shared__ unsigned long long s_prefix;
     stage_codes<ES>(sc, ct);
@@ -486,7 +488,7 @@ __global__ void __launch_bounds__(kEncThreads, 4) encode_kernel(const __grid_con
     uint32_t seg = seg0;
     RawElems next = load_raw<ES>(sg, c_begin * kEncChunk, c_begin * kEncChunk + tofs, n, seg);
     uint32_t range_total;
-    block_exclusive_scan<kEncThreads>(mine, s_warp, range_total);
+    block_exclusive_scan<kEncThreads>(mine, s_warp[0], range_total);
     // the range's first bit: one look-back per range; every earlier range's
     // CTA is already running (it holds an earlier ticket) and publishes its
     // aggregate as soon as it has its range's bits
@@ -505,7 +507,11 @@ __global__ void __launch_bounds__(kEncThreads, 4) encode_kernel(const __grid_con
             next = load_raw<ES>(sg, (c + 1) * kEncChunk, (c + 1) * kEncChunk + tofs, n, seg);
         }
         const uint64_t i0 = c * kEncChunk + tofs;
-        __syncthreads();  // s_words, s_gap, s_warp and s_pos of the last chunk are free
+        // 8-bit symbols: s_words, s_gap and s_warp of the last chunk are free.
+        // BF16 needs no barrier here: s_pos is the thread's own column, and
+        // the scan alternates between two s_warp rows (a warp writes a row
+        // again only after every warp has passed the scan in between).
+        if constexpr (ES == 1) __syncthreads();
         uint32_t w8[kWords<ES>];
         uint32_t valid = 0, bits = 0;
         uint32_t xhi = 0, xlo = 0;  // BF16: the thread's codes in a row, right-aligned (the last 64 bits)
@@ -536,11 +542,14 @@ __global__ void __launch_bounds__(kEncThreads, 4) encode_kernel(const __grid_con
                 bits = thread_bits<ES>(sc, w8, valid);
             }
         }
-        for (int j = threadIdx.x; j < kPackWords / 4; j += kEncThreads)
-            reinterpret_cast<uint4*>(s_words)[j] = make_uint4(0, 0, 0, 0);
-        for (int j = threadIdx.x; j < kGapWords; j += kEncThreads) s_gap[j] = 0;
+        if constexpr (ES == 1) {
+            for (int j = threadIdx.x; j < kPackWords / 4; j += kEncThreads)
+                reinterpret_cast<uint4*>(s_words)[j] = make_uint4(0, 0, 0, 0);
+            for (int j = threadIdx.x; j < kGapWords; j += kEncThreads) s_gap[j] = 0;
+        }
         uint32_t chunk_total;
-        const uint32_t my_off = block_exclusive_scan<kEncThreads>(bits, s_warp, chunk_total);
+        const uint32_t my_off =
+            block_exclusive_scan<kEncThreads>(bits, s_warp[ES == 2 ? uint32_t(c - c_begin) & 1u : 0u], chunk_total);
         const uint32_t lead = uint32_t(S & 31u);
         const uint64_t Sb = S & ~block_mask;  // a thread-block (and window) boundary
         // gap fields of this chunk: windows (S >> 6, (S + total - 1) >> 6], at
@@ -558,8 +567,13 @@ __global__ void __launch_bounds__(kEncThreads, 4) encode_kernel(const __grid_con
                 const uint32_t gb = uint32_t(gap_bit0 + int32_t(5 * j));
                 const uint32_t sh = gb & 31u;
                 const uint32_t k = gb >> 5;
-                atomicOr(&s_gap[k], g << sh);
-                if (sh > 27) atomicOr(&s_gap[k + 1], g >> (32 - sh));
+                if constexpr (ES == 2) {  // straight into the (cleared) Gaps array
+                    atomicOr(gaps32 + g0 + k, g << sh);
+                    if (sh > 27) atomicOr(gaps32 + g0 + k + 1, g >> (32 - sh));
+                } else {
+                    atomicOr(&s_gap[k], g << sh);
+                    if (sh > 27) atomicOr(&s_gap[k + 1], g >> (32 - sh));
+                }
             }
             const uint32_t br = r >> log2_block_bits;
             if ((r & uint32_t(block_mask)) == 0) {
@@ -568,10 +582,19 @@ __global__ void __launch_bounds__(kEncThreads, 4) encode_kernel(const __grid_con
                 block_off[blk_base + br + 1] = uint32_t(i + 1);
             }
         };
-        // Per-code packing: OR each code into the image at its own bit
-        // position: one shared-memory atomic, a second when the code runs into
-        // the next word (neighbouring threads share boundary words, hence the
-        // atomics).
+        // Word wi of the chunk's bits (counted from S rounded down to a word),
+        // MSB first: OR-ed into the shared image for 8-bit symbols, into the
+        // (cleared) EncodedExponent for BF16, where the words shared with
+        // neighbouring threads and chunks need no other care.
+        auto or_word = [&](uint32_t wi, uint32_t v) {
+            if constexpr (ES == 2) {
+                if (v) atomicOr(exp32 + (S >> 5) + wi, __byte_perm(v, 0, 0x0123));
+            } else {
+                atomicOr(&s_words[wi], v);
+            }
+        };
+        // Per-code packing: OR each code in at its own bit position, a second
+        // word when the code runs into the next one.
         auto pack_codes = [&](uint32_t pos, auto full_tag, auto note) {
             constexpr bool kFull = decltype(full_tag)::value;  // all kEncPerThread elements valid
 #pragma unroll
@@ -581,16 +604,16 @@ __global__ void __launch_bounds__(kEncThreads, 4) encode_kernel(const __grid_con
                 const uint32_t l = e.y;
                 const uint32_t t = ES == 2 ? __funnelshift_l(0u, e.x, 32u - l) : e.x;  // l = 32: shift 0
                 const uint32_t wi = pos >> 5, sh = pos & 31u;
-                atomicOr(&s_words[wi], t >> sh);
+                or_word(wi, t >> sh);
                 const uint32_t spill = __funnelshift_r(0u, t, sh);  // bits that did not fit
-                if (spill) atomicOr(&s_words[wi + 1], spill);
+                if (spill) or_word(wi + 1, spill);
                 note(k, l);
                 pos += l;
             }
         };
         if constexpr (ES == 2) {
             if (valid) {
-                const uint32_t pos = lead + my_off;  // bit position in the chunk image
+                const uint32_t pos = lead + my_off;  // from S rounded down to a word
                 if (bits <= 64) {
                     // the whole row of codes at once: at most three words
                     if (bits) {
@@ -598,11 +621,9 @@ __global__ void __launch_bounds__(kEncThreads, 4) encode_kernel(const __grid_con
                                                      << (64 - bits);
                         const uint32_t yh = uint32_t(y >> 32), yl = uint32_t(y);
                         const uint32_t wi = pos >> 5, sh = pos & 31u;
-                        atomicOr(&s_words[wi], yh >> sh);
-                        const uint32_t w1 = __funnelshift_r(yl, yh, sh);
-                        if (w1) atomicOr(&s_words[wi + 1], w1);
-                        const uint32_t w2 = __funnelshift_r(0u, yl, sh);
-                        if (w2) atomicOr(&s_words[wi + 2], w2);
+                        or_word(wi, yh >> sh);
+                        or_word(wi + 1, __funnelshift_r(yl, yh, sh));
+                        or_word(wi + 2, __funnelshift_r(0u, yl, sh));
                     }
                 } else {  // rare: more than 64 code bits in 16 elements
                     auto none = [](int, uint32_t) {};
@@ -678,45 +699,48 @@ __global__ void __launch_bounds__(kEncThreads, 4) encode_kernel(const __grid_con
                     if (uint32_t(k) < valid) sm[i0 + k] = uint8_t(smw[k >> 2] >> (8 * (k & 3)));
             }
         }
-        __syncthreads();
-        const uint32_t nwords = (lead + chunk_total + 31) >> 5;
-        const uint64_t W0 = S >> 5;
-        auto word = [&](uint32_t j) { return __byte_perm(s_words[j], 0, 0x0123); };  // MSB-first bytes
-        // the first and last words are shared with the neighbouring chunks
-        if (threadIdx.x == 0 || (threadIdx.x == 32 && nwords > 1)) {
-            const uint32_t j = threadIdx.x == 0 ? 0u : nwords - 1;
-            const uint32_t v = word(j);
-            if (v) atomicOr(exp32 + W0 + j, v);
-        }
-        // the words between: 16-byte stores from the first one at a 16-byte
-        // boundary of EncodedExponent, single words before and after
-        if (nwords > 2) {
-            const uint32_t jb = nwords - 1;                                // interior [1, jb)
-            const uint32_t ja = 1u + ((4u - uint32_t((W0 + 1) & 3u)) & 3u);  // W0 + ja is 4-word aligned
-            const uint32_t groups = ja < jb ? (jb - ja) / 4 : 0u;
-            const uint32_t jv = ja + 4 * groups;
-            if (threadIdx.x >= 64 && threadIdx.x < 70) {  // at most 3 words before, 3 after
-                const uint32_t k = threadIdx.x - 64;
-                const uint32_t j = k < 3 ? 1 + k : jv + (k - 3);
-                if (k < 3 ? j < min(ja, jb) : j < jb) exp32[W0 + j] = word(j);
+        if constexpr (ES == 1) {
+            __syncthreads();
+            const uint32_t nwords = (lead + chunk_total + 31) >> 5;
+            const uint64_t W0 = S >> 5;
+            auto word = [&](uint32_t j) { return __byte_perm(s_words[j], 0, 0x0123); };  // MSB-first bytes
+            // the first and last words are shared with the neighbouring chunks
+            if (threadIdx.x == 0 || (threadIdx.x == 32 && nwords > 1)) {
+                const uint32_t j = threadIdx.x == 0 ? 0u : nwords - 1;
+                const uint32_t v = word(j);
+                if (v) atomicOr(exp32 + W0 + j, v);
             }
-            for (uint32_t g = threadIdx.x; g < groups; g += kEncThreads) {
-                const uint32_t j = ja + 4 * g;
-                *reinterpret_cast<uint4*>(exp32 + W0 + j) = make_uint4(word(j), word(j + 1), word(j + 2), word(j + 3));
+            // the words between: 16-byte stores from the first one at a 16-byte
+            // boundary of EncodedExponent, single words before and after
+            if (nwords > 2) {
+                const uint32_t jb = nwords - 1;                                // interior [1, jb)
+                const uint32_t ja = 1u + ((4u - uint32_t((W0 + 1) & 3u)) & 3u);  // W0 + ja is 4-word aligned
+                const uint32_t groups = ja < jb ? (jb - ja) / 4 : 0u;
+                const uint32_t jv = ja + 4 * groups;
+                if (threadIdx.x >= 64 && threadIdx.x < 70) {  // at most 3 words before, 3 after
+                    const uint32_t k = threadIdx.x - 64;
+                    const uint32_t j = k < 3 ? 1 + k : jv + (k - 3);
+                    if (k < 3 ? j < min(ja, jb) : j < jb) exp32[W0 + j] = word(j);
+                }
+                for (uint32_t g = threadIdx.x; g < groups; g += kEncThreads) {
+                    const uint32_t j = ja + 4 * g;
+                    *reinterpret_cast<uint4*>(exp32 + W0 + j) =
+                        make_uint4(word(j), word(j + 1), word(j + 2), word(j + 3));
+                }
             }
-        }
-        if (gaps32) {
-            // gap words g0 .. g1; the first and last may hold other chunks' fields
-            const uint64_t w_last = (S + chunk_total - 1) >> 6;
-            const uint64_t g1 = (5 * w_last + 4) >> 5;
-            if (w_last > (S >> 6)) {
-                const uint32_t ng = uint32_t(g1 - g0 + 1);
-                for (uint32_t j = threadIdx.x; j < ng; j += kEncThreads) {
-                    const uint32_t v = s_gap[j];
-                    if (j == 0 || j == ng - 1) {
-                        if (v) atomicOr(gaps32 + g0 + j, v);
-                    } else {
-                        gaps32[g0 + j] = v;
+            if (gaps32) {
+                // gap words g0 .. g1; the first and last may hold other chunks' fields
+                const uint64_t w_last = (S + chunk_total - 1) >> 6;
+                const uint64_t g1 = (5 * w_last + 4) >> 5;
+                if (w_last > (S >> 6)) {
+                    const uint32_t ng = uint32_t(g1 - g0 + 1);
+                    for (uint32_t j = threadIdx.x; j < ng; j += kEncThreads) {
+                        const uint32_t v = s_gap[j];
+                        if (j == 0 || j == ng - 1) {
+                            if (v) atomicOr(gaps32 + g0 + j, v);
+                        } else {
+                            gaps32[g0 + j] = v;
+                        }
                     }
                 }
             }
