@@ -757,14 +757,25 @@ __global__ void mark_if_aborted(const uint32_t* abort_flag, uint32_t* lut_magic)
 
 // Persistent grid for an encode kernel: as many CTAs as can be resident on
 // every SM at once.
-template <typename Kernel>
-unsigned encode_grid(Kernel kernel, uint64_t chunks) {
-    int dev = 0, sms = 148, per_sm = 1;
+// (SMs × resident CTAs per SM, looked up once per device and kernel: the plan
+// and the encode of every compress call ask again.)
+constexpr int kMaxDevices = 64;
+template <int ES>
+unsigned encode_grid(uint64_t chunks) {
+    static std::atomic<uint32_t> cached[kMaxDevices];  // 0 = not yet
+    int dev = 0;
     cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kEncThreads, 0) != cudaSuccess || per_sm < 1)
-        per_sm = 1;
-    uint64_t want = uint64_t(sms) * uint64_t(per_sm);
+    uint32_t slots = dev >= 0 && dev < kMaxDevices ? cached[dev].load(std::memory_order_relaxed) : 0u;
+    if (!slots) {
+        int sms = 148, per_sm = 1;
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, encode_kernel<ES>, kEncThreads, 0) != cudaSuccess ||
+            per_sm < 1)
+            per_sm = 1;
+        slots = uint32_t(sms) * uint32_t(per_sm);
+        if (dev >= 0 && dev < kMaxDevices) cached[dev].store(slots, std::memory_order_relaxed);
+    }
+    uint64_t want = slots;
     if (want > kMaxEncRanges) want = kMaxEncRanges;
     return unsigned(chunks < want ? chunks : want);
 }
@@ -776,7 +787,7 @@ template <int ES>
 RangeTag encode_partition(uint64_t chunks) {
     RangeTag t{0u, 0u, 0u};
     if (!chunks) return t;
-    const uint64_t slots = encode_grid(encode_kernel<ES>, chunks);
+    const uint64_t slots = encode_grid<ES>(chunks);
     t.range_chunks = (chunks + slots - 1) / slots;
     t.n_ranges = uint32_t((chunks + t.range_chunks - 1) / t.range_chunks);
     return t;

@@ -9,7 +9,6 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
-#include <vector>
 
 #include "df11_internal.h"
 
@@ -103,10 +102,10 @@ const char* df11_last_error(void) { return g_err; }
 df11_status df11_code_lengths(const uint64_t* hist, uint32_t max_code_len, uint8_t* code_len) {
     if (!hist || !code_len) return fail(DF11_ERR_INVALID, "df11_code_lengths: null pointer");
     std::memset(code_len, 0, 256);
-    std::vector<int> sym;
+    int sym[256];
+    int m = 0;
     for (int s = 0; s < 256; s++)
-        if (hist[s]) sym.push_back(s);
-    const int m = int(sym.size());
+        if (hist[s]) sym[m++] = s;
     if (m == 0) return DF11_OK;
     if (max_code_len < 1 || max_code_len > 32)
         return fail(DF11_ERR_INVALID, "df11_code_lengths: max_code_len %u outside 1..32", max_code_len);
@@ -118,34 +117,42 @@ df11_status df11_code_lengths(const uint64_t* hist, uint32_t max_code_len, uint8
     if (L < 9 && (1 << L) < m)
         return fail(DF11_ERR_INVALID, "df11_code_lengths: %d values do not fit in %d-bit codes", m, L);
     // lighter first; equal counts: lower value first
-    std::stable_sort(sym.begin(), sym.end(), [&](int a, int b) { return hist[a] < hist[b]; });
+    std::sort(sym, sym + m, [&](int a, int b) { return hist[a] != hist[b] ? hist[a] < hist[b] : a < b; });
 
-    // is_leaf[d][i]: item i of the depth-d list is a leaf coin
-    std::vector<std::vector<uint8_t>> is_leaf(L + 1);
-    std::vector<uint64_t> prev(m), cur;
-    for (int i = 0; i < m; i++) prev[i] = hist[sym[i]];
-    is_leaf[L].assign(m, 1);
+    // is_leaf[d][i]: item i of the depth-d list is a leaf coin.  A list holds
+    // the m leaves and at most m - 1 packages (25 KB on the stack: no
+    // allocation)
+    uint8_t is_leaf[33][512];
+    uint64_t wbuf[2][512];
+    uint64_t* prev = wbuf[0];
+    uint64_t* cur = wbuf[1];
+    size_t n_prev = size_t(m), n_d1 = 0;
+    for (int i = 0; i < m; i++) {
+        prev[i] = hist[sym[i]];
+        is_leaf[L][i] = 1;
+    }
+    if (L == 1) n_d1 = size_t(m);
     for (int d = L - 1; d >= 1; d--) {
-        const size_t npk = prev.size() / 2;
-        cur.clear();
-        is_leaf[d].clear();
-        size_t li = 0, pi = 0;
+        const size_t npk = n_prev / 2;
+        size_t li = 0, pi = 0, nc = 0;
         while (li < size_t(m) || pi < npk) {
             const bool have_pk = pi < npk;
             const uint64_t pw = have_pk ? prev[2 * pi] + prev[2 * pi + 1] : 0;
             if (li < size_t(m) && (!have_pk || hist[sym[li]] <= pw)) {
-                cur.push_back(hist[sym[li++]]);
-                is_leaf[d].push_back(1);
+                cur[nc] = hist[sym[li++]];
+                is_leaf[d][nc++] = 1;
             } else {
-                cur.push_back(pw);
-                is_leaf[d].push_back(0);
+                cur[nc] = pw;
+                is_leaf[d][nc++] = 0;
                 pi++;
             }
         }
-        prev.swap(cur);
+        std::swap(prev, cur);
+        n_prev = nc;
+        if (d == 1) n_d1 = nc;
     }
     size_t k = size_t(2 * (m - 1));
-    if (is_leaf[1].size() < k) return fail(DF11_ERR_INVALID, "df11_code_lengths: too few items");
+    if (n_d1 < k) return fail(DF11_ERR_INVALID, "df11_code_lengths: too few items");
     for (int d = 1; d <= L && k; d++) {
         size_t j = 0;
         for (size_t i = 0; i < k; i++) j += is_leaf[d][i];
