@@ -633,22 +633,34 @@ __global__ void __launch_bounds__(kEncThreads, 4) encode_kernel(const __grid_con
                         pack_codes(pos, std::false_type{}, none);
                 }
                 if (gaps32) {
-                    // every window boundary 64 m (relative to Sb) in the
-                    // thread's bits [A, A + bits) is covered by one code: the
-                    // last one starting at or before it (binary search over
-                    // the thread's starts; starts past the valid elements
-                    // equal bits)
+                    // every window boundary in the thread's bits [A, A + bits)
+                    // (A relative to Sb), at q from the thread's first bit, is
+                    // covered by one code: the last one starting at or before
+                    // it (binary search over the thread's starts; starts past
+                    // the valid elements equal bits).  If that code starts
+                    // before the boundary, the window's gap is where the next
+                    // code starts (the gaps of windows that begin with a code
+                    // stay 0); at a thread-block boundary the block's first
+                    // element is that code's, or the next one's.
                     const uint32_t A = uint32_t(S - Sb) + my_off;
-                    for (uint32_t m = (A + 63) >> 6; 64 * m < A + bits; m++) {
-                        const uint32_t q = 64 * m - A;
+                    uint32_t* const gap_words = gaps32 + g0;
+                    for (uint32_t q = (64u - (A & 63u)) & 63u; q < bits; q += 64) {
                         uint32_t k = 0;
                         if (s_pos[k + 8][threadIdx.x] <= q) k += 8;
                         if (s_pos[k + 4][threadIdx.x] <= q) k += 4;
                         if (s_pos[k + 2][threadIdx.x] <= q) k += 2;
                         if (s_pos[k + 1][threadIdx.x] <= q) k += 1;
-                        const uint32_t a = s_pos[k][threadIdx.x];
-                        const uint32_t b = k + 1 < kEncPerThread ? s_pos[k + 1][threadIdx.x] : bits;
-                        window_event(A + a, b - a, uint32_t(i0) + k);
+                        const bool inside = s_pos[k][threadIdx.x] < q;  // the code starts before the boundary
+                        const uint32_t Bq = A + q;                       // the boundary, from Sb
+                        if (inside) {
+                            const uint32_t b = k + 1 < kEncPerThread ? s_pos[k + 1][threadIdx.x] : bits;
+                            const uint32_t gb = uint32_t(gap_bit0 + int32_t(5 * (Bq >> 6)));
+                            const uint32_t sh = gb & 31u, g = b - q;
+                            atomicOr(gap_words + (gb >> 5), g << sh);
+                            if (sh > 27) atomicOr(gap_words + (gb >> 5) + 1, g >> (32 - sh));
+                        }
+                        if ((Bq & uint32_t(block_mask)) == 0)
+                            block_off[blk_base + (Bq >> log2_block_bits)] = uint32_t(i0) + k + (inside ? 1u : 0u);
                     }
                 }
             }
