@@ -302,24 +302,32 @@ __device__ __forceinline__ uint32_t thread_bits(const SharedCodes& sc, const uin
 //   pack: chunk by chunk, each thread's bit offset by a CTA scan, and the
 //     chunk packed at the running prefix.
 //
-// Packing a chunk that starts at stream bit S: every code is OR-ed into a
-// shared-memory image of the chunk at its bit position (shared-memory
-// atomics; a code may run into the next word).  The image's interior words
-// are then stored to EncodedExponent and its two boundary words, shared with
-// the neighbouring chunks, are OR-ed into global memory.  The same pass
-// writes the sign+mantissa bytes, the gaps and the thread blocks' output
-// positions from each code's start bit s and length l:
+// Packing a chunk that starts at stream bit S.  Every code goes to its bit
+// position in EncodedExponent (MSB first); words shared with neighbouring
+// threads, chunks or ranges are OR-ed together:
+//   * BF16: each thread looks its 16 codes up once, appending them to a
+//     64-bit register row, and ORs the row into the (cleared) global array
+//     with at most three reductions after the scan; a thread with more than
+//     64 code bits ORs its codes one by one.
+//   * 8-bit symbols (16 codes overflow a row): per-code shared-memory atomics
+//     into an image of the chunk, whose interior words are then stored and
+//     whose two boundary words are OR-ed into global memory.
+// The same pass writes the sign+mantissa bytes, the gaps and the thread
+// blocks' output positions from each code's start bit s and length l:
 //   * a code that starts inside window w-1 and runs into window w sets
 //     gap[w] = s + l - 64w (gaps of windows that begin exactly at a code start
-//     stay 0); the chunk's gap fields are assembled in shared memory and
-//     stored as whole words, the two boundary words OR-ed in;
+//     stay 0); BF16 ORs the field into the (cleared) Gaps array, 8-bit
+//     symbols assemble the chunk's fields in shared memory and store whole
+//     words, the two boundary words OR-ed in;
 //   * a code that starts exactly at bit 64*T*b sets off[b] = i, one that runs
 //     over that bit sets off[b] = i + 1.
 // Positions are kept 32-bit relative to S rounded down to a thread-block
-// boundary; a code covers a window boundary exactly when (u >> 6) changes
-// across it, u = relative start + 63: one test per element marks the code in
-// a bit mask, and the marked codes' gap and offset writes follow the packing
-// loop, their positions read back from shared memory.
+// boundary.  BF16 finds the code covering each window boundary in the
+// thread's bits by a binary search over its codes' starts; for 8-bit symbols
+// a code covers a window boundary exactly when (u >> 6) changes across it,
+// u = relative start + 63: one test per element marks the code in a bit
+// mask, and the marked codes' gap and offset writes follow the packing loop,
+// their positions read back from shared memory.
 // ---------------------------------------------------------------------------
 constexpr int kPackWords = kEncChunk + 4;  // 32 bits per element at most, plus the misalignment
 // gap words a chunk can touch: 32 kEncChunk bits -> 512 kEncChunk / 64 + 2 windows of 5 bits
@@ -553,13 +561,15 @@ __global__ void __launch_bounds__(kEncThreads, 4) encode_kernel(const __grid_con
         const uint32_t lead = uint32_t(S & 31u);
         const uint64_t Sb = S & ~block_mask;  // a thread-block (and window) boundary
         // gap fields of this chunk: windows (S >> 6, (S + total - 1) >> 6], at
-        // gap array bits 5w .. 5w + 4; s_gap word 0 = gap array word g0
+        // gap array bits 5w .. 5w + 4, from gap array word g0 on (s_gap word 0)
         const uint64_t g0 = (5 * ((S >> 6) + 1)) >> 5;
         const uint64_t blk_base = Sb >> log2_block_bits;
-        // gap array bit 5w of window w = Sb / 64 + j, counted from s_gap's
+        // gap array bit 5w of window w = Sb / 64 + j, counted from word g0's
         // first bit: gap_bit0 + 5 j (small: Sb is at most one thread block,
         // 64 T bits, before the chunk's first window)
         const int32_t gap_bit0 = int32_t(int64_t(5 * (Sb >> 6)) - int64_t(32 * g0));
+        // 8-bit symbols: the gap and offset writes of the code at r (relative
+        // to Sb), l bits long, element i, when it covers a window boundary
         auto window_event = [&](uint32_t r, uint32_t l, uint32_t i) {
             if (r & 63u) {
                 const uint32_t j = (r >> 6) + 1;          // the window the code runs into, from Sb
@@ -567,13 +577,8 @@ __global__ void __launch_bounds__(kEncThreads, 4) encode_kernel(const __grid_con
                 const uint32_t gb = uint32_t(gap_bit0 + int32_t(5 * j));
                 const uint32_t sh = gb & 31u;
                 const uint32_t k = gb >> 5;
-                if constexpr (ES == 2) {  // straight into the (cleared) Gaps array
-                    atomicOr(gaps32 + g0 + k, g << sh);
-                    if (sh > 27) atomicOr(gaps32 + g0 + k + 1, g >> (32 - sh));
-                } else {
-                    atomicOr(&s_gap[k], g << sh);
-                    if (sh > 27) atomicOr(&s_gap[k + 1], g >> (32 - sh));
-                }
+                atomicOr(&s_gap[k], g << sh);
+                if (sh > 27) atomicOr(&s_gap[k + 1], g >> (32 - sh));
             }
             const uint32_t br = r >> log2_block_bits;
             if ((r & uint32_t(block_mask)) == 0) {
