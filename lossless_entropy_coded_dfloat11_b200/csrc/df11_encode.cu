@@ -979,6 +979,10 @@ df11_status compress_encode(const char* fn, const void* const* d_segs, const df1
         // this header's plan for this partition (the kernel compares tags)
         RangeTag expect = encode_partition<ES>(chunks);
         expect.token = range_hist && tag ? hdr->plan_token : 0u;
+        // a range's code bits are counted in 32 bits: at most 32 per element
+        if (expect.range_chunks * kEncChunk * 32 >= (uint64_t(1) << 32))
+            return fail(DF11_ERR_TOO_LARGE, "%s: %llu elements per encode range on this device", fn,
+                        (unsigned long long)(expect.range_chunks * kEncChunk));
         encode_kernel<ES><<<expect.n_ranges, kEncThreads, 0, s>>>(
             sg, ct, n, chunks, expect.range_chunks, log2_bb, desc, reinterpret_cast<uint32_t*>(desc + chunks),
             abort_flag, reinterpret_cast<uint32_t*>(d_exp), d_sm, reinterpret_cast<uint32_t*>(d_gaps),
