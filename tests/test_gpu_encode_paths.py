@@ -94,6 +94,21 @@ def test_bf16_range_histograms_match_counting(sizes):
     np.testing.assert_array_equal(got["off"], s.block_off)
 
 
+def test_bf16_sixty_four_ragged_segments():
+    """The most segments a stream may have, of random sizes: segment edges
+    fall anywhere inside the encode ranges, several segments per range."""
+    rng = np.random.default_rng(77)
+    sizes = [int(v) for v in rng.integers(1, 150_000, size=B.DF11_MAX_SEGMENTS)]
+    ts = _bf16_ragged(sizes, 78)
+    got = _three_ways([t.cuda() for t in ts], u8=False)
+    x = torch.cat(ts).view(torch.int16).numpy().view(np.uint16)
+    s = oracle.encode(x, threads_per_block=64)
+    np.testing.assert_array_equal(got["exp"], s.exp)
+    np.testing.assert_array_equal(got["sm"], s.sm)
+    np.testing.assert_array_equal(got["gaps"], s.gaps)
+    np.testing.assert_array_equal(got["off"], s.block_off)
+
+
 @pytest.mark.parametrize("sizes", [[3, 15, 16, 17, 70001], [2000001, 1999999]])
 def test_u8_range_histograms_match_counting(sizes):
     rng = np.random.default_rng(50 + len(sizes))
