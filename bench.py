@@ -771,7 +771,7 @@ def main(argv=None):
                     help="time the --config workload only, not the other workloads")
     ap.add_argument("--layout", choices=["gaps", "chunks"], default="gaps",
                     help="chunks: the independent-chunk variant of the container (an ablation)")
-    ap.add_argument("--compress-repeats", type=int, default=5)
+    ap.add_argument("--compress-repeats", type=int, default=11)
     ap.add_argument("--pipeline", action="store_true",
                     help="time decompress-into-consumer (BlockPrefetcher) instead of the decode alone")
     ap.add_argument("--pipeline-blocks", type=int, default=4)
