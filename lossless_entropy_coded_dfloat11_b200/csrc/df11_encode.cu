@@ -188,18 +188,11 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* s
 // exponent in every lane would serialise in the constant cache.)
 // ---------------------------------------------------------------------------
 struct SharedCodes {
-    // x = the code, right-aligned for BF16 input (appended to a register
-    // row), left-aligned in 32 bits for 8-bit symbols (OR-ed in place);
-    // y = its length (0 = absent)
-    uint2 e[256];
+    uint2 e[256];  // x = the code, right-aligned; y = its length (0 = absent)
 };
 
-template <int ES>
 __device__ __forceinline__ void stage_codes(SharedCodes& sc, const CodeTable& ct) {
-    for (int v = threadIdx.x; v < 256; v += blockDim.x) {
-        const uint32_t l = ct.len[v];
-        sc.e[v] = make_uint2(ES == 2 ? ct.code[v] : (l ? ct.code[v] << (32u - l) : 0u), l);
-    }
+    for (int v = threadIdx.x; v < 256; v += blockDim.x) sc.e[v] = make_uint2(ct.len[v] ? ct.code[v] : 0u, ct.len[v]);
 }
 
 // One thread's kEncPerThread elements packed in words (ES = 2: element 2j
@@ -303,36 +296,27 @@ __device__ __forceinline__ uint32_t thread_bits(const SharedCodes& sc, const uin
 //     chunk packed at the running prefix.
 //
 // Packing a chunk that starts at stream bit S.  Every code goes to its bit
-// position in EncodedExponent (MSB first); words shared with neighbouring
-// threads, chunks or ranges are OR-ed together:
-//   * BF16: each thread looks its 16 codes up once, appending them to a
-//     64-bit register row, and ORs the row into the (cleared) global array
-//     with at most three reductions after the scan; a thread with more than
-//     64 code bits ORs its codes one by one.
-//   * 8-bit symbols (16 codes overflow a row): per-code shared-memory atomics
-//     into an image of the chunk, whose interior words are then stored and
-//     whose two boundary words are OR-ed into global memory.
-// The same pass writes the sign+mantissa bytes, the gaps and the thread
-// blocks' output positions from each code's start bit s and length l:
+// position in EncodedExponent (MSB first): each thread looks its 16 codes up
+// once, appending them to a register row (2 words for BF16, 4 for 8-bit
+// symbols), and after the CTA scan ORs the row into the (cleared) global
+// array with one reduction per word it touches; a thread whose row
+// overflowed ORs its codes one by one.  Words shared with neighbouring
+// threads, chunks or ranges need no other care.  The same pass writes the
+// sign+mantissa bytes, the gaps and the thread blocks' output positions:
 //   * a code that starts inside window w-1 and runs into window w sets
-//     gap[w] = s + l - 64w (gaps of windows that begin exactly at a code start
-//     stay 0); BF16 ORs the field into the (cleared) Gaps array, 8-bit
-//     symbols assemble the chunk's fields in shared memory and store whole
-//     words, the two boundary words OR-ed in;
+//     gap[w] = s + l - 64w (s its start bit, l its length; gaps of windows
+//     that begin exactly at a code start stay 0), OR-ed into the (cleared)
+//     Gaps array;
 //   * a code that starts exactly at bit 64*T*b sets off[b] = i, one that runs
 //     over that bit sets off[b] = i + 1.
 // Positions are kept 32-bit relative to S rounded down to a thread-block
-// boundary.  BF16 finds the code covering each window boundary in the
-// thread's bits by a binary search over its codes' starts; for 8-bit symbols
-// a code covers a window boundary exactly when (u >> 6) changes across it,
-// u = relative start + 63: one test per element marks the code in a bit
-// mask, and the marked codes' gap and offset writes follow the packing loop,
-// their positions read back from shared memory.
+// boundary; the code covering each window boundary in a thread's bits is
+// found by a binary search over its codes' starts.
 // ---------------------------------------------------------------------------
-constexpr int kPackWords = kEncChunk + 4;  // 32 bits per element at most, plus the misalignment
-// gap words a chunk can touch: 32 kEncChunk bits -> 512 kEncChunk / 64 + 2 windows of 5 bits
-constexpr int kGapWords = (5 * (int(kEncChunk) * 32 / 64 + 2)) / 32 + 2;
-static_assert(kPackWords % 4 == 0, "image cleared in 16-byte stores");
+// Words in a thread's register row of codes: 16 exponent codes of ~2.6 bits
+// fit 64 bits, 16 codes of 8-bit symbols (~7 bits for quantized weights) 128.
+template <int ES>
+constexpr int kRowWords = ES == 2 ? 2 : 4;
 constexpr unsigned long long kDescAggregate = 1ull << 62, kDescInclusive = 2ull << 62;
 constexpr unsigned long long kDescValue = (1ull << 62) - 1;
 constexpr uint32_t kSpinLimit = 1u << 20;
@@ -434,17 +418,12 @@ __global__ void __launch_bounds__(kEncThreads, 4) encode_kernel(const __grid_con
                                                              const uint32_t* __restrict__ range_hist,
                                                              const RangeTag* __restrict__ tag, const RangeTag expect) {
     __shared__ SharedCodes sc;
-    // 8-bit symbols: the chunk's image and gap fields are assembled here
-    // (BF16 rows go to global memory directly)
-    __shared__ __align__(16) uint32_t s_words[ES == 1 ? kPackWords : 4];
-    __shared__ uint32_t s_gap[ES == 1 ? kGapWords : 1];
-    // per element: BF16, the code's start relative to its thread's first bit;
-    // 8-bit symbols, (start relative to Sb + 63) << 6 | length
+    // per element: its code's start relative to its thread's first bit
     __shared__ uint32_t s_pos[kEncPerThread][kEncThreads];
     __shared__ uint32_t s_warp[2][kEncThreads / 32];  // scan partials, two chunks apart
     __shared__ uint32_t s_ticket;
     __shared__ unsigned long long s_prefix;
-    stage_codes<ES>(sc, ct);
+    stage_codes(sc, ct);
     if (threadIdx.x == 0) s_ticket = atomicAdd(ticket, 1u);
     __syncthreads();
     const uint64_t block_mask = (uint64_t(1) << log2_block_bits) - 1;
@@ -507,7 +486,10 @@ __global__ void __launch_bounds__(kEncThreads, 4) encode_kernel(const __grid_con
     __syncthreads();
     uint64_t S = s_prefix;
 
-    // pack: each chunk at the running prefix
+    // pack: each chunk at the running prefix.  No barrier at the top of the
+    // loop: s_pos is the thread's own column, and the scan alternates between
+    // two s_warp rows (a warp writes a row again only after every warp has
+    // passed the scan in between).
     for (uint64_t c = c_begin; c < c_end; c++) {
         const RawElems cur = next;
         if (c + 1 < c_end) {
@@ -515,181 +497,117 @@ __global__ void __launch_bounds__(kEncThreads, 4) encode_kernel(const __grid_con
             next = load_raw<ES>(sg, (c + 1) * kEncChunk, (c + 1) * kEncChunk + tofs, n, seg);
         }
         const uint64_t i0 = c * kEncChunk + tofs;
-        // 8-bit symbols: s_words, s_gap and s_warp of the last chunk are free.
-        // BF16 needs no barrier here: s_pos is the thread's own column, and
-        // the scan alternates between two s_warp rows (a warp writes a row
-        // again only after every warp has passed the scan in between).
-        if constexpr (ES == 1) __syncthreads();
         uint32_t w8[kWords<ES>];
         uint32_t valid = 0, bits = 0;
-        uint32_t xhi = 0, xlo = 0;  // BF16: the thread's codes in a row, right-aligned (the last 64 bits)
+        // the thread's codes in a row, right-aligned: x[0] holds the last bits
+        uint32_t x[kRowWords<ES>];
+#pragma unroll
+        for (int j = 0; j < kRowWords<ES>; j++) x[j] = 0;
         if (i0 < n) {
             raw_words<ES>(sg, cur, i0, n, w8);
             const uint64_t left = n - i0;
             valid = left < kEncPerThread ? uint32_t(left) : kEncPerThread;
-            if constexpr (ES == 2) {
-                // one lookup per code: its start relative to the thread's
-                // first bit to s_pos, the code appended to xhi:xlo
-                auto gather = [&](auto full_tag) {
-                    constexpr bool kFull = decltype(full_tag)::value;
+            // one lookup per code: its start relative to the thread's first
+            // bit to s_pos, the code appended to the row
+            auto gather = [&](auto full_tag) {
+                constexpr bool kFull = decltype(full_tag)::value;
 #pragma unroll
-                    for (int k = 0; k < int(kEncPerThread); k++) {
-                        // code and length; 0, 0 past the valid elements
-                        const uint2 e = (kFull || uint32_t(k) < valid) ? sc.e[symbol<ES>(w8, k)] : make_uint2(0, 0);
-                        s_pos[k][threadIdx.x] = bits;
-                        xhi = __funnelshift_lc(xlo, xhi, e.y);
-                        xlo = __funnelshift_lc(0u, xlo, e.y) | e.x;  // e.x right-aligned
-                        bits += e.y;
-                    }
-                };
-                if (valid == kEncPerThread)
-                    gather(std::true_type{});
-                else
-                    gather(std::false_type{});
-            } else {
-                bits = thread_bits<ES>(sc, w8, valid);
-            }
-        }
-        if constexpr (ES == 1) {
-            for (int j = threadIdx.x; j < kPackWords / 4; j += kEncThreads)
-                reinterpret_cast<uint4*>(s_words)[j] = make_uint4(0, 0, 0, 0);
-            for (int j = threadIdx.x; j < kGapWords; j += kEncThreads) s_gap[j] = 0;
+                for (int k = 0; k < int(kEncPerThread); k++) {
+                    // code (right-aligned) and length; 0, 0 past the valid elements
+                    const uint2 e = (kFull || uint32_t(k) < valid) ? sc.e[symbol<ES>(w8, k)] : make_uint2(0, 0);
+                    s_pos[k][threadIdx.x] = bits;
+#pragma unroll
+                    for (int j = kRowWords<ES> - 1; j > 0; j--) x[j] = __funnelshift_lc(x[j - 1], x[j], e.y);
+                    x[0] = __funnelshift_lc(0u, x[0], e.y) | e.x;
+                    bits += e.y;
+                }
+            };
+            if (valid == kEncPerThread)
+                gather(std::true_type{});
+            else
+                gather(std::false_type{});
         }
         uint32_t chunk_total;
         const uint32_t my_off =
-            block_exclusive_scan<kEncThreads>(bits, s_warp[ES == 2 ? uint32_t(c - c_begin) & 1u : 0u], chunk_total);
+            block_exclusive_scan<kEncThreads>(bits, s_warp[uint32_t(c - c_begin) & 1u], chunk_total);
         const uint32_t lead = uint32_t(S & 31u);
         const uint64_t Sb = S & ~block_mask;  // a thread-block (and window) boundary
         // gap fields of this chunk: windows (S >> 6, (S + total - 1) >> 6], at
-        // gap array bits 5w .. 5w + 4, from gap array word g0 on (s_gap word 0)
+        // gap array bits 5w .. 5w + 4, from gap array word g0 on
         const uint64_t g0 = (5 * ((S >> 6) + 1)) >> 5;
         const uint64_t blk_base = Sb >> log2_block_bits;
         // gap array bit 5w of window w = Sb / 64 + j, counted from word g0's
         // first bit: gap_bit0 + 5 j (small: Sb is at most one thread block,
         // 64 T bits, before the chunk's first window)
         const int32_t gap_bit0 = int32_t(int64_t(5 * (Sb >> 6)) - int64_t(32 * g0));
-        // 8-bit symbols: the gap and offset writes of the code at r (relative
-        // to Sb), l bits long, element i, when it covers a window boundary
-        auto window_event = [&](uint32_t r, uint32_t l, uint32_t i) {
-            if (r & 63u) {
-                const uint32_t j = (r >> 6) + 1;          // the window the code runs into, from Sb
-                const uint32_t g = r + l - 64 * j;         // its gap
-                const uint32_t gb = uint32_t(gap_bit0 + int32_t(5 * j));
-                const uint32_t sh = gb & 31u;
-                const uint32_t k = gb >> 5;
-                atomicOr(&s_gap[k], g << sh);
-                if (sh > 27) atomicOr(&s_gap[k + 1], g >> (32 - sh));
-            }
-            const uint32_t br = r >> log2_block_bits;
-            if ((r & uint32_t(block_mask)) == 0) {
-                block_off[blk_base + br] = uint32_t(i);
-            } else if (((r + l - 1) >> log2_block_bits) != br) {
-                block_off[blk_base + br + 1] = uint32_t(i + 1);
-            }
-        };
         // Word wi of the chunk's bits (counted from S rounded down to a word),
-        // MSB first: OR-ed into the shared image for 8-bit symbols, into the
-        // (cleared) EncodedExponent for BF16, where the words shared with
-        // neighbouring threads and chunks need no other care.
+        // MSB first, OR-ed into the (cleared) EncodedExponent: words shared
+        // with neighbouring threads, chunks or ranges need no other care.
         auto or_word = [&](uint32_t wi, uint32_t v) {
-            if constexpr (ES == 2) {
-                if (v) atomicOr(exp32 + (S >> 5) + wi, __byte_perm(v, 0, 0x0123));
-            } else {
-                atomicOr(&s_words[wi], v);
-            }
+            if (v) atomicOr(exp32 + (S >> 5) + wi, __byte_perm(v, 0, 0x0123));
         };
-        // Per-code packing: OR each code in at its own bit position, a second
-        // word when the code runs into the next one.
-        auto pack_codes = [&](uint32_t pos, auto full_tag, auto note) {
-            constexpr bool kFull = decltype(full_tag)::value;  // all kEncPerThread elements valid
+        if (valid) {
+            const uint32_t pos = lead + my_off;  // from S rounded down to a word
+            if (bits <= 32u * kRowWords<ES>) {
+                // the whole row at once: with the row's end at bit e, the word
+                // k places before e's word holds row words k and k-1 shifted
+                // by 32 - e % 32 (no shift when e is word-aligned)
+                if (bits) {
+                    const uint32_t e = pos + bits, sh = 32u - (e & 31u), wl = (e - 1) >> 5;
+                    or_word(wl, __funnelshift_l(0u, x[0], sh));
 #pragma unroll
-            for (int k = 0; k < int(kEncPerThread); k++) {
-                // code, left-aligned, and length; l = 0, t = 0 past the valid elements
-                const uint2 e = (kFull || uint32_t(k) < valid) ? sc.e[symbol<ES>(w8, k)] : make_uint2(0, 0);
-                const uint32_t l = e.y;
-                const uint32_t t = ES == 2 ? __funnelshift_l(0u, e.x, 32u - l) : e.x;  // l = 32: shift 0
-                const uint32_t wi = pos >> 5, sh = pos & 31u;
-                or_word(wi, t >> sh);
-                const uint32_t spill = __funnelshift_r(0u, t, sh);  // bits that did not fit
-                if (spill) or_word(wi + 1, spill);
-                note(k, l);
-                pos += l;
-            }
-        };
-        if constexpr (ES == 2) {
-            if (valid) {
-                const uint32_t pos = lead + my_off;  // from S rounded down to a word
-                if (bits <= 64) {
-                    // the whole row of codes at once: at most three words
-                    if (bits) {
-                        const unsigned long long y = ((static_cast<unsigned long long>(xhi) << 32) | xlo)
-                                                     << (64 - bits);
-                        const uint32_t yh = uint32_t(y >> 32), yl = uint32_t(y);
-                        const uint32_t wi = pos >> 5, sh = pos & 31u;
-                        or_word(wi, yh >> sh);
-                        or_word(wi + 1, __funnelshift_r(yl, yh, sh));
-                        or_word(wi + 2, __funnelshift_r(0u, yl, sh));
-                    }
-                } else {  // rare: more than 64 code bits in 16 elements
-                    auto none = [](int, uint32_t) {};
-                    if (valid == kEncPerThread)
-                        pack_codes(pos, std::true_type{}, none);
-                    else
-                        pack_codes(pos, std::false_type{}, none);
+                    for (int k = 1; k < kRowWords<ES>; k++)
+                        if (uint32_t(k) <= wl) or_word(wl - k, __funnelshift_l(x[k - 1], x[k], sh));
+                    if (uint32_t(kRowWords<ES>) <= wl)
+                        or_word(wl - kRowWords<ES>, __funnelshift_l(x[kRowWords<ES> - 1], 0u, sh));
                 }
-                if (gaps32) {
-                    // every window boundary in the thread's bits [A, A + bits)
-                    // (A relative to Sb), at q from the thread's first bit, is
-                    // covered by one code: the last one starting at or before
-                    // it (binary search over the thread's starts; starts past
-                    // the valid elements equal bits).  If that code starts
-                    // before the boundary, the window's gap is where the next
-                    // code starts (the gaps of windows that begin with a code
-                    // stay 0); at a thread-block boundary the block's first
-                    // element is that code's, or the next one's.
-                    const uint32_t A = uint32_t(S - Sb) + my_off;
-                    uint32_t* const gap_words = gaps32 + g0;
-                    for (uint32_t q = (64u - (A & 63u)) & 63u; q < bits; q += 64) {
-                        uint32_t k = 0;
-                        if (s_pos[k + 8][threadIdx.x] <= q) k += 8;
-                        if (s_pos[k + 4][threadIdx.x] <= q) k += 4;
-                        if (s_pos[k + 2][threadIdx.x] <= q) k += 2;
-                        if (s_pos[k + 1][threadIdx.x] <= q) k += 1;
-                        const bool inside = s_pos[k][threadIdx.x] < q;  // the code starts before the boundary
-                        const uint32_t Bq = A + q;                       // the boundary, from Sb
-                        if (inside) {
-                            const uint32_t b = k + 1 < kEncPerThread ? s_pos[k + 1][threadIdx.x] : bits;
-                            const uint32_t gb = uint32_t(gap_bit0 + int32_t(5 * (Bq >> 6)));
-                            const uint32_t sh = gb & 31u, g = b - q;
-                            atomicOr(gap_words + (gb >> 5), g << sh);
-                            if (sh > 27) atomicOr(gap_words + (gb >> 5) + 1, g >> (32 - sh));
-                        }
-                        if ((Bq & uint32_t(block_mask)) == 0)
-                            block_off[blk_base + (Bq >> log2_block_bits)] = uint32_t(i0) + k + (inside ? 1u : 0u);
+            } else {  // rare: the row overflowed; code by code
+                uint32_t p = pos;
+                auto pack = [&](auto full_tag) {
+                    constexpr bool kFull = decltype(full_tag)::value;
+#pragma unroll
+                    for (int k = 0; k < int(kEncPerThread); k++) {
+                        const uint2 e = (kFull || uint32_t(k) < valid) ? sc.e[symbol<ES>(w8, k)] : make_uint2(0, 0);
+                        const uint32_t t = __funnelshift_l(0u, e.x, 32u - e.y);  // left-aligned (l = 32: shift 0)
+                        or_word(p >> 5, t >> (p & 31u));
+                        or_word((p >> 5) + 1, __funnelshift_r(0u, t, p & 31u));  // the bits that did not fit
+                        p += e.y;
                     }
-                }
+                };
+                if (valid == kEncPerThread)
+                    pack(std::true_type{});
+                else
+                    pack(std::false_type{});
             }
-        } else if (valid) {
-            // Every code's relative start and length go to the thread's
-            // column of s_pos and a bit of `cross` marks the codes that cover
-            // a window boundary; those few are handled after the loop.
-            uint32_t u = uint32_t(S - Sb) + my_off + 63u;  // relative start + 63
-            uint32_t cross = 0;
-            auto note = [&](int k, uint32_t l) {
-                const uint32_t nu = u + l;
-                s_pos[k][threadIdx.x] = (u << 6) | l;
-                cross |= uint32_t((u ^ nu) >= 64u) << k;
-                u = nu;
-            };
-            if (valid == kEncPerThread)
-                pack_codes(lead + my_off, std::true_type{}, note);
-            else
-                pack_codes(lead + my_off, std::false_type{}, note);
             if (gaps32) {
-                for (; cross; cross &= cross - 1) {
-                    const int k = __ffs(cross) - 1;
-                    const uint32_t e = s_pos[k][threadIdx.x];
-                    window_event((e >> 6) - 63u, e & 63u, uint32_t(i0) + uint32_t(k));
+                // every window boundary in the thread's bits [A, A + bits)
+                // (A relative to Sb), at q from the thread's first bit, is
+                // covered by one code: the last one starting at or before it
+                // (binary search over the thread's starts; starts past the
+                // valid elements equal bits).  If that code starts before the
+                // boundary, the window's gap is where the next code starts (the
+                // gaps of windows that begin with a code stay 0); at a
+                // thread-block boundary the block's first element is that
+                // code's, or the next one's.
+                const uint32_t A = uint32_t(S - Sb) + my_off;
+                uint32_t* const gap_words = gaps32 + g0;
+                for (uint32_t q = (64u - (A & 63u)) & 63u; q < bits; q += 64) {
+                    uint32_t k = 0;
+                    if (s_pos[k + 8][threadIdx.x] <= q) k += 8;
+                    if (s_pos[k + 4][threadIdx.x] <= q) k += 4;
+                    if (s_pos[k + 2][threadIdx.x] <= q) k += 2;
+                    if (s_pos[k + 1][threadIdx.x] <= q) k += 1;
+                    const bool inside = s_pos[k][threadIdx.x] < q;  // the code starts before the boundary
+                    const uint32_t Bq = A + q;                       // the boundary, from Sb
+                    if (inside) {
+                        const uint32_t b = k + 1 < kEncPerThread ? s_pos[k + 1][threadIdx.x] : bits;
+                        const uint32_t gb = uint32_t(gap_bit0 + int32_t(5 * (Bq >> 6)));
+                        const uint32_t sh = gb & 31u, g = b - q;
+                        atomicOr(gap_words + (gb >> 5), g << sh);
+                        if (sh > 27) atomicOr(gap_words + (gb >> 5) + 1, g >> (32 - sh));
+                    }
+                    if ((Bq & uint32_t(block_mask)) == 0)
+                        block_off[blk_base + (Bq >> log2_block_bits)] = uint32_t(i0) + k + (inside ? 1u : 0u);
                 }
             }
         }
@@ -714,52 +632,6 @@ __global__ void __launch_bounds__(kEncThreads, 4) encode_kernel(const __grid_con
 #pragma unroll
                 for (int k = 0; k < int(kEncPerThread); k++)
                     if (uint32_t(k) < valid) sm[i0 + k] = uint8_t(smw[k >> 2] >> (8 * (k & 3)));
-            }
-        }
-        if constexpr (ES == 1) {
-            __syncthreads();
-            const uint32_t nwords = (lead + chunk_total + 31) >> 5;
-            const uint64_t W0 = S >> 5;
-            auto word = [&](uint32_t j) { return __byte_perm(s_words[j], 0, 0x0123); };  // MSB-first bytes
-            // the first and last words are shared with the neighbouring chunks
-            if (threadIdx.x == 0 || (threadIdx.x == 32 && nwords > 1)) {
-                const uint32_t j = threadIdx.x == 0 ? 0u : nwords - 1;
-                const uint32_t v = word(j);
-                if (v) atomicOr(exp32 + W0 + j, v);
-            }
-            // the words between: 16-byte stores from the first one at a 16-byte
-            // boundary of EncodedExponent, single words before and after
-            if (nwords > 2) {
-                const uint32_t jb = nwords - 1;                                // interior [1, jb)
-                const uint32_t ja = 1u + ((4u - uint32_t((W0 + 1) & 3u)) & 3u);  // W0 + ja is 4-word aligned
-                const uint32_t groups = ja < jb ? (jb - ja) / 4 : 0u;
-                const uint32_t jv = ja + 4 * groups;
-                if (threadIdx.x >= 64 && threadIdx.x < 70) {  // at most 3 words before, 3 after
-                    const uint32_t k = threadIdx.x - 64;
-                    const uint32_t j = k < 3 ? 1 + k : jv + (k - 3);
-                    if (k < 3 ? j < min(ja, jb) : j < jb) exp32[W0 + j] = word(j);
-                }
-                for (uint32_t g = threadIdx.x; g < groups; g += kEncThreads) {
-                    const uint32_t j = ja + 4 * g;
-                    *reinterpret_cast<uint4*>(exp32 + W0 + j) =
-                        make_uint4(word(j), word(j + 1), word(j + 2), word(j + 3));
-                }
-            }
-            if (gaps32) {
-                // gap words g0 .. g1; the first and last may hold other chunks' fields
-                const uint64_t w_last = (S + chunk_total - 1) >> 6;
-                const uint64_t g1 = (5 * w_last + 4) >> 5;
-                if (w_last > (S >> 6)) {
-                    const uint32_t ng = uint32_t(g1 - g0 + 1);
-                    for (uint32_t j = threadIdx.x; j < ng; j += kEncThreads) {
-                        const uint32_t v = s_gap[j];
-                        if (j == 0 || j == ng - 1) {
-                            if (v) atomicOr(gaps32 + g0 + j, v);
-                        } else {
-                            gaps32[g0 + j] = v;
-                        }
-                    }
-                }
             }
         }
         S += chunk_total;
