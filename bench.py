@@ -634,8 +634,14 @@ def run_native(args, rank: int, world: int, local_rank: int) -> None:
                 continue
             base, var = EXTRA_VARIANTS.get(c, (c, {}))
             opts = df11.decode_options(peek_bits=var["peek_bits"]) if "peek_bits" in var else None
-            other = Prepared(df11, base, rank, dev, chunks=var.get("chunks", False), options=opts)
+            # the 8-bit-symbol workload also times its own compress call
+            # (compress_u8), the other extras share the headline's codec
+            repeats = args.compress_repeats if base in U8_CONFIGS and not var and not args.no_compress else 0
+            other = Prepared(df11, base, rank, dev, chunks=var.get("chunks", False), compress_repeats=repeats,
+                             options=opts)
             rec = measure(other, args.steps, args.warmup, stream, dev, world)
+            if other.compress is not None:
+                rec["compress"] = other.compress
             if var:
                 rec["variant"] = ("independent chunks of 64 elements (start-bit table), no gaps or scan"
                                   if var.get("chunks") else
