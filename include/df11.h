@@ -234,7 +234,7 @@ df11_status df11_decompress_sms(const df11_header* hdr, const uint8_t* d_exp, co
  * PackedSignMantissa array; EncodedExponent, Gaps, block offsets, the code
  * table, the header and its sizes are as for BF16 streams (bytes_sm is not
  * used).  Arguments as for the BF16 calls, with segments of n bytes.
- * T must be 32, or 64 when no code is 1 bit long (df11_decompress_u8
+ * T must be 32 or 64, or 128 when no code is 1 bit long (df11_decompress_u8
  * returns DF11_ERR_INVALID otherwise). */
 df11_status df11_compress_plan_u8(const void* const* d_segs, const uint64_t* seg_counts, uint32_t n_segs,
                                   uint32_t threads_per_block, uint32_t max_code_len, void* d_workspace,

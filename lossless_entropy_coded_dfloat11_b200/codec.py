@@ -394,9 +394,9 @@ class HostStream:
 def compress_u8(tensors, names=None, threads_per_block: int = DEFAULT_THREADS_PER_BLOCK, max_code_len: int = 32,
                 stream=None) -> CompressedStream:
     """Compress one uint8 tensor (e.g. per-tensor quantized weights), or a
-    list, coding each byte whole with one shared table; no side array.  T = 64
-    or 128 falls back to T = 32 when the code has a 1-bit symbol (the decoders
-    with two or four windows per lane need codes of 2 bits or more)."""
+    list, coding each byte whole with one shared table; no side array.  T = 128
+    falls back to T = 32 when the code has a 1-bit symbol (the decoder with
+    four windows per lane needs codes of 2 bits or more)."""
     segs = _as_segments(tensors, torch.uint8)
     device = segs[0].device
     n = sum(t.numel() for t in segs)
@@ -408,7 +408,7 @@ def compress_u8(tensors, names=None, threads_per_block: int = DEFAULT_THREADS_PE
     B.call("df11_compress_plan_u8", ptrs, counts, len(segs), threads_per_block, max_code_len, _ptr(ws),
            ws.numel(), ctypes.byref(hdr), sh)
     ln = np.frombuffer(bytes(hdr.code_len), dtype=np.uint8)
-    if threads_per_block in (64, 128) and n and ln[ln > 0].min() == 1:
+    if threads_per_block == 128 and n and ln[ln > 0].min() == 1:
         token = hdr.plan_token  # the plan's per-range histograms do not depend on T
         hdr = make_header(ln, int(hdr.n_elems), int(hdr.total_bits), 32, max_code_len,
                           [t.numel() for t in segs])

@@ -1275,6 +1275,8 @@ constexpr int kWarpsTwoWindowsU8 = 32;
 // four windows per lane with 2-bit codes: 8,384 bytes of slots and staging
 // per warp, so 20 warps fit beside the tables
 constexpr int kWarpsFourWindows = 20;
+// two windows per lane with a 1-bit code: the same 8,384 bytes per warp
+constexpr int kWarpsTwoWindowsOneBit = 20;
 
 // How one stream is decoded: which kernel, its CTA shape and its shared
 // memory.  Warp kernels take up to `warps` warps per CTA, one CTA per SM; a
@@ -1465,8 +1467,9 @@ df11_status plan_for(const char* fn, const df11_header* hdr, bool u8, uint32_t p
             *out = warp_plan<kWarpsTwoWindowsU8, 4, 2, true>(8);
             return DF11_OK;
         }
-        if (T == 64 && min_len >= 2) {
-            *out = warp_plan<kWarpsTwoWindows, 2, 2, true>(7);
+        if (T == 64) {
+            *out = min_len >= 2 ? warp_plan<kWarpsTwoWindows, 2, 2, true>(7)
+                                : warp_plan<kWarpsTwoWindowsOneBit, 1, 2, true>(13);
             return DF11_OK;
         }
         if (T == 128 && min_len >= 2) {  // four windows per lane
@@ -1475,7 +1478,7 @@ df11_status plan_for(const char* fn, const df11_header* hdr, bool u8, uint32_t p
             return DF11_OK;
         }
         return fail(DF11_ERR_INVALID,
-                    "%s: streams of 8-bit symbols decode with T = 32, or T = 64 or 128 when no code is 1 bit long",
+                    "%s: streams of 8-bit symbols decode with T = 32 or 64, or 128 when no code is 1 bit long",
                     fn);
     }
     switch (T) {
@@ -1494,7 +1497,8 @@ df11_status plan_for(const char* fn, const df11_header* hdr, bool u8, uint32_t p
             }
             if (peek_bits && peek_bits != uint32_t(kPeekBits))
                 return fail(DF11_ERR_INVALID, "%s: narrow tables need codes of 2 bits or more", fn);
-            *out = block_plan<64>(1);
+            // a 1-bit code: slots and staging for 128 codes per lane
+            *out = warp_plan<kWarpsTwoWindowsOneBit, 1, 2, false>(13);
             return DF11_OK;
         case 128:  // four windows per lane when every code has 2 bits or more
             *out = min_len >= 2 ? warp_plan<kWarpsFourWindows, 2, 4, false>(14) : block_plan<128>(2);

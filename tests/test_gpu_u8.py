@@ -40,7 +40,7 @@ def decode_u8(cs) -> np.ndarray:
 def both_directions(w: inputs.Workload, T: int = df11.DEFAULT_THREADS_PER_BLOCK):
     v = flat_u8(w)
     counts = [t.numel() for t in w.tensors]
-    # library encoder (T = 64 or 128 falls back to 32 when a code is 1 bit long)
+    # library encoder (T = 128 falls back to 32 when a code is 1 bit long)
     cs = df11.compress_u8([t.cuda() for t in w.tensors], threads_per_block=T)
     s = oracle_stream(v, cs.threads_per_block)
     # oracle stream -> library u8 kernel
@@ -125,11 +125,18 @@ def test_llama8b_block_quantized_one_launch():
         assert torch.equal(got.cpu(), ref)
 
 
-def test_one_bit_code_needs_t32():
+def test_one_bit_code_decodes_at_t64_and_is_refused_at_t128():
+    """A 1-bit code puts up to 128 codes in a lane's two windows (T = 64: the
+    kernel instance with buffers for them) and 256 in four (T = 128: no
+    8-bit-symbol decoder, an argument error)."""
     v = flat_u8(inputs.edge_case_u8(5000, "one_value", 3))
     s = oracle_stream(v, 64)
     assert s.code_len[s.code_len > 0].min() == 1
     cs = df11.from_arrays(s.code_len, s.n_elems, s.total_bits, 64, s.exp, None, s.gaps, s.block_off,
+                          symbols="u8")
+    np.testing.assert_array_equal(decode_u8(cs), v)
+    s = oracle_stream(v, 128)
+    cs = df11.from_arrays(s.code_len, s.n_elems, s.total_bits, 128, s.exp, None, s.gaps, s.block_off,
                           symbols="u8")
     with pytest.raises(B.DF11Error) as e:
         df11.decompress_u8(cs)
