@@ -358,22 +358,38 @@ def step_stats(per_step_ms: list[float]) -> dict:
     return {"median": v[len(v) // 2], "min": v[0], "max": v[-1], "n": len(v)}
 
 
+# how the per-step statistics of back-to-back workloads are taken
+PER_STEP_SOURCE = ("a second pass of the same steps right after the timed one, with an event between "
+                   "consecutive steps: such an event keeps each launch from overlapping the previous one "
+                   "(~3 us per launch here), so the total comes from a pass with events at its ends only")
+
+
 def time_steps(step, steps: int, warmup: int, stream, flush=None) -> tuple[float, list[float]]:
-    """Run `warmup` untimed steps, then time `steps` steps with one CUDA event
-    between consecutive steps on the launching stream.  Without `flush` the
-    steps run back to back and the total is the first-to-last event span; with
-    it, a write of the flush buffer (larger than L2) precedes every step and
-    only the steps are summed."""
+    """Run `warmup` untimed steps, then time `steps` steps on the launching
+    stream.  Without `flush` the steps run back to back: the total is the span
+    between an event before the first step and one after the last, and the
+    per-step times come from a second pass of the same steps with an event
+    between consecutive steps (PER_STEP_SOURCE).  With `flush`, a write of the
+    flush buffer (larger than L2) precedes every step and only the steps,
+    each between its own pair of events, are summed."""
     import torch
     for _ in range(warmup):
         step()
     torch.cuda.synchronize()
     if flush is None:
-        ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
         # a short device-side wait ahead of the first event lets the host queue
         # the first launches before the GPU reaches it, so the first step does
         # not include the host's launch latency (the GPU would otherwise idle
         # between the event and the kernel)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda._sleep(LEAD_CYCLES)
+        e0.record(stream)
+        for _ in range(steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        total = e0.elapsed_time(e1)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
         torch.cuda._sleep(LEAD_CYCLES)
         ev[0].record(stream)
         for i in range(steps):
@@ -381,7 +397,7 @@ def time_steps(step, steps: int, warmup: int, stream, flush=None) -> tuple[float
             ev[i + 1].record(stream)
         torch.cuda.synchronize()
         per = [ev[i].elapsed_time(ev[i + 1]) for i in range(steps)]
-        return ev[0].elapsed_time(ev[-1]), per
+        return total, per
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     for i, (e0, e1) in enumerate(evs):
         flush.fill_(i & 0xFF)
@@ -465,6 +481,7 @@ def measure(pw: Prepared, steps: int, warmup: int, stream, dev, world: int) -> d
     import torch
     flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev) if pw.alg_bytes < 2 * L2_BYTES else None
     elapsed, per = time_steps(lambda: pw.step(stream), steps, warmup, stream, flush)
+    flushed = flush is not None
     del flush
     elapsed = max_over_ranks(elapsed, dev)
     exact, scope = pw.check(0, stream)
@@ -478,6 +495,7 @@ def measure(pw: Prepared, steps: int, warmup: int, stream, dev, world: int) -> d
     return {
         "workload": CONFIGS[pw.config], "metric": METRIC_U8 if pw.u8 else METRIC, "value": agg["gbs"],
         "unit": UNIT, "ms_per_step": agg["ms_per_step"], "per_step_ms": step_stats(per),
+        "per_step_source": "each step between its own pair of events" if flushed else PER_STEP_SOURCE,
         "elements_per_step": pw.elements, "elements_per_s": agg["gbs"] * 1e9 / pw.esize,
         "launches_per_step": launches, "bit_exact": exact, "bit_exact_scope": scope,
         "compression_ratio": sum(c.compressed_bytes() for c in pw.streams) / pw.out_bytes,
@@ -533,6 +551,7 @@ def run_native(args, rank: int, world: int, local_rank: int) -> None:
         elapsed, per_step = time_steps(lambda: pw.step(stream), args.steps, 0, stream, flush)
     if world > 1:
         dist.barrier()
+    flushed = flush is not None
     del flush
     exact, exact_scope = pw.check(rank, stream)
     per_rank = [max_over_ranks(elapsed, dev)] * world
@@ -608,6 +627,7 @@ def run_native(args, rank: int, world: int, local_rank: int) -> None:
                           "per-step CUDA events time the decode alone"),
                    "parallelism": f"replicas x{world} (independent streams per rank)"},
         "per_step_ms": step_stats(per_step),
+        "per_step_source": "each step between its own pair of events" if flushed else PER_STEP_SOURCE,
         "bit_exact": exact, "bit_exact_scope": exact_scope,
         "elements_per_s": agg["gbs"] * 1e9 / pw.esize,
         "compression_ratio": sum(c.compressed_bytes() for c in pw.streams) / pw.out_bytes,
