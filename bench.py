@@ -576,7 +576,7 @@ def run_native(args, rank: int, world: int, local_rank: int) -> None:
         e1.record(stream)
         torch.cuda.synchronize()
         ems = max_over_ranks(e0.elapsed_time(e1), dev)
-        e2e_exact = bool(torch.equal(pw.bits(res), pw.originals[0].cpu()))
+        e2e_exact = min_over_ranks(bool(torch.equal(pw.bits(res), pw.originals[0].cpu())), dev)
         e2e = {"value": pw.esize * pw.streams[0].n_elems * k * world / (ems * 1e-3) / 1e9, "unit": UNIT,
                "h2d_bytes_per_step": hs.h2d_bytes(), "d2h_bytes_per_step": hs.d2h_bytes(),
                "steps": k, "bit_exact": e2e_exact}
