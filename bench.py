@@ -513,11 +513,15 @@ def measure(pw: Prepared, steps: int, warmup: int, stream, dev, world: int) -> d
 
 
 # the workloads measured besides the headline one in a default run; the
-# last two are the C3 block again, through the independent-chunk container
-# (an ablation of the gap layout) and through the pages' 8-bit first-level
-# table (an ablation of the 12-bit one)
-EXTRA_CONFIGS = ["c4", "c2", "c1", "c5", "edge_one_value", "edge_uniform", "edge_zipf", "c3_chunks", "c3_peek8"]
-EXTRA_VARIANTS = {"c3_chunks": ("c3", dict(chunks=True)), "c3_peek8": ("c3", dict(peek_bits=8))}
+# last three are the C3 block again, through the independent-chunk container
+# (an ablation of the gap layout), through the pages' 8-bit first-level table
+# (an ablation of the 12-bit one), and with early staging (each launch stages
+# its tables and first loads while the previous one finishes: the previous
+# launch, a decode of the same stream, writes none of its arrays)
+EXTRA_CONFIGS = ["c4", "c2", "c1", "c5", "edge_one_value", "edge_uniform", "edge_zipf", "c3_chunks", "c3_peek8",
+                 "c3_early"]
+EXTRA_VARIANTS = {"c3_chunks": ("c3", dict(chunks=True)), "c3_peek8": ("c3", dict(peek_bits=8)),
+                  "c3_early": ("c3", dict(early_staging=True))}
 
 
 def run_native(args, rank: int, world: int, local_rank: int) -> None:
@@ -653,7 +657,8 @@ def run_native(args, rank: int, world: int, local_rank: int) -> None:
             if c == args.config:
                 continue
             base, var = EXTRA_VARIANTS.get(c, (c, {}))
-            opts = df11.decode_options(peek_bits=var["peek_bits"]) if "peek_bits" in var else None
+            opts = (df11.decode_options(peek_bits=var.get("peek_bits", 0), early_staging=var.get("early_staging", False))
+                    if "peek_bits" in var or "early_staging" in var else None)
             # the 8-bit-symbol workload also times its own compress call
             # (compress_u8), the other extras share the headline's codec
             repeats = args.compress_repeats if base in U8_CONFIGS and not var and not args.no_compress else 0
@@ -665,6 +670,9 @@ def run_native(args, rank: int, world: int, local_rank: int) -> None:
             if var:
                 rec["variant"] = ("independent chunks of 64 elements (start-bit table), no gaps or scan"
                                   if var.get("chunks") else
+                                  "early staging: tables and first loads of each launch staged while the "
+                                  "previous launch (a decode of the same stream) finishes"
+                                  if var.get("early_staging") else
                                   f"first-level table of {var['peek_bits']} bits held in 16 shared-memory copies")
             rec["gpu_launches"] = args.steps * rec["launches_per_step"]  # in its own timed region
             rec.pop("_elapsed_ms")

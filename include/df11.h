@@ -317,7 +317,17 @@ typedef struct {
                                     block_end) only, exactly as
                                     df11_decompress_blocks (same reads, writes
                                     only those blocks' output elements)          */
-    uint32_t reserved[2];        /* must be zero                                  */
+    uint32_t early_staging;      /* 1: the caller states that the kernel launched
+                                    right before this decode on the stream writes
+                                    none of this stream's arrays (tables, exponent
+                                    stream, gaps, offsets, sign+mantissa bytes) --
+                                    the previous block's decode, say, or a consumer
+                                    GEMM.  The warp kernel then stages its tables
+                                    and first loads while that kernel finishes and
+                                    waits for it only before it writes (B200's
+                                    programmatic dependent launch).  0 = wait
+                                    first (other values: DF11_ERR_INVALID)        */
+    uint32_t reserved;           /* must be zero                                  */
 } df11_decode_options;
 
 /* df11_decompress (symbols_u8 = 0, d_out: n_elems uint16) or

@@ -56,7 +56,8 @@ class DecodeOptions(ctypes.Structure):
         ("ctas", ctypes.c_uint32),
         ("block_begin", ctypes.c_uint32),
         ("block_end", ctypes.c_uint32),
-        ("reserved", ctypes.c_uint32 * 2),
+        ("early_staging", ctypes.c_uint32),
+        ("reserved", ctypes.c_uint32),
     ]
 
 

@@ -221,10 +221,15 @@ def to_host(cs: CompressedStream) -> dict:
 
 
 def decode_options(peek_bits: int = 0, max_sms: int = 0, max_warps_per_cta: int = 0, ctas: int = 0,
-                   block_begin: int = 0, block_end: int = 0):
+                   block_begin: int = 0, block_end: int = 0, early_staging: bool = False):
     """df11_decode_options (all zero: the library's defaults; a block range
-    decodes only those thread blocks, as decompress_blocks)."""
-    return B.DecodeOptions(peek_bits, max_sms, max_warps_per_cta, ctas, block_begin, block_end)
+    decodes only those thread blocks, as decompress_blocks).  early_staging:
+    the caller states that the kernel launched just before the decode on its
+    stream writes none of the stream's arrays (e.g. the previous block's
+    decode, or a consumer GEMM), so the decode stages its tables and first
+    loads while that kernel finishes."""
+    return B.DecodeOptions(peek_bits, max_sms, max_warps_per_cta, ctas, block_begin, block_end,
+                           1 if early_staging else 0, 0)
 
 
 def decompress(cs: CompressedStream, out: torch.Tensor | None = None, status: torch.Tensor | None = None,

@@ -65,6 +65,7 @@ struct DecodeArgs {
     uint32_t block0;     // first thread block to decode
     uint32_t n_blocks;   // thread blocks to decode, from block0
     uint32_t last_wend;  // bits of the last window inside the stream, 1..64
+    uint32_t early;      // stage the tables and first loads before waiting for the prior grid
 };
 
 struct Tables {
@@ -400,6 +401,7 @@ __device__ __forceinline__ bool bulk_end(uint32_t bar) {
 // Kernels launched with programmatic stream serialisation start while the
 // previous kernel on the stream drains; nothing is read before this.
 __device__ __forceinline__ void wait_for_prior_grids() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void allow_next_grid() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 // After the table copy and a CTA barrier: false (and the stream reported
 // corrupt) when the staged tables do not carry the library's magic word -- a
@@ -770,7 +772,13 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_warp_kernel(const Decode
     __shared__ __align__(8) unsigned long long s_bar;
     __shared__ uint32_t s_abort;
     const uint32_t bar = uint32_t(__cvta_generic_to_shared(&s_bar));
-    wait_for_prior_grids();
+    // the next grid on the stream may start its CTAs as this grid's exit
+    // (it waits for this grid before touching memory)
+    allow_next_grid();
+    // Early staging (the caller's statement that the prior grid writes none
+    // of this stream's arrays): the tables and the first block's loads are
+    // staged while the prior grid finishes; every write comes after the wait.
+    if (!a.early) wait_for_prior_grids();
     if (threadIdx.x == 0) bulk_warp_tables<K>(smem, reinterpret_cast<const uint8_t*>(a.lut), bar);
     copy_narrow_decode<K>(smem, a.lut, int(blockDim.x));
     // the first block's loads overlap the table copy
@@ -783,6 +791,7 @@ __global__ void __launch_bounds__(WARPS * 32, 1) decode_warp_kernel(const Decode
     }
     if (threadIdx.x == 0) s_abort = bulk_end(bar) ? 0u : 1u;
     __syncthreads();
+    if (a.early) wait_for_prior_grids();
     if (s_abort) {
         if (threadIdx.x == 0 && a.status) atomicOr(a.status, uint32_t(DF11_ERR_CORRUPT));
         return;
@@ -1543,13 +1552,14 @@ df11_status decompress_on(const char* fn, bool u8, const df11_header* hdr, const
     a.block0 = uint32_t(block_begin);
     a.n_blocks = uint32_t(block_end - block_begin);
     a.last_wend = uint32_t(hdr->total_bits - 64 * (hdr->n_threads - 1));
+    a.early = opt.early_staging;
     Plan p;
     st = plan_for(fn, hdr, u8, opt.peek_bits, &p);
     if (st != DF11_OK) return st;
     return launch_plan(p, a, opt, reinterpret_cast<cudaStream_t>(stream));
 }
 
-constexpr df11_decode_options kDefaultOptions{0, 0, 0, 0, 0, 0, {0, 0}};
+constexpr df11_decode_options kDefaultOptions{0, 0, 0, 0, 0, 0, 0, 0};
 
 }  // namespace
 }  // namespace df11
@@ -1578,8 +1588,8 @@ extern "C" df11_status df11_decompress_opts(const df11_header* hdr, const uint8_
                                             const void* d_lut, void* d_out, uint32_t symbols_u8,
                                             const df11_decode_options* opt, uint32_t* d_status, void* stream) {
     if (!opt) return fail(DF11_ERR_INVALID, "df11_decompress_opts: null options");
-    for (uint32_t r : opt->reserved)
-        if (r) return fail(DF11_ERR_INVALID, "df11_decompress_opts: reserved fields must be zero");
+    if (opt->reserved) return fail(DF11_ERR_INVALID, "df11_decompress_opts: reserved field must be zero");
+    if (opt->early_staging > 1) return fail(DF11_ERR_INVALID, "df11_decompress_opts: early_staging is 0 or 1");
     if (opt->block_begin || opt->block_end)
         return decompress_on("df11_decompress_opts", symbols_u8 != 0, hdr, d_exp, d_sm, d_gaps, d_block_off, d_lut,
                              d_out, d_status, *opt, stream, opt->block_begin, opt->block_end);

@@ -137,7 +137,11 @@ def test_bad_options_are_rejected_on_the_host():
             df11.decompress(cs, options=opts)
         assert e.value.code == B.DF11_ERR_INVALID
     bad = df11.decode_options()
-    bad.reserved[1] = 1
+    bad.reserved = 1
+    with pytest.raises(df11.DF11Error):
+        df11.decompress(cs, options=bad)
+    bad = df11.decode_options()
+    bad.early_staging = 2
     with pytest.raises(df11.DF11Error):
         df11.decompress(cs, options=bad)
     # narrow tables: BF16 streams with T = 64 only
@@ -147,3 +151,31 @@ def test_bad_options_are_rejected_on_the_host():
     q = df11.compress_u8([inputs.quantize_u8(inputs.gaussian((256, 256), 0.02, 96)).cuda()])
     with pytest.raises(df11.DF11Error):
         df11.decompress_u8(q, options=df11.decode_options(peek_bits=10))
+
+
+def test_early_staging_back_to_back():
+    """Consecutive decodes with early staging (each stages its tables and
+    first loads while the previous one finishes): bit-exact, through one
+    reused output buffer and through alternating streams' buffers."""
+    w1 = inputs.llama_block(dict(hidden=512, intermediate=1408, kv=128), seed_base=131)
+    w2 = inputs.llama_block(dict(hidden=512, intermediate=1408, kv=128), seed_base=137)
+    c1 = df11.compress([t.cuda() for t in w1.tensors])
+    c2 = df11.compress([t.cuda() for t in w2.tensors])
+    opts = df11.decode_options(early_staging=True)
+    out = torch.empty(max(c1.n_elems, c2.n_elems), dtype=torch.bfloat16, device="cuda")
+    r1 = torch.cat([t.reshape(-1) for t in w1.tensors]).view(torch.int16)
+    r2 = torch.cat([t.reshape(-1) for t in w2.tensors]).view(torch.int16)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for k in range(6):
+        cs, ref = (c1, r1) if k % 2 == 0 else (c2, r2)
+        got = df11.decompress(cs, out=out[: cs.n_elems], status=status, options=opts)
+        if k >= 4:  # the last two: check each after its own launch
+            torch.cuda.synchronize()
+            assert torch.equal(got.view(torch.int16).cpu(), ref)
+    assert int(status.item()) == 0
+    q = df11.compress_u8([inputs.quantize_u8(inputs.gaussian((512, 384), 0.02, 138)).cuda()])
+    ref8 = inputs.quantize_u8(inputs.gaussian((512, 384), 0.02, 138)).reshape(-1)
+    for _ in range(3):
+        got8 = df11.decompress_u8(q, options=opts)
+    torch.cuda.synchronize()
+    assert torch.equal(got8.cpu(), ref8)
